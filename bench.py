@@ -1,0 +1,399 @@
+"""Benchmark of the attention forward path on B200 (one JSON line on rank 0).
+
+Workload timed as `value`: causal bf16 attention forward, B=1 H=32 S=8192 D=128
+(the sequence-length-8192 causal case, scale 1/sqrt(128)), inputs N(0,1) from a seed,
+resident in HBM. q, k, v, out total 256 MiB, larger than the 126 MB L2, so no flush is
+needed between steps. One step = one fa_fwd launch.
+
+Also reported on the same line:
+  e2e          the same TFLOPS through the C ABI with pinned HOST buffers: each step copies
+               q, k, v to the device, runs fa_fwd, and copies out + lse back.
+  varlen       the packed path at 32 sequences x 64 tokens, H=16, D=128, bf16, padded batch
+               (1, 4096, 16, 128): unpad(q), unpad(k), unpad(v), varlen forward, pad(out),
+               in microseconds per call (and per component).
+  roofline     tensor-bound: achieved TFLOPS of the attention kernel vs the measured bf16 peak.
+  cpu_baseline the float64 CPU oracle on a bounded sample of the same workload.
+
+Launch: `python bench.py [--gpus N --steps K --warmup W]`; for N > 1 under
+torch.distributed.run, every rank runs the same per-GPU workload (weak scaling, no
+collective on the data path) and the time is the max over ranks.
+`--impl reference` times the float64 CPU oracle (the only reference this path has).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import fa_inputs  # noqa: E402
+
+METRIC = "attention fwd TFLOPS and % of B200 tensor-core peak; varlen µs/call"
+WORKLOAD = "llm_causal_bf16"
+KERNEL_SOURCES = ["tiled_exact_attention_fwd_b200/csrc/fa_fwd.cu", "tiled_exact_attention_fwd_b200/csrc/fa_ptx.cuh"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["hbm_gbs"]), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every ~10 ms while running."""
+
+    REASONS = {
+        0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+        0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+    }
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_info():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws: int, device):
+    torch.cuda.synchronize(device)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[device.index])
+    torch.cuda.synchronize(device)
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+def oracle_sample(budget_s: float = 12.0, threads: int = 0):
+    """Times the float64 oracle on evenly spaced query rows of head 0 of the causal workload.
+
+    Returns (tflops, seconds, rows, flops, threads_used). Row i (causal) costs 4*D*(i+1) flops,
+    the same count the GPU figure uses (4*B*H*S*S*D/2 over all rows, up to the diagonal term).
+    """
+    import numpy as np
+
+    import oracle
+    w = fa_inputs.WORKLOADS[WORKLOAD]
+    B, S, H, D = w["B"], w["S"], w["H"], w["D"]
+    # one head is enough for a bounded sample: draw it directly
+    q, k, v = (fa_inputs.normal((B, S, 1, D), torch.bfloat16, 100 + s) for s in range(3))
+    nth = threads if threads > 0 else oracle.max_threads()
+
+    def run(nrows):
+        rows = np.stack([np.zeros(nrows, np.int64), np.zeros(nrows, np.int64),
+                         np.linspace(0, S - 1, nrows).astype(np.int64)], axis=1)
+        t0 = time.perf_counter()
+        oracle.attention_dense(q, k, v, causal=w["causal"], rows=rows, nthreads=nth)
+        dt = time.perf_counter() - t0
+        flops = float(sum(4 * D * (int(i) + 1) for i in rows[:, 2]))
+        return dt, flops
+
+    n = 64
+    dt, fl = run(n)
+    while dt < budget_s / 8 and n < S:
+        n = min(S, n * 2)
+        dt, fl = run(n)
+    if dt < budget_s / 2 and n < S:
+        n = min(S, int(n * (budget_s / max(dt, 1e-3))))
+        dt, fl = run(n)
+    return fl / dt / 1e12, dt, n, fl, nth
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args):
+    ws, rank, local = dist_info()
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import tiled_exact_attention_fwd_b200 as fa
+    fa.lib()  # raises if the CUDA library is missing: there is no fallback
+
+    w = fa_inputs.WORKLOADS[WORKLOAD]
+    B, S, H, D, causal = w["B"], w["S"], w["H"], w["D"], w["causal"]
+    dt = fa_inputs.DTYPES[w["dtype"]]
+    q_h, k_h, v_h = fa_inputs.dense_qkv(B, S, H, D, dt, seed=rank)
+    q, k, v = q_h.to(device), k_h.to(device), v_h.to(device)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, S), device=device, dtype=torch.float32)
+    flops = fa.attention_flops(B, H, S, S, D, causal)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        fa.fa_fwd(q, k, v, out=out, lse=lse, causal=causal, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    barrier(ws, device)
+    sampler = ClockSampler(device.index)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(ws, device)
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms_local, ws, device)
+    st, where = fa.fa_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} at {where}")
+    value = flops * ws / (ms * 1e-3) / 1e12
+    kernel_tflops = flops / (ms_local * 1e-3) / 1e12
+
+    # ---- end to end through the C ABI with pinned host buffers
+    qp, kp, vp = (t.pin_memory() for t in (q_h, k_h, v_h))
+    op = torch.empty(q_h.shape, dtype=dt).pin_memory()
+    lp = torch.empty((B, H, S), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        q.copy_(qp, non_blocking=True)
+        k.copy_(kp, non_blocking=True)
+        v.copy_(vp, non_blocking=True)
+        fa.fa_fwd(q, k, v, out=out, lse=lse, causal=causal, stream=stream)
+        op.copy_(out, non_blocking=True)
+        lp.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    barrier(ws, device)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(ws, device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws, device)
+    h2d = 3 * q_h.numel() * q_h.element_size()
+    d2h = op.numel() * op.element_size() + lp.numel() * 4
+
+    # ---- packed path (unpad x3, varlen forward, pad), microseconds per call
+    varlen = run_varlen_leg(fa, device, stream, max(args.steps, 20), args.warmup, ws)
+    del qp, kp, vp, op, lp
+
+    peak_tf, peak_bw, peak_kind = load_peaks()
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1))",
+        "config": {"workload": "causal attention fwd, B=1 H=32 S=8192 D=128 bf16, scale 1/sqrt(128)",
+                   "B": B, "H": H, "S": S, "D": D, "causal": causal,
+                   "flops_per_step": flops, "l2": "inputs larger than L2 (q,k,v,out = 256 MiB); no flush",
+                   "parallelism": f"replicas x{ws} (independent per-GPU problems)"},
+        "gpu_launches": args.steps,
+        "e2e": {"value": round(flops * ws / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": {"bound": "tensor", "achieved": round(kernel_tflops, 2), "peak": peak_tf,
+                     "unit": "TFLOP/s", "frac": round(kernel_tflops / peak_tf, 4),
+                     "peak_kind": f"{peak_kind} bf16 dense (burst)", "kernel": "fa_fwd_kernel<128,bf16,causal>",
+                     "traffic": recorded_traffic("fa_fwd_kernel_d128_bf16_causal")},
+        "varlen": varlen,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        tf, secs, nrows, fl, nth = oracle_sample()
+        result["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOPS", "cores": nth, "kind": "oracle",
+                                  "sample": f"{nrows} evenly spaced query rows of head 0 (causal, S=8192, D=128),"
+                                            f" {fl:.3g} flops in {secs:.1f} s, float64"}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_varlen_leg(fa, device, stream, iters, warmup, ws):
+    w = fa_inputs.WORKLOADS["varlen_bf16_32x64"]
+    case = fa_inputs.workload_inputs("varlen_bf16_32x64")
+    qp, kp, vp = case.q_pad.to(device), case.k_pad.to(device), case.v_pad.to(device)
+    idx, cu = case.indices.to(device), case.cu_seqlens.to(device)
+    H, D = w["H"], w["D"]
+    qu = torch.empty((case.nnz, H, D), device=device, dtype=qp.dtype)
+    ku, vu, ou = torch.empty_like(qu), torch.empty_like(qu), torch.empty_like(qu)
+    lse = torch.empty((H, case.nnz), device=device, dtype=torch.float32)
+    out_pad = torch.empty_like(qp)
+    # L2 flush buffer (2x L2) written between timed calls: the inputs here are L2-sized
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    def call():
+        fa.fa_unpad(qp, idx, out=qu, stream=stream)
+        fa.fa_unpad(kp, idx, out=ku, stream=stream)
+        fa.fa_unpad(vp, idx, out=vu, stream=stream)
+        fa.fa_varlen_fwd(qu, ku, vu, cu, case.max_seqlen, out=ou, lse=lse, stream=stream)
+        fa.fa_pad(ou, idx, 1, case.total_len, out=out_pad, stream=stream)
+
+    for _ in range(max(warmup, 3)):
+        call()
+    torch.cuda.synchronize(device)
+    n_ev = 6
+    tot = [0.0] * 5
+    whole = []
+    for it in range(iters):
+        flush.fill_(it & 0xFF)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+        ev[0].record(stream)
+        fa.fa_unpad(qp, idx, out=qu, stream=stream)
+        fa.fa_unpad(kp, idx, out=ku, stream=stream)
+        fa.fa_unpad(vp, idx, out=vu, stream=stream)
+        ev[1].record(stream)
+        fa.fa_varlen_fwd(qu, ku, vu, cu, case.max_seqlen, out=ou, lse=lse, stream=stream)
+        ev[2].record(stream)
+        fa.fa_pad(ou, idx, 1, case.total_len, out=out_pad, stream=stream)
+        ev[3].record(stream)
+        torch.cuda.synchronize(device)
+        whole.append(ev[0].elapsed_time(ev[3]) * 1e3)
+        tot[0] += ev[0].elapsed_time(ev[1]) * 1e3
+        tot[1] += ev[1].elapsed_time(ev[2]) * 1e3
+        tot[2] += ev[2].elapsed_time(ev[3]) * 1e3
+    flops = 4.0 * H * D * sum(int(x) ** 2 for x in (case.cu_seqlens[1:] - case.cu_seqlens[:-1]))
+    us = statistics.median(whole)
+    return {"value": round(us, 2), "unit": "us/call", "stat": f"median of {iters}, L2 flushed before each call",
+            "config": "32 seqs x 64 tokens, H=16 D=128 bf16, padded (1,4096,16,128), non-causal",
+            "components_us_mean": {"unpad_qkv": round(tot[0] / iters, 2), "varlen_fwd": round(tot[1] / iters, 2),
+                                   "pad_out": round(tot[2] / iters, 2)},
+            "varlen_fwd_tflops": round(flops / (tot[1] / iters * 1e-6) / 1e12, 2),
+            "gpu_launches_per_call": 5}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    ws, rank, local = dist_info()
+    if rank != 0:
+        return
+    import oracle
+    w = fa_inputs.WORKLOADS[WORKLOAD]
+    nth = oracle.max_threads()
+    # Each step: the oracle on a bounded sample (evenly spaced rows of head 0), ~2 s.
+    per = []
+    rows_used = flops_used = None
+    for i in range(args.warmup + args.steps):
+        tf, secs, nrows, fl, _ = oracle_sample(budget_s=2.0)
+        if i >= args.warmup:
+            per.append((tf, secs))
+            rows_used, flops_used = nrows, fl
+    value = statistics.mean(t for t, _ in per)
+    ms = statistics.mean(s for _, s in per) * 1e3
+    sample = (f"{rows_used} evenly spaced query rows of head 0 of the causal S=8192 D=128 workload, "
+              f"{flops_used:.3g} flops per step, float64")
+    res = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))", "impl": "reference",
+           "config": {"workload": "causal attention fwd, B=1 H=32 S=8192 D=128 bf16, scale 1/sqrt(128)",
+                      "B": w["B"], "H": w["H"], "S": w["S"], "D": w["D"], "causal": True},
+           "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": nth, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

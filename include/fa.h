@@ -1,0 +1,134 @@
+/*
+ * fa.h -- C ABI of libfa: exact attention forward computed tile by tile on one
+ * NVIDIA B200 (sm_100a), plus the unpad gather and pad scatter of the packed path.
+ *
+ * Every entry point is asynchronous on the caller's CUDA stream, allocates no
+ * device memory, never synchronises, and takes plain device pointers that the
+ * caller allocates and owns. Arguments are validated on the host before any
+ * launch; a rejected call launches nothing and returns a negative status.
+ *
+ * Definitions followed (pages are cited by title and section):
+ *   - standard attention, page "昇腾CANN跑大模型，FlashAttention这个算子你得认识一下",
+ *     section "传统实现到底慢在哪": O = softmax(Q K^T * scale) V, scale = 1/sqrt(d_k);
+ *   - tiling and the online softmax (running row max and row sum, correction of the
+ *     earlier partial output), same page, section "分块计算，这事没那么简单";
+ *   - causal masking fused with skipping of masked blocks, same page, section
+ *     "昇腾NPU上做了什么特殊优化";
+ *   - the packed path unpad -> flash_attn_varlen_func -> pad, page
+ *     "IAW 模型 FA2 vs FA3 实测", sections 1 and 2.
+ *
+ * Layouts (all contiguous, row-major, element type fp16 or bf16 unless stated):
+ *   dense  q, k, v, out : (B, S, H, D)         lse : (B, H, S)   float32
+ *   packed q, k, v, out : (total, H, D)        lse : (H, total)  float32
+ *   lse is the natural log of sum_j exp(scale * q.k_j) over the keys the row sees.
+ *
+ * Supported: D in {32, 64, 128, 256}; q, k, v, out 16-byte aligned; lse 4-byte
+ * aligned (may be NULL to skip it). Causal masking is aligned at the first token
+ * of each sequence (query and key lengths are equal per sequence).
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_NULL = -1,     /* a required pointer is NULL */
+    FA_ERR_SHAPE = -2,    /* a size is negative, zero where it must not be, or overflows */
+    FA_ERR_DTYPE = -3,    /* dtype is not FA_FP16 / FA_BF16 */
+    FA_ERR_HEADDIM = -4,  /* D is not 32, 64, 128 or 256 */
+    FA_ERR_ALIGN = -5,    /* a pointer or row size breaks the alignment rule */
+    FA_ERR_CUDA = -6,     /* a CUDA runtime/driver call failed (launch, tensor map) */
+    FA_ERR_TIMEOUT = -7,  /* a kernel's bounded wait ran out (reported by fa_device_status) */
+    FA_ERR_INDEX = -8     /* an index was out of range (reported by fa_device_status) */
+} fa_status;
+
+typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
+
+/*
+ * Dense attention forward.
+ *   q, k, v   (B, S, H, D) inputs, element type `dtype`.
+ *   out       (B, S, H, D) output, same type; every element is written.
+ *   lse       (B, H, S) float32 log-sum-exp, or NULL.
+ *   scale     score scale; <= 0 selects 1/sqrt(D).
+ *   causal    nonzero: query i sees keys 0..i only; fully masked key tiles are skipped.
+ *   stream    a cudaStream_t (NULL = the legacy default stream).
+ * B, H, S >= 1 (S may be any length; a ragged last tile is masked).
+ */
+FA_API fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
+                 int B, int H, int S, int D, float scale, int causal, fa_dtype dtype,
+                 void *stream);
+
+/*
+ * Packed variable-length attention forward (the flash_attn_varlen_func step).
+ *   q, k, v      (total, H, D) packed inputs; sequence s owns rows
+ *                [cu_seqlens[s], cu_seqlens[s+1]) and attends only inside itself.
+ *   cu_seqlens   device int32 array of num_seqs+1 non-decreasing offsets, cu_seqlens[0] = 0,
+ *                cu_seqlens[num_seqs] = total (read on the device; not checked on the host).
+ *   max_seqlen   an upper bound of every sequence length (sizes the launch grid).
+ *   out          (total, H, D); lse (H, total) float32 or NULL.
+ * Zero-length sequences are allowed and produce no rows. total may be 0 (no launch).
+ */
+FA_API fa_status fa_varlen_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqlens,
+                        int num_seqs, int max_seqlen, int total, void *out, float *lse, int H,
+                        int D, float scale, int causal, fa_dtype dtype, void *stream);
+
+/*
+ * Unpad (gather): out[r, :] = x[indices[r], :] for r < nnz, rows of `row_bytes` bytes.
+ *   x        (total_rows, row_bytes) padded input, e.g. (B*total_len, H*D*elt).
+ *   indices  device int64 [nnz], each in [0, total_rows).
+ *   out      (nnz, row_bytes).
+ * Bit-exact byte copy, so one call serves every dtype. Rows whose index is out of range
+ * are written as zeros and flag FA_ERR_INDEX for fa_device_status. 16-byte vectors are
+ * used when row_bytes and both pointers are 16-byte aligned; otherwise a byte loop.
+ */
+FA_API fa_status fa_unpad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
+                   int64_t row_bytes, void *out, void *stream);
+
+/*
+ * Pad (scatter + zero fill): out[indices[r], :] = x[r, :] for r < nnz and every other
+ * row of out (total_rows, row_bytes) is zero. Each output row is written exactly once.
+ *   indices  device int64 [nnz], strictly increasing, each in [0, total_rows)
+ *            (the order a nonzero() over a padding mask produces). Entries that break
+ *            this rule leave the affected rows unspecified but never cause an access
+ *            outside the buffers.
+ */
+FA_API fa_status fa_pad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
+                 int64_t row_bytes, void *out, void *stream);
+
+/*
+ * Device-side status of earlier launches: synchronises the device, returns FA_OK or the
+ * first FA_ERR_TIMEOUT / FA_ERR_INDEX recorded by a kernel since the last call, and
+ * clears it. `where` (may be NULL) receives a kernel-specific location code.
+ */
+FA_API fa_status fa_device_status(int *where);
+
+/*
+ * Self-test of the bounded wait used by every pipeline wait in the attention kernel:
+ * launches one CTA that waits on a barrier nothing ever completes, with a limit of
+ * `limit_ns` nanoseconds. The kernel gives up, records FA_ERR_TIMEOUT and returns, so
+ * fa_device_status must then report FA_ERR_TIMEOUT.
+ */
+FA_API fa_status fa_selftest_bounded_wait(uint64_t limit_ns, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+FA_API const char *fa_status_string(int status);
+
+/* Library version string (static storage). */
+FA_API const char *fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

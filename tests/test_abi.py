@@ -1,0 +1,91 @@
+"""The C-ABI library loads, exports every symbol include/fa.h declares, and its host-side
+argument validation rejects bad calls before any launch (CPU only: no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import tiled_exact_attention_fwd_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"FA_API\s+[^;(]*?\b(fa_\w+)\s*\(", text)
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tiled_exact_attention_fwd_b200 import build
+    build.build()
+    return fa.lib()
+
+
+def test_header_declares_the_boundary():
+    names = set(_declared_symbols())
+    for required in ("fa_fwd", "fa_varlen_fwd", "fa_unpad", "fa_pad"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_symbols()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code, name in fa.STATUS.items():
+        assert lib.fa_status_string(code).decode().startswith(name)
+    assert b"unknown" in lib.fa_status_string(12345)
+    assert b"sm_100a" in lib.fa_version()
+
+
+# Host-side validation returns before any CUDA call, so it is exercised here without a GPU.
+FAKE = 1 << 20  # a 16-byte aligned non-null address that is never dereferenced
+
+
+def test_fwd_rejects_null(lib):
+    assert lib.fa_fwd(None, FAKE, FAKE, FAKE, None, 1, 1, 128, 64, 0.0, 0, 0, None) == -1
+    assert lib.fa_fwd(FAKE, FAKE, FAKE, None, None, 1, 1, 128, 64, 0.0, 0, 0, None) == -1
+
+
+def test_fwd_rejects_head_dim_dtype_shape_align(lib):
+    assert lib.fa_fwd(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 128, 96, 0.0, 0, 0, None) == -4
+    assert lib.fa_fwd(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 128, 64, 0.0, 0, 7, None) == -3
+    assert lib.fa_fwd(FAKE, FAKE, FAKE, FAKE, None, 0, 1, 128, 64, 0.0, 0, 0, None) == -2
+    assert lib.fa_fwd(FAKE, FAKE, FAKE, FAKE, None, 1, 0, 128, 64, 0.0, 0, 0, None) == -2
+    assert lib.fa_fwd(FAKE, FAKE, FAKE, FAKE, None, 1, 1, -5, 64, 0.0, 0, 0, None) == -2
+    assert lib.fa_fwd(FAKE, FAKE, FAKE, FAKE, None, 70000, 1, 128, 64, 0.0, 0, 0, None) == -2
+    assert lib.fa_fwd(FAKE + 8, FAKE, FAKE, FAKE, None, 1, 1, 128, 64, 0.0, 0, 0, None) == -5
+    assert lib.fa_fwd(FAKE, FAKE, FAKE, FAKE, FAKE + 2, 1, 1, 128, 64, 0.0, 0, 0, None) == -5
+
+
+def test_varlen_validation(lib):
+    # empty problems are a successful no-op
+    assert lib.fa_varlen_fwd(None, None, None, None, 0, 0, 0, None, None, 4, 64, 0.0, 0, 1, None) == 0
+    assert lib.fa_varlen_fwd(FAKE, FAKE, FAKE, FAKE, 3, 0, 10, FAKE, None, 4, 64, 0.0, 0, 1, None) == -2
+    assert lib.fa_varlen_fwd(FAKE, FAKE, FAKE, None, 3, 8, 10, FAKE, None, 4, 64, 0.0, 0, 1, None) == -1
+    assert lib.fa_varlen_fwd(FAKE, FAKE, FAKE, FAKE, 3, 8, 10, FAKE, None, 4, 48, 0.0, 0, 1, None) == -4
+    assert lib.fa_varlen_fwd(FAKE, FAKE, FAKE, FAKE + 2, 3, 8, 10, FAKE, None, 4, 64, 0.0, 0, 1, None) == -5
+
+
+def test_pad_unpad_validation(lib):
+    assert lib.fa_unpad(None, None, 0, 10, 64, None, None) == 0
+    assert lib.fa_unpad(FAKE, None, 4, 10, 64, FAKE, None) == -1
+    assert lib.fa_unpad(FAKE, FAKE, -1, 10, 64, FAKE, None) == -2
+    assert lib.fa_unpad(FAKE, FAKE + 4, 4, 10, 64, FAKE, None) == -5
+    assert lib.fa_pad(FAKE, FAKE, 11, 10, 64, FAKE, None) == -2
+    assert lib.fa_pad(None, None, 0, 0, 64, None, None) == 0
+    assert lib.fa_pad(FAKE, FAKE, 4, 10, 0, FAKE, None) == -2
+    assert lib.fa_pad(FAKE, FAKE, 4, 10, 64, None, None) == -1
+
+
+def test_selftest_rejects_bad_limit(lib):
+    assert lib.fa_selftest_bounded_wait(0, None) == -2

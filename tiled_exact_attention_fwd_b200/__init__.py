@@ -1,0 +1,197 @@
+"""Python binding of libfa (include/fa.h): exact attention forward on B200 (sm_100a).
+
+This module only marshals torch CUDA tensors into the C ABI: every step of the
+computation runs in the library's kernels. There is no fallback: if libfa.so is not
+built, every call raises.
+
+    out, lse = fa_fwd(q, k, v, causal=True)                         # dense (B, S, H, D)
+    out, lse = fa_varlen_fwd(q, k, v, cu_seqlens, max_seqlen)        # packed (total, H, D)
+    x_unpad  = fa_unpad(x, indices)                                  # (B, L, H, D) -> (nnz, H, D)
+    x_pad    = fa_pad(x_unpad, indices, batch, total_len)            # (nnz, H, D) -> (B, L, H, D)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK = 0
+FA_FP16 = 0
+FA_BF16 = 1
+STATUS = {0: "FA_OK", -1: "FA_ERR_NULL", -2: "FA_ERR_SHAPE", -3: "FA_ERR_DTYPE", -4: "FA_ERR_HEADDIM",
+          -5: "FA_ERR_ALIGN", -6: "FA_ERR_CUDA", -7: "FA_ERR_TIMEOUT", -8: "FA_ERR_INDEX"}
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib().fa_status_string(status).decode()} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libfa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run `python -m tiled_exact_attention_fwd_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+        L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
+        L.fa_varlen_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, i32, i32, f32, i32, i32, vp]
+        L.fa_unpad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
+        L.fa_pad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
+        L.fa_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        L.fa_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
+        for f in (L.fa_fwd, L.fa_varlen_fwd, L.fa_unpad, L.fa_pad, L.fa_device_status,
+                  L.fa_selftest_bounded_wait):
+            f.restype = ctypes.c_int
+        L.fa_status_string.argtypes = [ctypes.c_int]
+        L.fa_status_string.restype = ctypes.c_char_p
+        L.fa_version.argtypes = []
+        L.fa_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != FA_OK:
+        raise FAError(status, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return FA_FP16
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; expected float16 or bfloat16")
+
+
+def _cuda_contig(name: str, t: torch.Tensor) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torch.Tensor] = None,
+           lse: Optional[torch.Tensor] = None, scale: Optional[float] = None, causal: bool = False,
+           return_lse: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Dense forward: q, k, v (B, S, H, D) -> out (B, S, H, D), lse (B, H, S) fp32."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _cuda_contig(n, t)
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one (B, S, H, D) shape and dtype")
+    B, S, H, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _cuda_contig("out", out)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
+    if lse is not None:
+        _cuda_contig("lse", lse)
+    st = lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                      float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
+    _check(st, "fa_fwd")
+    return out, lse
+
+
+def fa_varlen_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                  max_seqlen: int, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                  scale: Optional[float] = None, causal: bool = False, return_lse: bool = True,
+                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Packed forward: q, k, v (total, H, D) with int32 cu_seqlens -> out (total, H, D), lse (H, total)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("cu_seqlens", cu_seqlens)):
+        _cuda_contig(n, t)
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one (total, H, D) shape and dtype")
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor")
+    total, H, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _cuda_contig("out", out)
+    if return_lse and lse is None:
+        lse = torch.empty((H, total), device=q.device, dtype=torch.float32)
+    if lse is not None:
+        _cuda_contig("lse", lse)
+    st = lib().fa_varlen_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                             int(max_seqlen), total, _ptr(out), _ptr(lse), H, D,
+                             float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
+    _check(st, "fa_varlen_fwd")
+    return out, lse
+
+
+def fa_unpad(x: torch.Tensor, indices: torch.Tensor, out: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    """(B, L, H, D) (or any (..., H, D)) -> (nnz, H, D): rows taken by int64 indices."""
+    _cuda_contig("x", x)
+    _cuda_contig("indices", indices)
+    if indices.dtype != torch.int64:
+        raise ValueError("indices must be int64")
+    H, D = x.shape[-2], x.shape[-1]
+    row_bytes = H * D * x.element_size()
+    total_rows = x.numel() // (H * D)
+    nnz = indices.numel()
+    if out is None:
+        out = torch.empty((nnz, H, D), device=x.device, dtype=x.dtype)
+    _cuda_contig("out", out)
+    st = lib().fa_unpad(_ptr(x), _ptr(indices), nnz, total_rows, row_bytes, _ptr(out), _stream(stream))
+    _check(st, "fa_unpad")
+    return out
+
+
+def fa_pad(x: torch.Tensor, indices: torch.Tensor, batch: int, total_len: int,
+           out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """(nnz, H, D) -> (batch, total_len, H, D): rows put back by int64 indices, zeros elsewhere."""
+    _cuda_contig("x", x)
+    _cuda_contig("indices", indices)
+    if indices.dtype != torch.int64:
+        raise ValueError("indices must be int64")
+    nnz, H, D = x.shape
+    if out is None:
+        out = torch.empty((batch, total_len, H, D), device=x.device, dtype=x.dtype)
+    _cuda_contig("out", out)
+    st = lib().fa_pad(_ptr(x), _ptr(indices), nnz, batch * total_len, H * D * x.element_size(), _ptr(out),
+                      _stream(stream))
+    _check(st, "fa_pad")
+    return out
+
+
+def fa_device_status() -> Tuple[int, int]:
+    """(status, where) recorded by kernels since the last call (synchronises the device)."""
+    where = ctypes.c_int(0)
+    st = lib().fa_device_status(ctypes.byref(where))
+    return st, where.value
+
+
+def fa_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
+    _check(lib().fa_selftest_bounded_wait(int(limit_ns), _stream(stream)), "fa_selftest_bounded_wait")
+
+
+def version() -> str:
+    return lib().fa_version().decode()
+
+
+def attention_flops(B: int, H: int, Sq: int, Sk: int, D: int, causal: bool) -> float:
+    """4*B*H*Sq*Sk*D (two matmuls of 2*Sq*Sk*D each), halved for causal."""
+    f = 4.0 * B * H * Sq * Sk * D
+    return f / 2 if causal else f

@@ -1,0 +1,190 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument validation, TMA tensor-map
+// encoding and kernel dispatch. No entry point allocates, synchronises (except
+// fa_device_status, whose job it is) or touches host copies of tensor data.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#include <atomic>
+
+#include "fa.h"
+#include "fa_internal.h"
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static std::atomic<EncodeTiledFn> fn{nullptr};
+    EncodeTiledFn f = fn.load(std::memory_order_acquire);
+    if (!f) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess && p) {
+            f = reinterpret_cast<EncodeTiledFn>(p);
+            fn.store(f, std::memory_order_release);
+        }
+    }
+    return f;
+}
+
+uint64_t wait_limit_ns() {
+    static std::atomic<uint64_t> lim{0};
+    uint64_t v = lim.load(std::memory_order_relaxed);
+    if (v == 0) {
+        v = 2000000000ull;  // 2 s: every wait inside a CTA normally lasts microseconds
+        if (const char *e = getenv("FA_WAIT_LIMIT_NS")) {
+            const unsigned long long x = strtoull(e, nullptr, 10);
+            if (x > 0) v = x;
+        }
+        lim.store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool head_dim_ok(int D) { return D == 32 || D == 64 || D == 128 || D == 256; }
+
+// Token-major (N, H, D) 16-bit tensor seen by TMA as dims (D, H, N); one box is
+// `inner` elements of one head of `rows` consecutive tokens (a [rows][inner] tile).
+bool encode_map(CUtensorMap *m, const void *base, bool bf16, int D, int H, int64_t N, int inner, int rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(inner), 1, static_cast<cuuint32_t>(rows)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw = (inner * 2 == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUresult r = f(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                         const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
+                  const int32_t *cu_seqlens, int num_seqs, int seqlen_or_max, int64_t N, int H, int D,
+                  float scale, int causal, fa_dtype dtype, void *stream) {
+    const bool bf16 = dtype == FA_BF16;
+    const int inner = fa::fwd_box_inner_elems(D);
+    CUtensorMap tq, tk, tv;
+    if (!encode_map(&tq, q, bf16, D, H, N, inner, fa::fwd_tile_rows()) ||
+        !encode_map(&tk, k, bf16, D, H, N, inner, fa::fwd_kv_tile_rows(D)) ||
+        !encode_map(&tv, v, bf16, D, H, N, inner, fa::fwd_kv_tile_rows(D)))
+        return FA_ERR_CUDA;
+    if (!(scale > 0.f)) scale = 1.0f / sqrtf(static_cast<float>(D));
+    fa::FwdParams p;
+    p.out = out;
+    p.lse = lse;
+    p.cu_seqlens = cu_seqlens;
+    p.seqlen = seqlen_or_max;
+    p.H = H;
+    p.total_tokens = static_cast<int>(N);
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.timeout_ns = wait_limit_ns();
+    const int qtiles = (seqlen_or_max + fa::fwd_tile_rows() - 1) / fa::fwd_tile_rows();
+    const dim3 grid(static_cast<unsigned>(H), static_cast<unsigned>(qtiles), static_cast<unsigned>(num_seqs));
+    const cudaError_t e = fa::launch_fwd(D, bf16, causal != 0, tq, tk, tv, p, grid,
+                                         static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
+                 int D, float scale, int causal, fa_dtype dtype, void *stream) {
+    if (!q || !k || !v || !out) return FA_ERR_NULL;
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (!head_dim_ok(D)) return FA_ERR_HEADDIM;
+    if (B <= 0 || H <= 0 || S <= 0) return FA_ERR_SHAPE;
+    const int64_t N = static_cast<int64_t>(B) * S;
+    if (N > INT32_MAX || B > 65535 || (S + 127) / 128 > 65535) return FA_ERR_SHAPE;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
+        return FA_ERR_ALIGN;
+    return run_fwd(q, k, v, out, lse, nullptr, B, S, N, H, D, scale, causal, dtype, stream);
+}
+
+fa_status fa_varlen_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqlens, int num_seqs,
+                        int max_seqlen, int total, void *out, float *lse, int H, int D, float scale, int causal,
+                        fa_dtype dtype, void *stream) {
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (!head_dim_ok(D)) return FA_ERR_HEADDIM;
+    if (num_seqs < 0 || total < 0 || max_seqlen < 0 || H <= 0) return FA_ERR_SHAPE;
+    if (total == 0 || num_seqs == 0) return FA_OK;  // no rows, nothing to launch
+    if (!q || !k || !v || !out || !cu_seqlens) return FA_ERR_NULL;
+    if (max_seqlen == 0) return FA_ERR_SHAPE;
+    if (num_seqs > 65535 || (max_seqlen + 127) / 128 > 65535) return FA_ERR_SHAPE;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
+        !aligned(cu_seqlens, 4))
+        return FA_ERR_ALIGN;
+    return run_fwd(q, k, v, out, lse, cu_seqlens, num_seqs, max_seqlen, total, H, D, scale, causal, dtype,
+                   stream);
+}
+
+fa_status fa_unpad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows, int64_t row_bytes,
+                   void *out, void *stream) {
+    if (nnz < 0 || total_rows < 0 || row_bytes <= 0) return FA_ERR_SHAPE;
+    if (nnz == 0) return FA_OK;
+    if (!x || !indices || !out) return FA_ERR_NULL;
+    if (!aligned(indices, 8)) return FA_ERR_ALIGN;
+    const cudaError_t e = fa::launch_unpad(x, indices, nnz, total_rows, row_bytes, out,
+                                           static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_pad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows, int64_t row_bytes,
+                 void *out, void *stream) {
+    if (nnz < 0 || total_rows < 0 || row_bytes <= 0 || nnz > total_rows) return FA_ERR_SHAPE;
+    if (total_rows == 0) return FA_OK;
+    if (!out || (nnz > 0 && (!x || !indices))) return FA_ERR_NULL;
+    if (!aligned(indices, 8)) return FA_ERR_ALIGN;
+    const cudaError_t e = fa::launch_pad(x, indices, nnz, total_rows, row_bytes, out,
+                                         static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_device_status(int *where) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+    int c1 = 0, w1 = 0, c2 = 0, w2 = 0;
+    if (fa::fwd_take_device_error(&c1, &w1) != cudaSuccess) return FA_ERR_CUDA;
+    if (fa::pad_take_device_error(&c2, &w2) != cudaSuccess) return FA_ERR_CUDA;
+    if (where) *where = c1 ? w1 : w2;
+    if (c1) return static_cast<fa_status>(c1);
+    if (c2) return static_cast<fa_status>(c2);
+    return FA_OK;
+}
+
+fa_status fa_selftest_bounded_wait(uint64_t limit_ns, void *stream) {
+    if (limit_ns == 0 || limit_ns > 10000000000ull) return FA_ERR_SHAPE;
+    return fa::launch_selftest_wait(limit_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK
+                                                                                                : FA_ERR_CUDA;
+}
+
+const char *fa_status_string(int status) {
+    switch (status) {
+        case FA_OK: return "FA_OK";
+        case FA_ERR_NULL: return "FA_ERR_NULL: a required pointer is NULL";
+        case FA_ERR_SHAPE: return "FA_ERR_SHAPE: unsupported or inconsistent sizes";
+        case FA_ERR_DTYPE: return "FA_ERR_DTYPE: dtype must be FA_FP16 or FA_BF16";
+        case FA_ERR_HEADDIM: return "FA_ERR_HEADDIM: head dim must be 32, 64, 128 or 256";
+        case FA_ERR_ALIGN: return "FA_ERR_ALIGN: tensors must be 16-byte aligned (lse 4-byte)";
+        case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
+        case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a kernel's bounded wait ran out";
+        case FA_ERR_INDEX: return "FA_ERR_INDEX: an index was out of range";
+        default: return "unknown fa_status";
+    }
+}
+
+const char *fa_version(void) { return "fa-b200 0.1 (sm_100a: tcgen05 + TMEM + TMA)"; }
+
+}  // extern "C"

@@ -1,0 +1,38 @@
+// fa_internal.h -- declarations shared by the C-ABI layer and the kernel translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+// Kernel parameters of the attention forward (passed by value).
+struct FwdParams {
+    void *out;                  // token-major (N, H, D) output
+    float *lse;                 // dense: (B, H, S); packed: (H, total); may be null
+    const int32_t *cu_seqlens;  // null for dense (uniform sequences of `seqlen`)
+    int seqlen;                 // dense sequence length
+    int H;                      // heads
+    int total_tokens;           // N = rows of the token-major tensors
+    float scale_log2;           // scale * log2(e)
+    uint64_t timeout_ns;        // bound of every pipeline wait
+};
+
+// Attention forward: grid (H, ceil(max_len / 128), num_seqs), one CTA per query tile.
+cudaError_t launch_fwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
+                       const CUtensorMap &tv, const FwdParams &p, dim3 grid, cudaStream_t st);
+int fwd_tile_rows();
+int fwd_box_inner_elems(int D);
+int fwd_kv_tile_rows(int D);
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t st);
+cudaError_t fwd_take_device_error(int *code, int *where);
+
+// Unpad / pad (row gather / scatter + zero fill).
+cudaError_t launch_unpad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
+                         int64_t row_bytes, void *out, cudaStream_t st);
+cudaError_t launch_pad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
+                       int64_t row_bytes, void *out, cudaStream_t st);
+cudaError_t pad_take_device_error(int *code, int *where);
+
+}  // namespace fa

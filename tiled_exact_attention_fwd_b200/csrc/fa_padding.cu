@@ -1,0 +1,170 @@
+// fa_padding.cu -- unpad (row gather) and pad (row scatter with zero fill) kernels.
+//
+// Page "IAW 模型 FA2 vs FA3 实测": section 1 describes the packed path -- unpad drops the
+// padding tokens of a (B, total_len, H, D) tensor by taking rows by `indices`, pad puts
+// the compact rows back by `indices`; section 2 shows pad as a zero fill followed by an
+// index put. Here both are pure byte movement: one warp moves one row with 16-byte
+// vectors (several loads in flight per lane), and pad writes every output row exactly
+// once (copy when some index names it, zeros otherwise) instead of a fill plus a scatter.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fa.h"
+#include "fa_internal.h"
+
+namespace fa {
+
+static __device__ int g_pad_err_code;
+static __device__ int g_pad_err_where;
+
+__device__ __noinline__ void pad_record_error(int code, int where) {
+    if (atomicCAS(&g_pad_err_code, 0, code) == 0) atomicExch(&g_pad_err_where, where);
+}
+
+template <typename T>
+__device__ __forceinline__ T zero_of();
+template <>
+__device__ __forceinline__ uint4 zero_of<uint4>() { return make_uint4(0, 0, 0, 0); }
+template <>
+__device__ __forceinline__ uint8_t zero_of<uint8_t>() { return 0; }
+
+template <typename T>
+__device__ __forceinline__ T ld_stream(const T *p) { return __ldg(p); }
+
+// Copy one row of `n` elements of T with the lanes of a warp, 4 vectors in flight per lane.
+template <typename T>
+__device__ __forceinline__ void warp_copy_row(const T *__restrict__ src, T *__restrict__ dst,
+                                              int64_t n, int lane) {
+    int64_t c = lane;
+    for (; c + 96 < n; c += 128) {
+        const T a = ld_stream(src + c), b = ld_stream(src + c + 32);
+        const T d = ld_stream(src + c + 64), e = ld_stream(src + c + 96);
+        dst[c] = a;
+        dst[c + 32] = b;
+        dst[c + 64] = d;
+        dst[c + 96] = e;
+    }
+    for (; c < n; c += 32) dst[c] = ld_stream(src + c);
+}
+
+template <typename T>
+__device__ __forceinline__ void warp_zero_row(T *__restrict__ dst, int64_t n, int lane) {
+    const T z = zero_of<T>();
+    for (int64_t c = lane; c < n; c += 32) dst[c] = z;
+}
+
+// out[r] = x[indices[r]]: one warp per compact row r, grid-stride over rows.
+template <typename T>
+__global__ void __launch_bounds__(256) unpad_kernel(const T *__restrict__ x, const int64_t *__restrict__ idx,
+                                                    int64_t nnz, int64_t total_rows, int64_t per_row,
+                                                    T *__restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wpb = blockDim.x >> 5;
+    const int64_t nw = gridDim.x * wpb;
+    for (int64_t r = blockIdx.x * wpb + (threadIdx.x >> 5); r < nnz; r += nw) {
+        const int64_t src = __ldg(idx + r);
+        T *o = out + r * per_row;
+        if (src < 0 || src >= total_rows) {
+            warp_zero_row(o, per_row, lane);
+            if (lane == 0) pad_record_error(FA_ERR_INDEX, 1);
+            continue;
+        }
+        warp_copy_row(x + src * per_row, o, per_row, lane);
+    }
+}
+
+// Every output row t of [t0, t1) (one contiguous range per block, one warp per row):
+// copy x[r] if indices[r] == t for some r, zeros otherwise. With strictly increasing
+// indices, the r for row t lies in [r0, r0 + (t - t0)], r0 = lower_bound(indices, t0).
+template <typename T>
+__global__ void __launch_bounds__(256) pad_kernel(const T *__restrict__ x, const int64_t *__restrict__ idx,
+                                                  int64_t nnz, int64_t total_rows, int64_t per_row,
+                                                  int64_t rows_per_block, T *__restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * rows_per_block;
+    const int64_t t1 = min(total_rows, t0 + rows_per_block);
+    if (t0 >= t1) return;
+    int64_t lo = 0, hi = nnz;
+    while (lo < hi) {
+        const int64_t mid = (lo + hi) >> 1;
+        if (__ldg(idx + mid) < t0) lo = mid + 1; else hi = mid;
+    }
+    const int64_t r0 = lo;
+    const int64_t wpb = blockDim.x >> 5;
+    for (int64_t t = t0 + (threadIdx.x >> 5); t < t1; t += wpb) {
+        int64_t a = r0, b = min(nnz, r0 + (t - t0) + 1);
+        while (a < b) {
+            const int64_t mid = (a + b) >> 1;
+            if (__ldg(idx + mid) < t) a = mid + 1; else b = mid;
+        }
+        T *o = out + t * per_row;
+        if (a < nnz && __ldg(idx + a) == t)
+            warp_copy_row(x + a * per_row, o, per_row, lane);
+        else
+            warp_zero_row(o, per_row, lane);
+    }
+}
+
+static int num_sms() {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0, n = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+            sms = n;
+        else
+            return 148;
+    }
+    return sms;
+}
+
+static bool vec16_ok(const void *a, const void *b, int64_t row_bytes) {
+    return (row_bytes % 16) == 0 && (reinterpret_cast<uintptr_t>(a) % 16) == 0 &&
+           (reinterpret_cast<uintptr_t>(b) % 16) == 0;
+}
+
+cudaError_t launch_unpad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
+                         int64_t row_bytes, void *out, cudaStream_t st) {
+    if (nnz == 0) return cudaSuccess;
+    const int64_t want = (nnz + 7) / 8;
+    const int blocks = static_cast<int>(want < int64_t(num_sms()) * 8 ? want : int64_t(num_sms()) * 8);
+    if (vec16_ok(x, out, row_bytes))
+        unpad_kernel<uint4><<<blocks, 256, 0, st>>>(static_cast<const uint4 *>(x), indices, nnz, total_rows,
+                                                    row_bytes / 16, static_cast<uint4 *>(out));
+    else
+        unpad_kernel<uint8_t><<<blocks, 256, 0, st>>>(static_cast<const uint8_t *>(x), indices, nnz,
+                                                      total_rows, row_bytes, static_cast<uint8_t *>(out));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
+                       int64_t row_bytes, void *out, cudaStream_t st) {
+    if (total_rows == 0) return cudaSuccess;
+    const int64_t max_blocks = int64_t(num_sms()) * 8;
+    int64_t blocks = (total_rows + 15) / 16;
+    if (blocks > max_blocks) blocks = max_blocks;
+    const int64_t rows_per_block = (total_rows + blocks - 1) / blocks;
+    blocks = (total_rows + rows_per_block - 1) / rows_per_block;
+    if (vec16_ok(x ? x : out, out, row_bytes))
+        pad_kernel<uint4><<<static_cast<int>(blocks), 256, 0, st>>>(static_cast<const uint4 *>(x), indices, nnz,
+                                                                    total_rows, row_bytes / 16, rows_per_block,
+                                                                    static_cast<uint4 *>(out));
+    else
+        pad_kernel<uint8_t><<<static_cast<int>(blocks), 256, 0, st>>>(static_cast<const uint8_t *>(x), indices,
+                                                                      nnz, total_rows, row_bytes, rows_per_block,
+                                                                      static_cast<uint8_t *>(out));
+    return cudaGetLastError();
+}
+
+cudaError_t pad_take_device_error(int *code, int *where) {
+    int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(code, g_pad_err_code, sizeof(int));
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(where, g_pad_err_where, sizeof(int));
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyToSymbol(g_pad_err_code, &zero, sizeof(int));
+    if (e != cudaSuccess) return e;
+    return cudaMemcpyToSymbol(g_pad_err_where, &zero, sizeof(int));
+}
+
+}  // namespace fa
