@@ -91,7 +91,9 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = wait_limit_ns();
     const int qtiles = (seqlen_or_max + fa::fwd_tile_rows() - 1) / fa::fwd_tile_rows();
-    const dim3 grid(static_cast<unsigned>(H), static_cast<unsigned>(qtiles), static_cast<unsigned>(num_seqs));
+    const int per_cta = fa::fwd_tiles_per_cta(D);
+    const int ctas_y = (qtiles + per_cta - 1) / per_cta;
+    const dim3 grid(static_cast<unsigned>(H), static_cast<unsigned>(ctas_y), static_cast<unsigned>(num_seqs));
     const cudaError_t e = fa::launch_fwd(D, bf16, causal != 0, tq, tk, tv, p, grid,
                                          static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;

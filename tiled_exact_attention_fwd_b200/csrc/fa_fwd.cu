@@ -10,21 +10,25 @@
 // The packed case (page "IAW 模型 FA2 vs FA3 实测", section 1) is the same loop run inside
 // each sequence of cu_seqlens.
 //
-// B200 design (one CTA = one 128-row query tile of one head of one sequence):
-//   warp 0      TMA producer: Q once, then K_j / V_j tiles through an NS-stage ring of
-//               shared-memory slots guarded by full/empty mbarriers, in the exact order
-//               the MMA warp consumes them (K0, K1, V0, K2, V1, ..., V_last).
-//   warp 1      allocates TMEM; one thread issues every tcgen05.mma:
-//                 S_j = Q K_j^T    (A = Q, B = K_j, both K-major in SMEM, 128B swizzle)
-//                 O  += P_j V_j    (A = P_j read from TMEM, B = V_j MN-major in SMEM)
-//               S is double-buffered in TMEM so S_{j+1} is computed while the softmax
-//               warps work on S_j; P_j (16-bit) overwrites the first half of S_j's columns.
-//   warps 2-5   softmax: thread t owns query row t (TMEM lane t). It reads its S row
-//               with tcgen05.ld, masks, updates (m, l) with exp2 of scores pre-multiplied
-//               by scale*log2(e), writes P back to TMEM and, when its max grew by more than
-//               2^8, rescales its O row in TMEM (lazy rescale: between rescales every
-//               exponent uses the same stale max, which the final 1/l cancels exactly).
-//               At the end it normalises O by 1/l, stores O (fp16/bf16) and the LSE.
+// B200 design. One CTA owns up to two 128-row query tiles (A, B) of one head of one
+// sequence that share every K/V tile it loads (one tile when D = 256, where two O
+// accumulators do not fit in TMEM), which halves the K/V bytes moved per MMA flop:
+//   warps 0-7   two softmax warpgroups, warpgroup t for tile t; thread (warp w, lane l)
+//               owns row 32*(w%4)+l of its tile, the TMEM lane its warp may access. It
+//               reads its S row with tcgen05.ld, masks, updates (m, l) with exp2 of scores
+//               pre-multiplied by scale*log2(e), writes P (16-bit) over S in TMEM, and when
+//               its max grew by more than 2^8 rescales its O row in TMEM (lazy rescale:
+//               between rescales every exponent uses the same stale max, which the final
+//               1/l cancels exactly). At the end: O/l -> fp16/bf16 -> global, and the LSE.
+//   warp 8      TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ... through an
+//               NS-stage shared-memory ring guarded by full/empty mbarriers.
+//   warp 9      allocates TMEM; one thread issues every tcgen05.mma:
+//                 S_t = Q_t K_j^T   (A = Q_t, B = K_j, both K-major in SMEM, 128B swizzle)
+//                 O_t += P_t V_j    (A = P_t read from TMEM, B = V_j MN-major in SMEM)
+//               in the ping-pong order QK_A0, QK_B0, PV_A0, QK_A1, PV_B0, QK_B1, ..., so the
+//               tensor core works on one tile while the other tile's softmax runs. With a
+//               single tile the two S buffers are used alternately by that tile instead
+//               (order QK_0, QK_1, PV_0, QK_2, PV_1, ...).
 //
 // Every pipeline wait is bounded: after `timeout_ns` the waiting thread records
 // FA_ERR_TIMEOUT in a device word, raises a CTA-wide abort flag, and all roles drain
@@ -70,35 +74,47 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
 
 template <int D>
 struct Cfg {
-    static constexpr int BM = 128;                        // query rows per tile (MMA M)
-    static constexpr int BN = (D == 256) ? 64 : 128;      // key rows per tile
+    static constexpr int BM = 128;                           // query rows per tile (MMA M)
+    static constexpr int BN = (D == 256) ? 64 : 128;         // key rows per tile
+    static constexpr int MAXQ = (D == 256) ? 1 : 2;          // query tiles per CTA
     static constexpr int SW = (2 * D >= 128) ? 128 : 2 * D;  // swizzle span in bytes
-    static constexpr int SWE = SW / 2;                    // 16-bit elements per swizzle row
-    static constexpr int NBLK = D / SWE;                  // column blocks per tile row
+    static constexpr int SWE = SW / 2;                       // 16-bit elements per swizzle row
+    static constexpr int NBLK = D / SWE;                     // column blocks per tile row
     static constexpr int Q_BYTES = BM * D * 2;
     static constexpr int KV_BYTES = BN * D * 2;
-    static constexpr int NS = (D == 32) ? 8 : (D == 64) ? 6 : (D == 128) ? 5 : 4;
     static constexpr uint32_t LAYOUT = (SW == 128) ? kLayoutSw128 : kLayoutSw64;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t O_COL = 2 * BN;            // S0 at col 0, S1 at col BN, O after
-    static constexpr int NUM_THREADS = 192;
+    static constexpr uint32_t O_COL = 2 * BN;                // S0 at 0, S1 at BN, O_A, O_B after
+    static constexpr int NUM_SOFTMAX_WARPS = 4 * MAXQ;
+    static constexpr int WARP_TMA = NUM_SOFTMAX_WARPS;
+    static constexpr int WARP_MMA = NUM_SOFTMAX_WARPS + 1;
+    static constexpr int NUM_THREADS = 32 * (NUM_SOFTMAX_WARPS + 2);
+    // Column pairs (out of every 4) whose exp2 runs on the FMA pipe instead of MUFU.
+    static constexpr int EMU_PAIRS_OF_4 = 0;
     // shared memory map (offsets from a 1024-byte aligned base)
+    static constexpr int SMEM_LIMIT = 227 * 1024;
+    static constexpr int RESERVED = 1024 /*alignment*/ + 512 /*barriers, misc*/;
+    static constexpr int NS_FIT = (SMEM_LIMIT - RESERVED - MAXQ * Q_BYTES) / KV_BYTES;
+    static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_KV = Q_BYTES;
+    static constexpr int OFF_KV = MAXQ * Q_BYTES;
     static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
-    static constexpr int NUM_BARS = 1 + 2 * NS + 2 + 2 + 1 + 1;
+    // q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], drain
+    static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int USED = OFF_MISC + 16;
-    // Ask for more than half of the SM's shared memory so exactly one CTA (and one
-    // 512-column TMEM allocation) lives on an SM.
+    // More than half of the SM's shared memory, so exactly one CTA (and one 512-column
+    // TMEM allocation) lives on an SM.
     static constexpr int MIN_SMEM = 120 * 1024;
     static constexpr int SMEM_BYTES = (USED + 1024 > MIN_SMEM) ? USED + 1024 : MIN_SMEM;
-    static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
-    static_assert(USED + 1024 <= 227 * 1024, "shared memory budget");
+    static_assert(NS >= 3, "K/V ring too shallow");
+    static_assert(O_COL + MAXQ * D <= TMEM_COLS, "TMEM budget");
+    static_assert(USED + 1024 <= SMEM_LIMIT, "shared memory budget");
+    static_assert(NUM_BARS * 8 + 16 <= 512, "barrier area");
     static_assert(Q_BYTES % 1024 == 0 && KV_BYTES % 1024 == 0, "tile alignment");
 };
 
-// Position of load/consume step `idx` in the sequence K0, K1, V0, K2, V1, ..., V_{n-1}.
+// Single-tile order of MMA steps: K0, K1, V0, K2, V1, ..., V_{n-1} (QK runs one tile ahead).
 __device__ __forceinline__ void decode_step(int idx, int n, bool &is_v, int &j) {
     if (idx == 0) { is_v = false; j = 0; }
     else if (idx == 2 * n - 1) { is_v = true; j = n - 1; }
@@ -111,15 +127,135 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return BF16 ? pack2_bf16(lo, hi) : pack2_f16(lo, hi);
 }
 
+// 2^x evaluated on the FMA pipe instead of the MUFU unit. Cody-Waite style reduction
+// x = n + f with n = round(x) taken from the 1.5*2^23 shifter and f in [-1/2, 1/2]; 2^f by
+// a degree-3 polynomial fitted with the Remez algorithm for minimax relative error
+// (7.5e-5, below the 2^-11 rounding of the 16-bit P it feeds; gen_exp2_poly.py); 2^n is
+// added to the exponent field. Inputs below -126 are clamped (the result is then ~1e-38
+// instead of a smaller number, irrelevant next to the row sum, which is at least 1); it is
+// only used on tiles without masked (-inf) scores.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -126.0f);
+    const float t = x + 12582912.0f;
+    const float n = t - 12582912.0f;
+    const float f = x - n;
+    const float p = fmaf(fmaf(fmaf(5.517166853e-02f, f, 2.426111251e-01f), f, 6.932609677e-01f), f,
+                         9.999280572e-01f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// For each 64-column chunk of an S row (in registers): p = 2^(s*c + neg_m), accumulate the
+// row sum in four partial sums, pack pairs to 16 bits and store the chunk to TMEM.
+// Of every 4 column pairs, EMU of them use exp2_poly, the rest the MUFU ex2.
+template <int BN, bool BF16, int EMU>
+__device__ __forceinline__ void softmax_chunk_store(const uint32_t *sr, float c, float neg_m, float *rs,
+                                                    uint32_t p_addr) {
+#pragma unroll
+    for (int cc = 0; cc < BN / 64; ++cc) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int e = cc * 64 + 2 * i;
+            const float x0 = fmaf(__uint_as_float(sr[e]), c, neg_m);
+            const float x1 = fmaf(__uint_as_float(sr[e + 1]), c, neg_m);
+            float p0, p1;
+            if ((i & 3) >= 4 - EMU) {
+                p0 = exp2_poly(x0);
+                p1 = exp2_poly(x1);
+            } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+            }
+            rs[(2 * i) & 3] += p0;
+            rs[(2 * i + 1) & 3] += p1;
+            pk[i] = pack2<BF16>(p0, p1);
+        }
+        tmem_st32(p_addr + cc * 32, pk);
+    }
+}
+
+// Shared state of one CTA: shared-memory buffers, barriers, TMEM base and the plan.
+template <int D>
+struct Cta {
+    using C = Cfg<D>;
+    uint8_t *sQ, *sKV;
+    uint64_t *q_full, *kv_full, *kv_empty, *s_full, *p_full, *pv_done, *drain;
+    volatile int *abort_flag;
+    uint32_t tmem;
+    uint64_t lim;
+    int nA, nB;    // key tiles of query tile A and B (nB = 0 when B is absent)
+    bool two;      // two query tiles (ping-pong) or one (S double-buffered)
+    // S/P buffer and barrier phase used by tile t at key step j
+    __device__ __forceinline__ int buf(int t, int j) const { return two ? t : (j & 1); }
+    __device__ __forceinline__ uint32_t sphase(int j) const { return two ? (j & 1) : ((j >> 1) & 1); }
+};
+
+// One MMA step of the issuing thread. Returns false when a wait gave up.
+template <int D, bool BF16>
+__device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first_use, bool last_use) {
+    using C = Cfg<D>;
+    constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
+    constexpr uint32_t idesc = idesc_f16(BM, BN, BF16, false);
+    if (j == 0) {
+        if (!wait_bounded(&c.q_full[t], 0, c.abort_flag, c.lim, 200 + t)) return false;
+        tc_fence_after_sync();
+    }
+    const int L = 2 * j, stage = L % NS;
+    if (first_use) {
+        if (!wait_bounded(&c.kv_full[stage], (L / NS) & 1, c.abort_flag, c.lim, 220 + stage)) return false;
+        tc_fence_after_sync();
+    }
+    const uint32_t q_addr = smem_u32(c.sQ + t * C::Q_BYTES);
+    const uint32_t k_addr = smem_u32(c.sKV + stage * C::KV_BYTES);
+    const int b = c.buf(t, j);
+    const uint32_t d_tmem = c.tmem + b * BN;
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+        const uint32_t blk = (k * 32) / SW, off = (k * 32) % SW;
+        const uint64_t a = smem_desc(q_addr + blk * BM * SW + off, 16, 8 * SW, C::LAYOUT);
+        const uint64_t bd = smem_desc(k_addr + blk * BN * SW + off, 16, 8 * SW, C::LAYOUT);
+        umma_ss(d_tmem, a, bd, idesc, k > 0 ? 1u : 0u);
+    }
+    umma_commit(&c.s_full[b]);
+    if (last_use) umma_commit(&c.kv_empty[stage]);
+    return true;
+}
+
+template <int D, bool BF16>
+__device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first_use, bool last_use) {
+    using C = Cfg<D>;
+    constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
+    constexpr uint32_t idesc = idesc_f16(BM, D, BF16, true);
+    const int b = c.buf(t, j);
+    if (!wait_bounded(&c.p_full[b], c.sphase(j), c.abort_flag, c.lim, 210 + t)) return false;
+    tc_fence_after_sync();
+    const int L = 2 * j + 1, stage = L % NS;
+    if (first_use) {
+        if (!wait_bounded(&c.kv_full[stage], (L / NS) & 1, c.abort_flag, c.lim, 230 + stage)) return false;
+        tc_fence_after_sync();
+    }
+    const uint32_t v_addr = smem_u32(c.sKV + stage * C::KV_BYTES);
+    const uint32_t a_tmem = c.tmem + b * BN;
+    const uint32_t o_tmem = c.tmem + C::O_COL + t * D;
+#pragma unroll
+    for (int k = 0; k < BN / 16; ++k) {
+        const uint64_t bd = smem_desc(v_addr + k * 16 * SW, BN * SW, 8 * SW, C::LAYOUT);
+        umma_ts(o_tmem, a_tmem + k * 8, bd, idesc, (j > 0 || k > 0) ? 1u : 0u);
+    }
+    umma_commit(&c.pv_done[t]);
+    if (last_use) umma_commit(&c.kv_empty[stage]);
+    return true;
+}
+
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Cfg<D>::NUM_THREADS, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     using C = Cfg<D>;
     constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
 
     const int h = blockIdx.x;
-    const int qt = gridDim.y - 1 - blockIdx.y;  // longest (causal) tiles first
+    const int pair = gridDim.y - 1 - blockIdx.y;  // longest (causal) tiles first
     const int seq = blockIdx.z;
     int seq_start, seqlen;
     if (p.cu_seqlens) {
@@ -129,183 +265,190 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         seq_start = seq * p.seqlen;
         seqlen = p.seqlen;
     }
-    const int q0 = qt * BM;
-    if (q0 >= seqlen) return;  // uniform over the CTA, before any barrier exists
-    const int kv_end = CAUSAL ? min(seqlen, q0 + BM) : seqlen;
-    const int n_kv = (kv_end + BN - 1) / BN;
+    const int q0 = pair * C::MAXQ * BM;  // first row of tile A
+    if (q0 >= seqlen) return;            // uniform over the CTA, before any barrier exists
+
+    Cta<D> c;
+    c.two = (C::MAXQ == 2) && (q0 + BM < seqlen);
+    {
+        const int endA = CAUSAL ? min(seqlen, q0 + BM) : seqlen;
+        const int endB = CAUSAL ? min(seqlen, q0 + 2 * BM) : seqlen;
+        c.nA = (endA + BN - 1) / BN;
+        c.nB = c.two ? (endB + BN - 1) / BN : 0;
+    }
+    const int n_all = max(c.nA, c.nB);  // key tiles this CTA loads
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
-    uint8_t *sQ = smem + C::OFF_Q;
-    uint8_t *sKV = smem + C::OFF_KV;
+    c.sQ = smem + C::OFF_Q;
+    c.sKV = smem + C::OFF_KV;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *q_full = bars;
-    uint64_t *kv_full = bars + 1;
-    uint64_t *kv_empty = bars + 1 + NS;
-    uint64_t *s_full = bars + 1 + 2 * NS;
-    uint64_t *p_full = s_full + 2;
-    uint64_t *pv_done = p_full + 2;
-    uint64_t *drain = pv_done + 1;
+    c.q_full = bars;
+    c.kv_full = bars + 2;
+    c.kv_empty = c.kv_full + NS;
+    c.s_full = c.kv_empty + NS;
+    c.p_full = c.s_full + 2;
+    c.pv_done = c.p_full + 2;
+    c.drain = c.pv_done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    c.abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    c.lim = p.timeout_ns;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&c.q_full[t], 1);
+            mbar_init(&c.s_full[t], 1);
+            mbar_init(&c.p_full[t], 128);
+            mbar_init(&c.pv_done[t], 1);
+        }
         for (int s = 0; s < NS; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&c.kv_full[s], 1);
+            mbar_init(&c.kv_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 128);
-        }
-        mbar_init(pv_done, 1);
-        mbar_init(drain, 1);
-        *abort_flag = 0;
+        mbar_init(c.drain, 1);
+        *c.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == C::WARP_TMA && lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
-    if (warp == 1) {
+    if (warp == C::WARP_MMA) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
-    const uint64_t lim = p.timeout_ns;
+    c.tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp == C::WARP_TMA) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t pol_q = l2_policy_evict_first();
             const uint64_t pol_kv = l2_policy_evict_last();
-            mbar_arrive_expect_tx(q_full, C::Q_BYTES);
-#pragma unroll
-            for (int b = 0; b < C::NBLK; ++b)
-                tma_load_3d(sQ + b * BM * SW, &tm_q, q_full, b * C::SWE, h, seq_start + q0, pol_q);
-            const int steps = 2 * n_kv;
-            int issued = 0;
-            for (int idx = 0; idx < steps; ++idx) {
-                const int stage = idx % NS;
-                if (idx >= NS &&
-                    !wait_bounded(&kv_empty[stage], ((idx / NS) - 1) & 1, abort_flag, lim, 100 + stage))
-                    break;
-                bool is_v;
-                int j;
-                decode_step(idx, n_kv, is_v, j);
-                uint8_t *dst = sKV + stage * C::KV_BYTES;
-                mbar_arrive_expect_tx(&kv_full[stage], C::KV_BYTES);
-                const CUtensorMap *map = is_v ? &tm_v : &tm_k;
+            const int nq = c.two ? 2 : 1;
+            for (int t = 0; t < nq; ++t) {
+                mbar_arrive_expect_tx(&c.q_full[t], C::Q_BYTES);
 #pragma unroll
                 for (int b = 0; b < C::NBLK; ++b)
-                    tma_load_3d(dst + b * BN * SW, map, &kv_full[stage], b * C::SWE, h,
-                                seq_start + j * BN, pol_kv);
-                issued = idx + 1;
+                    tma_load_3d(c.sQ + t * C::Q_BYTES + b * BM * SW, &tm_q, &c.q_full[t], b * C::SWE, h,
+                                seq_start + q0 + t * BM, pol_q);
             }
-            if (*abort_flag) {
+            const int loads = 2 * n_all;  // K_0, V_0, K_1, V_1, ...
+            int issued = 0;
+            for (int L = 0; L < loads; ++L) {
+                const int stage = L % NS;
+                if (L >= NS &&
+                    !wait_bounded(&c.kv_empty[stage], ((L / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
+                    break;
+                const int j = L >> 1;
+                uint8_t *dst = c.sKV + stage * C::KV_BYTES;
+                mbar_arrive_expect_tx(&c.kv_full[stage], C::KV_BYTES);
+                const CUtensorMap *map = (L & 1) ? &tm_v : &tm_k;
+#pragma unroll
+                for (int b = 0; b < C::NBLK; ++b)
+                    tma_load_3d(dst + b * BN * SW, map, &c.kv_full[stage], b * C::SWE, h, seq_start + j * BN,
+                                pol_kv);
+                issued = L + 1;
+            }
+            if (*c.abort_flag) {
                 // Let the copies already issued land before the CTA's shared memory goes away.
-                wait_bounded(q_full, 0, abort_flag, lim, 190);
-                for (int idx = (issued > NS ? issued - NS : 0); idx < issued; ++idx) {
-                    const int stage = idx % NS;
+                for (int t = 0; t < nq; ++t) {
                     const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(&kv_full[stage], (idx / NS) & 1) &&
-                           global_timer_ns() - t0 < lim) {
+                    while (!mbar_try_wait(&c.q_full[t], 0) && global_timer_ns() - t0 < c.lim) {
+                    }
+                }
+                for (int L = (issued > NS ? issued - NS : 0); L < issued; ++L) {
+                    const int stage = L % NS;
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(&c.kv_full[stage], (L / NS) & 1) && global_timer_ns() - t0 < c.lim) {
                     }
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == C::WARP_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_f16(BM, BN, BF16, false);
-            constexpr uint32_t idesc_pv = idesc_f16(BM, D, BF16, true);
-            bool ok = wait_bounded(q_full, 0, abort_flag, lim, 200);
-            tc_fence_after_sync();
-            const uint32_t q_addr = smem_u32(sQ);
-            const int steps = 2 * n_kv;
-            for (int idx = 0; ok && idx < steps; ++idx) {
-                const int stage = idx % NS;
-                bool is_v;
-                int j;
-                decode_step(idx, n_kv, is_v, j);
-                if (is_v) {
-                    if (!wait_bounded(&p_full[j & 1], (j >> 1) & 1, abort_flag, lim, 210)) break;
-                    tc_fence_after_sync();
+            bool ok = true;
+            if (!c.two) {
+                const int n = c.nA;
+                for (int idx = 0; ok && idx < 2 * n; ++idx) {
+                    bool is_v;
+                    int j;
+                    decode_step(idx, n, is_v, j);
+                    ok = is_v ? mma_pv<D, BF16>(c, 0, j, true, true) : mma_qk<D, BF16>(c, 0, j, true, true);
                 }
-                if (!wait_bounded(&kv_full[stage], (idx / NS) & 1, abort_flag, lim, 220 + stage)) break;
-                tc_fence_after_sync();
-                const uint32_t kv_addr = smem_u32(sKV + stage * C::KV_BYTES);
-                if (!is_v) {
-                    const uint32_t d_tmem = tmem + (j & 1) * BN;
-#pragma unroll
-                    for (int t = 0; t < D / 16; ++t) {
-                        const uint32_t blk = (t * 32) / SW, off = (t * 32) % SW;
-                        const uint64_t a = smem_desc(q_addr + blk * BM * SW + off, 16, 8 * SW, C::LAYOUT);
-                        const uint64_t b = smem_desc(kv_addr + blk * BN * SW + off, 16, 8 * SW, C::LAYOUT);
-                        umma_ss(d_tmem, a, b, idesc_qk, t > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&kv_empty[stage]);
-                    umma_commit(&s_full[j & 1]);
-                } else {
-                    const uint32_t a_tmem = tmem + (j & 1) * BN;
-#pragma unroll
-                    for (int t = 0; t < BN / 16; ++t) {
-                        const uint64_t b = smem_desc(kv_addr + t * 16 * SW, BN * SW, 8 * SW, C::LAYOUT);
-                        umma_ts(tmem + C::O_COL, a_tmem + t * 8, b, idesc_pv, (j > 0 || t > 0) ? 1u : 0u);
-                    }
-                    umma_commit(&kv_empty[stage]);
-                    umma_commit(pv_done);
+            } else {
+                // Tile A needs key tiles [0, nA), tile B [0, nB), nA <= nB <= nA + 1. A key or
+                // value tile is waited for at its first use and released after its last.
+                const int nA = c.nA, nB = c.nB;
+                ok = mma_qk<D, BF16>(c, 0, 0, true, false) && mma_qk<D, BF16>(c, 1, 0, false, true);
+                for (int j = 1; ok && j < nB; ++j) {
+                    const bool a_prev = j - 1 < nA, a_cur = j < nA;
+                    if (a_prev) ok = mma_pv<D, BF16>(c, 0, j - 1, true, false);
+                    if (ok && a_cur) ok = mma_qk<D, BF16>(c, 0, j, true, false);
+                    if (ok) ok = mma_pv<D, BF16>(c, 1, j - 1, !a_prev, true);
+                    if (ok) ok = mma_qk<D, BF16>(c, 1, j, !a_cur, true);
                 }
+                if (ok && nB - 1 < nA) ok = mma_pv<D, BF16>(c, 0, nB - 1, true, false);
+                if (ok) ok = mma_pv<D, BF16>(c, 1, nB - 1, !(nB - 1 < nA), true);
             }
             // Every MMA issued above has finished once `drain` completes.
-            umma_commit(drain);
+            umma_commit(c.drain);
             const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < lim) {
+            while (!mbar_try_wait(c.drain, 0) && global_timer_ns() - t0 < c.lim) {
             }
         }
-    } else {
+    } else if (warp < C::NUM_SOFTMAX_WARPS) {
         // ------------------------------------------------------------ softmax + epilogue
+        const int t = warp >> 2;                      // query tile of this warpgroup
+        const int n = t ? c.nB : c.nA;
         const int quarter = warp & 3;                 // TMEM lanes this warp may access
         const int r = quarter * 32 + lane;            // row of the tile == TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        const int row_pos = q0 + r;                   // position inside the sequence
+        const int qt0 = q0 + t * BM;
+        const int row_pos = qt0 + r;                  // position inside the sequence
         const int row_lim = CAUSAL ? min(seqlen, row_pos + 1) : seqlen;  // keys [0, row_lim)
-        const float c = p.scale_log2;
+        const uint32_t o_col = C::O_COL + t * D;
+        const float sc = p.scale_log2;
         float m = -INFINITY;  // running max of scaled scores, log2 units (possibly stale)
-        float l = 0.f;        // running sum of 2^(t - m)
-        bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            if (!__all_sync(0xffffffffu, wait_bounded(&s_full[j & 1], (j >> 1) & 1, abort_flag, lim, 300))) {
+        float l = 0.f;        // running sum of 2^(s*sc - m)
+        bool ok = n > 0;
+        for (int j = 0; j < n; ++j) {
+            const int b = c.buf(t, j);
+            if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[b], c.sphase(j), c.abort_flag, c.lim, 300 + t))) {
                 ok = false;
                 break;
             }
             tc_fence_after_sync();
             uint32_t sr[BN];
 #pragma unroll
-            for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(tmem + lane_base + (j & 1) * BN + cc * 32, sr + cc * 32);
+            for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(c.tmem + lane_base + b * BN + cc * 32, sr + cc * 32);
             tmem_ld_wait();
             tmem_reg_fence<BN>(sr);
             const int kv0 = j * BN;
-            const bool need_mask = (kv0 + BN > seqlen) || (CAUSAL && kv0 + BN - 1 > q0);
+            const bool need_mask = (kv0 + BN > seqlen) || (CAUSAL && kv0 + BN - 1 > qt0);
             if (need_mask) {
                 const int valid = row_lim - kv0;  // columns [0, valid) of this tile are visible
 #pragma unroll
                 for (int i = 0; i < BN; ++i)
                     if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
             }
-            float mx = -INFINITY;
+            // Row max with 8 independent partial maxima (short dependency chains).
+            float mm[8];
 #pragma unroll
-            for (int i = 0; i < BN; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
-            const float m_cand = mx * c;
+            for (int k = 0; k < 8; ++k) mm[k] = __uint_as_float(sr[k]);
+#pragma unroll
+            for (int i = 8; i < BN; ++i) mm[i & 7] = fmaxf(mm[i & 7], __uint_as_float(sr[i]));
+            const float mx = fmaxf(fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3])),
+                                   fmaxf(fmaxf(mm[4], mm[5]), fmaxf(mm[6], mm[7])));
+            const float m_cand = mx * sc;
             const bool grow = m_cand > m + 8.0f;
             float alpha = 1.f;
             if (grow) {
@@ -313,46 +456,44 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 m = m_cand;
             }
             const bool warp_grow = __any_sync(0xffffffffu, grow);
-            float rs = 0.f;
-            uint32_t pk[BN / 2];
-#pragma unroll
-            for (int i = 0; i < BN / 2; ++i) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), c, -m));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), c, -m));
-                rs += p0 + p1;
-                pk[i] = pack2<BF16>(p0, p1);
+            // P = 2^(s*sc - m): written back to TMEM over S, 64 columns at a time.
+            const float neg_m = -m;
+            const uint32_t p_addr = c.tmem + lane_base + b * BN;
+            float rs[4] = {0.f, 0.f, 0.f, 0.f};
+            if (need_mask) {
+                softmax_chunk_store<BN, BF16, 0>(sr, sc, neg_m, rs, p_addr);  // -inf must give exactly 0
+            } else {
+                softmax_chunk_store<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, rs, p_addr);
             }
-            l = l * alpha + rs;
-#pragma unroll
-            for (int cc = 0; cc < BN / 64; ++cc) tmem_st32(tmem + lane_base + (j & 1) * BN + cc * 32, pk + cc * 32);
+            l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
             tmem_st_wait();
             if (j > 0) {
-                // PV_{j-1} is waited for on every tile (it has normally finished long before),
+                // PV_{j-1} is waited for on every step (it has normally finished long before),
                 // so this thread never falls two phases behind on pv_done.
-                if (!__all_sync(0xffffffffu, wait_bounded(pv_done, (j - 1) & 1, abort_flag, lim, 310))) {
+                if (!__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (j - 1) & 1, c.abort_flag, c.lim, 310 + t))) {
                     ok = false;
                     break;
                 }
-            }
-            if (warp_grow && j > 0) {
-                // O holds sum_{j' < j} P_j' V_j'; bring it to the new running max.
-                tc_fence_after_sync();
+                if (warp_grow) {
+                    // O holds sum_{j' < j} P_j' V_j'; bring it to the new running max.
+                    tc_fence_after_sync();
 #pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t o[32];
-                    tmem_ld32(tmem + lane_base + C::O_COL + cc * 32, o);
-                    tmem_ld_wait();
-                    tmem_reg_fence<32>(o);
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t o[32];
+                        tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
+                        tmem_ld_wait();
+                        tmem_reg_fence<32>(o);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(tmem + lane_base + C::O_COL + cc * 32, o);
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(c.tmem + lane_base + o_col + cc * 32, o);
+                    }
+                    tmem_st_wait();
                 }
-                tmem_st_wait();
             }
             tc_fence_before_sync();
-            mbar_arrive(&p_full[j & 1]);
+            mbar_arrive(&c.p_full[b]);
         }
-        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(pv_done, (n_kv - 1) & 1, abort_flag, lim, 320));
+        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (n - 1) & 1, c.abort_flag, c.lim, 320 + t));
         if (ok) {
             tc_fence_after_sync();
             const float inv_l = 1.f / l;
@@ -363,7 +504,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t o[32];
-                tmem_ld32(tmem + lane_base + C::O_COL + cc * 32, o);
+                tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
                 tmem_ld_wait();
                 tmem_reg_fence<32>(o);
                 uint32_t w[16];
@@ -387,9 +528,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == C::WARP_MMA) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem, C::TMEM_COLS);
+        tmem_dealloc(c.tmem, C::TMEM_COLS);
     }
 }
 
@@ -453,6 +594,8 @@ cudaError_t launch_fwd(int D, bool bf16, bool causal, const CUtensorMap &tq, con
 }
 
 int fwd_tile_rows() { return 128; }
+
+int fwd_tiles_per_cta(int D) { return (D == 256) ? 1 : 2; }
 
 int fwd_box_inner_elems(int D) { return (2 * D >= 128) ? 64 : D; }
 

@@ -19,10 +19,12 @@ struct FwdParams {
     uint64_t timeout_ns;        // bound of every pipeline wait
 };
 
-// Attention forward: grid (H, ceil(max_len / 128), num_seqs), one CTA per query tile.
+// Attention forward: grid (H, ceil(ceil(max_len / 128) / tiles_per_cta), num_seqs); a CTA
+// owns fwd_tiles_per_cta(D) consecutive 128-row query tiles.
 cudaError_t launch_fwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
                        const CUtensorMap &tv, const FwdParams &p, dim3 grid, cudaStream_t st);
 int fwd_tile_rows();
+int fwd_tiles_per_cta(int D);
 int fwd_box_inner_elems(int D);
 int fwd_kv_tile_rows(int D);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t st);
