@@ -271,6 +271,7 @@ def run_ours(args):
 
     # ---- packed path (unpad x3, varlen forward, pad), microseconds per call
     varlen = run_varlen_leg(fa, device, stream, max(args.steps, 20), args.warmup, ws)
+    padding = run_padding_hbm_leg(fa, device, stream, 20)
     del qp, kp, vp, op, lp
 
     peak_tf, peak_bw, peak_kind = load_peaks()
@@ -290,6 +291,7 @@ def run_ours(args):
                      "peak_kind": f"{peak_kind} bf16 dense (burst)", "kernel": "fa_fwd_kernel<128,bf16,causal>",
                      "traffic": recorded_traffic("fa_fwd_kernel_d128_bf16_causal")},
         "varlen": varlen,
+        "unpad_pad_hbm": padding,
         "clocks": sampler.summary(),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -355,6 +357,41 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
                                    "pad_out": round(tot[2] / iters, 2)},
             "varlen_fwd_tflops": round(flops / (tot[1] / iters * 1e-6) / 1e12, 2),
             "gpu_launches_per_call": 5}
+
+
+def run_padding_hbm_leg(fa, device, stream, iters):
+    """unpad / pad GB/s on the packed structure scaled past L2: (1, 262144, 16, 128) bf16 = 1 GiB
+    padded, half the positions valid. Algorithmic bytes: unpad reads and writes nnz rows plus the
+    indices; pad reads nnz rows and the indices and writes every one of the total rows."""
+    _, peak_bw, peak_kind = load_peaks()
+    L, H, D = 262144, 16, 128
+    nnz = L // 2
+    g = torch.Generator(device="cpu")
+    g.manual_seed(5)
+    x = torch.randn((1, L, H, D), generator=g, dtype=torch.float32).to(torch.bfloat16).to(device)
+    idx = fa_inputs.valid_indices(L, nnz, seed=6).to(device)
+    u = torch.empty((nnz, H, D), device=device, dtype=torch.bfloat16)
+    out = torch.empty_like(x)
+    row = H * D * 2
+    res = {}
+    for name, fn, nbytes in (
+            ("unpad", lambda: fa.fa_unpad(x, idx, out=u, stream=stream), 2 * nnz * row + 8 * nnz),
+            ("pad", lambda: fa.fa_pad(u, idx, 1, L, out=out, stream=stream), nnz * row + L * row + 8 * nnz)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        us = e0.elapsed_time(e1) / iters * 1e3
+        gbs = nbytes / (us * 1e-6) / 1e9
+        res[name] = {"us": round(us, 2), "bytes": nbytes, "achieved_gbs": round(gbs, 1), "peak_gbs": peak_bw,
+                     "frac": round(gbs / peak_bw, 4), "peak_kind": f"{peak_kind} HBM copy"}
+    res["config"] = "(1, 262144, 16, 128) bf16 padded (1 GiB), 131072 valid rows; inputs larger than L2"
+    return res
 
 
 # ----------------------------------------------------------------------------- reference arm

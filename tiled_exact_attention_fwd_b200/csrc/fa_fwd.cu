@@ -88,7 +88,16 @@ struct Cfg {
     static constexpr int NUM_SOFTMAX_WARPS = 4 * MAXQ;
     static constexpr int WARP_TMA = NUM_SOFTMAX_WARPS;
     static constexpr int WARP_MMA = NUM_SOFTMAX_WARPS + 1;
-    static constexpr int NUM_THREADS = 32 * (NUM_SOFTMAX_WARPS + 2);
+    // A full last warpgroup (two idle warps) so that per-warpgroup register limits apply.
+    static constexpr int NUM_THREADS = 32 * (NUM_SOFTMAX_WARPS + 4);
+    // Register split (two query tiles): 384 threads launch with LAUNCH_REGS each; the
+    // producer/MMA warpgroup drops to REGS_LOW and the softmax warpgroups rise to REGS_HIGH.
+    // The host refuses to launch unless the pool covers the split (it would otherwise wait).
+    static constexpr int LAUNCH_REGS = 168;
+    static constexpr int REGS_LOW = 56;
+    static constexpr int REGS_HIGH = 224;
+    static constexpr bool SPLIT_REGS = (MAXQ == 2);
+    static_assert(!SPLIT_REGS || 128 * REGS_LOW + 256 * REGS_HIGH <= NUM_THREADS * LAUNCH_REGS, "register split");
     // Column pairs (out of every 4) whose exp2 runs on the FMA pipe instead of MUFU.
     static constexpr int EMU_PAIRS_OF_4 = 0;
     // shared memory map (offsets from a 1024-byte aligned base)
@@ -144,20 +153,36 @@ __device__ __forceinline__ float exp2_poly(float x) {
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
-// For each 64-column chunk of an S row (in registers): p = 2^(s*c + neg_m), accumulate the
-// row sum in four partial sums, pack pairs to 16 bits and store the chunk to TMEM.
-// Of every 4 column pairs, EMU of them use exp2_poly, the rest the MUFU ex2.
+// Maximum of an S row held in registers: 8 independent chains of three-input maxima.
+template <int BN>
+__device__ __forceinline__ float row_max(const uint32_t *sr) {
+    float mm[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mm[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]));
+#pragma unroll
+    for (int i = 16; i < BN; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mm[k] = fmax3(mm[k], __uint_as_float(sr[i + k]), __uint_as_float(sr[i + 8 + k]));
+    return fmaxf(fmax3(mm[0], mm[1], mm[2]), fmax3(fmax3(mm[3], mm[4], mm[5]), mm[6], mm[7]));
+}
+
+// For each 64-column chunk of an S row (in registers): p = 2^(s*c + neg_m) (scaling done two
+// lanes at a time with fma.f32x2), row sum in four fp32x2 partial sums, pairs packed to
+// 16 bits and the chunk stored to TMEM at p_addr. Of every 4 column pairs, EMU use
+// exp2_poly, the rest the MUFU ex2. Returns the row sum of this tile.
 template <int BN, bool BF16, int EMU>
-__device__ __forceinline__ void softmax_chunk_store(const uint32_t *sr, float c, float neg_m, float *rs,
-                                                    uint32_t p_addr) {
+__device__ __forceinline__ float softmax_chunk_store(const uint32_t *sr, float c, float neg_m, uint32_t p_addr) {
+    const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
+    uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
     for (int cc = 0; cc < BN / 64; ++cc) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int e = cc * 64 + 2 * i;
-            const float x0 = fmaf(__uint_as_float(sr[e]), c, neg_m);
-            const float x1 = fmaf(__uint_as_float(sr[e + 1]), c, neg_m);
+            const uint64_t x2 = ffma2(f2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, nm2);
+            float x0, x1;
+            f2_split(x2, x0, x1);
             float p0, p1;
             if ((i & 3) >= 4 - EMU) {
                 p0 = exp2_poly(x0);
@@ -166,12 +191,15 @@ __device__ __forceinline__ void softmax_chunk_store(const uint32_t *sr, float c,
                 p0 = ex2_approx(x0);
                 p1 = ex2_approx(x1);
             }
-            rs[(2 * i) & 3] += p0;
-            rs[(2 * i + 1) & 3] += p1;
+            acc[i & 3] = fadd2(acc[i & 3], f2(p0, p1));
             pk[i] = pack2<BF16>(p0, p1);
         }
         tmem_st32(p_addr + cc * 32, pk);
     }
+    const uint64_t s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+    float lo, hi;
+    f2_split(s2, lo, hi);
+    return lo + hi;
 }
 
 // Shared state of one CTA: shared-memory buffers, barriers, TMEM base and the plan.
@@ -327,86 +355,91 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_after_sync();
     c.tmem = *tmem_slot;
 
-    if (warp == C::WARP_TMA) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            const uint64_t pol_q = l2_policy_evict_first();
-            const uint64_t pol_kv = l2_policy_evict_last();
-            const int nq = c.two ? 2 : 1;
-            for (int t = 0; t < nq; ++t) {
-                mbar_arrive_expect_tx(&c.q_full[t], C::Q_BYTES);
-#pragma unroll
-                for (int b = 0; b < C::NBLK; ++b)
-                    tma_load_3d(c.sQ + t * C::Q_BYTES + b * BM * SW, &tm_q, &c.q_full[t], b * C::SWE, h,
-                                seq_start + q0 + t * BM, pol_q);
-            }
-            const int loads = 2 * n_all;  // K_0, V_0, K_1, V_1, ...
-            int issued = 0;
-            for (int L = 0; L < loads; ++L) {
-                const int stage = L % NS;
-                if (L >= NS &&
-                    !wait_bounded(&c.kv_empty[stage], ((L / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
-                    break;
-                const int j = L >> 1;
-                uint8_t *dst = c.sKV + stage * C::KV_BYTES;
-                mbar_arrive_expect_tx(&c.kv_full[stage], C::KV_BYTES);
-                const CUtensorMap *map = (L & 1) ? &tm_v : &tm_k;
-#pragma unroll
-                for (int b = 0; b < C::NBLK; ++b)
-                    tma_load_3d(dst + b * BN * SW, map, &c.kv_full[stage], b * C::SWE, h, seq_start + j * BN,
-                                pol_kv);
-                issued = L + 1;
-            }
-            if (*c.abort_flag) {
-                // Let the copies already issued land before the CTA's shared memory goes away.
+    if (warp >= C::NUM_SOFTMAX_WARPS) {
+        // producer / MMA warpgroup (its two remaining warps idle)
+        if constexpr (C::SPLIT_REGS) regs_dec<C::REGS_LOW>();
+        if (warp == C::WARP_TMA) {
+            // ------------------------------------------------------------ TMA producer
+            if (lane == 0) {
+                const uint64_t pol_q = l2_policy_evict_first();
+                const uint64_t pol_kv = l2_policy_evict_last();
+                const int nq = c.two ? 2 : 1;
                 for (int t = 0; t < nq; ++t) {
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(&c.q_full[t], 0) && global_timer_ns() - t0 < c.lim) {
-                    }
+                    mbar_arrive_expect_tx(&c.q_full[t], C::Q_BYTES);
+    #pragma unroll
+                    for (int b = 0; b < C::NBLK; ++b)
+                        tma_load_3d(c.sQ + t * C::Q_BYTES + b * BM * SW, &tm_q, &c.q_full[t], b * C::SWE, h,
+                                    seq_start + q0 + t * BM, pol_q);
                 }
-                for (int L = (issued > NS ? issued - NS : 0); L < issued; ++L) {
+                const int loads = 2 * n_all;  // K_0, V_0, K_1, V_1, ...
+                int issued = 0;
+                for (int L = 0; L < loads; ++L) {
                     const int stage = L % NS;
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(&c.kv_full[stage], (L / NS) & 1) && global_timer_ns() - t0 < c.lim) {
+                    if (L >= NS &&
+                        !wait_bounded(&c.kv_empty[stage], ((L / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
+                        break;
+                    const int j = L >> 1;
+                    uint8_t *dst = c.sKV + stage * C::KV_BYTES;
+                    mbar_arrive_expect_tx(&c.kv_full[stage], C::KV_BYTES);
+                    const CUtensorMap *map = (L & 1) ? &tm_v : &tm_k;
+    #pragma unroll
+                    for (int b = 0; b < C::NBLK; ++b)
+                        tma_load_3d(dst + b * BN * SW, map, &c.kv_full[stage], b * C::SWE, h, seq_start + j * BN,
+                                    pol_kv);
+                    issued = L + 1;
+                }
+                if (*c.abort_flag) {
+                    // Let the copies already issued land before the CTA's shared memory goes away.
+                    for (int t = 0; t < nq; ++t) {
+                        const uint64_t t0 = global_timer_ns();
+                        while (!mbar_try_wait(&c.q_full[t], 0) && global_timer_ns() - t0 < c.lim) {
+                        }
+                    }
+                    for (int L = (issued > NS ? issued - NS : 0); L < issued; ++L) {
+                        const int stage = L % NS;
+                        const uint64_t t0 = global_timer_ns();
+                        while (!mbar_try_wait(&c.kv_full[stage], (L / NS) & 1) && global_timer_ns() - t0 < c.lim) {
+                        }
                     }
                 }
             }
-        }
-    } else if (warp == C::WARP_MMA) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            bool ok = true;
-            if (!c.two) {
-                const int n = c.nA;
-                for (int idx = 0; ok && idx < 2 * n; ++idx) {
-                    bool is_v;
-                    int j;
-                    decode_step(idx, n, is_v, j);
-                    ok = is_v ? mma_pv<D, BF16>(c, 0, j, true, true) : mma_qk<D, BF16>(c, 0, j, true, true);
+        } else if (warp == C::WARP_MMA) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                bool ok = true;
+                if (!c.two) {
+                    const int n = c.nA;
+                    for (int idx = 0; ok && idx < 2 * n; ++idx) {
+                        bool is_v;
+                        int j;
+                        decode_step(idx, n, is_v, j);
+                        ok = is_v ? mma_pv<D, BF16>(c, 0, j, true, true) : mma_qk<D, BF16>(c, 0, j, true, true);
+                    }
+                } else {
+                    // Tile A needs key tiles [0, nA), tile B [0, nB), nA <= nB <= nA + 1. A key or
+                    // value tile is waited for at its first use and released after its last.
+                    const int nA = c.nA, nB = c.nB;
+                    ok = mma_qk<D, BF16>(c, 0, 0, true, false) && mma_qk<D, BF16>(c, 1, 0, false, true);
+                    for (int j = 1; ok && j < nB; ++j) {
+                        const bool a_prev = j - 1 < nA, a_cur = j < nA;
+                        if (a_prev) ok = mma_pv<D, BF16>(c, 0, j - 1, true, false);
+                        if (ok && a_cur) ok = mma_qk<D, BF16>(c, 0, j, true, false);
+                        if (ok) ok = mma_pv<D, BF16>(c, 1, j - 1, !a_prev, true);
+                        if (ok) ok = mma_qk<D, BF16>(c, 1, j, !a_cur, true);
+                    }
+                    if (ok && nB - 1 < nA) ok = mma_pv<D, BF16>(c, 0, nB - 1, true, false);
+                    if (ok) ok = mma_pv<D, BF16>(c, 1, nB - 1, !(nB - 1 < nA), true);
                 }
-            } else {
-                // Tile A needs key tiles [0, nA), tile B [0, nB), nA <= nB <= nA + 1. A key or
-                // value tile is waited for at its first use and released after its last.
-                const int nA = c.nA, nB = c.nB;
-                ok = mma_qk<D, BF16>(c, 0, 0, true, false) && mma_qk<D, BF16>(c, 1, 0, false, true);
-                for (int j = 1; ok && j < nB; ++j) {
-                    const bool a_prev = j - 1 < nA, a_cur = j < nA;
-                    if (a_prev) ok = mma_pv<D, BF16>(c, 0, j - 1, true, false);
-                    if (ok && a_cur) ok = mma_qk<D, BF16>(c, 0, j, true, false);
-                    if (ok) ok = mma_pv<D, BF16>(c, 1, j - 1, !a_prev, true);
-                    if (ok) ok = mma_qk<D, BF16>(c, 1, j, !a_cur, true);
+                // Every MMA issued above has finished once `drain` completes.
+                umma_commit(c.drain);
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(c.drain, 0) && global_timer_ns() - t0 < c.lim) {
                 }
-                if (ok && nB - 1 < nA) ok = mma_pv<D, BF16>(c, 0, nB - 1, true, false);
-                if (ok) ok = mma_pv<D, BF16>(c, 1, nB - 1, !(nB - 1 < nA), true);
             }
-            // Every MMA issued above has finished once `drain` completes.
-            umma_commit(c.drain);
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(c.drain, 0) && global_timer_ns() - t0 < c.lim) {
-            }
-        }
-    } else if (warp < C::NUM_SOFTMAX_WARPS) {
+    }
+    } else {
         // ------------------------------------------------------------ softmax + epilogue
+        if constexpr (C::SPLIT_REGS) regs_inc<C::REGS_HIGH>();
         const int t = warp >> 2;                      // query tile of this warpgroup
         const int n = t ? c.nB : c.nA;
         const int quarter = warp & 3;                 // TMEM lanes this warp may access
@@ -440,14 +473,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 for (int i = 0; i < BN; ++i)
                     if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
             }
-            // Row max with 8 independent partial maxima (short dependency chains).
-            float mm[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mm[k] = __uint_as_float(sr[k]);
-#pragma unroll
-            for (int i = 8; i < BN; ++i) mm[i & 7] = fmaxf(mm[i & 7], __uint_as_float(sr[i]));
-            const float mx = fmaxf(fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3])),
-                                   fmaxf(fmaxf(mm[4], mm[5]), fmaxf(mm[6], mm[7])));
+            const float mx = row_max<BN>(sr);
             const float m_cand = mx * sc;
             const bool grow = m_cand > m + 8.0f;
             float alpha = 1.f;
@@ -459,13 +485,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // P = 2^(s*sc - m): written back to TMEM over S, 64 columns at a time.
             const float neg_m = -m;
             const uint32_t p_addr = c.tmem + lane_base + b * BN;
-            float rs[4] = {0.f, 0.f, 0.f, 0.f};
-            if (need_mask) {
-                softmax_chunk_store<BN, BF16, 0>(sr, sc, neg_m, rs, p_addr);  // -inf must give exactly 0
-            } else {
-                softmax_chunk_store<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, rs, p_addr);
-            }
-            l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+            const float rs = need_mask ? softmax_chunk_store<BN, BF16, 0>(sr, sc, neg_m, p_addr)  // -inf -> exactly 0
+                                       : softmax_chunk_store<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, p_addr);
+            l = fmaf(l, alpha, rs);
             tmem_st_wait();
             if (j > 0) {
                 // PV_{j-1} is waited for on every step (it has normally finished long before),
@@ -483,8 +505,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
                         tmem_ld_wait();
                         tmem_reg_fence<32>(o);
+                        const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        for (int i = 0; i < 16; ++i) {
+                            float lo, hi;
+                            f2_split(fmul2(f2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), lo, hi);
+                            o[2 * i] = __float_as_uint(lo);
+                            o[2 * i + 1] = __float_as_uint(hi);
+                        }
                         tmem_st32(c.tmem + lane_base + o_col + cc * 32, o);
                     }
                     tmem_st_wait();
@@ -560,6 +588,14 @@ static cudaError_t launch_t(const CUtensorMap &tq, const CUtensorMap &tk, const 
     if (e != cudaSuccess) return e;
     const uint64_t bit = uint64_t(1) << (dev & 63);
     if (!(__atomic_load_n(&attr_set_mask, __ATOMIC_ACQUIRE) & bit)) {
+        if (C::SPLIT_REGS) {
+            // The per-warpgroup register split draws on the registers the CTA launches with.
+            cudaFuncAttributes fa_attr;
+            e = cudaFuncGetAttributes(&fa_attr, kern);
+            if (e != cudaSuccess) return e;
+            if (fa_attr.numRegs * C::NUM_THREADS < 128 * C::REGS_LOW + 256 * C::REGS_HIGH)
+                return cudaErrorInvalidConfiguration;
+        }
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         __atomic_fetch_or(&attr_set_mask, bit, __ATOMIC_RELEASE);
