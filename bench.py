@@ -433,11 +433,17 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only-main", action="store_true", help="time the main kernel only (for profiling)")
+    ap.add_argument("--only-padding", action="store_true", help="run the unpad/pad HBM leg only (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.only_padding:
+        import tiled_exact_attention_fwd_b200 as fa
+        device = torch.device("cuda", 0)
+        torch.cuda.set_device(device)
+        print(json.dumps(run_padding_hbm_leg(fa, device, torch.cuda.current_stream(device), max(args.steps, 1))))
     else:
         run_ours(args)
 
