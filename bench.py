@@ -52,12 +52,20 @@ def kernel_source_hash() -> str:
 
 
 def load_peaks():
+    """(bf16 burst TF/s, HBM GB/s, kind, bf16 sustained TF/s) from MEASURED_PEAKS.json, else fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["bf16_tflops"]), float(d["hbm_gbs"]), "measured"
-    return 1590.0, 6650.0, "fallback"
+        return (float(d["bf16_tflops"]), float(d["hbm_gbs"]), "measured",
+                float(d.get("bf16_tflops_sustained", d["bf16_tflops"])))
+    return 1590.0, 6650.0, "fallback", 1400.0
+
+
+# A timed region longer than this runs into the 1 kW power cap on B200 (measured: the
+# causal forward loses ~8% between 100- and 200-launch windows), so it is compared with
+# the sustained GEMM figure rather than the burst one.
+BURST_WINDOW_MS = 50.0
 
 
 def recorded_traffic(kernel: str):
@@ -274,7 +282,13 @@ def run_ours(args):
     padding = run_padding_hbm_leg(fa, device, stream, 20)
     del qp, kp, vp, op, lp
 
-    peak_tf, peak_bw, peak_kind = load_peaks()
+    peak_burst, peak_bw, peak_kind, peak_sust = load_peaks()
+    clocks = sampler.summary()
+    timed_ms = ms_local * args.steps
+    long_region = timed_ms > BURST_WINDOW_MS or "sw_power_cap" in clocks.get("reasons", [])
+    peak_tf = peak_sust if long_region else peak_burst
+    peak_label = (f"{peak_kind} bf16 dense, {'sustained' if long_region else 'burst'} "
+                  f"(timed region {timed_ms:.0f} ms{', sw_power_cap seen' if 'sw_power_cap' in clocks.get('reasons', []) else ''})")
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
@@ -288,11 +302,13 @@ def run_ours(args):
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": {"bound": "tensor", "achieved": round(kernel_tflops, 2), "peak": peak_tf,
                      "unit": "TFLOP/s", "frac": round(kernel_tflops / peak_tf, 4),
-                     "peak_kind": f"{peak_kind} bf16 dense (burst)", "kernel": "fa_fwd_kernel<128,bf16,causal>",
+                     "peak_kind": peak_label, "frac_vs_burst": round(kernel_tflops / peak_burst, 4),
+                     "frac_vs_sustained": round(kernel_tflops / peak_sust, 4),
+                     "kernel": "fa_fwd_kernel<128,bf16,causal>",
                      "traffic": recorded_traffic("fa_fwd_kernel_d128_bf16_causal")},
         "varlen": varlen,
         "unpad_pad_hbm": padding,
-        "clocks": sampler.summary(),
+        "clocks": clocks,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         tf, secs, nheads, fl, nth = oracle_sample()
@@ -363,7 +379,7 @@ def run_padding_hbm_leg(fa, device, stream, iters):
     """unpad / pad GB/s on the packed structure scaled past L2: (1, 262144, 16, 128) bf16 = 1 GiB
     padded, half the positions valid. Algorithmic bytes: unpad reads and writes nnz rows plus the
     indices; pad reads nnz rows and the indices and writes every one of the total rows."""
-    _, peak_bw, peak_kind = load_peaks()
+    _, peak_bw, peak_kind, _ = load_peaks()
     L, H, D = 262144, 16, 128
     nnz = L // 2
     g = torch.Generator(device="cpu")
