@@ -84,7 +84,12 @@ struct Cfg {
     static constexpr int KV_BYTES = BN * D * 2;
     static constexpr uint32_t LAYOUT = (SW == 128) ? kLayoutSw128 : kLayoutSw64;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t O_COL = 2 * BN;                // S0 at 0, S1 at BN, O_A, O_B after
+    // TMEM columns: S0 at 0, S1 at BN. With D <= 64 two separate P buffers fit (P_COL + 64t)
+    // so a tile's next S = QK^T can be computed while its softmax still works on the last
+    // one ("decoupled"); otherwise P overwrites the first half of its S buffer.
+    static constexpr bool DECOUPLED = (MAXQ == 2) && (D <= 64);
+    static constexpr uint32_t P_COL = 2 * BN;
+    static constexpr uint32_t O_COL = 2 * BN + (DECOUPLED ? 128 : 0);  // O_A, O_B
     static constexpr int NUM_SOFTMAX_WARPS = 4 * MAXQ;
     static constexpr int WARP_TMA = NUM_SOFTMAX_WARPS;
     static constexpr int WARP_MMA = NUM_SOFTMAX_WARPS + 1;
@@ -108,8 +113,8 @@ struct Cfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = MAXQ * Q_BYTES;
     static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
-    // q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], drain
-    static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1;
+    // q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], drain, s_free[2]
+    static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int USED = OFF_MISC + 16;
     // More than half of the SM's shared memory, so exactly one CTA (and one 512-column
@@ -202,17 +207,46 @@ __device__ __forceinline__ float softmax_chunk_store(const uint32_t *sr, float c
     return lo + hi;
 }
 
+// A whole S row (in registers) to packed 16-bit P in registers pk[BN/2]:
+// p = 2^(s*c + neg_m), scaling two lanes at a time; returns the row sum.
+template <int BN, bool BF16, int EMU>
+__device__ __forceinline__ float softmax_row_to_regs(const uint32_t *sr, float c, float neg_m, uint32_t *pk) {
+    const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
+    uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
+    for (int i = 0; i < BN / 2; ++i) {
+        const uint64_t x2 = ffma2(f2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, nm2);
+        float x0, x1;
+        f2_split(x2, x0, x1);
+        float p0, p1;
+        if ((i & 3) >= 4 - EMU) {
+            p0 = exp2_poly(x0);
+            p1 = exp2_poly(x1);
+        } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+        }
+        acc[i & 3] = fadd2(acc[i & 3], f2(p0, p1));
+        pk[i] = pack2<BF16>(p0, p1);
+    }
+    const uint64_t s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+    float lo, hi;
+    f2_split(s2, lo, hi);
+    return lo + hi;
+}
+
 // Shared state of one CTA: shared-memory buffers, barriers, TMEM base and the plan.
 template <int D>
 struct Cta {
     using C = Cfg<D>;
     uint8_t *sQ, *sKV;
-    uint64_t *q_full, *kv_full, *kv_empty, *s_full, *p_full, *pv_done, *drain;
+    uint64_t *q_full, *kv_full, *kv_empty, *s_full, *p_full, *pv_done, *drain, *s_free;
     volatile int *abort_flag;
     uint32_t tmem;
     uint64_t lim;
     int nA, nB;    // key tiles of query tile A and B (nB = 0 when B is absent)
     bool two;      // two query tiles (ping-pong) or one (S double-buffered)
+    bool dec;      // two tiles with separate P buffers (Cfg::DECOUPLED)
     // S/P buffer and barrier phase used by tile t at key step j
     __device__ __forceinline__ int buf(int t, int j) const { return two ? t : (j & 1); }
     __device__ __forceinline__ uint32_t sphase(int j) const { return two ? (j & 1) : ((j >> 1) & 1); }
@@ -226,6 +260,10 @@ __device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first
     constexpr uint32_t idesc = idesc_f16(BM, BN, BF16, false);
     if (j == 0) {
         if (!wait_bounded(&c.q_full[t], 0, c.abort_flag, c.lim, 200 + t)) return false;
+        tc_fence_after_sync();
+    } else if (c.dec) {
+        // S_t is overwritten: the softmax warps must have read S_t(j-1)
+        if (!wait_bounded(&c.s_free[t], (j - 1) & 1, c.abort_flag, c.lim, 240 + t)) return false;
         tc_fence_after_sync();
     }
     const int L = 2 * j, stage = L % NS;
@@ -263,7 +301,7 @@ __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first
         tc_fence_after_sync();
     }
     const uint32_t v_addr = smem_u32(c.sKV + stage * C::KV_BYTES);
-    const uint32_t a_tmem = c.tmem + b * BN;
+    const uint32_t a_tmem = c.tmem + (c.dec ? C::P_COL + 64 * t : b * BN);
     const uint32_t o_tmem = c.tmem + C::O_COL + t * D;
 #pragma unroll
     for (int k = 0; k < BN / 16; ++k) {
@@ -298,6 +336,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     Cta<D> c;
     c.two = (C::MAXQ == 2) && (q0 + BM < seqlen);
+    c.dec = C::DECOUPLED && c.two;
     {
         const int endA = CAUSAL ? min(seqlen, q0 + BM) : seqlen;
         const int endB = CAUSAL ? min(seqlen, q0 + 2 * BM) : seqlen;
@@ -319,6 +358,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     c.p_full = c.s_full + 2;
     c.pv_done = c.p_full + 2;
     c.drain = c.pv_done + 2;
+    c.s_free = c.drain + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     c.abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     c.lim = p.timeout_ns;
@@ -332,6 +372,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_init(&c.s_full[t], 1);
             mbar_init(&c.p_full[t], 128);
             mbar_init(&c.pv_done[t], 1);
+            mbar_init(&c.s_free[t], 4);  // one arrival per softmax warp
         }
         for (int s = 0; s < NS; ++s) {
             mbar_init(&c.kv_full[s], 1);
@@ -415,6 +456,19 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         decode_step(idx, n, is_v, j);
                         ok = is_v ? mma_pv<D, BF16>(c, 0, j, true, true) : mma_qk<D, BF16>(c, 0, j, true, true);
                     }
+                } else if (c.dec) {
+                    // Separate P buffers: QK_t(j+1) only waits until the softmax warps have read
+                    // S_t(j), so it runs while they compute P_t(j). Order per step j:
+                    // QK_A(j+1), QK_B(j+1), PV_A(j), PV_B(j). Tile B (nB >= nA) is always the
+                    // last user of a key/value tile; tile A the first while j < nA.
+                    const int nA = c.nA, nB = c.nB;
+                    ok = mma_qk<D, BF16>(c, 0, 0, true, false) && mma_qk<D, BF16>(c, 1, 0, false, true);
+                    for (int j = 0; ok && j < nB; ++j) {
+                        if (j + 1 < nA) ok = mma_qk<D, BF16>(c, 0, j + 1, true, false);
+                        if (ok && j + 1 < nB) ok = mma_qk<D, BF16>(c, 1, j + 1, !(j + 1 < nA), true);
+                        if (ok && j < nA) ok = mma_pv<D, BF16>(c, 0, j, true, false);
+                        if (ok) ok = mma_pv<D, BF16>(c, 1, j, !(j < nA), true);
+                    }
                 } else {
                     // Tile A needs key tiles [0, nA), tile B [0, nB), nA <= nB <= nA + 1. A key or
                     // value tile is waited for at its first use and released after its last.
@@ -453,6 +507,76 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         float m = -INFINITY;  // running max of scaled scores, log2 units (possibly stale)
         float l = 0.f;        // running sum of 2^(s*sc - m)
         bool ok = n > 0;
+        if (c.dec) {
+            // Separate P buffer: S_t is released right after it is read, so QK_t(j+1) overlaps
+            // this step's exponentials; P_t(j) is written once PV_t(j-1) has consumed P_t(j-1).
+            const uint32_t p_addr = c.tmem + lane_base + C::P_COL + 64 * t;
+            for (int j = 0; j < n; ++j) {
+                if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[t], j & 1, c.abort_flag, c.lim, 330 + t))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                uint32_t sr[BN];
+#pragma unroll
+                for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(c.tmem + lane_base + t * BN + cc * 32, sr + cc * 32);
+                tmem_ld_wait();
+                tmem_reg_fence<BN>(sr);
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c.s_free[t]);
+                const int kv0 = j * BN;
+                const bool need_mask = (kv0 + BN > seqlen) || (CAUSAL && kv0 + BN - 1 > qt0);
+                if (need_mask) {
+                    const int valid = row_lim - kv0;
+#pragma unroll
+                    for (int i = 0; i < BN; ++i)
+                        if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
+                }
+                const float m_cand = row_max<BN>(sr) * sc;
+                const bool grow = m_cand > m + 8.0f;
+                float alpha = 1.f;
+                if (grow) {
+                    alpha = ex2_approx(m - m_cand);
+                    m = m_cand;
+                }
+                const bool warp_grow = __any_sync(0xffffffffu, grow);
+                uint32_t pk[BN / 2];
+                const float rs = need_mask ? softmax_row_to_regs<BN, BF16, 0>(sr, sc, -m, pk)
+                                           : softmax_row_to_regs<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, -m, pk);
+                l = fmaf(l, alpha, rs);
+                if (j > 0) {
+                    if (!__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (j - 1) & 1, c.abort_flag, c.lim, 340 + t))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    if (warp_grow) {
+                        const uint64_t a2 = f2(alpha, alpha);
+#pragma unroll 1
+                        for (int cc = 0; cc < D / 32; ++cc) {
+                            uint32_t o[32];
+                            tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
+                            tmem_ld_wait();
+                            tmem_reg_fence<32>(o);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                float lo, hi;
+                                f2_split(fmul2(f2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), lo, hi);
+                                o[2 * i] = __float_as_uint(lo);
+                                o[2 * i + 1] = __float_as_uint(hi);
+                            }
+                            tmem_st32(c.tmem + lane_base + o_col + cc * 32, o);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int cc = 0; cc < BN / 64; ++cc) tmem_st32(p_addr + cc * 32, pk + cc * 32);
+                tmem_st_wait();
+                tc_fence_before_sync();
+                mbar_arrive(&c.p_full[t]);
+            }
+        } else
         for (int j = 0; j < n; ++j) {
             const int b = c.buf(t, j);
             if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[b], c.sphase(j), c.abort_flag, c.lim, 300 + t))) {
