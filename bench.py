@@ -336,9 +336,7 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
 
     def call():
-        fa.fa_unpad(qp, idx, out=qu, stream=stream)
-        fa.fa_unpad(kp, idx, out=ku, stream=stream)
-        fa.fa_unpad(vp, idx, out=vu, stream=stream)
+        fa.fa_unpad_qkv(qp, kp, vp, idx, outs=(qu, ku, vu), stream=stream)
         fa.fa_varlen_fwd(qu, ku, vu, cu, case.max_seqlen, out=ou, lse=lse, stream=stream)
         fa.fa_pad(ou, idx, 1, case.total_len, out=out_pad, stream=stream)
 
@@ -352,9 +350,7 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
         flush.fill_(it & 0xFF)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
         ev[0].record(stream)
-        fa.fa_unpad(qp, idx, out=qu, stream=stream)
-        fa.fa_unpad(kp, idx, out=ku, stream=stream)
-        fa.fa_unpad(vp, idx, out=vu, stream=stream)
+        fa.fa_unpad_qkv(qp, kp, vp, idx, outs=(qu, ku, vu), stream=stream)
         ev[1].record(stream)
         fa.fa_varlen_fwd(qu, ku, vu, cu, case.max_seqlen, out=ou, lse=lse, stream=stream)
         ev[2].record(stream)
@@ -368,11 +364,12 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
     flops = 4.0 * H * D * sum(int(x) ** 2 for x in (case.cu_seqlens[1:] - case.cu_seqlens[:-1]))
     us = statistics.median(whole)
     return {"value": round(us, 2), "unit": "us/call", "stat": f"median of {iters}, L2 flushed before each call",
-            "config": "32 seqs x 64 tokens, H=16 D=128 bf16, padded (1,4096,16,128), non-causal",
+            "config": "32 seqs x 64 tokens, H=16 D=128 bf16, padded (1,4096,16,128), non-causal; "
+                      "fa_unpad_qkv + fa_varlen_fwd + fa_pad",
             "components_us_mean": {"unpad_qkv": round(tot[0] / iters, 2), "varlen_fwd": round(tot[1] / iters, 2),
                                    "pad_out": round(tot[2] / iters, 2)},
             "varlen_fwd_tflops": round(flops / (tot[1] / iters * 1e-6) / 1e12, 2),
-            "gpu_launches_per_call": 5}
+            "gpu_launches_per_call": 3}
 
 
 def run_padding_hbm_leg(fa, device, stream, iters):
@@ -408,6 +405,37 @@ def run_padding_hbm_leg(fa, device, stream, iters):
                      "frac": round(gbs / peak_bw, 4), "peak_kind": f"{peak_kind} HBM copy"}
     res["config"] = "(1, 262144, 16, 128) bf16 padded (1 GiB), 131072 valid rows; inputs larger than L2"
     return res
+
+
+def run_all_configs(args):
+    """TFLOPS of fa_fwd on every dense workload (informational; not the headline line)."""
+    import tiled_exact_attention_fwd_b200 as fa
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    peak_burst, _, _, _ = load_peaks()
+    for name, w in fa_inputs.WORKLOADS.items():
+        if w["kind"] != "dense":
+            continue
+        B, S, H, D, causal = w["B"], w["S"], w["H"], w["D"], w["causal"]
+        q, k, v = (t.to(device) for t in fa_inputs.dense_qkv(B, S, H, D, fa_inputs.DTYPES[w["dtype"]], seed=0))
+        out = torch.empty_like(q)
+        lse = torch.empty((B, H, S), device=device, dtype=torch.float32)
+        for _ in range(max(args.warmup, 3)):
+            fa.fa_fwd(q, k, v, out=out, lse=lse, causal=causal, stream=stream)
+        torch.cuda.synchronize(device)
+        n = max(1, min(args.steps, 50))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fa.fa_fwd(q, k, v, out=out, lse=lse, causal=causal, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms = e0.elapsed_time(e1) / n
+        tf = fa.attention_flops(B, H, S, S, D, causal) / (ms * 1e-3) / 1e12
+        print(json.dumps({"workload": name, "us": round(ms * 1e3, 1), "tflops": round(tf, 1),
+                          "frac_vs_burst": round(tf / peak_burst, 4), "launches": n}), flush=True)
+        del q, k, v, out, lse
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -450,11 +478,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only-main", action="store_true", help="time the main kernel only (for profiling)")
     ap.add_argument("--only-padding", action="store_true", help="run the unpad/pad HBM leg only (for profiling)")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="print one informational line per workload (dense/causal/head-dim sweep)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.all_configs:
+        run_all_configs(args)
     elif args.only_padding:
         import tiled_exact_attention_fwd_b200 as fa
         device = torch.device("cuda", 0)

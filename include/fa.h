@@ -75,9 +75,12 @@ FA_API fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, 
  *                [cu_seqlens[s], cu_seqlens[s+1]) and attends only inside itself.
  *   cu_seqlens   device int32 array of num_seqs+1 non-decreasing offsets, cu_seqlens[0] = 0,
  *                cu_seqlens[num_seqs] = total (read on the device; not checked on the host).
- *   max_seqlen   an upper bound of every sequence length (sizes the launch grid).
+ *   max_seqlen   the longest sequence (>= 1 when total > 0); kept for the interface of
+ *                flash_attn_varlen_func, the launch is sized by total.
  *   out          (total, H, D); lse (H, total) float32 or NULL.
- * Zero-length sequences are allowed and produce no rows. total may be 0 (no launch).
+ * Zero-length sequences are allowed and produce no rows. total may be 0 (no launch);
+ * total <= 65535 * 128. Work is split into tiles of 128 consecutive packed tokens, whatever
+ * sequences they hold (short sequences share a tile; each row only sees its own sequence).
  */
 FA_API fa_status fa_varlen_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqlens,
                         int num_seqs, int max_seqlen, int total, void *out, float *lse, int H,
@@ -94,6 +97,17 @@ FA_API fa_status fa_varlen_fwd(const void *q, const void *k, const void *v, cons
  */
 FA_API fa_status fa_unpad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
                    int64_t row_bytes, void *out, void *stream);
+
+/*
+ * Unpad of q, k and v in one launch: q_out[r] = q[indices[r]], k_out[r] = k[indices[r]],
+ * v_out[r] = v[indices[r]] for r < nnz. The packed path of page "IAW 模型 FA2 vs FA3 实测"
+ * (sections 1 and 6) gathers the three tensors with the same indices; one launch moves
+ * all three. Same argument rules and error behaviour as fa_unpad (all six pointers
+ * required; the 16-byte path needs all of them 16-byte aligned).
+ */
+FA_API fa_status fa_unpad_qkv(const void *q, const void *k, const void *v, const int64_t *indices,
+                              int64_t nnz, int64_t total_rows, int64_t row_bytes, void *q_out,
+                              void *k_out, void *v_out, void *stream);
 
 /*
  * Pad (scatter + zero fill): out[indices[r], :] = x[r, :] for r < nnz and every other

@@ -59,3 +59,17 @@ def test_unaligned_row_bytes_use_byte_path():
     assert torch.equal(u, oracle.unpad(x, idx))
     p = fa.fa_pad(u.to(dev), idx.to(dev), 1, 45).cpu()
     assert torch.equal(p, oracle.pad(u, idx, 1, 45))
+
+
+@pytest.mark.parametrize("shape", [(1, 4096, 16, 128), (2, 50, 3, 8), (1, 33, 1, 7)])
+def test_unpad_qkv_one_launch_bit_exact(shape):
+    B, L, H, D = shape
+    total = B * L
+    nnz = total // 2 + 1
+    q, k, v = (fa_inputs.normal(shape, torch.bfloat16, seed=s) for s in (1, 2, 3))
+    idx = fa_inputs.valid_indices(total, nnz, seed=9)
+    dev = torch.device("cuda:0")
+    outs = fa.fa_unpad_qkv(q.to(dev), k.to(dev), v.to(dev), idx.to(dev))
+    torch.cuda.synchronize()
+    for x, o in zip((q, k, v), outs):
+        assert torch.equal(_bits(o.cpu()), _bits(oracle.unpad(x, idx)))

@@ -47,9 +47,10 @@ def lib() -> ctypes.CDLL:
         L.fa_varlen_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, i32, i32, f32, i32, i32, vp]
         L.fa_unpad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fa_pad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
+        L.fa_unpad_qkv.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp]
         L.fa_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.fa_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
-        for f in (L.fa_fwd, L.fa_varlen_fwd, L.fa_unpad, L.fa_pad, L.fa_device_status,
+        for f in (L.fa_fwd, L.fa_varlen_fwd, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad, L.fa_device_status,
                   L.fa_selftest_bounded_wait):
             f.restype = ctypes.c_int
         L.fa_status_string.argtypes = [ctypes.c_int]
@@ -157,6 +158,27 @@ def fa_unpad(x: torch.Tensor, indices: torch.Tensor, out: Optional[torch.Tensor]
     st = lib().fa_unpad(_ptr(x), _ptr(indices), nnz, total_rows, row_bytes, _ptr(out), _stream(stream))
     _check(st, "fa_unpad")
     return out
+
+
+def fa_unpad_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, indices: torch.Tensor, outs=None,
+                 stream=None):
+    """The three gathers of the packed path in one launch: returns (q_unpad, k_unpad, v_unpad)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("indices", indices)):
+        _cuda_contig(n, t)
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one shape and dtype")
+    if indices.dtype != torch.int64:
+        raise ValueError("indices must be int64")
+    H, D = q.shape[-2], q.shape[-1]
+    nnz = indices.numel()
+    if outs is None:
+        outs = tuple(torch.empty((nnz, H, D), device=q.device, dtype=q.dtype) for _ in range(3))
+    for i, o in enumerate(outs):
+        _cuda_contig(f"outs[{i}]", o)
+    st = lib().fa_unpad_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(indices), nnz, q.numel() // (H * D),
+                            H * D * q.element_size(), _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), _stream(stream))
+    _check(st, "fa_unpad_qkv")
+    return outs
 
 
 def fa_pad(x: torch.Tensor, indices: torch.Tensor, batch: int, total_len: int,

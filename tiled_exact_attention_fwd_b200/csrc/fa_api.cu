@@ -71,7 +71,7 @@ bool encode_map(CUtensorMap *m, const void *base, bool bf16, int D, int H, int64
 }
 
 fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
-                  const int32_t *cu_seqlens, int num_seqs, int seqlen_or_max, int64_t N, int H, int D,
+                  const int32_t *cu_seqlens, int num_seqs, int seqlen, int64_t N, int H, int D,
                   float scale, int causal, fa_dtype dtype, void *stream) {
     const bool bf16 = dtype == FA_BF16;
     const int inner = fa::fwd_box_inner_elems(D);
@@ -85,15 +85,23 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     p.out = out;
     p.lse = lse;
     p.cu_seqlens = cu_seqlens;
-    p.seqlen = seqlen_or_max;
+    p.num_seqs = num_seqs;
+    p.seqlen = seqlen;
     p.H = H;
     p.total_tokens = static_cast<int>(N);
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = wait_limit_ns();
-    const int qtiles = (seqlen_or_max + fa::fwd_tile_rows() - 1) / fa::fwd_tile_rows();
-    const int per_cta = fa::fwd_tiles_per_cta(D);
-    const int ctas_y = (qtiles + per_cta - 1) / per_cta;
-    const dim3 grid(static_cast<unsigned>(H), static_cast<unsigned>(ctas_y), static_cast<unsigned>(num_seqs));
+    const int rows = fa::fwd_tile_rows();
+    dim3 grid;
+    if (cu_seqlens) {
+        // packed: one CTA per 128 consecutive tokens of the packed tensor
+        grid = dim3(static_cast<unsigned>(H), static_cast<unsigned>((N + rows - 1) / rows), 1);
+    } else {
+        const int qtiles = (seqlen + rows - 1) / rows;
+        const int per_cta = fa::fwd_tiles_per_cta(D);
+        grid = dim3(static_cast<unsigned>(H), static_cast<unsigned>((qtiles + per_cta - 1) / per_cta),
+                    static_cast<unsigned>(num_seqs));
+    }
     const cudaError_t e = fa::launch_fwd(D, bf16, causal != 0, tq, tk, tv, p, grid,
                                          static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -125,7 +133,7 @@ fa_status fa_varlen_fwd(const void *q, const void *k, const void *v, const int32
     if (total == 0 || num_seqs == 0) return FA_OK;  // no rows, nothing to launch
     if (!q || !k || !v || !out || !cu_seqlens) return FA_ERR_NULL;
     if (max_seqlen == 0) return FA_ERR_SHAPE;
-    if (num_seqs > 65535 || (max_seqlen + 127) / 128 > 65535) return FA_ERR_SHAPE;
+    if ((static_cast<int64_t>(total) + 127) / 128 > 65535) return FA_ERR_SHAPE;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
         !aligned(cu_seqlens, 4))
         return FA_ERR_ALIGN;
@@ -141,6 +149,18 @@ fa_status fa_unpad(const void *x, const int64_t *indices, int64_t nnz, int64_t t
     if (!aligned(indices, 8)) return FA_ERR_ALIGN;
     const cudaError_t e = fa::launch_unpad(x, indices, nnz, total_rows, row_bytes, out,
                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_unpad_qkv(const void *q, const void *k, const void *v, const int64_t *indices, int64_t nnz,
+                       int64_t total_rows, int64_t row_bytes, void *q_out, void *k_out, void *v_out, void *stream) {
+    if (nnz < 0 || total_rows < 0 || row_bytes <= 0) return FA_ERR_SHAPE;
+    if (nnz == 0) return FA_OK;
+    if (!q || !k || !v || !indices || !q_out || !k_out || !v_out) return FA_ERR_NULL;
+    if (!aligned(indices, 8)) return FA_ERR_ALIGN;
+    const void *const x[3] = {q, k, v};
+    void *const o[3] = {q_out, k_out, v_out};
+    const cudaError_t e = fa::launch_unpad3(x, indices, nnz, total_rows, row_bytes, o, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -128,6 +128,17 @@ struct Cfg {
     static_assert(Q_BYTES % 1024 == 0 && KV_BYTES % 1024 == 0, "tile alignment");
 };
 
+// Sequence that packed token `tok` belongs to: the s with cu[s] <= tok < cu[s+1]
+// (binary search over the num_seqs + 1 offsets; empty sequences are skipped).
+__device__ __forceinline__ int seq_of_token(const int32_t *cu, int num_seqs, int tok) {
+    int lo = 0, hi = num_seqs;  // invariant: cu[lo] <= tok < cu[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(cu + mid) <= tok) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
 // Single-tile order of MMA steps: K0, K1, V0, K2, V1, ..., V_{n-1} (QK runs one tile ahead).
 __device__ __forceinline__ void decode_step(int idx, int n, bool &is_v, int &j) {
     if (idx == 0) { is_v = false; j = 0; }
@@ -321,28 +332,42 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
 
     const int h = blockIdx.x;
-    const int pair = gridDim.y - 1 - blockIdx.y;  // longest (causal) tiles first
-    const int seq = blockIdx.z;
-    int seq_start, seqlen;
-    if (p.cu_seqlens) {
-        seq_start = p.cu_seqlens[seq];
-        seqlen = p.cu_seqlens[seq + 1] - seq_start;
-    } else {
-        seq_start = seq * p.seqlen;
+    // Rows of the CTA are tokens qbase + t*128 + r; keys are addressed from token kvbase.
+    //  dense : blockIdx.z is the batch entry; the CTA owns query tiles `pair` (two of them
+    //          when MAXQ = 2) of that sequence, longest (causal) tiles launched first.
+    //  packed: the CTA owns the 128 consecutive packed tokens of tile blockIdx.y, whatever
+    //          sequences they belong to; its keys are the union of those sequences' keys
+    //          (the device walks cu_seqlens), and each row is masked to its own sequence.
+    const bool packed = p.cu_seqlens != nullptr;
+    int seq_start = 0, seqlen = 0, q0 = 0, qbase, kvbase, kv_end_A, kv_end_B = 0;
+    bool two = false;
+    if (!packed) {
+        const int pair = gridDim.y - 1 - blockIdx.y;
+        seq_start = blockIdx.z * p.seqlen;
         seqlen = p.seqlen;
+        q0 = pair * C::MAXQ * BM;
+        if (q0 >= seqlen) return;  // uniform over the CTA, before any barrier exists
+        two = (C::MAXQ == 2) && (q0 + BM < seqlen);
+        qbase = seq_start + q0;
+        kvbase = seq_start;
+        kv_end_A = CAUSAL ? min(seqlen, q0 + BM) : seqlen;
+        if (two) kv_end_B = CAUSAL ? min(seqlen, q0 + 2 * BM) : seqlen;
+    } else {
+        qbase = blockIdx.y * BM;
+        if (qbase >= p.total_tokens) return;
+        const int tlast = min(qbase + BM, p.total_tokens) - 1;
+        const int s_first = seq_of_token(p.cu_seqlens, p.num_seqs, qbase);
+        const int s_last = seq_of_token(p.cu_seqlens, p.num_seqs, tlast);
+        kvbase = p.cu_seqlens[s_first];
+        const int kv_hi = CAUSAL ? min(p.cu_seqlens[s_last + 1], tlast + 1) : p.cu_seqlens[s_last + 1];
+        kv_end_A = kv_hi - kvbase;
     }
-    const int q0 = pair * C::MAXQ * BM;  // first row of tile A
-    if (q0 >= seqlen) return;            // uniform over the CTA, before any barrier exists
 
     Cta<D> c;
-    c.two = (C::MAXQ == 2) && (q0 + BM < seqlen);
+    c.two = two;
     c.dec = C::DECOUPLED && c.two;
-    {
-        const int endA = CAUSAL ? min(seqlen, q0 + BM) : seqlen;
-        const int endB = CAUSAL ? min(seqlen, q0 + 2 * BM) : seqlen;
-        c.nA = (endA + BN - 1) / BN;
-        c.nB = c.two ? (endB + BN - 1) / BN : 0;
-    }
+    c.nA = (kv_end_A + BN - 1) / BN;
+    c.nB = c.two ? (kv_end_B + BN - 1) / BN : 0;
     const int n_all = max(c.nA, c.nB);  // key tiles this CTA loads
 
     extern __shared__ uint8_t smem_raw[];
@@ -410,7 +435,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     #pragma unroll
                     for (int b = 0; b < C::NBLK; ++b)
                         tma_load_3d(c.sQ + t * C::Q_BYTES + b * BM * SW, &tm_q, &c.q_full[t], b * C::SWE, h,
-                                    seq_start + q0 + t * BM, pol_q);
+                                    qbase + t * BM, pol_q);
                 }
                 const int loads = 2 * n_all;  // K_0, V_0, K_1, V_1, ...
                 int issued = 0;
@@ -425,7 +450,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const CUtensorMap *map = (L & 1) ? &tm_v : &tm_k;
     #pragma unroll
                     for (int b = 0; b < C::NBLK; ++b)
-                        tma_load_3d(dst + b * BN * SW, map, &c.kv_full[stage], b * C::SWE, h, seq_start + j * BN,
+                        tma_load_3d(dst + b * BN * SW, map, &c.kv_full[stage], b * C::SWE, h, kvbase + j * BN,
                                     pol_kv);
                     issued = L + 1;
                 }
@@ -499,9 +524,22 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int quarter = warp & 3;                 // TMEM lanes this warp may access
         const int r = quarter * 32 + lane;            // row of the tile == TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        const int qt0 = q0 + t * BM;
-        const int row_pos = qt0 + r;                  // position inside the sequence
-        const int row_lim = CAUSAL ? min(seqlen, row_pos + 1) : seqlen;  // keys [0, row_lim)
+        // This row's token and its visible keys [klo, khi), counted from kvbase.
+        const int64_t tok = static_cast<int64_t>(qbase) + t * BM + r;
+        int klo = 0, khi = 1;
+        bool row_ok;
+        if (!packed) {
+            const int row_pos = q0 + t * BM + r;  // position inside the sequence
+            row_ok = row_pos < seqlen;
+            khi = CAUSAL ? min(seqlen, row_pos + 1) : seqlen;
+        } else {
+            row_ok = tok < p.total_tokens;
+            if (row_ok) {
+                const int s_r = seq_of_token(p.cu_seqlens, p.num_seqs, static_cast<int>(tok));
+                klo = p.cu_seqlens[s_r] - kvbase;
+                khi = (CAUSAL ? min(p.cu_seqlens[s_r + 1], static_cast<int>(tok) + 1) : p.cu_seqlens[s_r + 1]) - kvbase;
+            }
+        }
         const uint32_t o_col = C::O_COL + t * D;
         const float sc = p.scale_log2;
         float m = -INFINITY;  // running max of scaled scores, log2 units (possibly stale)
@@ -525,13 +563,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&c.s_free[t]);
-                const int kv0 = j * BN;
-                const bool need_mask = (kv0 + BN > seqlen) || (CAUSAL && kv0 + BN - 1 > qt0);
+                const int lo = klo - j * BN, hi = khi - j * BN;  // visible columns of this tile
+                const bool need_mask = __any_sync(0xffffffffu, lo > 0 || hi < BN);
                 if (need_mask) {
-                    const int valid = row_lim - kv0;
 #pragma unroll
                     for (int i = 0; i < BN; ++i)
-                        if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
+                        if (i < lo || i >= hi) sr[i] = __float_as_uint(-INFINITY);
                 }
                 const float m_cand = row_max<BN>(sr) * sc;
                 const bool grow = m_cand > m + 8.0f;
@@ -542,8 +579,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
                 const bool warp_grow = __any_sync(0xffffffffu, grow);
                 uint32_t pk[BN / 2];
-                const float rs = need_mask ? softmax_row_to_regs<BN, BF16, 0>(sr, sc, -m, pk)
-                                           : softmax_row_to_regs<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, -m, pk);
+                // a packed row may not have met any visible key yet (m = -inf): its P is 0
+                const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                const float rs = need_mask ? softmax_row_to_regs<BN, BF16, 0>(sr, sc, neg_m, pk)
+                                           : softmax_row_to_regs<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, pk);
                 l = fmaf(l, alpha, rs);
                 if (j > 0) {
                     if (!__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (j - 1) & 1, c.abort_flag, c.lim, 340 + t))) {
@@ -589,13 +628,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(c.tmem + lane_base + b * BN + cc * 32, sr + cc * 32);
             tmem_ld_wait();
             tmem_reg_fence<BN>(sr);
-            const int kv0 = j * BN;
-            const bool need_mask = (kv0 + BN > seqlen) || (CAUSAL && kv0 + BN - 1 > qt0);
+            const int lo = klo - j * BN, hi = khi - j * BN;  // visible columns of this tile
+            const bool need_mask = __any_sync(0xffffffffu, lo > 0 || hi < BN);
             if (need_mask) {
-                const int valid = row_lim - kv0;  // columns [0, valid) of this tile are visible
 #pragma unroll
                 for (int i = 0; i < BN; ++i)
-                    if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
+                    if (i < lo || i >= hi) sr[i] = __float_as_uint(-INFINITY);
             }
             const float mx = row_max<BN>(sr);
             const float m_cand = mx * sc;
@@ -607,7 +645,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             const bool warp_grow = __any_sync(0xffffffffu, grow);
             // P = 2^(s*sc - m): written back to TMEM over S, 64 columns at a time.
-            const float neg_m = -m;
+            // a packed row may not have met any visible key yet (m = -inf): its P is 0
+            const float neg_m = (m == -INFINITY) ? 0.f : -m;
             const uint32_t p_addr = c.tmem + lane_base + b * BN;
             const float rs = need_mask ? softmax_chunk_store<BN, BF16, 0>(sr, sc, neg_m, p_addr)  // -inf -> exactly 0
                                        : softmax_chunk_store<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, p_addr);
@@ -649,8 +688,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (ok) {
             tc_fence_after_sync();
             const float inv_l = 1.f / l;
-            const int64_t tok = static_cast<int64_t>(seq_start) + row_pos;
-            const bool row_ok = row_pos < seqlen && tok < p.total_tokens;
             uint4 *orow = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) +
                                                     (tok * p.H + h) * static_cast<int64_t>(D) * 2);
 #pragma unroll 1
@@ -671,8 +708,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             if (row_ok && p.lse) {
                 const float lse = m * 0.6931471805599453f + logf(l);
-                const int64_t li = p.cu_seqlens ? static_cast<int64_t>(h) * p.total_tokens + tok
-                                                : (static_cast<int64_t>(seq) * p.H + h) * p.seqlen + row_pos;
+                const int64_t li = packed ? static_cast<int64_t>(h) * p.total_tokens + tok
+                                          : (static_cast<int64_t>(blockIdx.z) * p.H + h) * p.seqlen + (tok - seq_start);
                 p.lse[li] = lse;
             }
         }

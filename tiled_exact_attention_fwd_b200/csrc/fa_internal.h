@@ -12,6 +12,7 @@ struct FwdParams {
     void *out;                  // token-major (N, H, D) output
     float *lse;                 // dense: (B, H, S); packed: (H, total); may be null
     const int32_t *cu_seqlens;  // null for dense (uniform sequences of `seqlen`)
+    int num_seqs;               // packed: entries of cu_seqlens minus one
     int seqlen;                 // dense sequence length
     int H;                      // heads
     int total_tokens;           // N = rows of the token-major tensors
@@ -19,8 +20,9 @@ struct FwdParams {
     uint64_t timeout_ns;        // bound of every pipeline wait
 };
 
-// Attention forward: grid (H, ceil(ceil(max_len / 128) / tiles_per_cta), num_seqs); a CTA
-// owns fwd_tiles_per_cta(D) consecutive 128-row query tiles.
+// Attention forward. Dense: grid (H, ceil(ceil(S / 128) / tiles_per_cta), B), a CTA owns
+// fwd_tiles_per_cta(D) consecutive 128-row query tiles of one sequence. Packed: grid
+// (H, ceil(total / 128), 1), a CTA owns 128 consecutive packed tokens.
 cudaError_t launch_fwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
                        const CUtensorMap &tv, const FwdParams &p, dim3 grid, cudaStream_t st);
 int fwd_tile_rows();
@@ -33,6 +35,8 @@ cudaError_t fwd_take_device_error(int *code, int *where);
 // Unpad / pad (row gather / scatter + zero fill).
 cudaError_t launch_unpad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
                          int64_t row_bytes, void *out, cudaStream_t st);
+cudaError_t launch_unpad3(const void *const x[3], const int64_t *indices, int64_t nnz, int64_t total_rows,
+                          int64_t row_bytes, void *const out[3], cudaStream_t st);
 cudaError_t launch_pad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
                        int64_t row_bytes, void *out, cudaStream_t st);
 cudaError_t pad_take_device_error(int *code, int *where);

@@ -73,6 +73,47 @@ __global__ void __launch_bounds__(256) unpad_kernel(const T *__restrict__ x, con
     }
 }
 
+// The three gathers of the packed path (q, k, v share one index list) in one launch: each
+// warp moves row r of all three tensors, so three rows' loads are in flight together.
+template <typename T>
+__global__ void __launch_bounds__(256) unpad3_kernel(const T *__restrict__ x0, const T *__restrict__ x1,
+                                                     const T *__restrict__ x2, const int64_t *__restrict__ idx,
+                                                     int64_t nnz, int64_t total_rows, int64_t per_row,
+                                                     T *__restrict__ o0, T *__restrict__ o1, T *__restrict__ o2) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wpb = blockDim.x >> 5;
+    const int64_t nw = gridDim.x * wpb;
+    for (int64_t r = blockIdx.x * wpb + (threadIdx.x >> 5); r < nnz; r += nw) {
+        const int64_t src = __ldg(idx + r);
+        const int64_t dst = r * per_row;
+        if (src < 0 || src >= total_rows) {
+            warp_zero_row(o0 + dst, per_row, lane);
+            warp_zero_row(o1 + dst, per_row, lane);
+            warp_zero_row(o2 + dst, per_row, lane);
+            if (lane == 0) pad_record_error(FA_ERR_INDEX, 3);
+            continue;
+        }
+        const int64_t so = src * per_row;
+        int64_t c = lane;
+        for (; c + 32 < per_row; c += 64) {
+            const T a0 = ld_stream(x0 + so + c), a1 = ld_stream(x1 + so + c), a2 = ld_stream(x2 + so + c);
+            const T b0 = ld_stream(x0 + so + c + 32), b1 = ld_stream(x1 + so + c + 32), b2 = ld_stream(x2 + so + c + 32);
+            o0[dst + c] = a0;
+            o1[dst + c] = a1;
+            o2[dst + c] = a2;
+            o0[dst + c + 32] = b0;
+            o1[dst + c + 32] = b1;
+            o2[dst + c + 32] = b2;
+        }
+        for (; c < per_row; c += 32) {
+            const T a0 = ld_stream(x0 + so + c), a1 = ld_stream(x1 + so + c), a2 = ld_stream(x2 + so + c);
+            o0[dst + c] = a0;
+            o1[dst + c] = a1;
+            o2[dst + c] = a2;
+        }
+    }
+}
+
 // Every output row t of [t0, t1) (one contiguous range per block, one warp per row):
 // copy x[r] if indices[r] == t for some r, zeros otherwise. With strictly increasing
 // indices, the r for row t lies in [r0, r0 + (t - t0)], r0 = lower_bound(indices, t0).
@@ -134,6 +175,26 @@ cudaError_t launch_unpad(const void *x, const int64_t *indices, int64_t nnz, int
     else
         unpad_kernel<uint8_t><<<blocks, 256, 0, st>>>(static_cast<const uint8_t *>(x), indices, nnz,
                                                       total_rows, row_bytes, static_cast<uint8_t *>(out));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unpad3(const void *const x[3], const int64_t *indices, int64_t nnz, int64_t total_rows,
+                          int64_t row_bytes, void *const out[3], cudaStream_t st) {
+    if (nnz == 0) return cudaSuccess;
+    const int64_t want = (nnz + 7) / 8;
+    const int blocks = static_cast<int>(want < int64_t(num_sms()) * 8 ? want : int64_t(num_sms()) * 8);
+    bool vec = true;
+    for (int i = 0; i < 3; ++i) vec = vec && vec16_ok(x[i], out[i], row_bytes);
+    if (vec)
+        unpad3_kernel<uint4><<<blocks, 256, 0, st>>>(
+            static_cast<const uint4 *>(x[0]), static_cast<const uint4 *>(x[1]), static_cast<const uint4 *>(x[2]),
+            indices, nnz, total_rows, row_bytes / 16, static_cast<uint4 *>(out[0]), static_cast<uint4 *>(out[1]),
+            static_cast<uint4 *>(out[2]));
+    else
+        unpad3_kernel<uint8_t><<<blocks, 256, 0, st>>>(
+            static_cast<const uint8_t *>(x[0]), static_cast<const uint8_t *>(x[1]), static_cast<const uint8_t *>(x[2]),
+            indices, nnz, total_rows, row_bytes, static_cast<uint8_t *>(out[0]), static_cast<uint8_t *>(out[1]),
+            static_cast<uint8_t *>(out[2]));
     return cudaGetLastError();
 }
 
