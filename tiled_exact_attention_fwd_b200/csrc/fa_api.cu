@@ -94,8 +94,9 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     const int rows = fa::fwd_tile_rows();
     dim3 grid;
     if (cu_seqlens) {
-        // packed: one CTA per 128 consecutive tokens of the packed tensor
-        grid = dim3(static_cast<unsigned>(H), static_cast<unsigned>((N + rows - 1) / rows), 1);
+        // packed: one CTA per tiles_per_cta x 128 consecutive tokens of the packed tensor
+        const int64_t span = static_cast<int64_t>(rows) * fa::fwd_tiles_per_cta(D);
+        grid = dim3(static_cast<unsigned>(H), static_cast<unsigned>((N + span - 1) / span), 1);
     } else {
         const int qtiles = (seqlen + rows - 1) / rows;
         const int per_cta = fa::fwd_tiles_per_cta(D);

@@ -255,7 +255,12 @@ struct Cta {
     volatile int *abort_flag;
     uint32_t tmem;
     uint64_t lim;
-    int nA, nB;    // key tiles of query tile A and B (nB = 0 when B is absent)
+    // Tile A visits key tiles [0, nA), tile B [jB0, nB) (nB = 0 when B is absent); key tile j
+    // covers tokens kvbase + [j*BN, (j+1)*BN). In dense sequences jB0 = 0; in packed ones
+    // B may begin a later sequence. Always jB0 <= nA <= nB, so the two ranges leave no gap.
+    int nA, nB, jB0;
+    __device__ __forceinline__ int j0(int t) const { return t ? jB0 : 0; }
+    __device__ __forceinline__ bool uses(int t, int j) const { return t ? (j >= jB0 && j < nB) : (j < nA); }
     bool two;      // two query tiles (ping-pong) or one (S double-buffered)
     bool dec;      // two tiles with separate P buffers (Cfg::DECOUPLED)
     // S/P buffer and barrier phase used by tile t at key step j
@@ -265,16 +270,18 @@ struct Cta {
 
 // One MMA step of the issuing thread. Returns false when a wait gave up.
 template <int D, bool BF16>
+// S_t = Q_t K_j^T for key tile j (tile-local step jj = j - j0(t)).
 __device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first_use, bool last_use) {
     using C = Cfg<D>;
     constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
     constexpr uint32_t idesc = idesc_f16(BM, BN, BF16, false);
-    if (j == 0) {
+    const int jj = j - c.j0(t);
+    if (jj == 0) {
         if (!wait_bounded(&c.q_full[t], 0, c.abort_flag, c.lim, 200 + t)) return false;
         tc_fence_after_sync();
     } else if (c.dec) {
-        // S_t is overwritten: the softmax warps must have read S_t(j-1)
-        if (!wait_bounded(&c.s_free[t], (j - 1) & 1, c.abort_flag, c.lim, 240 + t)) return false;
+        // S_t is overwritten: the softmax warps must have read the previous S_t
+        if (!wait_bounded(&c.s_free[t], (jj - 1) & 1, c.abort_flag, c.lim, 240 + t)) return false;
         tc_fence_after_sync();
     }
     const int L = 2 * j, stage = L % NS;
@@ -284,7 +291,7 @@ __device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first
     }
     const uint32_t q_addr = smem_u32(c.sQ + t * C::Q_BYTES);
     const uint32_t k_addr = smem_u32(c.sKV + stage * C::KV_BYTES);
-    const int b = c.buf(t, j);
+    const int b = c.buf(t, jj);
     const uint32_t d_tmem = c.tmem + b * BN;
 #pragma unroll
     for (int k = 0; k < D / 16; ++k) {
@@ -299,12 +306,14 @@ __device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first
 }
 
 template <int D, bool BF16>
+// O_t += P_t V_j for key tile j (tile-local step jj = j - j0(t)).
 __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first_use, bool last_use) {
     using C = Cfg<D>;
     constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
     constexpr uint32_t idesc = idesc_f16(BM, D, BF16, true);
-    const int b = c.buf(t, j);
-    if (!wait_bounded(&c.p_full[b], c.sphase(j), c.abort_flag, c.lim, 210 + t)) return false;
+    const int jj = j - c.j0(t);
+    const int b = c.buf(t, jj);
+    if (!wait_bounded(&c.p_full[b], c.sphase(jj), c.abort_flag, c.lim, 210 + t)) return false;
     tc_fence_after_sync();
     const int L = 2 * j + 1, stage = L % NS;
     if (first_use) {
@@ -317,7 +326,7 @@ __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first
 #pragma unroll
     for (int k = 0; k < BN / 16; ++k) {
         const uint64_t bd = smem_desc(v_addr + k * 16 * SW, BN * SW, 8 * SW, C::LAYOUT);
-        umma_ts(o_tmem, a_tmem + k * 8, bd, idesc, (j > 0 || k > 0) ? 1u : 0u);
+        umma_ts(o_tmem, a_tmem + k * 8, bd, idesc, (jj > 0 || k > 0) ? 1u : 0u);
     }
     umma_commit(&c.pv_done[t]);
     if (last_use) umma_commit(&c.kv_empty[stage]);
@@ -339,7 +348,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     //          sequences they belong to; its keys are the union of those sequences' keys
     //          (the device walks cu_seqlens), and each row is masked to its own sequence.
     const bool packed = p.cu_seqlens != nullptr;
-    int seq_start = 0, seqlen = 0, q0 = 0, qbase, kvbase, kv_end_A, kv_end_B = 0;
+    int seq_start = 0, seqlen = 0, q0 = 0, qbase, kvbase, kv_end_A, kv_end_B = 0, kv_start_B = 0;
     bool two = false;
     if (!packed) {
         const int pair = gridDim.y - 1 - blockIdx.y;
@@ -353,14 +362,21 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         kv_end_A = CAUSAL ? min(seqlen, q0 + BM) : seqlen;
         if (two) kv_end_B = CAUSAL ? min(seqlen, q0 + 2 * BM) : seqlen;
     } else {
-        qbase = blockIdx.y * BM;
+        qbase = blockIdx.y * C::MAXQ * BM;
         if (qbase >= p.total_tokens) return;
-        const int tlast = min(qbase + BM, p.total_tokens) - 1;
+        two = (C::MAXQ == 2) && (qbase + BM < p.total_tokens);
         const int s_first = seq_of_token(p.cu_seqlens, p.num_seqs, qbase);
-        const int s_last = seq_of_token(p.cu_seqlens, p.num_seqs, tlast);
         kvbase = p.cu_seqlens[s_first];
-        const int kv_hi = CAUSAL ? min(p.cu_seqlens[s_last + 1], tlast + 1) : p.cu_seqlens[s_last + 1];
-        kv_end_A = kv_hi - kvbase;
+        // keys of a tile end with its last row's sequence (or the causal limit)
+        auto kv_end = [&](int tlast) {
+            const int s_last = seq_of_token(p.cu_seqlens, p.num_seqs, tlast);
+            return (CAUSAL ? min(p.cu_seqlens[s_last + 1], tlast + 1) : p.cu_seqlens[s_last + 1]) - kvbase;
+        };
+        kv_end_A = kv_end(min(qbase + BM, p.total_tokens) - 1);
+        if (two) {
+            kv_end_B = kv_end(min(qbase + 2 * BM, p.total_tokens) - 1);
+            kv_start_B = p.cu_seqlens[seq_of_token(p.cu_seqlens, p.num_seqs, qbase + BM)] - kvbase;
+        }
     }
 
     Cta<D> c;
@@ -368,6 +384,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     c.dec = C::DECOUPLED && c.two;
     c.nA = (kv_end_A + BN - 1) / BN;
     c.nB = c.two ? (kv_end_B + BN - 1) / BN : 0;
+    c.jB0 = c.two ? kv_start_B / BN : 0;
     const int n_all = max(c.nA, c.nB);  // key tiles this CTA loads
 
     extern __shared__ uint8_t smem_raw[];
@@ -483,31 +500,31 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                 } else if (c.dec) {
                     // Separate P buffers: QK_t(j+1) only waits until the softmax warps have read
-                    // S_t(j), so it runs while they compute P_t(j). Order per step j:
-                    // QK_A(j+1), QK_B(j+1), PV_A(j), PV_B(j). Tile B (nB >= nA) is always the
-                    // last user of a key/value tile; tile A the first while j < nA.
-                    const int nA = c.nA, nB = c.nB;
-                    ok = mma_qk<D, BF16>(c, 0, 0, true, false) && mma_qk<D, BF16>(c, 1, 0, false, true);
+                    // S_t(j), so it runs while they compute P_t(j). Order per key tile j:
+                    // QK_A(j+1), QK_B(j+1), PV_A(j), PV_B(j), each when that tile uses key tile j.
+                    const int nB = c.nB;
+                    if (c.uses(0, 0)) ok = mma_qk<D, BF16>(c, 0, 0, true, !c.uses(1, 0));
+                    if (ok && c.uses(1, 0)) ok = mma_qk<D, BF16>(c, 1, 0, !c.uses(0, 0), true);
                     for (int j = 0; ok && j < nB; ++j) {
-                        if (j + 1 < nA) ok = mma_qk<D, BF16>(c, 0, j + 1, true, false);
-                        if (ok && j + 1 < nB) ok = mma_qk<D, BF16>(c, 1, j + 1, !(j + 1 < nA), true);
-                        if (ok && j < nA) ok = mma_pv<D, BF16>(c, 0, j, true, false);
-                        if (ok) ok = mma_pv<D, BF16>(c, 1, j, !(j < nA), true);
+                        const bool a1 = c.uses(0, j + 1), b1 = c.uses(1, j + 1), a0 = c.uses(0, j), b0 = c.uses(1, j);
+                        if (a1) ok = mma_qk<D, BF16>(c, 0, j + 1, true, !b1);
+                        if (ok && b1) ok = mma_qk<D, BF16>(c, 1, j + 1, !a1, true);
+                        if (ok && a0) ok = mma_pv<D, BF16>(c, 0, j, true, !b0);
+                        if (ok && b0) ok = mma_pv<D, BF16>(c, 1, j, !a0, true);
                     }
                 } else {
-                    // Tile A needs key tiles [0, nA), tile B [0, nB), nA <= nB <= nA + 1. A key or
+                    // Ping-pong over key tiles j: PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j). A key or
                     // value tile is waited for at its first use and released after its last.
-                    const int nA = c.nA, nB = c.nB;
-                    ok = mma_qk<D, BF16>(c, 0, 0, true, false) && mma_qk<D, BF16>(c, 1, 0, false, true);
-                    for (int j = 1; ok && j < nB; ++j) {
-                        const bool a_prev = j - 1 < nA, a_cur = j < nA;
-                        if (a_prev) ok = mma_pv<D, BF16>(c, 0, j - 1, true, false);
-                        if (ok && a_cur) ok = mma_qk<D, BF16>(c, 0, j, true, false);
-                        if (ok) ok = mma_pv<D, BF16>(c, 1, j - 1, !a_prev, true);
-                        if (ok) ok = mma_qk<D, BF16>(c, 1, j, !a_cur, true);
+                    const int nB = c.nB;
+                    if (c.uses(0, 0)) ok = mma_qk<D, BF16>(c, 0, 0, true, !c.uses(1, 0));
+                    if (ok && c.uses(1, 0)) ok = mma_qk<D, BF16>(c, 1, 0, !c.uses(0, 0), true);
+                    for (int j = 1; ok && j <= nB; ++j) {
+                        const bool ap = c.uses(0, j - 1), bp = c.uses(1, j - 1), ac = c.uses(0, j), bc = c.uses(1, j);
+                        if (ap) ok = mma_pv<D, BF16>(c, 0, j - 1, true, !bp);
+                        if (ok && ac) ok = mma_qk<D, BF16>(c, 0, j, true, !bc);
+                        if (ok && bp) ok = mma_pv<D, BF16>(c, 1, j - 1, !ap, true);
+                        if (ok && bc) ok = mma_qk<D, BF16>(c, 1, j, !ac, true);
                     }
-                    if (ok && nB - 1 < nA) ok = mma_pv<D, BF16>(c, 0, nB - 1, true, false);
-                    if (ok) ok = mma_pv<D, BF16>(c, 1, nB - 1, !(nB - 1 < nA), true);
                 }
                 // Every MMA issued above has finished once `drain` completes.
                 umma_commit(c.drain);
@@ -520,7 +537,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // ------------------------------------------------------------ softmax + epilogue
         if constexpr (C::SPLIT_REGS) regs_inc<C::REGS_HIGH>();
         const int t = warp >> 2;                      // query tile of this warpgroup
-        const int n = t ? c.nB : c.nA;
+        const int n = t ? c.nB - c.jB0 : c.nA;  // key tiles this warpgroup visits
+        const int j0 = c.j0(t);
         const int quarter = warp & 3;                 // TMEM lanes this warp may access
         const int r = quarter * 32 + lane;            // row of the tile == TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -549,8 +567,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // Separate P buffer: S_t is released right after it is read, so QK_t(j+1) overlaps
             // this step's exponentials; P_t(j) is written once PV_t(j-1) has consumed P_t(j-1).
             const uint32_t p_addr = c.tmem + lane_base + C::P_COL + 64 * t;
-            for (int j = 0; j < n; ++j) {
-                if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[t], j & 1, c.abort_flag, c.lim, 330 + t))) {
+            for (int jj = 0; jj < n; ++jj) {
+                const int j = j0 + jj;  // key tile
+                if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[t], jj & 1, c.abort_flag, c.lim, 330 + t))) {
                     ok = false;
                     break;
                 }
@@ -584,8 +603,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const float rs = need_mask ? softmax_row_to_regs<BN, BF16, 0>(sr, sc, neg_m, pk)
                                            : softmax_row_to_regs<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, pk);
                 l = fmaf(l, alpha, rs);
-                if (j > 0) {
-                    if (!__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (j - 1) & 1, c.abort_flag, c.lim, 340 + t))) {
+                if (jj > 0) {
+                    if (!__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (jj - 1) & 1, c.abort_flag, c.lim, 340 + t))) {
                         ok = false;
                         break;
                     }
@@ -616,9 +635,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 mbar_arrive(&c.p_full[t]);
             }
         } else
-        for (int j = 0; j < n; ++j) {
-            const int b = c.buf(t, j);
-            if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[b], c.sphase(j), c.abort_flag, c.lim, 300 + t))) {
+        for (int jj = 0; jj < n; ++jj) {
+            const int j = j0 + jj;  // key tile
+            const int b = c.buf(t, jj);
+            if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[b], c.sphase(jj), c.abort_flag, c.lim, 300 + t))) {
                 ok = false;
                 break;
             }
@@ -652,10 +672,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                        : softmax_chunk_store<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, p_addr);
             l = fmaf(l, alpha, rs);
             tmem_st_wait();
-            if (j > 0) {
-                // PV_{j-1} is waited for on every step (it has normally finished long before),
-                // so this thread never falls two phases behind on pv_done.
-                if (!__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (j - 1) & 1, c.abort_flag, c.lim, 310 + t))) {
+            if (jj > 0) {
+                // The previous PV is waited for on every step (it has normally finished long
+                // before), so this thread never falls two phases behind on pv_done.
+                if (!__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (jj - 1) & 1, c.abort_flag, c.lim, 310 + t))) {
                     ok = false;
                     break;
                 }

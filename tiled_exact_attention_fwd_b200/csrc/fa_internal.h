@@ -22,7 +22,7 @@ struct FwdParams {
 
 // Attention forward. Dense: grid (H, ceil(ceil(S / 128) / tiles_per_cta), B), a CTA owns
 // fwd_tiles_per_cta(D) consecutive 128-row query tiles of one sequence. Packed: grid
-// (H, ceil(total / 128), 1), a CTA owns 128 consecutive packed tokens.
+// (H, ceil(total / (128 * tiles_per_cta)), 1), a CTA owns that many consecutive packed tokens.
 cudaError_t launch_fwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
                        const CUtensorMap &tv, const FwdParams &p, dim3 grid, cudaStream_t st);
 int fwd_tile_rows();

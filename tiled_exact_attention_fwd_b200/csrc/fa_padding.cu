@@ -5,7 +5,8 @@
 // the compact rows back by `indices`; section 2 shows pad as a zero fill followed by an
 // index put. Here both are pure byte movement: one warp moves one row with 16-byte
 // vectors (several loads in flight per lane), and pad writes every output row exactly
-// once (copy when some index names it, zeros otherwise) instead of a fill plus a scatter.
+// once (copy when some index names it, zeros otherwise) instead of a fill plus a scatter;
+// the index searches are done by whole warps (32 probes per dependent load).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -114,33 +115,47 @@ __global__ void __launch_bounds__(256) unpad3_kernel(const T *__restrict__ x0, c
     }
 }
 
-// Every output row t of [t0, t1) (one contiguous range per block, one warp per row):
-// copy x[r] if indices[r] == t for some r, zeros otherwise. With strictly increasing
-// indices, the r for row t lies in [r0, r0 + (t - t0)], r0 = lower_bound(indices, t0).
+// First position r in the sorted idx[0, nnz) with idx[r] >= key, found by the 32 lanes of a
+// warp together: each round probes 32 evenly spaced entries at once, so the dependent-load
+// chain is log32(nnz) long instead of log2(nnz).
+__device__ __forceinline__ int64_t warp_lower_bound(const int64_t *__restrict__ idx, int64_t nnz, int64_t key,
+                                                    int lane) {
+    int64_t lo = 0, hi = nnz;  // answer in [lo, hi]
+    while (hi - lo > 32) {
+        const int64_t step = (hi - lo + 31) / 32;
+        const int64_t p = lo + lane * step;
+        const bool less = p < hi && __ldg(idx + p) < key;
+        const int c = __popc(__ballot_sync(0xffffffffu, less));  // probes below key form a prefix
+        const int64_t new_lo = (c == 0) ? lo : lo + (c - 1) * step + 1;
+        hi = min(hi, lo + c * step);
+        lo = new_lo;
+    }
+    const int64_t p = lo + lane;
+    const bool less = p < hi && __ldg(idx + p) < key;
+    return lo + __popc(__ballot_sync(0xffffffffu, less));
+}
+
+// Output rows [t0, t0 + 16) per block (8 warps, 2 rows each): copy x[r] if indices[r] == t for
+// some r, zeros otherwise. With strictly increasing indices, the r of row t lies in
+// [r0, r0 + (t - t0)] with r0 = lower_bound(indices, t0), so one 32-wide load of
+// indices[r0 .. r0 + 31] answers every row of the block with a ballot (ROWS <= 32).
 template <typename T>
 __global__ void __launch_bounds__(256) pad_kernel(const T *__restrict__ x, const int64_t *__restrict__ idx,
                                                   int64_t nnz, int64_t total_rows, int64_t per_row,
-                                                  int64_t rows_per_block, T *__restrict__ out) {
+                                                  T *__restrict__ out) {
+    constexpr int ROWS = 16;
     const int lane = threadIdx.x & 31;
-    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * rows_per_block;
-    const int64_t t1 = min(total_rows, t0 + rows_per_block);
-    if (t0 >= t1) return;
-    int64_t lo = 0, hi = nnz;
-    while (lo < hi) {
-        const int64_t mid = (lo + hi) >> 1;
-        if (__ldg(idx + mid) < t0) lo = mid + 1; else hi = mid;
-    }
-    const int64_t r0 = lo;
-    const int64_t wpb = blockDim.x >> 5;
-    for (int64_t t = t0 + (threadIdx.x >> 5); t < t1; t += wpb) {
-        int64_t a = r0, b = min(nnz, r0 + (t - t0) + 1);
-        while (a < b) {
-            const int64_t mid = (a + b) >> 1;
-            if (__ldg(idx + mid) < t) a = mid + 1; else b = mid;
-        }
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * ROWS;
+    if (t0 >= total_rows) return;
+    const int64_t r0 = warp_lower_bound(idx, nnz, t0, lane);
+    const int64_t cand = (r0 + lane < nnz) ? __ldg(idx + r0 + lane) : -1;
+    for (int k = threadIdx.x >> 5; k < ROWS; k += blockDim.x >> 5) {
+        const int64_t t = t0 + k;
+        if (t >= total_rows) break;
+        const unsigned hit = __ballot_sync(0xffffffffu, cand == t);
         T *o = out + t * per_row;
-        if (a < nnz && __ldg(idx + a) == t)
-            warp_copy_row(x + a * per_row, o, per_row, lane);
+        if (hit)
+            warp_copy_row(x + (r0 + __ffs(hit) - 1) * per_row, o, per_row, lane);
         else
             warp_zero_row(o, per_row, lane);
     }
@@ -201,19 +216,14 @@ cudaError_t launch_unpad3(const void *const x[3], const int64_t *indices, int64_
 cudaError_t launch_pad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
                        int64_t row_bytes, void *out, cudaStream_t st) {
     if (total_rows == 0) return cudaSuccess;
-    const int64_t max_blocks = int64_t(num_sms()) * 8;
-    int64_t blocks = (total_rows + 15) / 16;
-    if (blocks > max_blocks) blocks = max_blocks;
-    const int64_t rows_per_block = (total_rows + blocks - 1) / blocks;
-    blocks = (total_rows + rows_per_block - 1) / rows_per_block;
+    const int64_t blocks = (total_rows + 15) / 16;
+    if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
     if (vec16_ok(x ? x : out, out, row_bytes))
-        pad_kernel<uint4><<<static_cast<int>(blocks), 256, 0, st>>>(static_cast<const uint4 *>(x), indices, nnz,
-                                                                    total_rows, row_bytes / 16, rows_per_block,
-                                                                    static_cast<uint4 *>(out));
+        pad_kernel<uint4><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+            static_cast<const uint4 *>(x), indices, nnz, total_rows, row_bytes / 16, static_cast<uint4 *>(out));
     else
-        pad_kernel<uint8_t><<<static_cast<int>(blocks), 256, 0, st>>>(static_cast<const uint8_t *>(x), indices,
-                                                                      nnz, total_rows, row_bytes, rows_per_block,
-                                                                      static_cast<uint8_t *>(out));
+        pad_kernel<uint8_t><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+            static_cast<const uint8_t *>(x), indices, nnz, total_rows, row_bytes, static_cast<uint8_t *>(out));
     return cudaGetLastError();
 }
 
