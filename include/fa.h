@@ -87,6 +87,25 @@ FA_API fa_status fa_varlen_fwd(const void *q, const void *k, const void *v, cons
                         int D, float scale, int causal, fa_dtype dtype, void *stream);
 
 /*
+ * The whole packed path in one launch (unpad -> packed attention -> pad): the same result as
+ * fa_unpad of q, k, v, then fa_varlen_fwd, then fa_pad of the output, without the compact
+ * copies. Page "IAW 模型 FA2 vs FA3 实测", section 6, counts the separate gathers, fill and
+ * pads as ~18 us of a 118 us call; here the attention kernel gathers its Q/K/V tiles from
+ * the padded tensors and scatters O to the padded rows itself.
+ *   q, k, v      padded (padded_rows, H, D) inputs (e.g. (B * total_len, H, D)).
+ *   indices      device int64 [total]: padded row of packed token r, strictly increasing.
+ *   cu_seqlens   device int32 [num_seqs + 1] over the packed tokens (as in fa_varlen_fwd).
+ *   out          padded (padded_rows, H, D): row indices[r] receives token r's output, every
+ *                other row is zero.
+ *   lse          (H, total) float32 in packed order, or NULL.
+ * padded_rows < 2^31; total <= padded_rows. total == 0 writes an all-zero out.
+ */
+FA_API fa_status fa_varlen_fwd_padded(const void *q, const void *k, const void *v, const int64_t *indices,
+                                      const int32_t *cu_seqlens, int num_seqs, int max_seqlen, int total,
+                                      int64_t padded_rows, void *out, float *lse, int H, int D, float scale,
+                                      int causal, fa_dtype dtype, void *stream);
+
+/*
  * Unpad (gather): out[r, :] = x[indices[r], :] for r < nnz, rows of `row_bytes` bytes.
  *   x        (total_rows, row_bytes) padded input, e.g. (B*total_len, H*D*elt).
  *   indices  device int64 [nnz], each in [0, total_rows).

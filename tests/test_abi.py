@@ -89,3 +89,13 @@ def test_pad_unpad_validation(lib):
 
 def test_selftest_rejects_bad_limit(lib):
     assert lib.fa_selftest_bounded_wait(0, None) == -2
+
+
+def test_fused_varlen_validation(lib):
+    # all padding, nothing to attend: out is zero-filled (needs a device), here only shape checks
+    assert lib.fa_varlen_fwd_padded(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 10, 5, FAKE, None, 2, 64, 0.0, 0, 1, None) == -2
+    assert lib.fa_varlen_fwd_padded(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 10, 20, None, None, 2, 64, 0.0, 0, 1, None) == -1
+    assert lib.fa_varlen_fwd_padded(FAKE, FAKE, FAKE, None, FAKE, 2, 8, 10, 20, FAKE, None, 2, 64, 0.0, 0, 1, None) == -1
+    assert lib.fa_varlen_fwd_padded(FAKE, FAKE, FAKE, FAKE + 4, FAKE, 2, 8, 10, 20, FAKE, None, 2, 64, 0.0, 0, 1, None) == -5
+    assert lib.fa_varlen_fwd_padded(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 10, 20, FAKE, None, 2, 48, 0.0, 0, 1, None) == -4
+    assert lib.fa_varlen_fwd_padded(None, None, None, None, None, 0, 0, 0, 0, None, None, 2, 64, 0.0, 0, 1, None) == 0

@@ -246,3 +246,60 @@ def test_workload_varlen_pipeline_all_rows():
     assert_lse_close(lse.cpu(), L, "varlen workload")
     p_ref = oracle.pad(ou.cpu(), case.indices, 1, case.total_len)
     assert torch.equal(op.cpu().view(torch.int16), p_ref.view(torch.int16))
+
+
+# ----------------------------------------------------------------------------- fused packed path
+def _fused_case(lengths, total_len, H, D, dtype, causal, seed):
+    case = fa_inputs.varlen_case(lengths, total_len, H, D, dtype, seed=seed)
+    dev = torch.device("cuda:0")
+    qp, kp, vp = case.q_pad.to(dev), case.k_pad.to(dev), case.v_pad.to(dev)
+    idx, cu = case.indices.to(dev), case.cu_seqlens.to(dev)
+    out = torch.full_like(qp, float("nan"))  # every element must be written
+    out, lse = fa.fa_varlen_fwd_padded(qp, kp, vp, idx, cu, max(case.max_seqlen, 1), out=out, causal=causal)
+    # the same path in three launches
+    qu, ku, vu = fa.fa_unpad_qkv(qp, kp, vp, idx)
+    ou, lu = fa.fa_varlen_fwd(qu, ku, vu, cu, max(case.max_seqlen, 1), causal=causal)
+    ref_pad = fa.fa_pad(ou, idx, 1, total_len)
+    torch.cuda.synchronize()
+    return case, out.cpu(), lse.cpu(), ref_pad.cpu(), lu.cpu()
+
+
+@pytest.mark.parametrize("D,dtype", [(128, torch.bfloat16), (64, torch.float16), (32, torch.bfloat16),
+                                     (256, torch.float16)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fused_padded_path(D, dtype, causal):
+    lengths = [1, 70, 0, 130, 255, 64, 3]
+    case, out, lse, ref_pad, ref_lse = _fused_case(lengths, 1000, 2, D, dtype, causal, seed=D)
+    # identical to unpad -> varlen forward -> pad on the GPU, bit for bit
+    assert torch.equal(out.view(torch.int16), ref_pad.view(torch.int16))
+    assert torch.equal(lse, ref_lse)
+    # and within tolerance of the oracle; padding rows exactly zero
+    O, L = oracle.attention_varlen(oracle.unpad(case.q_pad, case.indices), oracle.unpad(case.k_pad, case.indices),
+                                   oracle.unpad(case.v_pad, case.indices), case.cu_seqlens, causal=causal)
+    flat = out.view(-1, 2, D)
+    assert_o_close(flat[case.indices], O, dtype, "fused")
+    assert_lse_close(lse, L, "fused")
+    mask = torch.ones(flat.shape[0], dtype=torch.bool)
+    mask[case.indices] = False
+    assert (flat[mask].view(torch.int16) == 0).all()
+
+
+def test_fused_workload_32x64():
+    w = fa_inputs.WORKLOADS["varlen_bf16_32x64"]
+    case, out, lse, ref_pad, ref_lse = _fused_case(w["lengths"], w["total_len"], w["H"], w["D"], torch.bfloat16,
+                                                   False, seed=0)
+    assert torch.equal(out.view(torch.int16), ref_pad.view(torch.int16))
+    assert torch.equal(lse, ref_lse)
+
+
+def test_fused_edge_cases():
+    dev = torch.device("cuda:0")
+    # no valid token: all zeros
+    x = fa_inputs.normal((1, 300, 2, 64), torch.bfloat16, 1).to(dev)
+    idx = torch.zeros(0, dtype=torch.int64, device=dev)
+    cu = torch.zeros(1, dtype=torch.int32, device=dev)
+    out, _ = fa.fa_varlen_fwd_padded(x, x, x, idx, cu, 0, out=torch.full_like(x, 7.0))
+    assert float(out.abs().max()) == 0.0
+    # no padding at all: equals the plain packed call
+    case, out, lse, ref_pad, ref_lse = _fused_case([100, 156], 256, 2, 64, torch.bfloat16, True, seed=3)
+    assert torch.equal(out.view(torch.int16), ref_pad.view(torch.int16))

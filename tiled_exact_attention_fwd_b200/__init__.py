@@ -48,9 +48,12 @@ def lib() -> ctypes.CDLL:
         L.fa_unpad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fa_pad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fa_unpad_qkv.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp]
+        L.fa_varlen_fwd_padded.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i64, vp, vp, i32, i32, f32, i32, i32,
+                                           vp]
         L.fa_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.fa_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
-        for f in (L.fa_fwd, L.fa_varlen_fwd, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad, L.fa_device_status,
+        for f in (L.fa_fwd, L.fa_varlen_fwd, L.fa_varlen_fwd_padded, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad,
+                  L.fa_device_status,
                   L.fa_selftest_bounded_wait):
             f.restype = ctypes.c_int
         L.fa_status_string.argtypes = [ctypes.c_int]
@@ -138,6 +141,36 @@ def fa_varlen_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens:
                              int(max_seqlen), total, _ptr(out), _ptr(lse), H, D,
                              float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
     _check(st, "fa_varlen_fwd")
+    return out, lse
+
+
+def fa_varlen_fwd_padded(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, indices: torch.Tensor,
+                         cu_seqlens: torch.Tensor, max_seqlen: int, out: Optional[torch.Tensor] = None,
+                         lse: Optional[torch.Tensor] = None, scale: Optional[float] = None, causal: bool = False,
+                         return_lse: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Fused unpad -> packed attention -> pad: padded q, k, v (..., H, D) with the int64 padded row
+    of every packed token -> padded out (zeros at padding rows), lse (H, total)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("indices", indices), ("cu_seqlens", cu_seqlens)):
+        _cuda_contig(n, t)
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one shape and dtype")
+    if indices.dtype != torch.int64 or cu_seqlens.dtype != torch.int32:
+        raise ValueError("indices must be int64 and cu_seqlens int32")
+    H, D = q.shape[-2], q.shape[-1]
+    padded_rows = q.numel() // (H * D)
+    total = indices.numel()
+    if out is None:
+        out = torch.empty_like(q)
+    _cuda_contig("out", out)
+    if return_lse and lse is None:
+        lse = torch.empty((H, total), device=q.device, dtype=torch.float32)
+    if lse is not None:
+        _cuda_contig("lse", lse)
+    st = lib().fa_varlen_fwd_padded(_ptr(q), _ptr(k), _ptr(v), _ptr(indices), _ptr(cu_seqlens),
+                                    cu_seqlens.numel() - 1, int(max_seqlen), total, padded_rows, _ptr(out), _ptr(lse),
+                                    H, D, float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q),
+                                    _stream(stream))
+    _check(st, "fa_varlen_fwd_padded")
     return out, lse
 
 

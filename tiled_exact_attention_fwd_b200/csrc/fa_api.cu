@@ -72,13 +72,15 @@ bool encode_map(CUtensorMap *m, const void *base, bool bf16, int D, int H, int64
 
 fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
                   const int32_t *cu_seqlens, int num_seqs, int seqlen, int64_t N, int H, int D,
-                  float scale, int causal, fa_dtype dtype, void *stream) {
+                  float scale, int causal, fa_dtype dtype, void *stream,
+                  const int64_t *gather = nullptr, int64_t padded_rows = 0) {
     const bool bf16 = dtype == FA_BF16;
     const int inner = fa::fwd_box_inner_elems(D);
     CUtensorMap tq, tk, tv;
-    if (!encode_map(&tq, q, bf16, D, H, N, inner, fa::fwd_tile_rows()) ||
-        !encode_map(&tk, k, bf16, D, H, N, inner, fa::fwd_kv_tile_rows(D)) ||
-        !encode_map(&tv, v, bf16, D, H, N, inner, fa::fwd_kv_tile_rows(D)))
+    const int64_t map_rows = gather ? padded_rows : N;  // the fused path's copy threads do not use the maps
+    if (!encode_map(&tq, q, bf16, D, H, map_rows, inner, fa::fwd_tile_rows()) ||
+        !encode_map(&tk, k, bf16, D, H, map_rows, inner, fa::fwd_kv_tile_rows(D)) ||
+        !encode_map(&tv, v, bf16, D, H, map_rows, inner, fa::fwd_kv_tile_rows(D)))
         return FA_ERR_CUDA;
     if (!(scale > 0.f)) scale = 1.0f / sqrtf(static_cast<float>(D));
     fa::FwdParams p;
@@ -86,6 +88,11 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     p.lse = lse;
     p.cu_seqlens = cu_seqlens;
     p.num_seqs = num_seqs;
+    p.gather = gather;
+    p.padded_rows = padded_rows;
+    p.q = q;
+    p.k = k;
+    p.v = v;
     p.seqlen = seqlen;
     p.H = H;
     p.total_tokens = static_cast<int>(N);
@@ -140,6 +147,32 @@ fa_status fa_varlen_fwd(const void *q, const void *k, const void *v, const int32
         return FA_ERR_ALIGN;
     return run_fwd(q, k, v, out, lse, cu_seqlens, num_seqs, max_seqlen, total, H, D, scale, causal, dtype,
                    stream);
+}
+
+fa_status fa_varlen_fwd_padded(const void *q, const void *k, const void *v, const int64_t *indices,
+                               const int32_t *cu_seqlens, int num_seqs, int max_seqlen, int total,
+                               int64_t padded_rows, void *out, float *lse, int H, int D, float scale, int causal,
+                               fa_dtype dtype, void *stream) {
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (!head_dim_ok(D)) return FA_ERR_HEADDIM;
+    if (num_seqs < 0 || total < 0 || max_seqlen < 0 || H <= 0 || padded_rows < 0) return FA_ERR_SHAPE;
+    if (total > padded_rows || padded_rows > INT32_MAX) return FA_ERR_SHAPE;
+    if (padded_rows == 0) return FA_OK;
+    if (!out) return FA_ERR_NULL;
+    if (!aligned(out, 16)) return FA_ERR_ALIGN;
+    if (total == 0 || num_seqs == 0) {
+        // no valid token: the padded output is all zeros
+        const size_t bytes = static_cast<size_t>(padded_rows) * H * D * 2;
+        return cudaMemsetAsync(out, 0, bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    }
+    if (!q || !k || !v || !cu_seqlens || !indices) return FA_ERR_NULL;
+    if (max_seqlen == 0) return FA_ERR_SHAPE;
+    if ((static_cast<int64_t>(total) + 127) / 128 > 65535) return FA_ERR_SHAPE;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(lse, 4) || !aligned(cu_seqlens, 4) ||
+        !aligned(indices, 8))
+        return FA_ERR_ALIGN;
+    return run_fwd(q, k, v, out, lse, cu_seqlens, num_seqs, max_seqlen, total, H, D, scale, causal, dtype, stream,
+                   indices, padded_rows);
 }
 
 fa_status fa_unpad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows, int64_t row_bytes,

@@ -263,6 +263,7 @@ struct Cta {
     __device__ __forceinline__ bool uses(int t, int j) const { return t ? (j >= jB0 && j < nB) : (j < nA); }
     bool two;      // two query tiles (ping-pong) or one (S double-buffered)
     bool dec;      // two tiles with separate P buffers (Cfg::DECOUPLED)
+    bool fused;    // Q/K/V tiles written by threads (cp.async), not TMA: fence before the MMA reads them
     // S/P buffer and barrier phase used by tile t at key step j
     __device__ __forceinline__ int buf(int t, int j) const { return two ? t : (j & 1); }
     __device__ __forceinline__ uint32_t sphase(int j) const { return two ? (j & 1) : ((j >> 1) & 1); }
@@ -279,6 +280,7 @@ __device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first
     if (jj == 0) {
         if (!wait_bounded(&c.q_full[t], 0, c.abort_flag, c.lim, 200 + t)) return false;
         tc_fence_after_sync();
+        if (c.fused) fence_proxy_async_smem();
     } else if (c.dec) {
         // S_t is overwritten: the softmax warps must have read the previous S_t
         if (!wait_bounded(&c.s_free[t], (jj - 1) & 1, c.abort_flag, c.lim, 240 + t)) return false;
@@ -288,6 +290,7 @@ __device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first
     if (first_use) {
         if (!wait_bounded(&c.kv_full[stage], (L / NS) & 1, c.abort_flag, c.lim, 220 + stage)) return false;
         tc_fence_after_sync();
+        if (c.fused) fence_proxy_async_smem();
     }
     const uint32_t q_addr = smem_u32(c.sQ + t * C::Q_BYTES);
     const uint32_t k_addr = smem_u32(c.sKV + stage * C::KV_BYTES);
@@ -319,6 +322,7 @@ __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first
     if (first_use) {
         if (!wait_bounded(&c.kv_full[stage], (L / NS) & 1, c.abort_flag, c.lim, 230 + stage)) return false;
         tc_fence_after_sync();
+        if (c.fused) fence_proxy_async_smem();
     }
     const uint32_t v_addr = smem_u32(c.sKV + stage * C::KV_BYTES);
     const uint32_t a_tmem = c.tmem + (c.dec ? C::P_COL + 64 * t : b * BN);
@@ -382,6 +386,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     Cta<D> c;
     c.two = two;
     c.dec = C::DECOUPLED && c.two;
+    c.fused = p.gather != nullptr;
     c.nA = (kv_end_A + BN - 1) / BN;
     c.nB = c.two ? (kv_end_B + BN - 1) / BN : 0;
     c.jB0 = c.two ? kv_start_B / BN : 0;
@@ -409,15 +414,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
+        const int fill_arrivals = p.gather ? 96 : 1;  // fused: the 96 copy threads arrive
         for (int t = 0; t < 2; ++t) {
-            mbar_init(&c.q_full[t], 1);
+            mbar_init(&c.q_full[t], fill_arrivals);
             mbar_init(&c.s_full[t], 1);
             mbar_init(&c.p_full[t], 128);
             mbar_init(&c.pv_done[t], 1);
             mbar_init(&c.s_free[t], 4);  // one arrival per softmax warp
         }
         for (int s = 0; s < NS; ++s) {
-            mbar_init(&c.kv_full[s], 1);
+            mbar_init(&c.kv_full[s], fill_arrivals);
             mbar_init(&c.kv_empty[s], 1);
         }
         mbar_init(c.drain, 1);
@@ -441,21 +447,60 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (warp >= C::NUM_SOFTMAX_WARPS) {
         // producer / MMA warpgroup (its two remaining warps idle)
         if constexpr (C::SPLIT_REGS) regs_dec<C::REGS_LOW>();
-        if (warp == C::WARP_TMA) {
+        if (warp == C::WARP_TMA || (p.gather && warp > C::WARP_MMA)) {
             // ------------------------------------------------------------ TMA producer
-            if (lane == 0) {
+            // (with the fused packed path also warps 10 and 11: copy producers)
+            const int nq = c.two ? 2 : 1;
+            const int loads = 2 * n_all;  // K_0, V_0, K_1, V_1, ...
+            int issued = 0;
+            if (p.gather) {
+                // Fused packed path: warps 8, 10 and 11 (96 threads) copy every tile row from
+                // the padded tensor (row = padded row of the packed token; rows past the last
+                // token read row 0, which the masks then ignore) with 16-byte cp.async into the
+                // same swizzled layout the TMA would produce; each thread's copies arrive on the
+                // tile's barrier when they land, and the MMA thread fences the async proxy.
+                const int pt = (warp == C::WARP_TMA) ? lane : (warp - C::WARP_MMA) * 32 + lane;  // 0..95
+                constexpr int CPR = D * 2 / 16;          // 16-byte chunks per row of one head
+                constexpr int CPB = SW / 16;             // chunks per swizzle row (column block)
+                auto fill_tile = [&](uint8_t *dst, const void *src, uint64_t *bar, int tok0, int rows) {
+                    const int total_chunks = rows * CPR;
+                    const uint32_t dst_u32 = smem_u32(dst);
+#pragma unroll 4
+                    for (int ci = pt; ci < total_chunks; ci += 96) {
+                        const int r = ci / CPR, ch = ci % CPR;
+                        const int tok = tok0 + r;
+                        int64_t prow = (tok >= 0 && tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
+                        if (prow < 0 || prow >= p.padded_rows) prow = 0;  // never read outside q/k/v
+                        const int blk = ch / CPB, cc = ch % CPB;
+                        const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
+                        cp_async_16(dst_u32 + blk * rows * SW + r * SW + ((cc ^ swz) << 4),
+                                    static_cast<const uint8_t *>(src) + (prow * p.H + h) * static_cast<int64_t>(D) * 2 +
+                                        ch * 16);
+                    }
+                    cp_async_mbar_arrive(bar);  // arrives once this thread's copies have landed
+                };
+                for (int t = 0; t < nq; ++t) fill_tile(c.sQ + t * C::Q_BYTES, p.q, &c.q_full[t], qbase + t * BM, BM);
+                for (int L = 0; L < loads; ++L) {
+                    const int stage = L % NS;
+                    if (L >= NS &&
+                        !wait_bounded(&c.kv_empty[stage], ((L / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
+                        break;
+                    fill_tile(c.sKV + stage * C::KV_BYTES, (L & 1) ? p.v : p.k, &c.kv_full[stage],
+                              kvbase + (L >> 1) * BN, BN);
+                    issued = L + 1;
+                }
+                cp_async_wait_all();  // nothing of this thread is left in flight at exit
+                issued = 0;
+            } else if (lane == 0) {
                 const uint64_t pol_q = l2_policy_evict_first();
                 const uint64_t pol_kv = l2_policy_evict_last();
-                const int nq = c.two ? 2 : 1;
                 for (int t = 0; t < nq; ++t) {
                     mbar_arrive_expect_tx(&c.q_full[t], C::Q_BYTES);
-    #pragma unroll
+#pragma unroll
                     for (int b = 0; b < C::NBLK; ++b)
                         tma_load_3d(c.sQ + t * C::Q_BYTES + b * BM * SW, &tm_q, &c.q_full[t], b * C::SWE, h,
                                     qbase + t * BM, pol_q);
                 }
-                const int loads = 2 * n_all;  // K_0, V_0, K_1, V_1, ...
-                int issued = 0;
                 for (int L = 0; L < loads; ++L) {
                     const int stage = L % NS;
                     if (L >= NS &&
@@ -465,24 +510,24 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     uint8_t *dst = c.sKV + stage * C::KV_BYTES;
                     mbar_arrive_expect_tx(&c.kv_full[stage], C::KV_BYTES);
                     const CUtensorMap *map = (L & 1) ? &tm_v : &tm_k;
-    #pragma unroll
+#pragma unroll
                     for (int b = 0; b < C::NBLK; ++b)
                         tma_load_3d(dst + b * BN * SW, map, &c.kv_full[stage], b * C::SWE, h, kvbase + j * BN,
                                     pol_kv);
                     issued = L + 1;
                 }
-                if (*c.abort_flag) {
-                    // Let the copies already issued land before the CTA's shared memory goes away.
-                    for (int t = 0; t < nq; ++t) {
-                        const uint64_t t0 = global_timer_ns();
-                        while (!mbar_try_wait(&c.q_full[t], 0) && global_timer_ns() - t0 < c.lim) {
-                        }
+            }
+            if (warp == C::WARP_TMA && lane == 0 && *c.abort_flag) {
+                // Let the copies already issued land before the CTA's shared memory goes away.
+                for (int t = 0; t < nq; ++t) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(&c.q_full[t], 0) && global_timer_ns() - t0 < c.lim) {
                     }
-                    for (int L = (issued > NS ? issued - NS : 0); L < issued; ++L) {
-                        const int stage = L % NS;
-                        const uint64_t t0 = global_timer_ns();
-                        while (!mbar_try_wait(&c.kv_full[stage], (L / NS) & 1) && global_timer_ns() - t0 < c.lim) {
-                        }
+                }
+                for (int L = (issued > NS ? issued - NS : 0); L < issued; ++L) {
+                    const int stage = L % NS;
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(&c.kv_full[stage], (L / NS) & 1) && global_timer_ns() - t0 < c.lim) {
                     }
                 }
             }
@@ -708,8 +753,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (ok) {
             tc_fence_after_sync();
             const float inv_l = 1.f / l;
+            int64_t orow_idx = (p.gather && row_ok) ? __ldg(p.gather + tok) : tok;  // fused: padded row
+            const bool store_ok = row_ok && (!p.gather || (orow_idx >= 0 && orow_idx < p.padded_rows));
             uint4 *orow = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) +
-                                                    (tok * p.H + h) * static_cast<int64_t>(D) * 2);
+                                                    (orow_idx * p.H + h) * static_cast<int64_t>(D) * 2);
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t o[32];
@@ -720,7 +767,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     w[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-                if (row_ok) {
+                if (store_ok) {
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4)
                         orow[cc * 4 + v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
@@ -731,6 +778,27 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const int64_t li = packed ? static_cast<int64_t>(h) * p.total_tokens + tok
                                           : (static_cast<int64_t>(blockIdx.z) * p.H + h) * p.seqlen + (tok - seq_start);
                 p.lse[li] = lse;
+            }
+            if (p.gather) {
+                // Fused pad: this warp's 32 tokens own the padded rows from just after the
+                // previous token's row up to their last row (through the end of the tensor for
+                // the last token, from row 0 for the first); rows no token maps to become 0.
+                const int64_t tw0 = static_cast<int64_t>(qbase) + t * BM + quarter * 32;
+                if (tw0 < p.total_tokens) {
+                    const int64_t tw1 = min(tw0 + 32, static_cast<int64_t>(p.total_tokens)) - 1;
+                    const int64_t g_lane = (tw0 + lane <= tw1) ? __ldg(p.gather + tw0 + lane) : -1;
+                    const int64_t lo_row = max(int64_t(0), (tw0 == 0) ? int64_t(0) : __ldg(p.gather + tw0 - 1) + 1);
+                    const int64_t hi_row =
+                        min(p.padded_rows, (tw1 == p.total_tokens - 1) ? p.padded_rows : __ldg(p.gather + tw1));
+                    constexpr int VEC = D * 2 / 16;  // 16-byte vectors per row of one head
+                    for (int64_t pr = lo_row; pr < hi_row; ++pr) {
+                        const bool mapped = __any_sync(0xffffffffu, g_lane == pr);
+                        if (!mapped && lane < VEC)
+                            reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) +
+                                                      (pr * p.H + h) * static_cast<int64_t>(D) * 2)[lane] =
+                                make_uint4(0, 0, 0, 0);
+                    }
+                }
             }
         }
     }

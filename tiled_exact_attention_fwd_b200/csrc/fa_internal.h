@@ -13,6 +13,10 @@ struct FwdParams {
     float *lse;                 // dense: (B, H, S); packed: (H, total); may be null
     const int32_t *cu_seqlens;  // null for dense (uniform sequences of `seqlen`)
     int num_seqs;               // packed: entries of cu_seqlens minus one
+    const int64_t *gather;      // fused packed path: padded row of every packed token (else null);
+                                // q/k/v/out are then padded (padded_rows, H, D) and read by threads
+    int64_t padded_rows;
+    const void *q, *k, *v;      // the inputs (used by the fused path's copy threads)
     int seqlen;                 // dense sequence length
     int H;                      // heads
     int total_tokens;           // N = rows of the token-major tensors
