@@ -139,6 +139,41 @@ __device__ __forceinline__ int seq_of_token(const int32_t *cu, int num_seqs, int
     return lo;
 }
 
+// seq_of_token for a token shared by the whole warp: 32 probes per dependent load.
+__device__ __forceinline__ int warp_seq_of_token(const int32_t *cu, int num_seqs, int tok, int lane) {
+    int lo = 0, hi = num_seqs;  // answer s in [lo, hi - 1]: the last s with cu[s] <= tok
+    while (hi - lo > 32) {
+        const int step = (hi - lo + 31) / 32;
+        const int p = lo + lane * step;
+        const bool le = p < hi && __ldg(cu + p) <= tok;
+        const int c = __popc(__ballot_sync(0xffffffffu, le));  // probes <= tok form a prefix (c >= 1)
+        const int new_lo = lo + (c - 1) * step;
+        hi = min(hi, lo + c * step);
+        lo = new_lo;
+    }
+    const int p = lo + lane;
+    const bool le = p < hi && __ldg(cu + p) <= tok;
+    return lo + __popc(__ballot_sync(0xffffffffu, le)) - 1;
+}
+
+// Sequence of each lane's token `tok` (tokens of one warp, >= cu[s0] where s0 is the sequence
+// of the warp's first token): one 32-wide load of cu[s0 + 1 ..] and a 5-step search over the
+// lanes; falls back to the plain search when the warp's tokens span more than 32 sequences.
+__device__ __forceinline__ int lane_seq_of_token(const int32_t *cu, int num_seqs, int s0, int tok, int lane) {
+    const int wi = s0 + 1 + lane;
+    const int w = (wi <= num_seqs) ? __ldg(cu + wi) : 0x7fffffff;
+    int lo = 0, hi = 32;  // count of window entries <= tok, in [lo, hi]
+#pragma unroll
+    for (int k = 0; k < 6; ++k) {
+        const int mid = (lo + hi + 1) >> 1;
+        const int v = __shfl_sync(0xffffffffu, w, (mid - 1) & 31);
+        if (mid <= hi && lo < hi) {
+            if (v <= tok) lo = mid; else hi = mid - 1;
+        }
+    }
+    return (lo < 32) ? s0 + lo : seq_of_token(cu, num_seqs, tok);
+}
+
 // Single-tile order of MMA steps: K0, K1, V0, K2, V1, ..., V_{n-1} (QK runs one tile ahead).
 __device__ __forceinline__ void decode_step(int idx, int n, bool &is_v, int &j) {
     if (idx == 0) { is_v = false; j = 0; }
@@ -369,17 +404,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         qbase = blockIdx.y * C::MAXQ * BM;
         if (qbase >= p.total_tokens) return;
         two = (C::MAXQ == 2) && (qbase + BM < p.total_tokens);
-        const int s_first = seq_of_token(p.cu_seqlens, p.num_seqs, qbase);
+        const int ln = threadIdx.x & 31;
+        const int s_first = warp_seq_of_token(p.cu_seqlens, p.num_seqs, qbase, ln);
         kvbase = p.cu_seqlens[s_first];
         // keys of a tile end with its last row's sequence (or the causal limit)
         auto kv_end = [&](int tlast) {
-            const int s_last = seq_of_token(p.cu_seqlens, p.num_seqs, tlast);
+            const int s_last = warp_seq_of_token(p.cu_seqlens, p.num_seqs, tlast, ln);
             return (CAUSAL ? min(p.cu_seqlens[s_last + 1], tlast + 1) : p.cu_seqlens[s_last + 1]) - kvbase;
         };
         kv_end_A = kv_end(min(qbase + BM, p.total_tokens) - 1);
         if (two) {
             kv_end_B = kv_end(min(qbase + 2 * BM, p.total_tokens) - 1);
-            kv_start_B = p.cu_seqlens[seq_of_token(p.cu_seqlens, p.num_seqs, qbase + BM)] - kvbase;
+            kv_start_B = p.cu_seqlens[warp_seq_of_token(p.cu_seqlens, p.num_seqs, qbase + BM, ln)] - kvbase;
         }
     }
 
@@ -459,23 +495,29 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // token read row 0, which the masks then ignore) with 16-byte cp.async into the
                 // same swizzled layout the TMA would produce; each thread's copies arrive on the
                 // tile's barrier when they land, and the MMA thread fences the async proxy.
-                const int pt = (warp == C::WARP_TMA) ? lane : (warp - C::WARP_MMA) * 32 + lane;  // 0..95
                 constexpr int CPR = D * 2 / 16;          // 16-byte chunks per row of one head
                 constexpr int CPB = SW / 16;             // chunks per swizzle row (column block)
+                const int pw = (warp == C::WARP_TMA) ? 0 : warp - C::WARP_MMA;  // producer warp 0..2
                 auto fill_tile = [&](uint8_t *dst, const void *src, uint64_t *bar, int tok0, int rows) {
-                    const int total_chunks = rows * CPR;
                     const uint32_t dst_u32 = smem_u32(dst);
-#pragma unroll 4
-                    for (int ci = pt; ci < total_chunks; ci += 96) {
-                        const int r = ci / CPR, ch = ci % CPR;
-                        const int tok = tok0 + r;
+                    // 32-row groups round-robin over the three warps: one coalesced load of the
+                    // group's padded rows, then every lane issues CPR 16-byte copies.
+                    for (int g = pw; g * 32 < rows; g += 3) {
+                        const int tok = tok0 + g * 32 + lane;
                         int64_t prow = (tok >= 0 && tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
                         if (prow < 0 || prow >= p.padded_rows) prow = 0;  // never read outside q/k/v
-                        const int blk = ch / CPB, cc = ch % CPB;
-                        const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
-                        cp_async_16(dst_u32 + blk * rows * SW + r * SW + ((cc ^ swz) << 4),
-                                    static_cast<const uint8_t *>(src) + (prow * p.H + h) * static_cast<int64_t>(D) * 2 +
-                                        ch * 16);
+#pragma unroll 4
+                        for (int i = 0; i < CPR; ++i) {
+                            const int idx = i * 32 + lane;
+                            const int rr = idx / CPR, ch = idx % CPR;
+                            const int64_t pr = __shfl_sync(0xffffffffu, prow, rr);
+                            const int r = g * 32 + rr;
+                            const int blk = ch / CPB, cc = ch % CPB;
+                            const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
+                            cp_async_16(dst_u32 + blk * rows * SW + r * SW + ((cc ^ swz) << 4),
+                                        static_cast<const uint8_t *>(src) + (pr * p.H + h) * static_cast<int64_t>(D) * 2 +
+                                            ch * 16);
+                        }
                     }
                     cp_async_mbar_arrive(bar);  // arrives once this thread's copies have landed
                 };
@@ -597,8 +639,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             khi = CAUSAL ? min(seqlen, row_pos + 1) : seqlen;
         } else {
             row_ok = tok < p.total_tokens;
+            const int tw0 = qbase + t * BM + quarter * 32;  // this warp's first token
+            int s_lane = 0;
+            if (tw0 < p.total_tokens) {  // warp-uniform
+                const int s_w = warp_seq_of_token(p.cu_seqlens, p.num_seqs, tw0, lane);
+                s_lane = lane_seq_of_token(p.cu_seqlens, p.num_seqs, s_w,
+                                           static_cast<int>(min(tok, static_cast<int64_t>(p.total_tokens - 1))), lane);
+            }
             if (row_ok) {
-                const int s_r = seq_of_token(p.cu_seqlens, p.num_seqs, static_cast<int>(tok));
+                const int s_r = s_lane;
                 klo = p.cu_seqlens[s_r] - kvbase;
                 khi = (CAUSAL ? min(p.cu_seqlens[s_r + 1], static_cast<int>(tok) + 1) : p.cu_seqlens[s_r + 1]) - kvbase;
             }
@@ -786,17 +835,28 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const int64_t tw0 = static_cast<int64_t>(qbase) + t * BM + quarter * 32;
                 if (tw0 < p.total_tokens) {
                     const int64_t tw1 = min(tw0 + 32, static_cast<int64_t>(p.total_tokens)) - 1;
-                    const int64_t g_lane = (tw0 + lane <= tw1) ? __ldg(p.gather + tw0 + lane) : -1;
+                    // padded rows of this warp's tokens, sorted (lanes past the last token: +inf)
+                    const int64_t g_lane = (tw0 + lane <= tw1) ? __ldg(p.gather + tw0 + lane) : INT64_MAX;
                     const int64_t lo_row = max(int64_t(0), (tw0 == 0) ? int64_t(0) : __ldg(p.gather + tw0 - 1) + 1);
                     const int64_t hi_row =
                         min(p.padded_rows, (tw1 == p.total_tokens - 1) ? p.padded_rows : __ldg(p.gather + tw1));
                     constexpr int VEC = D * 2 / 16;  // 16-byte vectors per row of one head
-                    for (int64_t pr = lo_row; pr < hi_row; ++pr) {
-                        const bool mapped = __any_sync(0xffffffffu, g_lane == pr);
-                        if (!mapped && lane < VEC)
-                            reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) +
-                                                      (pr * p.H + h) * static_cast<int64_t>(D) * 2)[lane] =
-                                make_uint4(0, 0, 0, 0);
+                    for (int64_t base = lo_row; base < hi_row; base += 32) {
+                        const int64_t pr = base + lane;
+                        // is pr one of the 32 mapped rows? binary search over the lanes' sorted values
+                        int lo = 0;
+#pragma unroll
+                        for (int step = 16; step >= 1; step >>= 1) {
+                            const int64_t v = __shfl_sync(0xffffffffu, g_lane, lo + step - 1);
+                            if (v < pr) lo += step;
+                        }
+                        const bool mapped = __shfl_sync(0xffffffffu, g_lane, lo & 31) == pr;
+                        if (pr < hi_row && !mapped) {
+                            uint4 *row = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) +
+                                                                   (pr * p.H + h) * static_cast<int64_t>(D) * 2);
+#pragma unroll
+                            for (int v4 = 0; v4 < VEC; ++v4) row[v4] = make_uint4(0, 0, 0, 0);
+                        }
                     }
                 }
             }
