@@ -80,7 +80,7 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     const int64_t map_rows = gather ? padded_rows : N;  // the fused path's copy threads do not use the maps
     if (!encode_map(&tq, q, bf16, D, H, map_rows, inner, fa::fwd_tile_rows()) ||
         !encode_map(&tk, k, bf16, D, H, map_rows, inner, fa::fwd_kv_tile_rows(D)) ||
-        !encode_map(&tv, v, bf16, D, H, map_rows, inner, fa::fwd_kv_tile_rows(D)))
+        !encode_map(&tv, v, bf16, D, H, map_rows, inner, fa::fwd_v_box_rows(D)))
         return FA_ERR_CUDA;
     if (!(scale > 0.f)) scale = 1.0f / sqrtf(static_cast<float>(D));
     fa::FwdParams p;

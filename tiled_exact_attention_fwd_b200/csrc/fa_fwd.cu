@@ -40,6 +40,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "fa.h"
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
@@ -75,13 +77,20 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
 template <int D>
 struct Cfg {
     static constexpr int BM = 128;                           // query rows per tile (MMA M)
-    static constexpr int BN = (D == 256) ? 64 : 128;         // key rows per tile
+    static constexpr int BN = 128;                           // key rows per tile
     static constexpr int MAXQ = (D == 256) ? 1 : 2;          // query tiles per CTA
     static constexpr int SW = (2 * D >= 128) ? 128 : 2 * D;  // swizzle span in bytes
     static constexpr int SWE = SW / 2;                       // 16-bit elements per swizzle row
     static constexpr int NBLK = D / SWE;                     // column blocks per tile row
     static constexpr int Q_BYTES = BM * D * 2;
     static constexpr int KV_BYTES = BN * D * 2;
+    // The K/V ring moves tiles in UNITS parts (D = 256: 64 KB tiles in two 32 KB parts, so
+    // the ring keeps 5 stages): part u of K_j holds column blocks [u*NBLK/UNITS, ...) of all
+    // rows, part u of V_j rows [u*BN/UNITS, ...) of all column blocks.
+    static constexpr int UNITS = (D == 256) ? 2 : 1;
+    static constexpr int UNIT_BYTES = KV_BYTES / UNITS;
+    static constexpr int KBLK_PER_UNIT = NBLK / UNITS;   // K column blocks per part
+    static constexpr int VROWS_PER_UNIT = BN / UNITS;    // V rows per part
     static constexpr uint32_t LAYOUT = (SW == 128) ? kLayoutSw128 : kLayoutSw64;
     static constexpr uint32_t TMEM_COLS = 512;
     // TMEM columns: S0 at 0, S1 at BN. With D <= 64 two separate P buffers fit (P_COL + 64t)
@@ -108,11 +117,11 @@ struct Cfg {
     // shared memory map (offsets from a 1024-byte aligned base)
     static constexpr int SMEM_LIMIT = 227 * 1024;
     static constexpr int RESERVED = 1024 /*alignment*/ + 512 /*barriers, misc*/;
-    static constexpr int NS_FIT = (SMEM_LIMIT - RESERVED - MAXQ * Q_BYTES) / KV_BYTES;
+    static constexpr int NS_FIT = (SMEM_LIMIT - RESERVED - MAXQ * Q_BYTES) / UNIT_BYTES;
     static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = MAXQ * Q_BYTES;
-    static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_KV + NS * UNIT_BYTES;
     // q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], drain, s_free[2]
     static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -125,7 +134,9 @@ struct Cfg {
     static_assert(O_COL + MAXQ * D <= TMEM_COLS, "TMEM budget");
     static_assert(USED + 1024 <= SMEM_LIMIT, "shared memory budget");
     static_assert(NUM_BARS * 8 + 16 <= 512, "barrier area");
-    static_assert(Q_BYTES % 1024 == 0 && KV_BYTES % 1024 == 0, "tile alignment");
+    static_assert(Q_BYTES % 1024 == 0 && UNIT_BYTES % 1024 == 0, "tile alignment");
+    // The MMA thread waits for K_{j+1} while V_j is still held: the ring needs both, plus a part.
+    static_assert(NS >= 2 * UNITS + 1, "K/V ring too shallow");
 };
 
 // Sequence that packed token `tok` belongs to: the s with cu[s] <= tok < cu[s+1]
@@ -321,25 +332,35 @@ __device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first
         if (!wait_bounded(&c.s_free[t], (jj - 1) & 1, c.abort_flag, c.lim, 240 + t)) return false;
         tc_fence_after_sync();
     }
-    const int L = 2 * j, stage = L % NS;
-    if (first_use) {
-        if (!wait_bounded(&c.kv_full[stage], (L / NS) & 1, c.abort_flag, c.lim, 220 + stage)) return false;
-        tc_fence_after_sync();
-        if (c.fused) fence_proxy_async_smem();
-    }
+    constexpr int UK = D / 16 / C::UNITS;  // k-steps per K part
     const uint32_t q_addr = smem_u32(c.sQ + t * C::Q_BYTES);
-    const uint32_t k_addr = smem_u32(c.sKV + stage * C::KV_BYTES);
     const int b = c.buf(t, jj);
     const uint32_t d_tmem = c.tmem + b * BN;
 #pragma unroll
-    for (int k = 0; k < D / 16; ++k) {
-        const uint32_t blk = (k * 32) / SW, off = (k * 32) % SW;
-        const uint64_t a = smem_desc(q_addr + blk * BM * SW + off, 16, 8 * SW, C::LAYOUT);
-        const uint64_t bd = smem_desc(k_addr + blk * BN * SW + off, 16, 8 * SW, C::LAYOUT);
-        umma_ss(d_tmem, a, bd, idesc, k > 0 ? 1u : 0u);
+    for (int u = 0; u < C::UNITS; ++u) {
+        const int U = 2 * j * C::UNITS + u, stage = U % NS;  // ring part holding K_j part u
+        if (first_use) {
+            if (!wait_bounded(&c.kv_full[stage], (U / NS) & 1, c.abort_flag, c.lim, 220 + stage)) return false;
+            tc_fence_after_sync();
+            if (c.fused) fence_proxy_async_smem();
+        }
+        const uint32_t k_addr = smem_u32(c.sKV + stage * C::UNIT_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < UK; ++kk) {
+            const int k = u * UK + kk;
+            const uint32_t blk = (k * 32) / SW, off = (k * 32) % SW;
+            const uint32_t lb = blk - u * C::KBLK_PER_UNIT;  // column block inside the part
+            const uint64_t a = smem_desc(q_addr + blk * BM * SW + off, 16, 8 * SW, C::LAYOUT);
+            const uint64_t bd = smem_desc(k_addr + lb * BN * SW + off, 16, 8 * SW, C::LAYOUT);
+            umma_ss(d_tmem, a, bd, idesc, k > 0 ? 1u : 0u);
+        }
+        if (u + 1 < C::UNITS) {
+            if (last_use) umma_commit(&c.kv_empty[stage]);  // release this part early
+        } else {
+            umma_commit(&c.s_full[b]);  // the softmax waits on S first
+            if (last_use) umma_commit(&c.kv_empty[stage]);
+        }
     }
-    umma_commit(&c.s_full[b]);
-    if (last_use) umma_commit(&c.kv_empty[stage]);
     return true;
 }
 
@@ -353,22 +374,31 @@ __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first
     const int b = c.buf(t, jj);
     if (!wait_bounded(&c.p_full[b], c.sphase(jj), c.abort_flag, c.lim, 210 + t)) return false;
     tc_fence_after_sync();
-    const int L = 2 * j + 1, stage = L % NS;
-    if (first_use) {
-        if (!wait_bounded(&c.kv_full[stage], (L / NS) & 1, c.abort_flag, c.lim, 230 + stage)) return false;
-        tc_fence_after_sync();
-        if (c.fused) fence_proxy_async_smem();
-    }
-    const uint32_t v_addr = smem_u32(c.sKV + stage * C::KV_BYTES);
+    constexpr int UV = BN / 16 / C::UNITS;  // k-steps per V part
     const uint32_t a_tmem = c.tmem + (c.dec ? C::P_COL + 64 * t : b * BN);
     const uint32_t o_tmem = c.tmem + C::O_COL + t * D;
 #pragma unroll
-    for (int k = 0; k < BN / 16; ++k) {
-        const uint64_t bd = smem_desc(v_addr + k * 16 * SW, BN * SW, 8 * SW, C::LAYOUT);
-        umma_ts(o_tmem, a_tmem + k * 8, bd, idesc, (jj > 0 || k > 0) ? 1u : 0u);
+    for (int u = 0; u < C::UNITS; ++u) {
+        const int U = (2 * j + 1) * C::UNITS + u, stage = U % NS;  // ring part holding V_j part u
+        if (first_use) {
+            if (!wait_bounded(&c.kv_full[stage], (U / NS) & 1, c.abort_flag, c.lim, 230 + stage)) return false;
+            tc_fence_after_sync();
+            if (c.fused) fence_proxy_async_smem();
+        }
+        const uint32_t v_addr = smem_u32(c.sKV + stage * C::UNIT_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < UV; ++kk) {
+            const int k = u * UV + kk;
+            const uint64_t bd = smem_desc(v_addr + kk * 16 * SW, C::VROWS_PER_UNIT * SW, 8 * SW, C::LAYOUT);
+            umma_ts(o_tmem, a_tmem + k * 8, bd, idesc, (jj > 0 || k > 0) ? 1u : 0u);
+        }
+        if (u + 1 < C::UNITS) {
+            if (last_use) umma_commit(&c.kv_empty[stage]);
+        } else {
+            umma_commit(&c.pv_done[t]);
+            if (last_use) umma_commit(&c.kv_empty[stage]);
+        }
     }
-    umma_commit(&c.pv_done[t]);
-    if (last_use) umma_commit(&c.kv_empty[stage]);
     return true;
 }
 
@@ -487,7 +517,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // ------------------------------------------------------------ TMA producer
             // (with the fused packed path also warps 10 and 11: copy producers)
             const int nq = c.two ? 2 : 1;
-            const int loads = 2 * n_all;  // K_0, V_0, K_1, V_1, ...
+            const int loads = 2 * n_all * C::UNITS;  // parts of K_0, V_0, K_1, V_1, ...
             int issued = 0;
             if (p.gather) {
                 // Fused packed path: warps 8, 10 and 11 (96 threads) copy every tile row from
@@ -495,10 +525,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // token read row 0, which the masks then ignore) with 16-byte cp.async into the
                 // same swizzled layout the TMA would produce; each thread's copies arrive on the
                 // tile's barrier when they land, and the MMA thread fences the async proxy.
-                constexpr int CPR = D * 2 / 16;          // 16-byte chunks per row of one head
-                constexpr int CPB = SW / 16;             // chunks per swizzle row (column block)
+                constexpr int CPB = SW / 16;  // 16-byte chunks per swizzle row (column block)
                 const int pw = (warp == C::WARP_TMA) ? 0 : warp - C::WARP_MMA;  // producer warp 0..2
-                auto fill_tile = [&](uint8_t *dst, const void *src, uint64_t *bar, int tok0, int rows) {
+                // Copies rows [tok0, tok0 + rows) x column blocks [b0, b0 + NB) into dst laid out
+                // as [NB][rows][SW].
+                auto fill = [&](auto nb_c, uint8_t *dst, const void *src, uint64_t *bar, int tok0, int rows,
+                                int b0) {
+                    constexpr int CPR = decltype(nb_c)::value * CPB;  // chunks per row
                     const uint32_t dst_u32 = smem_u32(dst);
                     // 32-row groups round-robin over the three warps: one coalesced load of the
                     // group's padded rows, then every lane issues CPR 16-byte copies.
@@ -506,6 +539,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         const int tok = tok0 + g * 32 + lane;
                         int64_t prow = (tok >= 0 && tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
                         if (prow < 0 || prow >= p.padded_rows) prow = 0;  // never read outside q/k/v
+                        const uint8_t *srow = static_cast<const uint8_t *>(src) + b0 * SW;
 #pragma unroll 4
                         for (int i = 0; i < CPR; ++i) {
                             const int idx = i * 32 + lane;
@@ -515,21 +549,28 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             const int blk = ch / CPB, cc = ch % CPB;
                             const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
                             cp_async_16(dst_u32 + blk * rows * SW + r * SW + ((cc ^ swz) << 4),
-                                        static_cast<const uint8_t *>(src) + (pr * p.H + h) * static_cast<int64_t>(D) * 2 +
-                                            ch * 16);
+                                        srow + (pr * p.H + h) * static_cast<int64_t>(D) * 2 + ch * 16);
                         }
                     }
                     cp_async_mbar_arrive(bar);  // arrives once this thread's copies have landed
                 };
-                for (int t = 0; t < nq; ++t) fill_tile(c.sQ + t * C::Q_BYTES, p.q, &c.q_full[t], qbase + t * BM, BM);
-                for (int L = 0; L < loads; ++L) {
-                    const int stage = L % NS;
-                    if (L >= NS &&
-                        !wait_bounded(&c.kv_empty[stage], ((L / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
+                using AllBlk = std::integral_constant<int, C::NBLK>;
+                using KBlk = std::integral_constant<int, C::KBLK_PER_UNIT>;
+                for (int t = 0; t < nq; ++t)
+                    fill(AllBlk{}, c.sQ + t * C::Q_BYTES, p.q, &c.q_full[t], qbase + t * BM, BM, 0);
+                for (int U = 0; U < loads; ++U) {
+                    const int stage = U % NS;
+                    if (U >= NS &&
+                        !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
                         break;
-                    fill_tile(c.sKV + stage * C::KV_BYTES, (L & 1) ? p.v : p.k, &c.kv_full[stage],
-                              kvbase + (L >> 1) * BN, BN);
-                    issued = L + 1;
+                    const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
+                    uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
+                    if (L & 1)
+                        fill(AllBlk{}, dst, p.v, &c.kv_full[stage], kvbase + j * BN + u * C::VROWS_PER_UNIT,
+                             C::VROWS_PER_UNIT, 0);
+                    else
+                        fill(KBlk{}, dst, p.k, &c.kv_full[stage], kvbase + j * BN, BN, u * C::KBLK_PER_UNIT);
+                    issued = U + 1;
                 }
                 cp_async_wait_all();  // nothing of this thread is left in flight at exit
                 issued = 0;
@@ -543,20 +584,28 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         tma_load_3d(c.sQ + t * C::Q_BYTES + b * BM * SW, &tm_q, &c.q_full[t], b * C::SWE, h,
                                     qbase + t * BM, pol_q);
                 }
-                for (int L = 0; L < loads; ++L) {
-                    const int stage = L % NS;
-                    if (L >= NS &&
-                        !wait_bounded(&c.kv_empty[stage], ((L / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
+                for (int U = 0; U < loads; ++U) {
+                    const int stage = U % NS;
+                    if (U >= NS &&
+                        !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
                         break;
-                    const int j = L >> 1;
-                    uint8_t *dst = c.sKV + stage * C::KV_BYTES;
-                    mbar_arrive_expect_tx(&c.kv_full[stage], C::KV_BYTES);
-                    const CUtensorMap *map = (L & 1) ? &tm_v : &tm_k;
+                    const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
+                    uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
+                    mbar_arrive_expect_tx(&c.kv_full[stage], C::UNIT_BYTES);
+                    if (L & 1) {
+                        // V part u: rows [u*VROWS_PER_UNIT, ...) of the tile, every column block
 #pragma unroll
-                    for (int b = 0; b < C::NBLK; ++b)
-                        tma_load_3d(dst + b * BN * SW, map, &c.kv_full[stage], b * C::SWE, h, kvbase + j * BN,
-                                    pol_kv);
-                    issued = L + 1;
+                        for (int b = 0; b < C::NBLK; ++b)
+                            tma_load_3d(dst + b * C::VROWS_PER_UNIT * SW, &tm_v, &c.kv_full[stage], b * C::SWE, h,
+                                        kvbase + j * BN + u * C::VROWS_PER_UNIT, pol_kv);
+                    } else {
+                        // K part u: column blocks [u*KBLK_PER_UNIT, ...) of every tile row
+#pragma unroll
+                        for (int b = 0; b < C::KBLK_PER_UNIT; ++b)
+                            tma_load_3d(dst + b * BN * SW, &tm_k, &c.kv_full[stage],
+                                        (u * C::KBLK_PER_UNIT + b) * C::SWE, h, kvbase + j * BN, pol_kv);
+                    }
+                    issued = U + 1;
                 }
             }
             if (warp == C::WARP_TMA && lane == 0 && *c.abort_flag) {
@@ -566,10 +615,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     while (!mbar_try_wait(&c.q_full[t], 0) && global_timer_ns() - t0 < c.lim) {
                     }
                 }
-                for (int L = (issued > NS ? issued - NS : 0); L < issued; ++L) {
-                    const int stage = L % NS;
+                for (int U = (issued > NS ? issued - NS : 0); U < issued; ++U) {
+                    const int stage = U % NS;
                     const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(&c.kv_full[stage], (L / NS) & 1) && global_timer_ns() - t0 < c.lim) {
+                    while (!mbar_try_wait(&c.kv_full[stage], (U / NS) & 1) && global_timer_ns() - t0 < c.lim) {
                     }
                 }
             }
@@ -944,7 +993,8 @@ int fwd_tiles_per_cta(int D) { return (D == 256) ? 1 : 2; }
 
 int fwd_box_inner_elems(int D) { return (2 * D >= 128) ? 64 : D; }
 
-int fwd_kv_tile_rows(int D) { return (D == 256) ? 64 : 128; }
+int fwd_kv_tile_rows(int D) { return 128; }
+int fwd_v_box_rows(int D) { return (D == 256) ? 64 : 128; }
 
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t st) {
     fa_selftest_wait_kernel<<<1, 32, 0, st>>>(limit_ns);

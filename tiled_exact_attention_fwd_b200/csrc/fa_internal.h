@@ -33,6 +33,8 @@ int fwd_tile_rows();
 int fwd_tiles_per_cta(int D);
 int fwd_box_inner_elems(int D);
 int fwd_kv_tile_rows(int D);
+// Rows of one V box the producer copies (a V tile may move as several row parts).
+int fwd_v_box_rows(int D);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t st);
 cudaError_t fwd_take_device_error(int *code, int *where);
 
