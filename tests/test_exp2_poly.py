@@ -15,7 +15,7 @@ SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
 
 def _coeffs():
     text = open(SRC).read()
-    body = text[text.index("float exp2_poly(float x)"):]
+    body = text[text.index("void exp2_poly2("):]
     body = body[:body.index("}")]
     nums = [float(x) for x in re.findall(r"([0-9]\.[0-9]+e[-+][0-9]+)f", body)]
     c3, c2, c1, c0 = nums[:4]

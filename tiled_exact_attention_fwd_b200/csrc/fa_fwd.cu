@@ -198,21 +198,29 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return BF16 ? pack2_bf16(lo, hi) : pack2_f16(lo, hi);
 }
 
-// 2^x evaluated on the FMA pipe instead of the MUFU unit. Cody-Waite style reduction
-// x = n + f with n = round(x) taken from the 1.5*2^23 shifter and f in [-1/2, 1/2]; 2^f by
-// a degree-3 polynomial fitted with the Remez algorithm for minimax relative error
-// (7.5e-5, below the 2^-11 rounding of the 16-bit P it feeds; gen_exp2_poly.py); 2^n is
-// added to the exponent field. Inputs below -126 are clamped (the result is then ~1e-38
+// 2^x for a pair of scores, evaluated on the FMA pipe instead of the MUFU unit. Cody-Waite
+// style reduction x = n + f with n = round(x) taken from the 1.5*2^23 shifter and f in
+// [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted with the Remez algorithm for minimax
+// relative error (7.5e-5, below the 2^-11 rounding of the 16-bit P it feeds;
+// gen_exp2_poly.py); 2^n is added to the exponent field. The float arithmetic runs two
+// lanes at a time (add/fma .f32x2). Inputs below -126 are clamped (the result is then ~1e-38
 // instead of a smaller number, irrelevant next to the row sum, which is at least 1); it is
 // only used on tiles without masked (-inf) scores.
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -126.0f);
-    const float t = x + 12582912.0f;
-    const float n = t - 12582912.0f;
-    const float f = x - n;
-    const float p = fmaf(fmaf(fmaf(5.517166853e-02f, f, 2.426111251e-01f), f, 6.932609677e-01f), f,
-                         9.999280572e-01f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float &y1) {
+    constexpr float c3 = 5.517166853e-02f, c2 = 2.426111251e-01f, c1 = 6.932609677e-01f, c0 = 9.999280572e-01f;
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    const uint64_t x2 = f2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+    const uint64_t t2 = fadd2(x2, f2(kShift, kShift));
+    const uint64_t n2 = fadd2(t2, f2(-kShift, -kShift));
+    const uint64_t r2 = ffma2(n2, f2(-1.0f, -1.0f), x2);  // x - n, exact
+    uint64_t p2 = ffma2(f2(c3, c3), r2, f2(c2, c2));
+    p2 = ffma2(p2, r2, f2(c1, c1));
+    p2 = ffma2(p2, r2, f2(c0, c0));
+    float t0, t1, p0, p1;
+    f2_split(t2, t0, t1);
+    f2_split(p2, p0, p1);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 // Maximum of an S row held in registers: 8 independent chains of three-input maxima.
@@ -247,8 +255,7 @@ __device__ __forceinline__ float softmax_chunk_store(const uint32_t *sr, float c
             f2_split(x2, x0, x1);
             float p0, p1;
             if ((i & 3) >= 4 - EMU) {
-                p0 = exp2_poly(x0);
-                p1 = exp2_poly(x1);
+                exp2_poly2(x0, x1, p0, p1);
             } else {
                 p0 = ex2_approx(x0);
                 p1 = ex2_approx(x1);
@@ -277,8 +284,7 @@ __device__ __forceinline__ float softmax_row_to_regs(const uint32_t *sr, float c
         f2_split(x2, x0, x1);
         float p0, p1;
         if ((i & 3) >= 4 - EMU) {
-            p0 = exp2_poly(x0);
-            p1 = exp2_poly(x1);
+            exp2_poly2(x0, x1, p0, p1);
         } else {
             p0 = ex2_approx(x0);
             p1 = ex2_approx(x1);
