@@ -130,6 +130,32 @@ WORKLOADS = {
 }
 
 
+def paged_kv(k: torch.Tensor, v: torch.Tensor, page_size: int, seed: int, spare_pages: int = 3,
+             extra_table_cols: int = 1, fill: float = float("nan")):
+    """Scatter contiguous (B, S, H, D) k and v into page pools of ``page_size`` rows.
+
+    Pages are assigned in a seeded random order; ``spare_pages`` pages belong to no sequence.
+    Rows of the pools that hold no key (spare pages, the tail of each sequence's last page)
+    are set to ``fill``. The int32 block table has ``extra_table_cols`` more columns than a
+    sequence needs, set to -1 (never read). Returns (k_cache, v_cache, block_table).
+    """
+    B, S, H, D = k.shape
+    per_seq = (S + page_size - 1) // page_size
+    num_pages = B * per_seq + spare_pages
+    order = torch.randperm(num_pages, generator=generator(seed))
+    table = torch.full((B, per_seq + extra_table_cols), -1, dtype=torch.int32)
+    table[:, :per_seq] = order[:B * per_seq].reshape(B, per_seq).to(torch.int32)
+    k_cache = torch.full((num_pages, page_size, H, D), fill, dtype=k.dtype)
+    v_cache = torch.full((num_pages, page_size, H, D), fill, dtype=v.dtype)
+    for b in range(B):
+        for lp in range(per_seq):
+            n = min(page_size, S - lp * page_size)
+            pg = int(table[b, lp])
+            k_cache[pg, :n] = k[b, lp * page_size:lp * page_size + n]
+            v_cache[pg, :n] = v[b, lp * page_size:lp * page_size + n]
+    return k_cache, v_cache, table
+
+
 def workload_inputs(name: str, seed: int = 0):
     """CPU inputs of a named workload (dense: (q, k, v); varlen: VarlenCase)."""
     w = WORKLOADS[name]

@@ -70,6 +70,31 @@ FA_API fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, 
                  void *stream);
 
 /*
+ * Dense attention forward with K and V in a paged pool (the PagedAttention layout that page
+ * hwcomputing.csdn.net "FlashAttention 的加速玄学", section 5, recommends for long contexts;
+ * the page gives no layout, so this one is the common block-table form). Same result as
+ * fa_fwd on the contiguous K/V that the block table describes.
+ *   q            (B, S, H, D) queries, element type `dtype`.
+ *   k_cache,
+ *   v_cache      pools (num_pages, page_size, H, D): page n holds page_size consecutive token
+ *                rows of some sequence.
+ *   block_table  device int32 (B, max_blocks_per_seq): key position pos of batch entry b is
+ *                row pos % page_size of page block_table[b * max_blocks_per_seq + pos / page_size].
+ *                Entries past ceil(S / page_size) are never read. An entry outside
+ *                [0, num_pages) is not dereferenced: page 0 is read instead (that output is
+ *                wrong) and FA_ERR_INDEX is left for fa_device_status.
+ *   page_size    a power of two, 16 <= page_size <= 2^20; max_blocks_per_seq * page_size >= S;
+ *                num_pages * page_size < 2^31.
+ *   out, lse     as fa_fwd: (B, S, H, D) and (B, H, S) float32 or NULL.
+ * Queries and keys have the same length S per batch entry (causal masks key j > query i).
+ * The caller owns every buffer; nothing is allocated; asynchronous on `stream`.
+ */
+FA_API fa_status fa_fwd_paged(const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *block_table, int max_blocks_per_seq, int page_size,
+                              int num_pages, void *out, float *lse, int B, int H, int S, int D,
+                              float scale, int causal, fa_dtype dtype, void *stream);
+
+/*
  * Packed variable-length attention forward (the flash_attn_varlen_func step).
  *   q, k, v      (total, H, D) packed inputs; sequence s owns rows
  *                [cu_seqlens[s], cu_seqlens[s+1]) and attends only inside itself.

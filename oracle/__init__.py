@@ -147,6 +147,35 @@ def attention_dense(q, k, v, scale: Optional[float] = None, causal: bool = False
     return O, L
 
 
+def paged_to_contiguous(cache: torch.Tensor, block_table, S: int) -> torch.Tensor:
+    """Key positions 0..S-1 of every batch entry read out of a page pool: (B, S, H, D).
+
+    Page hwcomputing.csdn.net "FlashAttention 的加速玄学", section 5, recommends PagedAttention
+    without giving a layout; the block-table reading is: position pos of entry b is row
+    pos % page_size of page block_table[b][pos // page_size] of the (num_pages, page_size,
+    H, D) pool. A plain copy, page by page.
+    """
+    bt = _i64(block_table)
+    B = bt.shape[0]
+    page_size = cache.shape[1]
+    out = torch.empty((B, S) + tuple(cache.shape[2:]), dtype=cache.dtype)
+    for b in range(B):
+        for lp in range((S + page_size - 1) // page_size):
+            n = min(page_size, S - lp * page_size)
+            out[b, lp * page_size:lp * page_size + n] = cache[int(bt[b, lp]), :n]
+    return out
+
+
+def attention_paged(q, k_cache, v_cache, block_table, scale: Optional[float] = None, causal: bool = False,
+                    rows=None, nthreads: int = 0):
+    """Dense attention of q (B, S, H, D) over K/V held in page pools: the dense definition
+    applied to the keys and values the block table describes (``paged_to_contiguous``)."""
+    S = q.shape[1]
+    k = paged_to_contiguous(k_cache, block_table, S)
+    v = paged_to_contiguous(v_cache, block_table, S)
+    return attention_dense(q, k, v, scale=scale, causal=causal, rows=rows, nthreads=nthreads)
+
+
 def varlen_row_spec(cu_seqlens, H: int, rows=None):
     """(tok, head, lo, hi) for packed rows; rows None = all, else an (n, 2) array of (token, head)."""
     cu = _i64(cu_seqlens)

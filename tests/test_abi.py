@@ -99,3 +99,30 @@ def test_fused_varlen_validation(lib):
     assert lib.fa_varlen_fwd_padded(FAKE, FAKE, FAKE, FAKE + 4, FAKE, 2, 8, 10, 20, FAKE, None, 2, 64, 0.0, 0, 1, None) == -5
     assert lib.fa_varlen_fwd_padded(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 10, 20, FAKE, None, 2, 48, 0.0, 0, 1, None) == -4
     assert lib.fa_varlen_fwd_padded(None, None, None, None, None, 0, 0, 0, 0, None, None, 2, 64, 0.0, 0, 1, None) == 0
+
+
+def test_paged_validation(lib):
+    f = lib.fa_fwd_paged
+    # q, k_cache, v_cache, table, max_blocks, page_size, num_pages, out, lse, B, H, S, D, scale, causal, dtype
+    ok = [FAKE, FAKE, FAKE, FAKE, 3, 64, 10, FAKE, None, 2, 4, 130, 128, 0.0, 0, 1, None]
+
+    def call(**kw):
+        a = list(ok)
+        names = ["q", "k", "v", "table", "max_blocks", "page", "pages", "out", "lse", "B", "H", "S", "D",
+                 "scale", "causal", "dtype", "stream"]
+        for n, val in kw.items():
+            a[names.index(n)] = val
+        return f(*a)
+
+    assert call(table=None) == -1
+    assert call(out=None) == -1
+    assert call(D=96) == -4
+    assert call(dtype=5) == -3
+    for bad_page in (0, 8, 24, 48, 96, 200, 384):
+        assert call(page=bad_page) == -2, bad_page
+    assert call(max_blocks=2) == -2          # 2 * 64 < 130 keys
+    assert call(pages=0) == -2
+    assert call(pages=1 << 26, page=64) == -2  # pool rows past 2^31
+    assert call(table=FAKE + 2) == -5
+    assert call(q=FAKE + 8) == -5
+    assert call(B=0) == -2

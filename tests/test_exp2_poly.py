@@ -10,7 +10,7 @@ import re
 import numpy as np
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
-                   "tiled_exact_attention_fwd_b200", "csrc", "fa_fwd.cu")
+                   "tiled_exact_attention_fwd_b200", "csrc", "fa_fwd_kernel.cuh")
 
 
 def _coeffs():

@@ -6,6 +6,7 @@ built, every call raises.
 
     out, lse = fa_fwd(q, k, v, causal=True)                         # dense (B, S, H, D)
     out, lse = fa_varlen_fwd(q, k, v, cu_seqlens, max_seqlen)        # packed (total, H, D)
+    out, lse = fa_fwd_paged(q, k_cache, v_cache, block_table)        # K/V in a page pool
     x_unpad  = fa_unpad(x, indices)                                  # (B, L, H, D) -> (nnz, H, D)
     x_pad    = fa_pad(x_unpad, indices, batch, total_len)            # (nnz, H, D) -> (B, L, H, D)
 """
@@ -45,6 +46,7 @@ def lib() -> ctypes.CDLL:
         vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
         L.fa_varlen_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, i32, i32, f32, i32, i32, vp]
+        L.fa_fwd_paged.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
         L.fa_unpad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fa_pad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fa_unpad_qkv.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp]
@@ -52,7 +54,7 @@ def lib() -> ctypes.CDLL:
                                            vp]
         L.fa_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.fa_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
-        for f in (L.fa_fwd, L.fa_varlen_fwd, L.fa_varlen_fwd_padded, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad,
+        for f in (L.fa_fwd, L.fa_fwd_paged, L.fa_varlen_fwd, L.fa_varlen_fwd_padded, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad,
                   L.fa_device_status,
                   L.fa_selftest_bounded_wait):
             f.restype = ctypes.c_int
@@ -115,6 +117,38 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torc
     st = lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
                       float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
     _check(st, "fa_fwd")
+    return out, lse
+
+
+def fa_fwd_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.Tensor,
+                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                 scale: Optional[float] = None, causal: bool = False, return_lse: bool = True,
+                 stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Dense forward with paged K/V: q (B, S, H, D); k_cache, v_cache (num_pages, page_size, H, D);
+    block_table int32 (B, max_blocks_per_seq) -> out (B, S, H, D), lse (B, H, S) fp32."""
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("block_table", block_table)):
+        _cuda_contig(n, t)
+    if q.dim() != 4 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("q must be (B, S, H, D) and k_cache, v_cache one (num_pages, page_size, H, D) shape")
+    if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise ValueError("q, k_cache, v_cache must share one dtype")
+    B, S, H, D = q.shape
+    num_pages, page_size = k_cache.shape[0], k_cache.shape[1]
+    if tuple(k_cache.shape[2:]) != (H, D):
+        raise ValueError("k_cache and v_cache pages must hold (H, D) rows like q")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be an int32 (B, max_blocks_per_seq) tensor")
+    if out is None:
+        out = torch.empty_like(q)
+    _cuda_contig("out", out)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
+    if lse is not None:
+        _cuda_contig("lse", lse)
+    st = lib().fa_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
+                            page_size, num_pages, _ptr(out), _ptr(lse), B, H, S, D,
+                            float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
+    _check(st, "fa_fwd_paged")
     return out, lse
 
 

@@ -70,17 +70,25 @@ bool encode_map(CUtensorMap *m, const void *base, bool bf16, int D, int H, int64
     return r == CUDA_SUCCESS;
 }
 
+struct Paging {
+    const int32_t *block_table;
+    int max_blocks, page_size, num_pages;
+};
+
 fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
                   const int32_t *cu_seqlens, int num_seqs, int seqlen, int64_t N, int H, int D,
                   float scale, int causal, fa_dtype dtype, void *stream,
-                  const int64_t *gather = nullptr, int64_t padded_rows = 0) {
+                  const int64_t *gather = nullptr, int64_t padded_rows = 0, const Paging *paging = nullptr) {
     const bool bf16 = dtype == FA_BF16;
     const int inner = fa::fwd_box_inner_elems(D);
     CUtensorMap tq, tk, tv;
     const int64_t map_rows = gather ? padded_rows : N;  // the fused path's copy threads do not use the maps
+    const int64_t kv_rows = paging ? static_cast<int64_t>(paging->num_pages) * paging->page_size : map_rows;
+    const int k_box = paging ? fa::fwd_paged_k_box_rows(D, paging->page_size) : fa::fwd_kv_tile_rows(D);
+    const int v_box = paging ? fa::fwd_paged_v_box_rows(D, paging->page_size) : fa::fwd_v_box_rows(D);
     if (!encode_map(&tq, q, bf16, D, H, map_rows, inner, fa::fwd_tile_rows()) ||
-        !encode_map(&tk, k, bf16, D, H, map_rows, inner, fa::fwd_kv_tile_rows(D)) ||
-        !encode_map(&tv, v, bf16, D, H, map_rows, inner, fa::fwd_v_box_rows(D)))
+        !encode_map(&tk, k, bf16, D, H, kv_rows, inner, k_box) ||
+        !encode_map(&tv, v, bf16, D, H, kv_rows, inner, v_box))
         return FA_ERR_CUDA;
     if (!(scale > 0.f)) scale = 1.0f / sqrtf(static_cast<float>(D));
     fa::FwdParams p;
@@ -98,6 +106,12 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     p.total_tokens = static_cast<int>(N);
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = wait_limit_ns();
+    p.block_table = paging ? paging->block_table : nullptr;
+    p.max_blocks = paging ? paging->max_blocks : 0;
+    p.page_size = paging ? paging->page_size : 0;
+    p.page_shift = 0;
+    while (paging && (1 << p.page_shift) < paging->page_size) ++p.page_shift;
+    p.num_pages = paging ? paging->num_pages : 0;
     const int rows = fa::fwd_tile_rows();
     dim3 grid;
     if (cu_seqlens) {
@@ -110,8 +124,10 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
         grid = dim3(static_cast<unsigned>(H), static_cast<unsigned>((qtiles + per_cta - 1) / per_cta),
                     static_cast<unsigned>(num_seqs));
     }
-    const cudaError_t e = fa::launch_fwd(D, bf16, causal != 0, tq, tk, tv, p, grid,
-                                         static_cast<cudaStream_t>(stream));
+    const cudaError_t e = paging ? fa::launch_fwd_paged(D, bf16, causal != 0, tq, tk, tv, p, grid,
+                                                        static_cast<cudaStream_t>(stream))
+                                 : fa::launch_fwd(D, bf16, causal != 0, tq, tk, tv, p, grid,
+                                                  static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -130,6 +146,28 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, float *
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
         return FA_ERR_ALIGN;
     return run_fwd(q, k, v, out, lse, nullptr, B, S, N, H, D, scale, causal, dtype, stream);
+}
+
+fa_status fa_fwd_paged(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+                       int max_blocks_per_seq, int page_size, int num_pages, void *out, float *lse, int B, int H,
+                       int S, int D, float scale, int causal, fa_dtype dtype, void *stream) {
+    if (!q || !k_cache || !v_cache || !block_table || !out) return FA_ERR_NULL;
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (!head_dim_ok(D)) return FA_ERR_HEADDIM;
+    if (B <= 0 || H <= 0 || S <= 0 || num_pages <= 0 || max_blocks_per_seq <= 0) return FA_ERR_SHAPE;
+    // a power of two of at least 16 rows: a page is a whole number of 16-row boxes, and a
+    // 128-row key tile either holds whole pages or lies inside one
+    if (page_size < 16 || page_size > (1 << 20) || (page_size & (page_size - 1)) != 0) return FA_ERR_SHAPE;
+    if (static_cast<int64_t>(max_blocks_per_seq) * page_size < S) return FA_ERR_SHAPE;
+    if (static_cast<int64_t>(num_pages) * page_size > INT32_MAX) return FA_ERR_SHAPE;
+    const int64_t N = static_cast<int64_t>(B) * S;
+    if (N > INT32_MAX || B > 65535 || (S + 127) / 128 > 65535) return FA_ERR_SHAPE;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+        !aligned(lse, 4) || !aligned(block_table, 4))
+        return FA_ERR_ALIGN;
+    const Paging paging{block_table, max_blocks_per_seq, page_size, num_pages};
+    return run_fwd(q, k_cache, v_cache, out, lse, nullptr, B, S, N, H, D, scale, causal, dtype, stream, nullptr, 0,
+                   &paging);
 }
 
 fa_status fa_varlen_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqlens, int num_seqs,
@@ -211,12 +249,17 @@ fa_status fa_pad(const void *x, const int64_t *indices, int64_t nnz, int64_t tot
 
 fa_status fa_device_status(int *where) {
     if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
-    int c1 = 0, w1 = 0, c2 = 0, w2 = 0;
-    if (fa::fwd_take_device_error(&c1, &w1) != cudaSuccess) return FA_ERR_CUDA;
-    if (fa::pad_take_device_error(&c2, &w2) != cudaSuccess) return FA_ERR_CUDA;
-    if (where) *where = c1 ? w1 : w2;
-    if (c1) return static_cast<fa_status>(c1);
-    if (c2) return static_cast<fa_status>(c2);
+    // every kernel family keeps its own word; all are read (and so cleared), the first set wins
+    int code[3] = {0, 0, 0}, w[3] = {0, 0, 0};
+    if (fa::fwd_take_device_error(&code[0], &w[0]) != cudaSuccess) return FA_ERR_CUDA;
+    if (fa::fwd_paged_take_device_error(&code[1], &w[1]) != cudaSuccess) return FA_ERR_CUDA;
+    if (fa::pad_take_device_error(&code[2], &w[2]) != cudaSuccess) return FA_ERR_CUDA;
+    for (int i = 0; i < 3; ++i)
+        if (code[i]) {
+            if (where) *where = w[i];
+            return static_cast<fa_status>(code[i]);
+        }
+    if (where) *where = 0;
     return FA_OK;
 }
 

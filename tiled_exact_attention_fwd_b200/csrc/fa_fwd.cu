@@ -1,930 +1,9 @@
-// fa_fwd.cu -- exact attention forward, tile by tile, on sm_100a.
-//
-// What is computed (page "昇腾CANN跑大模型，FlashAttention这个算子你得认识一下"):
-//   section "传统实现到底慢在哪": O = softmax(Q K^T * scale) V;
-//   section "分块计算，这事没那么简单": Q, K, V are cut into tiles that stay on chip and
-//     only O is written back; each row keeps a running max m and sum l, and a new key
-//     tile updates (m, l) and corrects the partial output computed so far;
-//   section "昇腾NPU上做了什么特殊优化": the causal mask is fused, key tiles that are fully
-//     masked are never loaded or multiplied.
-// The packed case (page "IAW 模型 FA2 vs FA3 实测", section 1) is the same loop run inside
-// each sequence of cu_seqlens.
-//
-// B200 design. One CTA owns up to two 128-row query tiles (A, B) of one head of one
-// sequence that share every K/V tile it loads (one tile when D = 256, where two O
-// accumulators do not fit in TMEM), which halves the K/V bytes moved per MMA flop:
-//   warps 0-7   two softmax warpgroups, warpgroup t for tile t; thread (warp w, lane l)
-//               owns row 32*(w%4)+l of its tile, the TMEM lane its warp may access. It
-//               reads its S row with tcgen05.ld, masks, updates (m, l) with exp2 of scores
-//               pre-multiplied by scale*log2(e), writes P (16-bit) over S in TMEM, and when
-//               its max grew by more than 2^8 rescales its O row in TMEM (lazy rescale:
-//               between rescales every exponent uses the same stale max, which the final
-//               1/l cancels exactly). At the end: O/l -> fp16/bf16 -> global, and the LSE.
-//   warp 8      TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ... through an
-//               NS-stage shared-memory ring guarded by full/empty mbarriers.
-//   warp 9      allocates TMEM; one thread issues every tcgen05.mma:
-//                 S_t = Q_t K_j^T   (A = Q_t, B = K_j, both K-major in SMEM, 128B swizzle)
-//                 O_t += P_t V_j    (A = P_t read from TMEM, B = V_j MN-major in SMEM)
-//               in the ping-pong order QK_A0, QK_B0, PV_A0, QK_A1, PV_B0, QK_B1, ..., so the
-//               tensor core works on one tile while the other tile's softmax runs. With a
-//               single tile the two S buffers are used alternately by that tile instead
-//               (order QK_0, QK_1, PV_0, QK_2, PV_1, ...).
-//
-// Every pipeline wait is bounded: after `timeout_ns` the waiting thread records
-// FA_ERR_TIMEOUT in a device word, raises a CTA-wide abort flag, and all roles drain
-// their in-flight copies/MMAs (again with a bound) before TMEM is released.
-#include <cuda.h>
-#include <cuda_bf16.h>
-#include <cuda_fp16.h>
-#include <cuda_runtime.h>
-#include <math.h>
-#include <stdint.h>
-
-#include <type_traits>
-
-#include "fa.h"
-#include "fa_internal.h"
-#include "fa_ptx.cuh"
+// fa_fwd.cu -- the attention forward over contiguous K/V (dense and packed sequences, and the
+// fused packed path): instantiations of the kernel in fa_fwd_kernel.cuh, the bounded-wait
+// self-test, and the host-side tile geometry shared with fa_api.cu.
+#include "fa_fwd_kernel.cuh"
 
 namespace fa {
-
-static __device__ int g_err_code;
-static __device__ int g_err_where;
-
-__device__ __noinline__ void record_error(int code, int where) {
-    if (atomicCAS(&g_err_code, 0, code) == 0) atomicExch(&g_err_where, where);
-}
-
-// Wait for phase `parity` of `bar`, giving up after limit_ns or when another role aborted.
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             uint64_t limit_ns, int where) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-#pragma unroll 1
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 31u) == 0) {
-            if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > limit_ns) {
-                *abort_flag = 1;
-                record_error(FA_ERR_TIMEOUT, where);
-                return false;
-            }
-        }
-    }
-}
-
-template <int D>
-struct Cfg {
-    static constexpr int BM = 128;                           // query rows per tile (MMA M)
-    static constexpr int BN = 128;                           // key rows per tile
-    static constexpr int MAXQ = (D == 256) ? 1 : 2;          // query tiles per CTA
-    static constexpr int SW = (2 * D >= 128) ? 128 : 2 * D;  // swizzle span in bytes
-    static constexpr int SWE = SW / 2;                       // 16-bit elements per swizzle row
-    static constexpr int NBLK = D / SWE;                     // column blocks per tile row
-    static constexpr int Q_BYTES = BM * D * 2;
-    static constexpr int KV_BYTES = BN * D * 2;
-    // The K/V ring moves tiles in UNITS parts (D = 256: 64 KB tiles in two 32 KB parts, so
-    // the ring keeps 5 stages): part u of K_j holds column blocks [u*NBLK/UNITS, ...) of all
-    // rows, part u of V_j rows [u*BN/UNITS, ...) of all column blocks.
-    static constexpr int UNITS = (D == 256) ? 2 : 1;
-    static constexpr int UNIT_BYTES = KV_BYTES / UNITS;
-    static constexpr int KBLK_PER_UNIT = NBLK / UNITS;   // K column blocks per part
-    static constexpr int VROWS_PER_UNIT = BN / UNITS;    // V rows per part
-    static constexpr uint32_t LAYOUT = (SW == 128) ? kLayoutSw128 : kLayoutSw64;
-    static constexpr uint32_t TMEM_COLS = 512;
-    // TMEM columns: S0 at 0, S1 at BN. With D <= 64 two separate P buffers fit (P_COL + 64t)
-    // so a tile's next S = QK^T can be computed while its softmax still works on the last
-    // one ("decoupled"); otherwise P overwrites the first half of its S buffer.
-    static constexpr bool DECOUPLED = (MAXQ == 2) && (D <= 64);
-    static constexpr uint32_t P_COL = 2 * BN;
-    static constexpr uint32_t O_COL = 2 * BN + (DECOUPLED ? 128 : 0);  // O_A, O_B
-    static constexpr int NUM_SOFTMAX_WARPS = 4 * MAXQ;
-    static constexpr int WARP_TMA = NUM_SOFTMAX_WARPS;
-    static constexpr int WARP_MMA = NUM_SOFTMAX_WARPS + 1;
-    // A full last warpgroup (two idle warps) so that per-warpgroup register limits apply.
-    static constexpr int NUM_THREADS = 32 * (NUM_SOFTMAX_WARPS + 4);
-    // Register split (two query tiles): 384 threads launch with LAUNCH_REGS each; the
-    // producer/MMA warpgroup drops to REGS_LOW and the softmax warpgroups rise to REGS_HIGH.
-    // The host refuses to launch unless the pool covers the split (it would otherwise wait).
-    static constexpr int LAUNCH_REGS = 168;
-    static constexpr int REGS_LOW = 56;
-    static constexpr int REGS_HIGH = 224;
-    static constexpr bool SPLIT_REGS = (MAXQ == 2);
-    static_assert(!SPLIT_REGS || 128 * REGS_LOW + 256 * REGS_HIGH <= NUM_THREADS * LAUNCH_REGS, "register split");
-    // Column pairs (out of every 4) whose exp2 runs on the FMA pipe instead of MUFU.
-    static constexpr int EMU_PAIRS_OF_4 = 0;
-    // shared memory map (offsets from a 1024-byte aligned base)
-    static constexpr int SMEM_LIMIT = 227 * 1024;
-    static constexpr int RESERVED = 1024 /*alignment*/ + 512 /*barriers, misc*/;
-    static constexpr int NS_FIT = (SMEM_LIMIT - RESERVED - MAXQ * Q_BYTES) / UNIT_BYTES;
-    static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_KV = MAXQ * Q_BYTES;
-    static constexpr int OFF_BAR = OFF_KV + NS * UNIT_BYTES;
-    // q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], drain, s_free[2]
-    static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1 + 2;
-    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-    static constexpr int USED = OFF_MISC + 16;
-    // More than half of the SM's shared memory, so exactly one CTA (and one 512-column
-    // TMEM allocation) lives on an SM.
-    static constexpr int MIN_SMEM = 120 * 1024;
-    static constexpr int SMEM_BYTES = (USED + 1024 > MIN_SMEM) ? USED + 1024 : MIN_SMEM;
-    static_assert(NS >= 3, "K/V ring too shallow");
-    static_assert(O_COL + MAXQ * D <= TMEM_COLS, "TMEM budget");
-    static_assert(USED + 1024 <= SMEM_LIMIT, "shared memory budget");
-    static_assert(NUM_BARS * 8 + 16 <= 512, "barrier area");
-    static_assert(Q_BYTES % 1024 == 0 && UNIT_BYTES % 1024 == 0, "tile alignment");
-    // The MMA thread waits for K_{j+1} while V_j is still held: the ring needs both, plus a part.
-    static_assert(NS >= 2 * UNITS + 1, "K/V ring too shallow");
-};
-
-// Sequence that packed token `tok` belongs to: the s with cu[s] <= tok < cu[s+1]
-// (binary search over the num_seqs + 1 offsets; empty sequences are skipped).
-__device__ __forceinline__ int seq_of_token(const int32_t *cu, int num_seqs, int tok) {
-    int lo = 0, hi = num_seqs;  // invariant: cu[lo] <= tok < cu[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(cu + mid) <= tok) lo = mid; else hi = mid;
-    }
-    return lo;
-}
-
-// seq_of_token for a token shared by the whole warp: 32 probes per dependent load.
-__device__ __forceinline__ int warp_seq_of_token(const int32_t *cu, int num_seqs, int tok, int lane) {
-    int lo = 0, hi = num_seqs;  // answer s in [lo, hi - 1]: the last s with cu[s] <= tok
-    while (hi - lo > 32) {
-        const int step = (hi - lo + 31) / 32;
-        const int p = lo + lane * step;
-        const bool le = p < hi && __ldg(cu + p) <= tok;
-        const int c = __popc(__ballot_sync(0xffffffffu, le));  // probes <= tok form a prefix (c >= 1)
-        const int new_lo = lo + (c - 1) * step;
-        hi = min(hi, lo + c * step);
-        lo = new_lo;
-    }
-    const int p = lo + lane;
-    const bool le = p < hi && __ldg(cu + p) <= tok;
-    return lo + __popc(__ballot_sync(0xffffffffu, le)) - 1;
-}
-
-// Sequence of each lane's token `tok` (tokens of one warp, >= cu[s0] where s0 is the sequence
-// of the warp's first token): one 32-wide load of cu[s0 + 1 ..] and a 5-step search over the
-// lanes; falls back to the plain search when the warp's tokens span more than 32 sequences.
-__device__ __forceinline__ int lane_seq_of_token(const int32_t *cu, int num_seqs, int s0, int tok, int lane) {
-    const int wi = s0 + 1 + lane;
-    const int w = (wi <= num_seqs) ? __ldg(cu + wi) : 0x7fffffff;
-    int lo = 0, hi = 32;  // count of window entries <= tok, in [lo, hi]
-#pragma unroll
-    for (int k = 0; k < 6; ++k) {
-        const int mid = (lo + hi + 1) >> 1;
-        const int v = __shfl_sync(0xffffffffu, w, (mid - 1) & 31);
-        if (mid <= hi && lo < hi) {
-            if (v <= tok) lo = mid; else hi = mid - 1;
-        }
-    }
-    return (lo < 32) ? s0 + lo : seq_of_token(cu, num_seqs, tok);
-}
-
-// Single-tile order of MMA steps: K0, K1, V0, K2, V1, ..., V_{n-1} (QK runs one tile ahead).
-__device__ __forceinline__ void decode_step(int idx, int n, bool &is_v, int &j) {
-    if (idx == 0) { is_v = false; j = 0; }
-    else if (idx == 2 * n - 1) { is_v = true; j = n - 1; }
-    else if (idx & 1) { is_v = false; j = (idx + 1) >> 1; }
-    else { is_v = true; j = (idx >> 1) - 1; }
-}
-
-template <bool BF16>
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-    return BF16 ? pack2_bf16(lo, hi) : pack2_f16(lo, hi);
-}
-
-// 2^x for a pair of scores, evaluated on the FMA pipe instead of the MUFU unit. Cody-Waite
-// style reduction x = n + f with n = round(x) taken from the 1.5*2^23 shifter and f in
-// [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted with the Remez algorithm for minimax
-// relative error (7.5e-5, below the 2^-11 rounding of the 16-bit P it feeds;
-// gen_exp2_poly.py); 2^n is added to the exponent field. The float arithmetic runs two
-// lanes at a time (add/fma .f32x2). Inputs below -126 are clamped (the result is then ~1e-38
-// instead of a smaller number, irrelevant next to the row sum, which is at least 1); it is
-// only used on tiles without masked (-inf) scores.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float &y1) {
-    constexpr float c3 = 5.517166853e-02f, c2 = 2.426111251e-01f, c1 = 6.932609677e-01f, c0 = 9.999280572e-01f;
-    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-    const uint64_t x2 = f2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-    const uint64_t t2 = fadd2(x2, f2(kShift, kShift));
-    const uint64_t n2 = fadd2(t2, f2(-kShift, -kShift));
-    const uint64_t r2 = ffma2(n2, f2(-1.0f, -1.0f), x2);  // x - n, exact
-    uint64_t p2 = ffma2(f2(c3, c3), r2, f2(c2, c2));
-    p2 = ffma2(p2, r2, f2(c1, c1));
-    p2 = ffma2(p2, r2, f2(c0, c0));
-    float t0, t1, p0, p1;
-    f2_split(t2, t0, t1);
-    f2_split(p2, p0, p1);
-    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
-// Maximum of an S row held in registers: 8 independent chains of three-input maxima.
-template <int BN>
-__device__ __forceinline__ float row_max(const uint32_t *sr) {
-    float mm[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) mm[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]));
-#pragma unroll
-    for (int i = 16; i < BN; i += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mm[k] = fmax3(mm[k], __uint_as_float(sr[i + k]), __uint_as_float(sr[i + 8 + k]));
-    return fmaxf(fmax3(mm[0], mm[1], mm[2]), fmax3(fmax3(mm[3], mm[4], mm[5]), mm[6], mm[7]));
-}
-
-// For each 64-column chunk of an S row (in registers): p = 2^(s*c + neg_m) (scaling done two
-// lanes at a time with fma.f32x2), row sum in four fp32x2 partial sums, pairs packed to
-// 16 bits and the chunk stored to TMEM at p_addr. Of every 4 column pairs, EMU use
-// exp2_poly, the rest the MUFU ex2. Returns the row sum of this tile.
-template <int BN, bool BF16, int EMU>
-__device__ __forceinline__ float softmax_chunk_store(const uint32_t *sr, float c, float neg_m, uint32_t p_addr) {
-    const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
-    uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
-#pragma unroll
-    for (int cc = 0; cc < BN / 64; ++cc) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int e = cc * 64 + 2 * i;
-            const uint64_t x2 = ffma2(f2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, nm2);
-            float x0, x1;
-            f2_split(x2, x0, x1);
-            float p0, p1;
-            if ((i & 3) >= 4 - EMU) {
-                exp2_poly2(x0, x1, p0, p1);
-            } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-            }
-            acc[i & 3] = fadd2(acc[i & 3], f2(p0, p1));
-            pk[i] = pack2<BF16>(p0, p1);
-        }
-        tmem_st32(p_addr + cc * 32, pk);
-    }
-    const uint64_t s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-    float lo, hi;
-    f2_split(s2, lo, hi);
-    return lo + hi;
-}
-
-// A whole S row (in registers) to packed 16-bit P in registers pk[BN/2]:
-// p = 2^(s*c + neg_m), scaling two lanes at a time; returns the row sum.
-template <int BN, bool BF16, int EMU>
-__device__ __forceinline__ float softmax_row_to_regs(const uint32_t *sr, float c, float neg_m, uint32_t *pk) {
-    const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
-    uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
-#pragma unroll
-    for (int i = 0; i < BN / 2; ++i) {
-        const uint64_t x2 = ffma2(f2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, nm2);
-        float x0, x1;
-        f2_split(x2, x0, x1);
-        float p0, p1;
-        if ((i & 3) >= 4 - EMU) {
-            exp2_poly2(x0, x1, p0, p1);
-        } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-        }
-        acc[i & 3] = fadd2(acc[i & 3], f2(p0, p1));
-        pk[i] = pack2<BF16>(p0, p1);
-    }
-    const uint64_t s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-    float lo, hi;
-    f2_split(s2, lo, hi);
-    return lo + hi;
-}
-
-// Shared state of one CTA: shared-memory buffers, barriers, TMEM base and the plan.
-template <int D>
-struct Cta {
-    using C = Cfg<D>;
-    uint8_t *sQ, *sKV;
-    uint64_t *q_full, *kv_full, *kv_empty, *s_full, *p_full, *pv_done, *drain, *s_free;
-    volatile int *abort_flag;
-    uint32_t tmem;
-    uint64_t lim;
-    // Tile A visits key tiles [0, nA), tile B [jB0, nB) (nB = 0 when B is absent); key tile j
-    // covers tokens kvbase + [j*BN, (j+1)*BN). In dense sequences jB0 = 0; in packed ones
-    // B may begin a later sequence. Always jB0 <= nA <= nB, so the two ranges leave no gap.
-    int nA, nB, jB0;
-    __device__ __forceinline__ int j0(int t) const { return t ? jB0 : 0; }
-    __device__ __forceinline__ bool uses(int t, int j) const { return t ? (j >= jB0 && j < nB) : (j < nA); }
-    bool two;      // two query tiles (ping-pong) or one (S double-buffered)
-    bool dec;      // two tiles with separate P buffers (Cfg::DECOUPLED)
-    bool fused;    // Q/K/V tiles written by threads (cp.async), not TMA: fence before the MMA reads them
-    // S/P buffer and barrier phase used by tile t at key step j
-    __device__ __forceinline__ int buf(int t, int j) const { return two ? t : (j & 1); }
-    __device__ __forceinline__ uint32_t sphase(int j) const { return two ? (j & 1) : ((j >> 1) & 1); }
-};
-
-// One MMA step of the issuing thread. Returns false when a wait gave up.
-template <int D, bool BF16>
-// S_t = Q_t K_j^T for key tile j (tile-local step jj = j - j0(t)).
-__device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first_use, bool last_use) {
-    using C = Cfg<D>;
-    constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
-    constexpr uint32_t idesc = idesc_f16(BM, BN, BF16, false);
-    const int jj = j - c.j0(t);
-    if (jj == 0) {
-        if (!wait_bounded(&c.q_full[t], 0, c.abort_flag, c.lim, 200 + t)) return false;
-        tc_fence_after_sync();
-        if (c.fused) fence_proxy_async_smem();
-    } else if (c.dec) {
-        // S_t is overwritten: the softmax warps must have read the previous S_t
-        if (!wait_bounded(&c.s_free[t], (jj - 1) & 1, c.abort_flag, c.lim, 240 + t)) return false;
-        tc_fence_after_sync();
-    }
-    constexpr int UK = D / 16 / C::UNITS;  // k-steps per K part
-    const uint32_t q_addr = smem_u32(c.sQ + t * C::Q_BYTES);
-    const int b = c.buf(t, jj);
-    const uint32_t d_tmem = c.tmem + b * BN;
-#pragma unroll
-    for (int u = 0; u < C::UNITS; ++u) {
-        const int U = 2 * j * C::UNITS + u, stage = U % NS;  // ring part holding K_j part u
-        if (first_use) {
-            if (!wait_bounded(&c.kv_full[stage], (U / NS) & 1, c.abort_flag, c.lim, 220 + stage)) return false;
-            tc_fence_after_sync();
-            if (c.fused) fence_proxy_async_smem();
-        }
-        const uint32_t k_addr = smem_u32(c.sKV + stage * C::UNIT_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < UK; ++kk) {
-            const int k = u * UK + kk;
-            const uint32_t blk = (k * 32) / SW, off = (k * 32) % SW;
-            const uint32_t lb = blk - u * C::KBLK_PER_UNIT;  // column block inside the part
-            const uint64_t a = smem_desc(q_addr + blk * BM * SW + off, 16, 8 * SW, C::LAYOUT);
-            const uint64_t bd = smem_desc(k_addr + lb * BN * SW + off, 16, 8 * SW, C::LAYOUT);
-            umma_ss(d_tmem, a, bd, idesc, k > 0 ? 1u : 0u);
-        }
-        if (u + 1 < C::UNITS) {
-            if (last_use) umma_commit(&c.kv_empty[stage]);  // release this part early
-        } else {
-            umma_commit(&c.s_full[b]);  // the softmax waits on S first
-            if (last_use) umma_commit(&c.kv_empty[stage]);
-        }
-    }
-    return true;
-}
-
-template <int D, bool BF16>
-// O_t += P_t V_j for key tile j (tile-local step jj = j - j0(t)).
-__device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first_use, bool last_use) {
-    using C = Cfg<D>;
-    constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
-    constexpr uint32_t idesc = idesc_f16(BM, D, BF16, true);
-    const int jj = j - c.j0(t);
-    const int b = c.buf(t, jj);
-    if (!wait_bounded(&c.p_full[b], c.sphase(jj), c.abort_flag, c.lim, 210 + t)) return false;
-    tc_fence_after_sync();
-    constexpr int UV = BN / 16 / C::UNITS;  // k-steps per V part
-    const uint32_t a_tmem = c.tmem + (c.dec ? C::P_COL + 64 * t : b * BN);
-    const uint32_t o_tmem = c.tmem + C::O_COL + t * D;
-#pragma unroll
-    for (int u = 0; u < C::UNITS; ++u) {
-        const int U = (2 * j + 1) * C::UNITS + u, stage = U % NS;  // ring part holding V_j part u
-        if (first_use) {
-            if (!wait_bounded(&c.kv_full[stage], (U / NS) & 1, c.abort_flag, c.lim, 230 + stage)) return false;
-            tc_fence_after_sync();
-            if (c.fused) fence_proxy_async_smem();
-        }
-        const uint32_t v_addr = smem_u32(c.sKV + stage * C::UNIT_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < UV; ++kk) {
-            const int k = u * UV + kk;
-            const uint64_t bd = smem_desc(v_addr + kk * 16 * SW, C::VROWS_PER_UNIT * SW, 8 * SW, C::LAYOUT);
-            umma_ts(o_tmem, a_tmem + k * 8, bd, idesc, (jj > 0 || k > 0) ? 1u : 0u);
-        }
-        if (u + 1 < C::UNITS) {
-            if (last_use) umma_commit(&c.kv_empty[stage]);
-        } else {
-            umma_commit(&c.pv_done[t]);
-            if (last_use) umma_commit(&c.kv_empty[stage]);
-        }
-    }
-    return true;
-}
-
-template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(Cfg<D>::NUM_THREADS, 1)
-fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using C = Cfg<D>;
-    constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
-
-    const int h = blockIdx.x;
-    // Rows of the CTA are tokens qbase + t*128 + r; keys are addressed from token kvbase.
-    //  dense : blockIdx.z is the batch entry; the CTA owns query tiles `pair` (two of them
-    //          when MAXQ = 2) of that sequence, longest (causal) tiles launched first.
-    //  packed: the CTA owns the 128 consecutive packed tokens of tile blockIdx.y, whatever
-    //          sequences they belong to; its keys are the union of those sequences' keys
-    //          (the device walks cu_seqlens), and each row is masked to its own sequence.
-    const bool packed = p.cu_seqlens != nullptr;
-    int seq_start = 0, seqlen = 0, q0 = 0, qbase, kvbase, kv_end_A, kv_end_B = 0, kv_start_B = 0;
-    bool two = false;
-    if (!packed) {
-        const int pair = gridDim.y - 1 - blockIdx.y;
-        seq_start = blockIdx.z * p.seqlen;
-        seqlen = p.seqlen;
-        q0 = pair * C::MAXQ * BM;
-        if (q0 >= seqlen) return;  // uniform over the CTA, before any barrier exists
-        two = (C::MAXQ == 2) && (q0 + BM < seqlen);
-        qbase = seq_start + q0;
-        kvbase = seq_start;
-        kv_end_A = CAUSAL ? min(seqlen, q0 + BM) : seqlen;
-        if (two) kv_end_B = CAUSAL ? min(seqlen, q0 + 2 * BM) : seqlen;
-    } else {
-        qbase = blockIdx.y * C::MAXQ * BM;
-        if (qbase >= p.total_tokens) return;
-        two = (C::MAXQ == 2) && (qbase + BM < p.total_tokens);
-        const int ln = threadIdx.x & 31;
-        const int s_first = warp_seq_of_token(p.cu_seqlens, p.num_seqs, qbase, ln);
-        kvbase = p.cu_seqlens[s_first];
-        // keys of a tile end with its last row's sequence (or the causal limit)
-        auto kv_end = [&](int tlast) {
-            const int s_last = warp_seq_of_token(p.cu_seqlens, p.num_seqs, tlast, ln);
-            return (CAUSAL ? min(p.cu_seqlens[s_last + 1], tlast + 1) : p.cu_seqlens[s_last + 1]) - kvbase;
-        };
-        kv_end_A = kv_end(min(qbase + BM, p.total_tokens) - 1);
-        if (two) {
-            kv_end_B = kv_end(min(qbase + 2 * BM, p.total_tokens) - 1);
-            kv_start_B = p.cu_seqlens[warp_seq_of_token(p.cu_seqlens, p.num_seqs, qbase + BM, ln)] - kvbase;
-        }
-    }
-
-    Cta<D> c;
-    c.two = two;
-    c.dec = C::DECOUPLED && c.two;
-    c.fused = p.gather != nullptr;
-    c.nA = (kv_end_A + BN - 1) / BN;
-    c.nB = c.two ? (kv_end_B + BN - 1) / BN : 0;
-    c.jB0 = c.two ? kv_start_B / BN : 0;
-    const int n_all = max(c.nA, c.nB);  // key tiles this CTA loads
-
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~uintptr_t(1023));
-    c.sQ = smem + C::OFF_Q;
-    c.sKV = smem + C::OFF_KV;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    c.q_full = bars;
-    c.kv_full = bars + 2;
-    c.kv_empty = c.kv_full + NS;
-    c.s_full = c.kv_empty + NS;
-    c.p_full = c.s_full + 2;
-    c.pv_done = c.p_full + 2;
-    c.drain = c.pv_done + 2;
-    c.s_free = c.drain + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
-    c.abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
-    c.lim = p.timeout_ns;
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-
-    if (threadIdx.x == 0) {
-        const int fill_arrivals = p.gather ? 96 : 1;  // fused: the 96 copy threads arrive
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(&c.q_full[t], fill_arrivals);
-            mbar_init(&c.s_full[t], 1);
-            mbar_init(&c.p_full[t], 128);
-            mbar_init(&c.pv_done[t], 1);
-            mbar_init(&c.s_free[t], 4);  // one arrival per softmax warp
-        }
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(&c.kv_full[s], fill_arrivals);
-            mbar_init(&c.kv_empty[s], 1);
-        }
-        mbar_init(c.drain, 1);
-        *c.abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == C::WARP_TMA && lane == 0) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-    }
-    if (warp == C::WARP_MMA) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    c.tmem = *tmem_slot;
-
-    if (warp >= C::NUM_SOFTMAX_WARPS) {
-        // producer / MMA warpgroup (its two remaining warps idle)
-        if constexpr (C::SPLIT_REGS) regs_dec<C::REGS_LOW>();
-        if (warp == C::WARP_TMA || (p.gather && warp > C::WARP_MMA)) {
-            // ------------------------------------------------------------ TMA producer
-            // (with the fused packed path also warps 10 and 11: copy producers)
-            const int nq = c.two ? 2 : 1;
-            const int loads = 2 * n_all * C::UNITS;  // parts of K_0, V_0, K_1, V_1, ...
-            int issued = 0;
-            if (p.gather) {
-                // Fused packed path: warps 8, 10 and 11 (96 threads) copy every tile row from
-                // the padded tensor (row = padded row of the packed token; rows past the last
-                // token read row 0, which the masks then ignore) with 16-byte cp.async into the
-                // same swizzled layout the TMA would produce; each thread's copies arrive on the
-                // tile's barrier when they land, and the MMA thread fences the async proxy.
-                constexpr int CPB = SW / 16;  // 16-byte chunks per swizzle row (column block)
-                const int pw = (warp == C::WARP_TMA) ? 0 : warp - C::WARP_MMA;  // producer warp 0..2
-                // Copies rows [tok0, tok0 + rows) x column blocks [b0, b0 + NB) into dst laid out
-                // as [NB][rows][SW].
-                auto fill = [&](auto nb_c, uint8_t *dst, const void *src, uint64_t *bar, int tok0, int rows,
-                                int b0) {
-                    constexpr int CPR = decltype(nb_c)::value * CPB;  // chunks per row
-                    const uint32_t dst_u32 = smem_u32(dst);
-                    // 32-row groups round-robin over the three warps: one coalesced load of the
-                    // group's padded rows, then every lane issues CPR 16-byte copies.
-                    for (int g = pw; g * 32 < rows; g += 3) {
-                        const int tok = tok0 + g * 32 + lane;
-                        int64_t prow = (tok >= 0 && tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
-                        if (prow < 0 || prow >= p.padded_rows) prow = 0;  // never read outside q/k/v
-                        const uint8_t *srow = static_cast<const uint8_t *>(src) + b0 * SW;
-#pragma unroll 4
-                        for (int i = 0; i < CPR; ++i) {
-                            const int idx = i * 32 + lane;
-                            const int rr = idx / CPR, ch = idx % CPR;
-                            const int64_t pr = __shfl_sync(0xffffffffu, prow, rr);
-                            const int r = g * 32 + rr;
-                            const int blk = ch / CPB, cc = ch % CPB;
-                            const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
-                            cp_async_16(dst_u32 + blk * rows * SW + r * SW + ((cc ^ swz) << 4),
-                                        srow + (pr * p.H + h) * static_cast<int64_t>(D) * 2 + ch * 16);
-                        }
-                    }
-                    cp_async_mbar_arrive(bar);  // arrives once this thread's copies have landed
-                };
-                using AllBlk = std::integral_constant<int, C::NBLK>;
-                using KBlk = std::integral_constant<int, C::KBLK_PER_UNIT>;
-                for (int t = 0; t < nq; ++t)
-                    fill(AllBlk{}, c.sQ + t * C::Q_BYTES, p.q, &c.q_full[t], qbase + t * BM, BM, 0);
-                for (int U = 0; U < loads; ++U) {
-                    const int stage = U % NS;
-                    if (U >= NS &&
-                        !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
-                        break;
-                    const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
-                    uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
-                    if (L & 1)
-                        fill(AllBlk{}, dst, p.v, &c.kv_full[stage], kvbase + j * BN + u * C::VROWS_PER_UNIT,
-                             C::VROWS_PER_UNIT, 0);
-                    else
-                        fill(KBlk{}, dst, p.k, &c.kv_full[stage], kvbase + j * BN, BN, u * C::KBLK_PER_UNIT);
-                    issued = U + 1;
-                }
-                cp_async_wait_all();  // nothing of this thread is left in flight at exit
-                issued = 0;
-            } else if (lane == 0) {
-                const uint64_t pol_q = l2_policy_evict_first();
-                const uint64_t pol_kv = l2_policy_evict_last();
-                for (int t = 0; t < nq; ++t) {
-                    mbar_arrive_expect_tx(&c.q_full[t], C::Q_BYTES);
-#pragma unroll
-                    for (int b = 0; b < C::NBLK; ++b)
-                        tma_load_3d(c.sQ + t * C::Q_BYTES + b * BM * SW, &tm_q, &c.q_full[t], b * C::SWE, h,
-                                    qbase + t * BM, pol_q);
-                }
-                for (int U = 0; U < loads; ++U) {
-                    const int stage = U % NS;
-                    if (U >= NS &&
-                        !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
-                        break;
-                    const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
-                    uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
-                    mbar_arrive_expect_tx(&c.kv_full[stage], C::UNIT_BYTES);
-                    if (L & 1) {
-                        // V part u: rows [u*VROWS_PER_UNIT, ...) of the tile, every column block
-#pragma unroll
-                        for (int b = 0; b < C::NBLK; ++b)
-                            tma_load_3d(dst + b * C::VROWS_PER_UNIT * SW, &tm_v, &c.kv_full[stage], b * C::SWE, h,
-                                        kvbase + j * BN + u * C::VROWS_PER_UNIT, pol_kv);
-                    } else {
-                        // K part u: column blocks [u*KBLK_PER_UNIT, ...) of every tile row
-#pragma unroll
-                        for (int b = 0; b < C::KBLK_PER_UNIT; ++b)
-                            tma_load_3d(dst + b * BN * SW, &tm_k, &c.kv_full[stage],
-                                        (u * C::KBLK_PER_UNIT + b) * C::SWE, h, kvbase + j * BN, pol_kv);
-                    }
-                    issued = U + 1;
-                }
-            }
-            if (warp == C::WARP_TMA && lane == 0 && *c.abort_flag) {
-                // Let the copies already issued land before the CTA's shared memory goes away.
-                for (int t = 0; t < nq; ++t) {
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(&c.q_full[t], 0) && global_timer_ns() - t0 < c.lim) {
-                    }
-                }
-                for (int U = (issued > NS ? issued - NS : 0); U < issued; ++U) {
-                    const int stage = U % NS;
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(&c.kv_full[stage], (U / NS) & 1) && global_timer_ns() - t0 < c.lim) {
-                    }
-                }
-            }
-        } else if (warp == C::WARP_MMA) {
-            // ------------------------------------------------------------ MMA issuer
-            if (lane == 0) {
-                bool ok = true;
-                if (!c.two) {
-                    const int n = c.nA;
-                    for (int idx = 0; ok && idx < 2 * n; ++idx) {
-                        bool is_v;
-                        int j;
-                        decode_step(idx, n, is_v, j);
-                        ok = is_v ? mma_pv<D, BF16>(c, 0, j, true, true) : mma_qk<D, BF16>(c, 0, j, true, true);
-                    }
-                } else if (c.dec) {
-                    // Separate P buffers: QK_t(j+1) only waits until the softmax warps have read
-                    // S_t(j), so it runs while they compute P_t(j). Order per key tile j:
-                    // QK_A(j+1), QK_B(j+1), PV_A(j), PV_B(j), each when that tile uses key tile j.
-                    const int nB = c.nB;
-                    if (c.uses(0, 0)) ok = mma_qk<D, BF16>(c, 0, 0, true, !c.uses(1, 0));
-                    if (ok && c.uses(1, 0)) ok = mma_qk<D, BF16>(c, 1, 0, !c.uses(0, 0), true);
-                    for (int j = 0; ok && j < nB; ++j) {
-                        const bool a1 = c.uses(0, j + 1), b1 = c.uses(1, j + 1), a0 = c.uses(0, j), b0 = c.uses(1, j);
-                        if (a1) ok = mma_qk<D, BF16>(c, 0, j + 1, true, !b1);
-                        if (ok && b1) ok = mma_qk<D, BF16>(c, 1, j + 1, !a1, true);
-                        if (ok && a0) ok = mma_pv<D, BF16>(c, 0, j, true, !b0);
-                        if (ok && b0) ok = mma_pv<D, BF16>(c, 1, j, !a0, true);
-                    }
-                } else {
-                    // Ping-pong over key tiles j: PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j). A key or
-                    // value tile is waited for at its first use and released after its last.
-                    const int nB = c.nB;
-                    if (c.uses(0, 0)) ok = mma_qk<D, BF16>(c, 0, 0, true, !c.uses(1, 0));
-                    if (ok && c.uses(1, 0)) ok = mma_qk<D, BF16>(c, 1, 0, !c.uses(0, 0), true);
-                    for (int j = 1; ok && j <= nB; ++j) {
-                        const bool ap = c.uses(0, j - 1), bp = c.uses(1, j - 1), ac = c.uses(0, j), bc = c.uses(1, j);
-                        if (ap) ok = mma_pv<D, BF16>(c, 0, j - 1, true, !bp);
-                        if (ok && ac) ok = mma_qk<D, BF16>(c, 0, j, true, !bc);
-                        if (ok && bp) ok = mma_pv<D, BF16>(c, 1, j - 1, !ap, true);
-                        if (ok && bc) ok = mma_qk<D, BF16>(c, 1, j, !ac, true);
-                    }
-                }
-                // Every MMA issued above has finished once `drain` completes.
-                umma_commit(c.drain);
-                const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(c.drain, 0) && global_timer_ns() - t0 < c.lim) {
-                }
-            }
-    }
-    } else {
-        // ------------------------------------------------------------ softmax + epilogue
-        if constexpr (C::SPLIT_REGS) regs_inc<C::REGS_HIGH>();
-        const int t = warp >> 2;                      // query tile of this warpgroup
-        const int n = t ? c.nB - c.jB0 : c.nA;  // key tiles this warpgroup visits
-        const int j0 = c.j0(t);
-        const int quarter = warp & 3;                 // TMEM lanes this warp may access
-        const int r = quarter * 32 + lane;            // row of the tile == TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        // This row's token and its visible keys [klo, khi), counted from kvbase.
-        const int64_t tok = static_cast<int64_t>(qbase) + t * BM + r;
-        int klo = 0, khi = 1;
-        bool row_ok;
-        if (!packed) {
-            const int row_pos = q0 + t * BM + r;  // position inside the sequence
-            row_ok = row_pos < seqlen;
-            khi = CAUSAL ? min(seqlen, row_pos + 1) : seqlen;
-        } else {
-            row_ok = tok < p.total_tokens;
-            const int tw0 = qbase + t * BM + quarter * 32;  // this warp's first token
-            int s_lane = 0;
-            if (tw0 < p.total_tokens) {  // warp-uniform
-                const int s_w = warp_seq_of_token(p.cu_seqlens, p.num_seqs, tw0, lane);
-                s_lane = lane_seq_of_token(p.cu_seqlens, p.num_seqs, s_w,
-                                           static_cast<int>(min(tok, static_cast<int64_t>(p.total_tokens - 1))), lane);
-            }
-            if (row_ok) {
-                const int s_r = s_lane;
-                klo = p.cu_seqlens[s_r] - kvbase;
-                khi = (CAUSAL ? min(p.cu_seqlens[s_r + 1], static_cast<int>(tok) + 1) : p.cu_seqlens[s_r + 1]) - kvbase;
-            }
-        }
-        const uint32_t o_col = C::O_COL + t * D;
-        const float sc = p.scale_log2;
-        float m = -INFINITY;  // running max of scaled scores, log2 units (possibly stale)
-        float l = 0.f;        // running sum of 2^(s*sc - m)
-        bool ok = n > 0;
-        if (c.dec) {
-            // Separate P buffer: S_t is released right after it is read, so QK_t(j+1) overlaps
-            // this step's exponentials; P_t(j) is written once PV_t(j-1) has consumed P_t(j-1).
-            const uint32_t p_addr = c.tmem + lane_base + C::P_COL + 64 * t;
-            for (int jj = 0; jj < n; ++jj) {
-                const int j = j0 + jj;  // key tile
-                if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[t], jj & 1, c.abort_flag, c.lim, 330 + t))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                uint32_t sr[BN];
-#pragma unroll
-                for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(c.tmem + lane_base + t * BN + cc * 32, sr + cc * 32);
-                tmem_ld_wait();
-                tmem_reg_fence<BN>(sr);
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&c.s_free[t]);
-                const int lo = klo - j * BN, hi = khi - j * BN;  // visible columns of this tile
-                const bool need_mask = __any_sync(0xffffffffu, lo > 0 || hi < BN);
-                if (need_mask) {
-#pragma unroll
-                    for (int i = 0; i < BN; ++i)
-                        if (i < lo || i >= hi) sr[i] = __float_as_uint(-INFINITY);
-                }
-                const float m_cand = row_max<BN>(sr) * sc;
-                const bool grow = m_cand > m + 8.0f;
-                float alpha = 1.f;
-                if (grow) {
-                    alpha = ex2_approx(m - m_cand);
-                    m = m_cand;
-                }
-                const bool warp_grow = __any_sync(0xffffffffu, grow);
-                uint32_t pk[BN / 2];
-                // a packed row may not have met any visible key yet (m = -inf): its P is 0
-                const float neg_m = (m == -INFINITY) ? 0.f : -m;
-                const float rs = need_mask ? softmax_row_to_regs<BN, BF16, 0>(sr, sc, neg_m, pk)
-                                           : softmax_row_to_regs<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, pk);
-                l = fmaf(l, alpha, rs);
-                if (jj > 0) {
-                    if (!__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (jj - 1) & 1, c.abort_flag, c.lim, 340 + t))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    if (warp_grow) {
-                        const uint64_t a2 = f2(alpha, alpha);
-#pragma unroll 1
-                        for (int cc = 0; cc < D / 32; ++cc) {
-                            uint32_t o[32];
-                            tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
-                            tmem_ld_wait();
-                            tmem_reg_fence<32>(o);
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                float lo, hi;
-                                f2_split(fmul2(f2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), lo, hi);
-                                o[2 * i] = __float_as_uint(lo);
-                                o[2 * i + 1] = __float_as_uint(hi);
-                            }
-                            tmem_st32(c.tmem + lane_base + o_col + cc * 32, o);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int cc = 0; cc < BN / 64; ++cc) tmem_st32(p_addr + cc * 32, pk + cc * 32);
-                tmem_st_wait();
-                tc_fence_before_sync();
-                mbar_arrive(&c.p_full[t]);
-            }
-        } else
-        for (int jj = 0; jj < n; ++jj) {
-            const int j = j0 + jj;  // key tile
-            const int b = c.buf(t, jj);
-            if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[b], c.sphase(jj), c.abort_flag, c.lim, 300 + t))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after_sync();
-            uint32_t sr[BN];
-#pragma unroll
-            for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(c.tmem + lane_base + b * BN + cc * 32, sr + cc * 32);
-            tmem_ld_wait();
-            tmem_reg_fence<BN>(sr);
-            const int lo = klo - j * BN, hi = khi - j * BN;  // visible columns of this tile
-            const bool need_mask = __any_sync(0xffffffffu, lo > 0 || hi < BN);
-            if (need_mask) {
-#pragma unroll
-                for (int i = 0; i < BN; ++i)
-                    if (i < lo || i >= hi) sr[i] = __float_as_uint(-INFINITY);
-            }
-            const float mx = row_max<BN>(sr);
-            const float m_cand = mx * sc;
-            const bool grow = m_cand > m + 8.0f;
-            float alpha = 1.f;
-            if (grow) {
-                alpha = ex2_approx(m - m_cand);
-                m = m_cand;
-            }
-            const bool warp_grow = __any_sync(0xffffffffu, grow);
-            // P = 2^(s*sc - m): written back to TMEM over S, 64 columns at a time.
-            // a packed row may not have met any visible key yet (m = -inf): its P is 0
-            const float neg_m = (m == -INFINITY) ? 0.f : -m;
-            const uint32_t p_addr = c.tmem + lane_base + b * BN;
-            const float rs = need_mask ? softmax_chunk_store<BN, BF16, 0>(sr, sc, neg_m, p_addr)  // -inf -> exactly 0
-                                       : softmax_chunk_store<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, p_addr);
-            l = fmaf(l, alpha, rs);
-            tmem_st_wait();
-            if (jj > 0) {
-                // The previous PV is waited for on every step (it has normally finished long
-                // before), so this thread never falls two phases behind on pv_done.
-                if (!__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (jj - 1) & 1, c.abort_flag, c.lim, 310 + t))) {
-                    ok = false;
-                    break;
-                }
-                if (warp_grow) {
-                    // O holds sum_{j' < j} P_j' V_j'; bring it to the new running max.
-                    tc_fence_after_sync();
-#pragma unroll 1
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
-                        tmem_ld_wait();
-                        tmem_reg_fence<32>(o);
-                        const uint64_t a2 = f2(alpha, alpha);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float lo, hi;
-                            f2_split(fmul2(f2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), lo, hi);
-                            o[2 * i] = __float_as_uint(lo);
-                            o[2 * i + 1] = __float_as_uint(hi);
-                        }
-                        tmem_st32(c.tmem + lane_base + o_col + cc * 32, o);
-                    }
-                    tmem_st_wait();
-                }
-            }
-            tc_fence_before_sync();
-            mbar_arrive(&c.p_full[b]);
-        }
-        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (n - 1) & 1, c.abort_flag, c.lim, 320 + t));
-        if (ok) {
-            tc_fence_after_sync();
-            const float inv_l = 1.f / l;
-            int64_t orow_idx = (p.gather && row_ok) ? __ldg(p.gather + tok) : tok;  // fused: padded row
-            const bool store_ok = row_ok && (!p.gather || (orow_idx >= 0 && orow_idx < p.padded_rows));
-            uint4 *orow = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) +
-                                                    (orow_idx * p.H + h) * static_cast<int64_t>(D) * 2);
-#pragma unroll 1
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t o[32];
-                tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
-                tmem_ld_wait();
-                tmem_reg_fence<32>(o);
-                uint32_t w[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    w[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-                if (store_ok) {
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        orow[cc * 4 + v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
-                }
-            }
-            if (row_ok && p.lse) {
-                const float lse = m * 0.6931471805599453f + logf(l);
-                const int64_t li = packed ? static_cast<int64_t>(h) * p.total_tokens + tok
-                                          : (static_cast<int64_t>(blockIdx.z) * p.H + h) * p.seqlen + (tok - seq_start);
-                p.lse[li] = lse;
-            }
-            if (p.gather) {
-                // Fused pad: this warp's 32 tokens own the padded rows from just after the
-                // previous token's row up to their last row (through the end of the tensor for
-                // the last token, from row 0 for the first); rows no token maps to become 0.
-                const int64_t tw0 = static_cast<int64_t>(qbase) + t * BM + quarter * 32;
-                if (tw0 < p.total_tokens) {
-                    const int64_t tw1 = min(tw0 + 32, static_cast<int64_t>(p.total_tokens)) - 1;
-                    // padded rows of this warp's tokens, sorted (lanes past the last token: +inf)
-                    const int64_t g_lane = (tw0 + lane <= tw1) ? __ldg(p.gather + tw0 + lane) : INT64_MAX;
-                    const int64_t lo_row = max(int64_t(0), (tw0 == 0) ? int64_t(0) : __ldg(p.gather + tw0 - 1) + 1);
-                    const int64_t hi_row =
-                        min(p.padded_rows, (tw1 == p.total_tokens - 1) ? p.padded_rows : __ldg(p.gather + tw1));
-                    constexpr int VEC = D * 2 / 16;  // 16-byte vectors per row of one head
-                    for (int64_t base = lo_row; base < hi_row; base += 32) {
-                        const int64_t pr = base + lane;
-                        // is pr one of the 32 mapped rows? binary search over the lanes' sorted values
-                        int lo = 0;
-#pragma unroll
-                        for (int step = 16; step >= 1; step >>= 1) {
-                            const int64_t v = __shfl_sync(0xffffffffu, g_lane, lo + step - 1);
-                            if (v < pr) lo += step;
-                        }
-                        const bool mapped = __shfl_sync(0xffffffffu, g_lane, lo & 31) == pr;
-                        if (pr < hi_row && !mapped) {
-                            uint4 *row = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) +
-                                                                   (pr * p.H + h) * static_cast<int64_t>(D) * 2);
-#pragma unroll
-                            for (int v4 = 0; v4 < VEC; ++v4) row[v4] = make_uint4(0, 0, 0, 0);
-                        }
-                    }
-                }
-            }
-        }
-    }
-
-    tc_fence_before_sync();
-    __syncthreads();
-    if (warp == C::WARP_MMA) {
-        tc_fence_after_sync();
-        tmem_dealloc(c.tmem, C::TMEM_COLS);
-    }
-}
 
 // One CTA waits on a barrier that nothing completes; the bounded wait must give up.
 __global__ void fa_selftest_wait_kernel(uint64_t limit_ns) {
@@ -939,40 +18,11 @@ __global__ void fa_selftest_wait_kernel(uint64_t limit_ns) {
     if (threadIdx.x == 0) wait_bounded(&bar, 0, &abort_flag, limit_ns, 900);
 }
 
-// ------------------------------------------------------------------ host launchers
-template <int D, bool BF16, bool CAUSAL>
-static cudaError_t launch_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                            const FwdParams &p, dim3 grid, cudaStream_t st) {
-    using C = Cfg<D>;
-    auto kern = fa_fwd_kernel<D, BF16, CAUSAL>;
-    // The shared-memory opt-in is a per-device function attribute; setting it twice is harmless.
-    static uint64_t attr_set_mask = 0;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    const uint64_t bit = uint64_t(1) << (dev & 63);
-    if (!(__atomic_load_n(&attr_set_mask, __ATOMIC_ACQUIRE) & bit)) {
-        if (C::SPLIT_REGS) {
-            // The per-warpgroup register split draws on the registers the CTA launches with.
-            cudaFuncAttributes fa_attr;
-            e = cudaFuncGetAttributes(&fa_attr, kern);
-            if (e != cudaSuccess) return e;
-            if (fa_attr.numRegs * C::NUM_THREADS < 128 * C::REGS_LOW + 256 * C::REGS_HIGH)
-                return cudaErrorInvalidConfiguration;
-        }
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        __atomic_fetch_or(&attr_set_mask, bit, __ATOMIC_RELEASE);
-    }
-    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
-    return cudaGetLastError();
-}
-
 template <int D, bool BF16>
 static cudaError_t launch_c(bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
                             const CUtensorMap &tv, const FwdParams &p, dim3 grid, cudaStream_t st) {
-    return causal ? launch_t<D, BF16, true>(tq, tk, tv, p, grid, st)
-                  : launch_t<D, BF16, false>(tq, tk, tv, p, grid, st);
+    return causal ? launch_t<D, BF16, true, false>(tq, tk, tv, p, grid, st)
+                  : launch_t<D, BF16, false, false>(tq, tk, tv, p, grid, st);
 }
 
 template <int D>
@@ -1001,21 +51,14 @@ int fwd_box_inner_elems(int D) { return (2 * D >= 128) ? 64 : D; }
 
 int fwd_kv_tile_rows(int D) { return 128; }
 int fwd_v_box_rows(int D) { return (D == 256) ? 64 : 128; }
+int fwd_paged_k_box_rows(int D, int page_size) { return page_size < fwd_kv_tile_rows(D) ? page_size : fwd_kv_tile_rows(D); }
+int fwd_paged_v_box_rows(int D, int page_size) { return page_size < fwd_v_box_rows(D) ? page_size : fwd_v_box_rows(D); }
 
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t st) {
     fa_selftest_wait_kernel<<<1, 32, 0, st>>>(limit_ns);
     return cudaGetLastError();
 }
 
-cudaError_t fwd_take_device_error(int *code, int *where) {
-    int zero = 0;
-    cudaError_t e = cudaMemcpyFromSymbol(code, g_err_code, sizeof(int));
-    if (e != cudaSuccess) return e;
-    e = cudaMemcpyFromSymbol(where, g_err_where, sizeof(int));
-    if (e != cudaSuccess) return e;
-    e = cudaMemcpyToSymbol(g_err_code, &zero, sizeof(int));
-    if (e != cudaSuccess) return e;
-    return cudaMemcpyToSymbol(g_err_where, &zero, sizeof(int));
-}
+cudaError_t fwd_take_device_error(int *code, int *where) { return take_device_error(code, where); }
 
 }  // namespace fa

@@ -22,6 +22,14 @@ struct FwdParams {
     int total_tokens;           // N = rows of the token-major tensors
     float scale_log2;           // scale * log2(e)
     uint64_t timeout_ns;        // bound of every pipeline wait
+    // Paged K/V (dense queries only; null otherwise): k and v are pools of num_pages pages of
+    // page_size token rows, (num_pages * page_size, H, D); key position pos of batch entry b
+    // lives in page block_table[b * max_blocks + pos / page_size], row pos % page_size.
+    const int32_t *block_table;
+    int max_blocks;
+    int page_size;   // a power of two
+    int page_shift;  // log2(page_size)
+    int num_pages;
 };
 
 // Attention forward. Dense: grid (H, ceil(ceil(S / 128) / tiles_per_cta), B), a CTA owns
@@ -29,14 +37,21 @@ struct FwdParams {
 // (H, ceil(total / (128 * tiles_per_cta)), 1), a CTA owns that many consecutive packed tokens.
 cudaError_t launch_fwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
                        const CUtensorMap &tv, const FwdParams &p, dim3 grid, cudaStream_t st);
+// The same with p.block_table set (paged K/V; maps tk/tv cover the page pools).
+cudaError_t launch_fwd_paged(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
+                             const CUtensorMap &tv, const FwdParams &p, dim3 grid, cudaStream_t st);
 int fwd_tile_rows();
 int fwd_tiles_per_cta(int D);
 int fwd_box_inner_elems(int D);
 int fwd_kv_tile_rows(int D);
 // Rows of one V box the producer copies (a V tile may move as several row parts).
 int fwd_v_box_rows(int D);
+// Paged K/V: rows per K box / V box for a page size (a box never crosses a page).
+int fwd_paged_k_box_rows(int D, int page_size);
+int fwd_paged_v_box_rows(int D, int page_size);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t st);
 cudaError_t fwd_take_device_error(int *code, int *where);
+cudaError_t fwd_paged_take_device_error(int *code, int *where);
 
 // Unpad / pad (row gather / scatter + zero fill).
 cudaError_t launch_unpad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
