@@ -277,6 +277,9 @@ def run_ours(args):
     h2d = 3 * q_h.numel() * q_h.element_size()
     d2h = op.numel() * op.element_size() + lp.numel() * 4
 
+    # ---- the same problem with K/V in page pools (block table), per page size
+    paged = run_paged_leg(fa, device, stream, q, k_h, v_h, causal, flops, args.warmup, rank)
+
     # ---- packed path (unpad x3, varlen forward, pad), microseconds per call
     varlen = run_varlen_leg(fa, device, stream, max(args.steps, 20), args.warmup, ws)
     padding = run_padding_hbm_leg(fa, device, stream, 20)
@@ -307,6 +310,7 @@ def run_ours(args):
                      "kernel": "fa_fwd_kernel<128,bf16,causal>",
                      "traffic": recorded_traffic("fa_fwd_kernel_d128_bf16_causal")},
         "varlen": varlen,
+        "paged": paged,
         "unpad_pad_hbm": padding,
         "clocks": clocks,
     }
@@ -320,6 +324,39 @@ def run_ours(args):
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_paged_leg(fa, device, stream, q, k_h, v_h, causal, flops, warmup, rank, iters=20):
+    """fa_fwd_paged on the main workload with K/V scattered over shuffled page pools."""
+    res = {"what": "the main workload with K/V in page pools (shuffled page order, block table), "
+                   "fa_fwd_paged; TFLOPS and fraction of contiguous fa_fwd timed the same way",
+           "launches_per_size": iters}
+    out = torch.empty_like(q)
+    k, v = k_h.to(device), v_h.to(device)
+
+    def timed(call):
+        for _ in range(warmup):
+            call()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return flops / (e0.elapsed_time(e1) / iters * 1e-3) / 1e12
+
+    dense_tflops = timed(lambda: fa.fa_fwd(q, k, v, out=out, causal=causal, return_lse=False, stream=stream))
+    res["contiguous_tflops"] = round(dense_tflops, 1)
+    del k, v
+    for ps in (16, 64, 256):
+        kc, vc, table = fa_inputs.paged_kv(k_h, v_h, ps, seed=rank + 1, fill=0.0)
+        kc, vc, table = kc.to(device), vc.to(device), table.to(device)
+        tf = timed(lambda: fa.fa_fwd_paged(q, kc, vc, table, out=out, causal=causal, return_lse=False,
+                                           stream=stream))
+        res[f"page_{ps}"] = {"tflops": round(tf, 1), "frac_of_contiguous": round(tf / dense_tflops, 3)}
+        del kc, vc, table
+    return res
 
 
 def run_varlen_leg(fa, device, stream, iters, warmup, ws):
