@@ -277,6 +277,9 @@ def run_ours(args):
     h2d = 3 * q_h.numel() * q_h.element_size()
     d2h = op.numel() * op.element_size() + lp.numel() * 4
 
+    # ---- the backward pass of the same problem (recomputation from the saved LSE)
+    backward = run_backward_leg(fa, device, stream, q, k, v, out, lse, causal, args.warmup, rank)
+
     # ---- the same problem with K/V in page pools (block table), per page size
     paged = run_paged_leg(fa, device, stream, q, k_h, v_h, causal, flops, args.warmup, rank)
 
@@ -311,6 +314,7 @@ def run_ours(args):
                      "traffic": recorded_traffic("fa_fwd_kernel_d128_bf16_causal")},
         "varlen": varlen,
         "paged": paged,
+        "backward": backward,
         "unpad_pad_hbm": padding,
         "clocks": clocks,
     }
@@ -324,6 +328,39 @@ def run_ours(args):
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_backward_leg(fa, device, stream, q, k, v, out, lse, causal, warmup, rank, iters=10):
+    """fa_bwd on the main workload: TFLOPS by the usual 2.5x-forward convention."""
+    B, S, H, D = q.shape
+    do = fa_inputs.normal(tuple(q.shape), q.dtype, seed=rank + 100).to(device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    delta = torch.empty((B, H, S), device=device, dtype=torch.float32)
+    fa.fa_fwd(q, k, v, out=out, lse=lse, causal=causal, stream=stream)
+
+    def call():
+        fa.fa_bwd(q, k, v, out, do, lse, dq=dq, dk=dk, dv=dv, delta=delta, causal=causal, stream=stream)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(iters):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / iters
+    flops = fa.attention_bwd_flops(B, H, S, D, causal)
+    st, where = fa.fa_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} at {where} after the backward leg")
+    peak_burst, _, _, _ = load_peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"what": "fa_bwd (delta, dK/dV and dQ kernels) on the main workload; FLOPs = 2.5x the forward's "
+                    "(five S x S x D products; the dQ kernel recomputes two of them, not counted)",
+            "ms": round(ms, 4), "tflops": round(tf, 1), "frac_vs_burst": round(tf / peak_burst, 4),
+            "launches": 3 * iters}
 
 
 def run_paged_leg(fa, device, stream, q, k_h, v_h, causal, flops, warmup, rank, iters=20):

@@ -95,6 +95,25 @@ FA_API fa_status fa_fwd_paged(const void *q, const void *k_cache, const void *v_
                               float scale, int causal, fa_dtype dtype, void *stream);
 
 /*
+ * Dense attention backward: the gradients of out = softmax(scale * q k^T) v (causal mask as
+ * in fa_fwd) with respect to q, k and v, by recomputation from the forward's LSE (page
+ * "昇腾CANN跑大模型，FlashAttention这个算子你得认识一下", section "分块计算，这事没那么简单",
+ * second pitfall: the scores are not stored, the backward pass computes them again).
+ *   q, k, v, out   (B, S, H, D) forward inputs and output, element type `dtype`.
+ *   dout           (B, S, H, D) gradient of the loss with respect to out.
+ *   lse            (B, H, S) float32 log-sum-exp written by fa_fwd for the same inputs.
+ *   dq, dk, dv     (B, S, H, D) outputs, element type `dtype`; every element is written.
+ *   delta          (B, H, S) float32 caller-owned workspace; on return it holds
+ *                  rowsum(dout * out), the per-row term of the softmax derivative.
+ *   scale          <= 0 selects 1/sqrt(D); must be the value the forward used.
+ * D in {32, 64, 128} (the dK and dV accumulators of a 128-key tile share TMEM; D = 256 is
+ * FA_ERR_HEADDIM). Three launches on `stream` (delta, dK/dV, dQ); nothing is allocated.
+ */
+FA_API fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
+                        const float *lse, void *dq, void *dk, void *dv, float *delta, int B, int H, int S,
+                        int D, float scale, int causal, fa_dtype dtype, void *stream);
+
+/*
  * Packed variable-length attention forward (the flash_attn_varlen_func step).
  *   q, k, v      (total, H, D) packed inputs; sequence s owns rows
  *                [cu_seqlens[s], cu_seqlens[s+1]) and attends only inside itself.

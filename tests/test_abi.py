@@ -126,3 +126,26 @@ def test_paged_validation(lib):
     assert call(table=FAKE + 2) == -5
     assert call(q=FAKE + 8) == -5
     assert call(B=0) == -2
+
+
+def test_bwd_validation(lib):
+    f = lib.fa_bwd
+    # q, k, v, out, dout, lse, dq, dk, dv, delta, B, H, S, D, scale, causal, dtype, stream
+    ok = [FAKE] * 10 + [2, 4, 130, 128, 0.0, 1, 1, None]
+
+    def call(i=None, val=None):
+        a = list(ok)
+        if i is not None:
+            a[i] = val
+        return f(*a)
+
+    for i in range(10):
+        assert call(i, None) == -1, i
+    assert call(13, 256) == -4   # dK and dV accumulators would not fit in TMEM
+    assert call(13, 96) == -4
+    assert call(16, 3) == -3
+    assert call(10, 0) == -2
+    assert call(12, 0) == -2
+    assert call(0, FAKE + 8) == -5
+    assert call(5, FAKE + 2) == -5
+    assert call(9, FAKE + 2) == -5

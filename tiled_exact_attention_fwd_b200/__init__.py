@@ -7,6 +7,7 @@ built, every call raises.
     out, lse = fa_fwd(q, k, v, causal=True)                         # dense (B, S, H, D)
     out, lse = fa_varlen_fwd(q, k, v, cu_seqlens, max_seqlen)        # packed (total, H, D)
     out, lse = fa_fwd_paged(q, k_cache, v_cache, block_table)        # K/V in a page pool
+    dq, dk, dv = fa_bwd(q, k, v, out, dout, lse, causal=True)        # gradients (recomputation)
     x_unpad  = fa_unpad(x, indices)                                  # (B, L, H, D) -> (nnz, H, D)
     x_pad    = fa_pad(x_unpad, indices, batch, total_len)            # (nnz, H, D) -> (B, L, H, D)
 """
@@ -47,6 +48,7 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
         L.fa_varlen_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, i32, i32, f32, i32, i32, vp]
         L.fa_fwd_paged.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
+        L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
         L.fa_unpad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fa_pad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fa_unpad_qkv.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp]
@@ -54,7 +56,7 @@ def lib() -> ctypes.CDLL:
                                            vp]
         L.fa_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.fa_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
-        for f in (L.fa_fwd, L.fa_fwd_paged, L.fa_varlen_fwd, L.fa_varlen_fwd_padded, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad,
+        for f in (L.fa_fwd, L.fa_fwd_paged, L.fa_bwd, L.fa_varlen_fwd, L.fa_varlen_fwd_padded, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad,
                   L.fa_device_status,
                   L.fa_selftest_bounded_wait):
             f.restype = ctypes.c_int
@@ -118,6 +120,38 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torc
                       float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
     _check(st, "fa_fwd")
     return out, lse
+
+
+def fa_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
+           lse: torch.Tensor, dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+           dv: Optional[torch.Tensor] = None, delta: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+           causal: bool = False, stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Dense backward: gradients (dq, dk, dv), each (B, S, H, D), of out = fa_fwd(q, k, v) given
+    dout and the forward's lse (B, H, S). `delta` is an optional fp32 (B, H, S) workspace."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse)):
+        _cuda_contig(n, t)
+    if q.dim() != 4 or any(t.shape != q.shape or t.dtype != q.dtype for t in (k, v, out, dout)):
+        raise ValueError("q, k, v, out, dout must share one (B, S, H, D) shape and dtype")
+    B, S, H, D = q.shape
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, S):
+        raise ValueError("lse must be float32 (B, H, S)")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if delta is None:
+        delta = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv), ("delta", delta)):
+        _cuda_contig(n, t)
+    st = lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                      _ptr(delta), B, H, S, D, float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q),
+                      _stream(stream))
+    _check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def attention_bwd_flops(B: int, H: int, S: int, D: int, causal: bool) -> float:
+    """Backward FLOPs by the usual convention: 2.5x the forward (five S x S x D products)."""
+    return 2.5 * attention_flops(B, H, S, S, D, causal)
 
 
 def fa_fwd_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.Tensor,

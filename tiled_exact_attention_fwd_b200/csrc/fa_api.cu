@@ -170,6 +170,43 @@ fa_status fa_fwd_paged(const void *q, const void *k_cache, const void *v_cache, 
                    &paging);
 }
 
+fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+                 void *dq, void *dk, void *dv, float *delta, int B, int H, int S, int D, float scale, int causal,
+                 fa_dtype dtype, void *stream) {
+    if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !delta) return FA_ERR_NULL;
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;  // dK and dV accumulators share TMEM
+    if (B <= 0 || H <= 0 || S <= 0) return FA_ERR_SHAPE;
+    const int64_t N = static_cast<int64_t>(B) * S;
+    if (N > INT32_MAX || B > 65535 || (S + 127) / 128 > 65535) return FA_ERR_SHAPE;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(dout, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(delta, 4))
+        return FA_ERR_ALIGN;
+    const bool bf16 = dtype == FA_BF16;
+    const int inner = fa::fwd_box_inner_elems(D);
+    CUtensorMap tq, tk, tv, tdo;
+    if (!encode_map(&tq, q, bf16, D, H, N, inner, 128) || !encode_map(&tk, k, bf16, D, H, N, inner, 128) ||
+        !encode_map(&tv, v, bf16, D, H, N, inner, 128) || !encode_map(&tdo, dout, bf16, D, H, N, inner, 128))
+        return FA_ERR_CUDA;
+    if (!(scale > 0.f)) scale = 1.0f / sqrtf(static_cast<float>(D));
+    fa::BwdParams p;
+    p.out = out;
+    p.dout = dout;
+    p.lse = lse;
+    p.delta = delta;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.B = B;
+    p.H = H;
+    p.seqlen = S;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.timeout_ns = wait_limit_ns();
+    const cudaError_t e = fa::launch_bwd(D, bf16, causal != 0, tq, tk, tv, tdo, p, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status fa_varlen_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqlens, int num_seqs,
                         int max_seqlen, int total, void *out, float *lse, int H, int D, float scale, int causal,
                         fa_dtype dtype, void *stream) {
@@ -250,11 +287,12 @@ fa_status fa_pad(const void *x, const int64_t *indices, int64_t nnz, int64_t tot
 fa_status fa_device_status(int *where) {
     if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
     // every kernel family keeps its own word; all are read (and so cleared), the first set wins
-    int code[3] = {0, 0, 0}, w[3] = {0, 0, 0};
+    int code[4] = {0, 0, 0, 0}, w[4] = {0, 0, 0, 0};
     if (fa::fwd_take_device_error(&code[0], &w[0]) != cudaSuccess) return FA_ERR_CUDA;
     if (fa::fwd_paged_take_device_error(&code[1], &w[1]) != cudaSuccess) return FA_ERR_CUDA;
-    if (fa::pad_take_device_error(&code[2], &w[2]) != cudaSuccess) return FA_ERR_CUDA;
-    for (int i = 0; i < 3; ++i)
+    if (fa::bwd_take_device_error(&code[2], &w[2]) != cudaSuccess) return FA_ERR_CUDA;
+    if (fa::pad_take_device_error(&code[3], &w[3]) != cudaSuccess) return FA_ERR_CUDA;
+    for (int i = 0; i < 4; ++i)
         if (code[i]) {
             if (where) *where = w[i];
             return static_cast<fa_status>(code[i]);

@@ -1,0 +1,477 @@
+// fa_bwd.cu -- attention backward on sm_100a: gradients dQ, dK, dV of O = softmax(Z) V,
+// Z = scale * Q K^T, by recomputation (page "昇腾CANN跑大模型，FlashAttention这个算子你得认识一下",
+// section "分块计算，这事没那么简单", second pitfall: the score matrix is never stored, the
+// backward pass recomputes it from Q, K and the saved log-sum-exp).
+//
+// Per (batch, head), with P = exp(Z - lse) recomputed tile by tile:
+//   delta_i = sum_d dO_id O_id                    (bwd_delta_kernel; equals rowsum(P * dP))
+//   dV = P^T dO,  dP = dO V^T,  dZ = P * (dP - delta),  dQ = scale dZ K,  dK = scale dZ^T Q
+//
+// Two tcgen05 kernels, one template (no atomics, no accumulation workspace):
+//   dK/dV: a CTA owns one 128-row key tile j (K_j, V_j stay in shared memory) and streams the
+//          query tiles i >= j (causal) or all of them through a two-stage TMA ring:
+//            S^T  = K_j Q_i^T, dP^T = V_j dO_i^T        (SS MMAs, fp32 in TMEM)
+//            P^T, dZ^T (16-bit) over S^T, dP^T in TMEM  (4 elementwise warps, thread = key)
+//            dV  += P^T dO_i,  dK += dZ^T Q_i           (TS MMAs, A from TMEM)
+//   dQ:    a CTA owns one 128-row query tile i (Q_i, dO_i stay) and streams key tiles j <= i:
+//            S = Q_i K_j^T, dP = dO_i V_j^T;  dZ over S;  dQ += dZ K_j
+// Warps 0-3 do the elementwise work (thread = TMEM lane = one row), warp 4 lane 0 issues the
+// TMA loads, warp 5 allocates TMEM and lane 0 issues every MMA. Every wait is bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "fa.h"
+#include "fa_internal.h"
+#include "fa_ptx.cuh"
+#include "fa_sync.cuh"
+
+namespace fa {
+namespace {
+
+template <int D>
+struct BwdCfg {
+    static constexpr int BM = 128;                           // rows of every tile
+    static constexpr int SW = (2 * D >= 128) ? 128 : 2 * D;  // swizzle span in bytes
+    static constexpr int SWE = SW / 2;                       // 16-bit elements per swizzle row
+    static constexpr int NBLK = D / SWE;                     // column blocks per tile row
+    static constexpr int TILE_BYTES = BM * D * 2;
+    static constexpr uint32_t LAYOUT = (SW == 128) ? kLayoutSw128 : kLayoutSw64;
+    static constexpr int NUM_THREADS = 192;
+    static constexpr int WARP_TMA = 4, WARP_MMA = 5;
+    // shared memory: fixed tiles A0, A1; ring stages s = 0, 1 holding tiles B0, B1;
+    // per-column statistics (dK/dV kernel) in two slots; barriers; misc
+    static constexpr int OFF_FIX = 0;
+    static constexpr int OFF_RING = 2 * TILE_BYTES;
+    static constexpr int OFF_STAT = OFF_RING + 4 * TILE_BYTES;  // [slot][-lse*log2e | -delta][128]
+    static constexpr int OFF_BAR = OFF_STAT + 2 * 2 * BM * 4;
+    // fix_full, ring_full[2], ring_empty[2], s_full, p_ready, done, drain, stats_ready[2]
+    static constexpr int NUM_BARS = 11;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int USED = OFF_MISC + 16;
+    static constexpr int MIN_SMEM = 120 * 1024;  // one CTA (and one TMEM allocation) per SM
+    static constexpr int SMEM_BYTES = (USED + 1024 > MIN_SMEM) ? USED + 1024 : MIN_SMEM;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr int COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
+    static_assert(USED + 1024 <= 227 * 1024, "shared memory budget");
+    static_assert(COL_ACC1 + D <= (int)TMEM_COLS, "TMEM budget (dK and dV accumulators)");
+    static_assert(TILE_BYTES % 1024 == 0, "tile alignment");
+};
+
+// Loads of one 128-row tile of a token-major (N, H, D) tensor: NBLK boxes side by side.
+template <int D>
+__device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int h, int row,
+                                          uint64_t pol) {
+    using C = BwdCfg<D>;
+#pragma unroll
+    for (int b = 0; b < C::NBLK; ++b) tma_load_3d(dst + b * C::BM * C::SW, map, bar, b * C::SWE, h, row, pol);
+}
+
+// D_out (+)= A B^T over the head dimension: A, B K-major 128-row tiles in shared memory.
+template <int D, bool BF16>
+__device__ __forceinline__ void mma_rows(uint32_t d_tmem, const uint8_t *a, const uint8_t *b) {
+    using C = BwdCfg<D>;
+    constexpr uint32_t idesc = idesc_f16(C::BM, C::BM, BF16, false);
+    const uint32_t a0 = smem_u32(a), b0 = smem_u32(b);
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+        const uint32_t blk = (k * 32) / C::SW, off = (k * 32) % C::SW;
+        umma_ss(d_tmem, smem_desc(a0 + blk * C::BM * C::SW + off, 16, 8 * C::SW, C::LAYOUT),
+                smem_desc(b0 + blk * C::BM * C::SW + off, 16, 8 * C::SW, C::LAYOUT), idesc, k > 0 ? 1u : 0u);
+    }
+}
+
+// D_out (+)= A_tmem B over 128 rows: A (128 x 128, 16-bit) in TMEM, B a 128-row tile read
+// MN-major (its D columns are the output columns).
+template <int D, bool BF16>
+__device__ __forceinline__ void mma_acc(uint32_t d_tmem, uint32_t a_tmem, const uint8_t *b, bool accumulate) {
+    using C = BwdCfg<D>;
+    constexpr uint32_t idesc = idesc_f16(C::BM, D, BF16, true);
+    const uint32_t b0 = smem_u32(b);
+#pragma unroll
+    for (int k = 0; k < C::BM / 16; ++k)
+        umma_ts(d_tmem, a_tmem + k * 8, smem_desc(b0 + k * 16 * C::SW, C::BM * C::SW, 8 * C::SW, C::LAYOUT), idesc,
+                (accumulate || k > 0) ? 1u : 0u);
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2b(float lo, float hi) {
+    return BF16 ? pack2_bf16(lo, hi) : pack2_f16(lo, hi);
+}
+
+// One row of a TMEM accumulator (D fp32 columns) times `mul` -> 16-bit -> global.
+template <int D, bool BF16>
+__device__ __forceinline__ void store_row(uint32_t taddr, float mul, uint8_t *grow, bool store) {
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(taddr + cc * 32, o);
+        tmem_ld_wait();
+        tmem_reg_fence<32>(o);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = pack2b<BF16>(__uint_as_float(o[2 * i]) * mul, __uint_as_float(o[2 * i + 1]) * mul);
+        if (store) {
+            uint4 *g = reinterpret_cast<uint4 *>(grow) + cc * 4;
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) g[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+        }
+    }
+}
+
+// DKDV: the CTA owns key tile j = blockIdx.y; fixed A0 = K_j, A1 = V_j; ring B0 = Q_i, B1 = dO_i.
+// !DKDV: the CTA owns query tile i (longest first); fixed A0 = Q_i, A1 = dO_i; ring B0 = K_j, B1 = V_j.
+template <int D, bool BF16, bool CAUSAL, bool DKDV>
+__global__ void __launch_bounds__(BwdCfg<D>::NUM_THREADS, 1)
+fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+              const BwdParams p) {
+    using C = BwdCfg<D>;
+    constexpr int BM = C::BM;
+    const int h = blockIdx.x, b = blockIdx.z, S = p.seqlen;
+    const int ntiles = (S + BM - 1) / BM;
+    const int own = DKDV ? static_cast<int>(blockIdx.y) : ntiles - 1 - static_cast<int>(blockIdx.y);
+    // tiles streamed through the ring: [t0, t1)
+    const int t0 = (DKDV && CAUSAL) ? own : 0;
+    const int t1 = (!DKDV && CAUSAL) ? own + 1 : ntiles;
+    const int n = t1 - t0;
+    const int64_t row0 = static_cast<int64_t>(b) * S;  // first token row of this batch entry
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *fixA0 = smem + C::OFF_FIX, *fixA1 = fixA0 + C::TILE_BYTES;
+    float *stats = reinterpret_cast<float *>(smem + C::OFF_STAT);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *fix_full = bars, *ring_full = bars + 1, *ring_empty = bars + 3, *s_full = bars + 5,
+             *p_ready = bars + 6, *done = bars + 7, *drain = bars + 8, *stats_ready = bars + 9;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    const uint64_t lim = p.timeout_ns;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto ring_tile = [&](int stage, int which) { return smem + C::OFF_RING + (2 * stage + which) * C::TILE_BYTES; };
+
+    if (threadIdx.x == 0) {
+        mbar_init(fix_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&ring_full[s], 1);
+            mbar_init(&ring_empty[s], 1);
+            mbar_init(&stats_ready[s], 128);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_ready, 128);
+        mbar_init(done, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == C::WARP_TMA && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_do);
+    }
+    if (warp == C::WARP_MMA) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+
+    if (warp == C::WARP_TMA) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0 && n > 0) {
+            const uint64_t pol_fix = l2_policy_evict_first();
+            const uint64_t pol_ring = l2_policy_evict_last();
+            const CUtensorMap *fa0 = DKDV ? &tm_k : &tm_q, *fa1 = DKDV ? &tm_v : &tm_do;
+            const CUtensorMap *rb0 = DKDV ? &tm_q : &tm_k, *rb1 = DKDV ? &tm_do : &tm_v;
+            mbar_arrive_expect_tx(fix_full, 2 * C::TILE_BYTES);
+            load_tile<D>(fixA0, fa0, fix_full, h, static_cast<int>(row0 + own * BM), pol_fix);
+            load_tile<D>(fixA1, fa1, fix_full, h, static_cast<int>(row0 + own * BM), pol_fix);
+            int issued = 0;
+            for (int t = 0; t < n; ++t) {
+                const int s = t & 1;
+                if (t >= 2 && !wait_bounded(&ring_empty[s], ((t >> 1) - 1) & 1, abort_flag, lim, 400 + s)) break;
+                mbar_arrive_expect_tx(&ring_full[s], 2 * C::TILE_BYTES);
+                const int row = static_cast<int>(row0 + (t0 + t) * BM);
+                load_tile<D>(ring_tile(s, 0), rb0, &ring_full[s], h, row, pol_ring);
+                load_tile<D>(ring_tile(s, 1), rb1, &ring_full[s], h, row, pol_ring);
+                issued = t + 1;
+            }
+            if (*abort_flag) {
+                // let the copies already issued land before shared memory goes away
+                const uint64_t g0 = global_timer_ns();
+                while (!mbar_try_wait(fix_full, 0) && global_timer_ns() - g0 < lim) {
+                }
+                for (int t = (issued > 2 ? issued - 2 : 0); t < issued; ++t) {
+                    const uint64_t g1 = global_timer_ns();
+                    while (!mbar_try_wait(&ring_full[t & 1], (t >> 1) & 1) && global_timer_ns() - g1 < lim) {
+                    }
+                }
+            }
+        }
+    } else if (warp == C::WARP_MMA) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && n > 0) {
+            ok = wait_bounded(fix_full, 0, abort_flag, lim, 410);
+            if (ok) tc_fence_after_sync();
+            for (int t = 0; ok && t < n; ++t) {
+                const int s = t & 1;
+                if (!(ok = wait_bounded(&ring_full[s], (t >> 1) & 1, abort_flag, lim, 420 + s))) break;
+                tc_fence_after_sync();
+                mma_rows<D, BF16>(tmem + C::COL_S, fixA0, ring_tile(s, 0));   // S (or S^T)
+                mma_rows<D, BF16>(tmem + C::COL_DP, fixA1, ring_tile(s, 1));  // dP (or dP^T)
+                umma_commit(s_full);
+                if (!(ok = wait_bounded(p_ready, t & 1, abort_flag, lim, 430))) break;
+                tc_fence_after_sync();
+                if (DKDV) {
+                    mma_acc<D, BF16>(tmem + C::COL_ACC0, tmem + C::COL_S, ring_tile(s, 1), t > 0);   // dV += P^T dO
+                    mma_acc<D, BF16>(tmem + C::COL_ACC1, tmem + C::COL_DP, ring_tile(s, 0), t > 0);  // dK += dZ^T Q
+                } else {
+                    mma_acc<D, BF16>(tmem + C::COL_ACC0, tmem + C::COL_S, ring_tile(s, 0), t > 0);   // dQ += dZ K
+                }
+                umma_commit(&ring_empty[s]);
+            }
+            if (ok) umma_commit(done);
+            umma_commit(drain);  // every MMA issued above has finished once this arrives
+            const uint64_t g0 = global_timer_ns();
+            while (!mbar_try_wait(drain, 0) && global_timer_ns() - g0 < lim) {
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ elementwise warps 0-3
+        const int r = warp * 32 + lane;  // TMEM lane = row of the owned tile
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const int own_pos = own * BM + r;  // sequence position of this row (key or query)
+        const float sl2 = p.scale_log2;
+        constexpr float kLog2e = 1.4426950408889634f;
+        const int64_t stat_base = (static_cast<int64_t>(b) * p.H + h) * S;
+        // statistics of a query position: -lse*log2(e) and -delta (0 past the sequence end, which
+        // makes every weight of that query exactly 0)
+        auto query_stats = [&](int qpos, float &nl, float &nd) {
+            if (qpos < S) {
+                nl = -__ldg(p.lse + stat_base + qpos) * kLog2e;
+                nd = -__ldg(p.delta + stat_base + qpos);
+            } else {
+                nl = -INFINITY;
+                nd = 0.f;
+            }
+        };
+        float my_nl = 0.f, my_nd = 0.f;  // dQ: this row's statistics; dK/dV: prefetched column stats
+        if (DKDV) {
+            if (n > 0) query_stats(t0 * BM + r, my_nl, my_nd);
+        } else {
+            query_stats(own_pos, my_nl, my_nd);
+        }
+        for (int t = 0; ok && t < n; ++t) {
+            const int other = t0 + t;  // the streamed tile (query tile for dK/dV, key tile for dQ)
+            const int slot = t & 1;
+            float *snl = stats + slot * 2 * BM, *snd = snl + BM;
+            if (DKDV) {
+                // publish this thread's query column statistics, prefetch the next tile's
+                snl[r] = my_nl;
+                snd[r] = my_nd;
+                mbar_arrive(&stats_ready[slot]);
+                if (t + 1 < n) query_stats((other + 1) * BM + r, my_nl, my_nd);
+                if (!(ok = __all_sync(0xffffffffu, wait_bounded(&stats_ready[slot], (t >> 1) & 1, abort_flag, lim, 440))))
+                    break;
+            }
+            if (!(ok = __all_sync(0xffffffffu, wait_bounded(s_full, t & 1, abort_flag, lim, 450)))) break;
+            tc_fence_after_sync();
+            const bool diag = CAUSAL && other == own;
+            // dQ: keys past the sequence end weigh 0
+            const int key_hi = DKDV ? BM : min(BM, S - other * BM);
+#pragma unroll 1
+            for (int cc = 0; cc < BM / 32; ++cc) {
+                uint32_t sv[32], dv[32];
+                tmem_ld32(tmem + lane_base + C::COL_S + cc * 32, sv);
+                tmem_ld32(tmem + lane_base + C::COL_DP + cc * 32, dv);
+                tmem_ld_wait();
+                tmem_reg_fence<32>(sv);
+                tmem_reg_fence<32>(dv);
+                uint32_t pk[16], zk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int col = cc * 32 + 2 * i;
+                    float nl0, nl1, nd0, nd1;
+                    if (DKDV) {
+                        const float2 a = *reinterpret_cast<const float2 *>(snl + col);
+                        const float2 c2 = *reinterpret_cast<const float2 *>(snd + col);
+                        nl0 = a.x, nl1 = a.y, nd0 = c2.x, nd1 = c2.y;
+                    } else {
+                        nl0 = nl1 = my_nl;
+                        nd0 = nd1 = my_nd;
+                    }
+                    const uint64_t x2 = ffma2(f2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])),
+                                              f2(sl2, sl2), f2(nl0, nl1));
+                    float x0, x1;
+                    f2_split(x2, x0, x1);
+                    float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    // causal: key position > query position weighs 0 (only on the diagonal tile;
+                    // dK/dV rows are keys and columns queries, dQ the other way round)
+                    if (diag) {
+                        if (DKDV ? (r > col) : (col > r)) p0 = 0.f;
+                        if (DKDV ? (r > col + 1) : (col + 1 > r)) p1 = 0.f;
+                    }
+                    if (!DKDV) {
+                        if (col >= key_hi) p0 = 0.f;
+                        if (col + 1 >= key_hi) p1 = 0.f;
+                    }
+                    const uint64_t z2 = fmul2(f2(p0, p1), fadd2(f2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])),
+                                                                f2(nd0, nd1)));
+                    float z0, z1;
+                    f2_split(z2, z0, z1);
+                    pk[i] = pack2b<BF16>(p0, p1);
+                    zk[i] = pack2b<BF16>(z0, z1);
+                }
+                if (DKDV) {
+                    tmem_st16(tmem + lane_base + C::COL_S + cc * 16, pk);   // P^T over S^T
+                    tmem_st16(tmem + lane_base + C::COL_DP + cc * 16, zk);  // dZ^T over dP^T
+                } else {
+                    tmem_st16(tmem + lane_base + C::COL_S + cc * 16, zk);   // dZ over S
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before_sync();
+            mbar_arrive(p_ready);
+        }
+        if (ok && n > 0) ok = __all_sync(0xffffffffu, wait_bounded(done, 0, abort_flag, lim, 460));
+        if (ok) {
+            tc_fence_after_sync();
+            const bool store = own_pos < S;
+            const int64_t grow = (row0 + own_pos) * p.H + h;  // token row, head
+            if (DKDV) {
+                if (n > 0) {
+                    store_row<D, BF16>(tmem + lane_base + C::COL_ACC0, 1.f,
+                                       static_cast<uint8_t *>(p.dv) + grow * D * 2, store);
+                    store_row<D, BF16>(tmem + lane_base + C::COL_ACC1, p.scale,
+                                       static_cast<uint8_t *>(p.dk) + grow * D * 2, store);
+                } else if (store) {
+                    // no query sees these keys: zero gradients
+                    uint4 *gv = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.dv) + grow * D * 2);
+                    uint4 *gk = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.dk) + grow * D * 2);
+                    for (int i = 0; i < D / 8; ++i) gv[i] = gk[i] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            } else {
+                store_row<D, BF16>(tmem + lane_base + C::COL_ACC0, p.scale, static_cast<uint8_t *>(p.dq) + grow * D * 2,
+                                   store);
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == C::WARP_MMA) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// delta[b, h, s] = sum_d dO[b, s, h, d] * O[b, s, h, d] in fp32: D/8 lanes per (row, head),
+// 16-byte loads, a shuffle reduction. Warps stride over groups of 32/(D/8) consecutive
+// (row, head) items, so every lane of a warp runs the same number of iterations.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) bwd_delta_kernel(const void *out, const void *dout, float *delta, int64_t rows,
+                                                        int H, int S) {
+    constexpr int LPH = D / 8;           // lanes per (row, head)
+    constexpr int PER_WARP = 32 / LPH;   // items per warp and iteration
+    const int64_t items = rows * H;
+    const int lane = threadIdx.x & 31, sub = lane % LPH;
+    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * blockDim.x / 32;
+    for (int64_t base = warp0 * PER_WARP; base < items; base += nwarps * PER_WARP) {
+        const int64_t it = base + lane / LPH;
+        const bool live = it < items;
+        float acc = 0.f;
+        if (live) {
+            const uint4 o4 = ld_nc_v4(static_cast<const uint8_t *>(out) + (it * D + sub * 8) * 2);
+            const uint4 g4 = ld_nc_v4(static_cast<const uint8_t *>(dout) + (it * D + sub * 8) * 2);
+            const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w}, gw[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float2 of, gf;
+                if (BF16) {
+                    of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ow[i]));
+                    gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gw[i]));
+                } else {
+                    of = __half22float2(*reinterpret_cast<const __half2 *>(&ow[i]));
+                    gf = __half22float2(*reinterpret_cast<const __half2 *>(&gw[i]));
+                }
+                acc = fmaf(of.x, gf.x, acc);
+                acc = fmaf(of.y, gf.y, acc);
+            }
+        }
+#pragma unroll
+        for (int off = LPH / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (live && sub == 0) {
+            const int64_t row = it / H;  // token row b*S + s
+            const int hh = static_cast<int>(it % H);
+            const int64_t bb = row / S, ss = row % S;
+            delta[(bb * H + hh) * S + ss] = acc;
+        }
+    }
+}
+
+template <int D, bool BF16, bool CAUSAL, bool DKDV>
+cudaError_t launch_bwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
+                         const BwdParams &p, dim3 grid, cudaStream_t st) {
+    using C = BwdCfg<D>;
+    auto kern = fa_bwd_kernel<D, BF16, CAUSAL, DKDV>;
+    static uint64_t attr_set_mask = 0;  // per-device shared-memory opt-in done
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = uint64_t(1) << (dev & 63);
+    if (!(__atomic_load_n(&attr_set_mask, __ATOMIC_ACQUIRE) & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        __atomic_fetch_or(&attr_set_mask, bit, __ATOMIC_RELEASE);
+    }
+    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, tdo, p);
+    return cudaGetLastError();
+}
+
+template <int D, bool BF16>
+cudaError_t launch_bwd_d(bool causal, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                         const CUtensorMap &tdo, const BwdParams &p, cudaStream_t st) {
+    const int rows = p.B * p.seqlen;
+    const int64_t items = static_cast<int64_t>(rows) * p.H;
+    const int threads = 256;
+    int64_t blocks = (items * (D / 8) + threads - 1) / threads;  // one (row, head) per D/8 lanes
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    bwd_delta_kernel<D, BF16><<<static_cast<unsigned>(blocks), threads, 0, st>>>(p.out, p.dout, p.delta, rows, p.H,
+                                                                                 p.seqlen);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int ntiles = (p.seqlen + 127) / 128;
+    const dim3 grid(static_cast<unsigned>(p.H), static_cast<unsigned>(ntiles), static_cast<unsigned>(p.B));
+    e = causal ? launch_bwd_t<D, BF16, true, true>(tq, tk, tv, tdo, p, grid, st)
+               : launch_bwd_t<D, BF16, false, true>(tq, tk, tv, tdo, p, grid, st);
+    if (e != cudaSuccess) return e;
+    return causal ? launch_bwd_t<D, BF16, true, false>(tq, tk, tv, tdo, p, grid, st)
+                  : launch_bwd_t<D, BF16, false, false>(tq, tk, tv, tdo, p, grid, st);
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
+                       const CUtensorMap &tv, const CUtensorMap &tdo, const BwdParams &p, cudaStream_t st) {
+    switch (D) {
+        case 32: return bf16 ? launch_bwd_d<32, true>(causal, tq, tk, tv, tdo, p, st)
+                             : launch_bwd_d<32, false>(causal, tq, tk, tv, tdo, p, st);
+        case 64: return bf16 ? launch_bwd_d<64, true>(causal, tq, tk, tv, tdo, p, st)
+                             : launch_bwd_d<64, false>(causal, tq, tk, tv, tdo, p, st);
+        case 128: return bf16 ? launch_bwd_d<128, true>(causal, tq, tk, tv, tdo, p, st)
+                              : launch_bwd_d<128, false>(causal, tq, tk, tv, tdo, p, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t bwd_take_device_error(int *code, int *where) { return take_device_error(code, where); }
+
+}  // namespace fa

@@ -49,36 +49,9 @@
 #include "fa.h"
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
+#include "fa_sync.cuh"
 
 namespace fa {
-
-// Error word of this compilation unit's kernels (each unit that includes this header has its
-// own copy; take_device_error reads and clears it).
-static __device__ int g_err_code;
-static __device__ int g_err_where;
-
-static __device__ __noinline__ void record_error(int code, int where) {
-    if (atomicCAS(&g_err_code, 0, code) == 0) atomicExch(&g_err_where, where);
-}
-
-// Wait for phase `parity` of `bar`, giving up after limit_ns or when another role aborted.
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             uint64_t limit_ns, int where) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-#pragma unroll 1
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 31u) == 0) {
-            if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > limit_ns) {
-                *abort_flag = 1;
-                record_error(FA_ERR_TIMEOUT, where);
-                return false;
-            }
-        }
-    }
-}
 
 template <int D>
 struct Cfg {
@@ -1033,18 +1006,6 @@ static cudaError_t launch_t(const CUtensorMap &tq, const CUtensorMap &tk, const 
     }
     kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
     return cudaGetLastError();
-}
-
-// Reads and clears this compilation unit's error word.
-static cudaError_t take_device_error(int *code, int *where) {
-    int zero = 0;
-    cudaError_t e = cudaMemcpyFromSymbol(code, g_err_code, sizeof(int));
-    if (e != cudaSuccess) return e;
-    e = cudaMemcpyFromSymbol(where, g_err_where, sizeof(int));
-    if (e != cudaSuccess) return e;
-    e = cudaMemcpyToSymbol(g_err_code, &zero, sizeof(int));
-    if (e != cudaSuccess) return e;
-    return cudaMemcpyToSymbol(g_err_where, &zero, sizeof(int));
 }
 
 }  // namespace fa

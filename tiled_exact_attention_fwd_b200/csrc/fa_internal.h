@@ -53,6 +53,22 @@ cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t st);
 cudaError_t fwd_take_device_error(int *code, int *where);
 cudaError_t fwd_paged_take_device_error(int *code, int *where);
 
+// Attention backward (fa_bwd.cu): dQ, dK, dV from q, k, v, out, dout and the forward's LSE.
+struct BwdParams {
+    const void *out, *dout;  // (B, S, H, D), read by the delta kernel
+    const float *lse;        // (B, H, S) from the forward
+    float *delta;            // (B, H, S) workspace: rowsum(dO * O)
+    void *dq, *dk, *dv;      // (B, S, H, D) gradients
+    int B, H, seqlen;
+    float scale;             // softmax scale
+    float scale_log2;        // scale * log2(e)
+    uint64_t timeout_ns;     // bound of every pipeline wait
+};
+// tq, tk, tv, tdo: TMA maps of q, k, v, dout as for the forward (128-row boxes).
+cudaError_t launch_bwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
+                       const CUtensorMap &tv, const CUtensorMap &tdo, const BwdParams &p, cudaStream_t st);
+cudaError_t bwd_take_device_error(int *code, int *where);
+
 // Unpad / pad (row gather / scatter + zero fill).
 cudaError_t launch_unpad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
                          int64_t row_bytes, void *out, cudaStream_t st);

@@ -1,0 +1,51 @@
+// fa_sync.cuh -- the device error word and the bounded mbarrier wait shared by the kernels.
+// Each compilation unit that includes this header gets its own error word (static device
+// variables); take_device_error reads and clears the word of the unit that calls it.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fa.h"
+#include "fa_ptx.cuh"
+
+namespace fa {
+
+static __device__ int g_err_code;
+static __device__ int g_err_where;
+
+static __device__ __noinline__ void record_error(int code, int where) {
+    if (atomicCAS(&g_err_code, 0, code) == 0) atomicExch(&g_err_where, where);
+}
+
+// Wait for phase `parity` of `bar`, giving up after limit_ns or when another role aborted.
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             uint64_t limit_ns, int where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+#pragma unroll 1
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 31u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > limit_ns) {
+                *abort_flag = 1;
+                record_error(FA_ERR_TIMEOUT, where);
+                return false;
+            }
+        }
+    }
+}
+
+// Reads and clears this compilation unit's error word.
+static cudaError_t take_device_error(int *code, int *where) {
+    int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(code, g_err_code, sizeof(int));
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(where, g_err_where, sizeof(int));
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyToSymbol(g_err_code, &zero, sizeof(int));
+    if (e != cudaSuccess) return e;
+    return cudaMemcpyToSymbol(g_err_where, &zero, sizeof(int));
+}
+
+}  // namespace fa
