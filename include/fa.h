@@ -114,6 +114,24 @@ FA_API fa_status fa_bwd(const void *q, const void *k, const void *v, const void 
                         int D, float scale, int causal, fa_dtype dtype, void *stream);
 
 /*
+ * fa_bwd without the caller's delta workspace: the same computation and results, with the
+ * workspace taken from a fixed device array that is part of the library (64 MiB, room for
+ * B * H * S <= 2^24 rows; larger problems return FA_ERR_SHAPE before any launch). The pages
+ * have no counterpart to this entry point; it exists for callers that may not allocate
+ * (nothing here calls cudaMalloc or any allocating routine).
+ *   Set-up: the first call on each device looks the array's address up (this loads the
+ *   library's module on that device); make that first call outside any stream capture. Later
+ *   calls only launch kernels and may be captured into a CUDA graph.
+ *   Nothing has to start at zero: every call overwrites the rows it reads.
+ *   Calls that overlap in time (different streams, or concurrent graph nodes) share the one
+ *   array and race; serialise them.
+ * Arguments as fa_bwd, minus `delta`.
+ */
+FA_API fa_status fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *out, const void *dout,
+                                const float *lse, void *dq, void *dk, void *dv, int B, int H, int S, int D,
+                                float scale, int causal, fa_dtype dtype, void *stream);
+
+/*
  * Packed variable-length attention forward (the flash_attn_varlen_func step).
  *   q, k, v      (total, H, D) packed inputs; sequence s owns rows
  *                [cu_seqlens[s], cu_seqlens[s+1]) and attends only inside itself.

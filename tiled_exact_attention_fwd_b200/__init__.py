@@ -49,6 +49,7 @@ def lib() -> ctypes.CDLL:
         L.fa_varlen_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, i32, i32, f32, i32, i32, vp]
         L.fa_fwd_paged.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
         L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
+        L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
         L.fa_unpad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fa_pad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fa_unpad_qkv.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp]
@@ -56,7 +57,7 @@ def lib() -> ctypes.CDLL:
                                            vp]
         L.fa_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.fa_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
-        for f in (L.fa_fwd, L.fa_fwd_paged, L.fa_bwd, L.fa_varlen_fwd, L.fa_varlen_fwd_padded, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad,
+        for f in (L.fa_fwd, L.fa_fwd_paged, L.fa_bwd, L.fa_bwd_noalloc, L.fa_varlen_fwd, L.fa_varlen_fwd_padded, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad,
                   L.fa_device_status,
                   L.fa_selftest_bounded_wait):
             f.restype = ctypes.c_int
@@ -147,6 +148,21 @@ def fa_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                       _stream(stream))
     _check(st, "fa_bwd")
     return dq, dk, dv
+
+
+def fa_bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
+                   lse: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor,
+                   scale: Optional[float] = None, causal: bool = False, stream=None) -> None:
+    """fa_bwd into caller-given dq, dk, dv with the library's fixed delta buffer (no
+    allocation by the library; concurrent calls share that buffer and must be serialised)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse), ("dq", dq),
+                 ("dk", dk), ("dv", dv)):
+        _cuda_contig(n, t)
+    B, S, H, D = q.shape
+    st = lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                              _ptr(dv), B, H, S, D, float(scale) if scale else 0.0, int(bool(causal)),
+                              _dtype_code(q), _stream(stream))
+    _check(st, "fa_bwd_noalloc")
 
 
 def attention_bwd_flops(B: int, H: int, S: int, D: int, causal: bool) -> float:

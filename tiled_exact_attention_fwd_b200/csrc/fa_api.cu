@@ -207,6 +207,20 @@ fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, c
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+fa_status fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *out, const void *dout,
+                         const float *lse, void *dq, void *dk, void *dv, int B, int H, int S, int D, float scale,
+                         int causal, fa_dtype dtype, void *stream) {
+    // the fixed delta buffer holds B * H * S floats at most; larger problems are refused
+    if (B > 0 && H > 0 && S > 0 && static_cast<int64_t>(B) * H * S > fa::kNoallocDeltaFloats) return FA_ERR_SHAPE;
+    if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv) return FA_ERR_NULL;
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;
+    if (B <= 0 || H <= 0 || S <= 0) return FA_ERR_SHAPE;
+    float *delta = nullptr;
+    if (fa::noalloc_delta_buffer(&delta) != cudaSuccess) return FA_ERR_CUDA;
+    return fa_bwd(q, k, v, out, dout, lse, dq, dk, dv, delta, B, H, S, D, scale, causal, dtype, stream);
+}
+
 fa_status fa_varlen_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqlens, int num_seqs,
                         int max_seqlen, int total, void *out, float *lse, int H, int D, float scale, int causal,
                         fa_dtype dtype, void *stream) {

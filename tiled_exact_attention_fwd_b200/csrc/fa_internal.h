@@ -68,6 +68,10 @@ struct BwdParams {
 cudaError_t launch_bwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
                        const CUtensorMap &tv, const CUtensorMap &tdo, const BwdParams &p, cudaStream_t st);
 cudaError_t bwd_take_device_error(int *code, int *where);
+// The fixed delta buffer of fa_bwd_noalloc: kNoallocDeltaFloats floats (64 MiB) in device
+// memory that belongs to the library's module image; its address on the current device.
+constexpr int64_t kNoallocDeltaFloats = int64_t(1) << 24;
+cudaError_t noalloc_delta_buffer(float **ptr);
 
 // Unpad / pad (row gather / scatter + zero fill).
 cudaError_t launch_unpad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
