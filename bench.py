@@ -571,6 +571,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only-main", action="store_true", help="time the main kernel only (for profiling)")
     ap.add_argument("--only-padding", action="store_true", help="run the unpad/pad HBM leg only (for profiling)")
+    ap.add_argument("--only-backward", action="store_true", help="run the backward leg only (for profiling)")
     ap.add_argument("--all-configs", action="store_true",
                     help="print one informational line per workload (dense/causal/head-dim sweep)")
     args = ap.parse_args()
@@ -580,6 +581,17 @@ def main():
         run_reference(args)
     elif args.all_configs:
         run_all_configs(args)
+    elif args.only_backward:
+        import tiled_exact_attention_fwd_b200 as fa
+        device = torch.device("cuda", 0)
+        torch.cuda.set_device(device)
+        w = fa_inputs.WORKLOADS[WORKLOAD]
+        B, S, H, D, causal = w["B"], w["S"], w["H"], w["D"], w["causal"]
+        q, k, v = (t.to(device) for t in fa_inputs.dense_qkv(B, S, H, D, fa_inputs.DTYPES[w["dtype"]], seed=0))
+        out = torch.empty_like(q)
+        lse = torch.empty((B, H, S), device=device, dtype=torch.float32)
+        print(json.dumps(run_backward_leg(fa, device, torch.cuda.current_stream(device), q, k, v, out, lse, causal,
+                                          args.warmup, 0, iters=max(args.steps, 1))))
     elif args.only_padding:
         import tiled_exact_attention_fwd_b200 as fa
         device = torch.device("cuda", 0)
