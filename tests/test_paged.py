@@ -36,6 +36,7 @@ def test_oracle_paged_attention_is_dense_attention():
 CASES = [  # (D, page_size, dtype, causal)
     (32, 16, torch.bfloat16, True), (64, 64, torch.float16, False), (64, 16, torch.bfloat16, True),
     (128, 128, torch.bfloat16, True), (128, 32, torch.float16, False), (128, 256, torch.bfloat16, False),
+    (128, 16, torch.bfloat16, True), (64, 32, torch.float16, True),
     (256, 64, torch.float16, True), (256, 128, torch.bfloat16, False), (256, 16, torch.bfloat16, True),
 ]
 
@@ -60,13 +61,15 @@ def test_paged_matches_oracle_and_dense(cuda_device, D, page_size, dtype, causal
 
 
 @pytest.mark.gpu
-def test_paged_full_size_matches_dense(cuda_device):
-    """The causal bf16 B1 H32 S8192 D128 workload with 64-row pages, against fa_fwd on the
-    contiguous tensors (bit for bit) and sampled rows of the oracle."""
+@pytest.mark.parametrize("page_size", [16, 64])
+def test_paged_full_size_matches_dense(cuda_device, page_size):
+    """The causal bf16 B1 H32 S8192 D128 workload in 16-row pages (copy producers) and 64-row
+    pages (TMA), against fa_fwd on the contiguous tensors (bit for bit) and sampled rows of the
+    oracle."""
     import tiled_exact_attention_fwd_b200 as fa
     B, S, H, D = 1, 8192, 32, 128
     q, k, v = fa_inputs.dense_qkv(B, S, H, D, torch.bfloat16, seed=0)
-    kc, vc, table = fa_inputs.paged_kv(k, v, 64, seed=1, fill=0.0)
+    kc, vc, table = fa_inputs.paged_kv(k, v, page_size, seed=1, fill=0.0)
     dev = cuda_device
     out, lse = fa.fa_fwd_paged(q.to(dev), kc.to(dev), vc.to(dev), table.to(dev), causal=True)
     ref_out, ref_lse = fa.fa_fwd(q.to(dev), k.to(dev), v.to(dev), causal=True)

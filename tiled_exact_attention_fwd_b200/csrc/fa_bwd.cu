@@ -15,14 +15,17 @@
 //            dV  += P^T dO_i,  dK += dZ^T Q_i           (TS MMAs, A from TMEM)
 //   dQ:    a CTA owns one 128-row query tile i (Q_i, dO_i stay) and streams key tiles j <= i:
 //            S = Q_i K_j^T, dP = dO_i V_j^T;  dZ over S;  dQ += dZ K_j
-// Warps 0-3 do the elementwise work (thread = TMEM lane = one row), warp 4 lane 0 issues the
-// TMA loads, warp 5 allocates TMEM and lane 0 issues every MMA. Every wait is bounded.
+// Warps 0-7 do the elementwise work (two threads per TMEM lane = row, each on half of the
+// columns), warp 8 lane 0 issues the TMA loads, warp 9 allocates TMEM and lane 0 issues
+// every MMA. Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "fa.h"
 #include "fa_internal.h"
@@ -40,8 +43,10 @@ struct BwdCfg {
     static constexpr int NBLK = D / SWE;                     // column blocks per tile row
     static constexpr int TILE_BYTES = BM * D * 2;
     static constexpr uint32_t LAYOUT = (SW == 128) ? kLayoutSw128 : kLayoutSw64;
-    static constexpr int NUM_THREADS = 192;
-    static constexpr int WARP_TMA = 4, WARP_MMA = 5;
+    // warps 0-7 elementwise (warp w: TMEM lanes 32*(w%4).., columns half w/4), 8 TMA, 9 MMA
+    static constexpr int NUM_EW = 256;
+    static constexpr int NUM_THREADS = NUM_EW + 64;
+    static constexpr int WARP_TMA = 8, WARP_MMA = 9;
     // shared memory: fixed tiles A0, A1; ring stages s = 0, 1 holding tiles B0, B1;
     // per-column statistics (dK/dV kernel) in two slots; barriers; misc
     static constexpr int OFF_FIX = 0;
@@ -85,7 +90,9 @@ __device__ __forceinline__ void mma_rows(uint32_t d_tmem, const uint8_t *a, cons
 }
 
 // D_out (+)= A_tmem B over 128 rows: A (128 x 128, 16-bit) in TMEM, B a 128-row tile read
-// MN-major (its D columns are the output columns).
+// MN-major (its D columns are the output columns). A's packed columns 0-31 (elements 0-63)
+// sit at a_tmem + [0, 32) and columns 32-63 at a_tmem + [64, 96): each half was written by
+// its own thread over the fp32 columns it had read.
 template <int D, bool BF16>
 __device__ __forceinline__ void mma_acc(uint32_t d_tmem, uint32_t a_tmem, const uint8_t *b, bool accumulate) {
     using C = BwdCfg<D>;
@@ -93,7 +100,8 @@ __device__ __forceinline__ void mma_acc(uint32_t d_tmem, uint32_t a_tmem, const 
     const uint32_t b0 = smem_u32(b);
 #pragma unroll
     for (int k = 0; k < C::BM / 16; ++k)
-        umma_ts(d_tmem, a_tmem + k * 8, smem_desc(b0 + k * 16 * C::SW, C::BM * C::SW, 8 * C::SW, C::LAYOUT), idesc,
+        umma_ts(d_tmem, a_tmem + k * 8 + (k >= 4 ? 32 : 0),
+                smem_desc(b0 + k * 16 * C::SW, C::BM * C::SW, 8 * C::SW, C::LAYOUT), idesc,
                 (accumulate || k > 0) ? 1u : 0u);
 }
 
@@ -102,11 +110,12 @@ __device__ __forceinline__ uint32_t pack2b(float lo, float hi) {
     return BF16 ? pack2_bf16(lo, hi) : pack2_f16(lo, hi);
 }
 
-// One row of a TMEM accumulator (D fp32 columns) times `mul` -> 16-bit -> global.
+// One row of a TMEM accumulator (D fp32 columns) times `mul` -> 16-bit -> global; the two
+// threads of a row take alternate 32-column chunks (half = 0, 1).
 template <int D, bool BF16>
-__device__ __forceinline__ void store_row(uint32_t taddr, float mul, uint8_t *grow, bool store) {
+__device__ __forceinline__ void store_row(uint32_t taddr, float mul, uint8_t *grow, bool store, int half) {
 #pragma unroll 1
-    for (int cc = 0; cc < D / 32; ++cc) {
+    for (int cc = half; cc < D / 32; cc += 2) {
         uint32_t o[32];
         tmem_ld32(taddr + cc * 32, o);
         tmem_ld_wait();
@@ -158,10 +167,10 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int s = 0; s < 2; ++s) {
             mbar_init(&ring_full[s], 1);
             mbar_init(&ring_empty[s], 1);
-            mbar_init(&stats_ready[s], 128);
+            mbar_init(&stats_ready[s], BM);  // the column-half-0 threads publish 128 columns
         }
         mbar_init(s_full, 1);
-        mbar_init(p_ready, 128);
+        mbar_init(p_ready, C::NUM_EW);
         mbar_init(done, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -244,9 +253,10 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         }
     } else {
-        // ------------------------------------------------------------ elementwise warps 0-3
-        const int r = warp * 32 + lane;  // TMEM lane = row of the owned tile
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        // ------------------------------------------------------------ elementwise warps 0-7
+        const int quarter = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
+        const int r = quarter * 32 + lane;                // TMEM lane = row of the owned tile
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         const int own_pos = own * BM + r;  // sequence position of this row (key or query)
         const float sl2 = p.scale_log2;
         constexpr float kLog2e = 1.4426950408889634f;
@@ -262,79 +272,94 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 nd = 0.f;
             }
         };
+        const bool publisher = DKDV && half == 0;  // publishes the statistics of query column r
         float my_nl = 0.f, my_nd = 0.f;  // dQ: this row's statistics; dK/dV: prefetched column stats
-        if (DKDV) {
+        if (publisher) {
             if (n > 0) query_stats(t0 * BM + r, my_nl, my_nd);
-        } else {
+        } else if (!DKDV) {
             query_stats(own_pos, my_nl, my_nd);
         }
+        // P (or P^T) and dZ for 32 columns starting at col0; MASK applies the causal diagonal
+        // and (dQ) the keys past the sequence end.
+        auto chunk = [&](auto mask_c, int col0, const float *snl, const float *snd, int key_hi, bool diag) {
+            constexpr bool MASK = decltype(mask_c)::value;
+            uint32_t sv[32], dv[32];
+            tmem_ld32(tmem + lane_base + C::COL_S + col0, sv);
+            tmem_ld32(tmem + lane_base + C::COL_DP + col0, dv);
+            tmem_ld_wait();
+            tmem_reg_fence<32>(sv);
+            tmem_reg_fence<32>(dv);
+            uint32_t pk[16], zk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int col = col0 + 2 * i;
+                float nl0, nl1, nd0, nd1;
+                if (DKDV) {
+                    const float2 a = *reinterpret_cast<const float2 *>(snl + col);
+                    const float2 c2 = *reinterpret_cast<const float2 *>(snd + col);
+                    nl0 = a.x, nl1 = a.y, nd0 = c2.x, nd1 = c2.y;
+                } else {
+                    nl0 = nl1 = my_nl;
+                    nd0 = nd1 = my_nd;
+                }
+                const uint64_t x2 = ffma2(f2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])),
+                                          f2(sl2, sl2), f2(nl0, nl1));
+                float x0, x1;
+                f2_split(x2, x0, x1);
+                float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                if constexpr (MASK) {
+                    // key position > query position weighs 0 (dK/dV rows are keys and columns
+                    // queries, dQ the other way round); dQ: keys past the sequence end weigh 0
+                    if (DKDV ? (diag && r > col) : ((diag && col > r) || col >= key_hi)) p0 = 0.f;
+                    if (DKDV ? (diag && r > col + 1) : ((diag && col + 1 > r) || col + 1 >= key_hi)) p1 = 0.f;
+                }
+                const uint64_t z2 = fmul2(f2(p0, p1), fadd2(f2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])),
+                                                            f2(nd0, nd1)));
+                float z0, z1;
+                f2_split(z2, z0, z1);
+                pk[i] = pack2b<BF16>(p0, p1);
+                zk[i] = pack2b<BF16>(z0, z1);
+            }
+            // packed columns of this half start at its own first column (32 * half packed
+            // columns further on for half 1), so neither thread of the row overwrites
+            // columns the other one has yet to read
+            const int pcol = col0 / 2 + 32 * half;
+            if (DKDV) {
+                tmem_st16(tmem + lane_base + C::COL_S + pcol, pk);   // P^T over S^T
+                tmem_st16(tmem + lane_base + C::COL_DP + pcol, zk);  // dZ^T over dP^T
+            } else {
+                tmem_st16(tmem + lane_base + C::COL_S + pcol, zk);   // dZ over S
+            }
+        };
         for (int t = 0; ok && t < n; ++t) {
             const int other = t0 + t;  // the streamed tile (query tile for dK/dV, key tile for dQ)
             const int slot = t & 1;
-            float *snl = stats + slot * 2 * BM, *snd = snl + BM;
+            const float *snl = stats + slot * 2 * BM, *snd = snl + BM;
             if (DKDV) {
-                // publish this thread's query column statistics, prefetch the next tile's
-                snl[r] = my_nl;
-                snd[r] = my_nd;
-                mbar_arrive(&stats_ready[slot]);
-                if (t + 1 < n) query_stats((other + 1) * BM + r, my_nl, my_nd);
+                if (publisher) {
+                    // publish this thread's query column statistics, prefetch the next tile's
+                    stats[slot * 2 * BM + r] = my_nl;
+                    stats[slot * 2 * BM + BM + r] = my_nd;
+                    mbar_arrive(&stats_ready[slot]);
+                    if (t + 1 < n) query_stats((other + 1) * BM + r, my_nl, my_nd);
+                }
                 if (!(ok = __all_sync(0xffffffffu, wait_bounded(&stats_ready[slot], (t >> 1) & 1, abort_flag, lim, 440))))
                     break;
             }
             if (!(ok = __all_sync(0xffffffffu, wait_bounded(s_full, t & 1, abort_flag, lim, 450)))) break;
             tc_fence_after_sync();
-            const bool diag = CAUSAL && other == own;
-            // dQ: keys past the sequence end weigh 0
             const int key_hi = DKDV ? BM : min(BM, S - other * BM);
+            const bool diag = CAUSAL && other == own;
+            const bool masked = diag || key_hi < BM;
+            // this thread's 64 columns: [64*half, 64*half + 64), two chunks; each chunk's
+            // results are stored over columns this thread has already read
 #pragma unroll 1
-            for (int cc = 0; cc < BM / 32; ++cc) {
-                uint32_t sv[32], dv[32];
-                tmem_ld32(tmem + lane_base + C::COL_S + cc * 32, sv);
-                tmem_ld32(tmem + lane_base + C::COL_DP + cc * 32, dv);
-                tmem_ld_wait();
-                tmem_reg_fence<32>(sv);
-                tmem_reg_fence<32>(dv);
-                uint32_t pk[16], zk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int col = cc * 32 + 2 * i;
-                    float nl0, nl1, nd0, nd1;
-                    if (DKDV) {
-                        const float2 a = *reinterpret_cast<const float2 *>(snl + col);
-                        const float2 c2 = *reinterpret_cast<const float2 *>(snd + col);
-                        nl0 = a.x, nl1 = a.y, nd0 = c2.x, nd1 = c2.y;
-                    } else {
-                        nl0 = nl1 = my_nl;
-                        nd0 = nd1 = my_nd;
-                    }
-                    const uint64_t x2 = ffma2(f2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])),
-                                              f2(sl2, sl2), f2(nl0, nl1));
-                    float x0, x1;
-                    f2_split(x2, x0, x1);
-                    float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                    // causal: key position > query position weighs 0 (only on the diagonal tile;
-                    // dK/dV rows are keys and columns queries, dQ the other way round)
-                    if (diag) {
-                        if (DKDV ? (r > col) : (col > r)) p0 = 0.f;
-                        if (DKDV ? (r > col + 1) : (col + 1 > r)) p1 = 0.f;
-                    }
-                    if (!DKDV) {
-                        if (col >= key_hi) p0 = 0.f;
-                        if (col + 1 >= key_hi) p1 = 0.f;
-                    }
-                    const uint64_t z2 = fmul2(f2(p0, p1), fadd2(f2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])),
-                                                                f2(nd0, nd1)));
-                    float z0, z1;
-                    f2_split(z2, z0, z1);
-                    pk[i] = pack2b<BF16>(p0, p1);
-                    zk[i] = pack2b<BF16>(z0, z1);
-                }
-                if (DKDV) {
-                    tmem_st16(tmem + lane_base + C::COL_S + cc * 16, pk);   // P^T over S^T
-                    tmem_st16(tmem + lane_base + C::COL_DP + cc * 16, zk);  // dZ^T over dP^T
-                } else {
-                    tmem_st16(tmem + lane_base + C::COL_S + cc * 16, zk);   // dZ over S
-                }
+            for (int c = 0; c < 2; ++c) {
+                const int col0 = half * 64 + c * 32;
+                if (masked)
+                    chunk(std::integral_constant<bool, true>{}, col0, snl, snd, key_hi, diag);
+                else
+                    chunk(std::integral_constant<bool, false>{}, col0, snl, snd, key_hi, diag);
             }
             tmem_st_wait();
             tc_fence_before_sync();
@@ -346,20 +371,13 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const bool store = own_pos < S;
             const int64_t grow = (row0 + own_pos) * p.H + h;  // token row, head
             if (DKDV) {
-                if (n > 0) {
-                    store_row<D, BF16>(tmem + lane_base + C::COL_ACC0, 1.f,
-                                       static_cast<uint8_t *>(p.dv) + grow * D * 2, store);
-                    store_row<D, BF16>(tmem + lane_base + C::COL_ACC1, p.scale,
-                                       static_cast<uint8_t *>(p.dk) + grow * D * 2, store);
-                } else if (store) {
-                    // no query sees these keys: zero gradients
-                    uint4 *gv = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.dv) + grow * D * 2);
-                    uint4 *gk = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.dk) + grow * D * 2);
-                    for (int i = 0; i < D / 8; ++i) gv[i] = gk[i] = make_uint4(0u, 0u, 0u, 0u);
-                }
+                store_row<D, BF16>(tmem + lane_base + C::COL_ACC0, 1.f, static_cast<uint8_t *>(p.dv) + grow * D * 2,
+                                   store, half);
+                store_row<D, BF16>(tmem + lane_base + C::COL_ACC1, p.scale, static_cast<uint8_t *>(p.dk) + grow * D * 2,
+                                   store, half);
             } else {
                 store_row<D, BF16>(tmem + lane_base + C::COL_ACC0, p.scale, static_cast<uint8_t *>(p.dq) + grow * D * 2,
-                                   store);
+                                   store, half);
             }
         }
     }

@@ -445,7 +445,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // after they land, so the MMA thread fences the async proxy after its waits. (The paged
     // path's zeroed page tails are fenced by the writing thread itself before it releases
     // the stage.)
-    c.fused = p.gather != nullptr;
+    // Paged K/V in 16-row pages: TMA boxes that small run at half the copy rate, so the fused
+    // path's copy threads fetch Q, K and V instead (the same fence applies).
+    const bool copy_pages = PAGED && p.page_size < 32;
+    c.fused = p.gather != nullptr || copy_pages;
     c.nA = (kv_end_A + BN - 1) / BN;
     c.nB = c.two ? (kv_end_B + BN - 1) / BN : 0;
     c.jB0 = c.two ? kv_start_B / BN : 0;
@@ -474,7 +477,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        const int fill_arrivals = p.gather ? 96 : 1;  // fused: the 96 copy threads arrive
+        const int fill_arrivals = c.fused ? 96 : 1;  // copy producers: the 96 copy threads arrive
         for (int t = 0; t < 2; ++t) {
             mbar_init(&c.q_full[t], fill_arrivals);
             mbar_init(&c.s_full[t], 1);
@@ -508,14 +511,83 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (warp >= C::NUM_SOFTMAX_WARPS) {
         // producer / MMA warpgroup (its two remaining warps idle)
         if constexpr (C::SPLIT_REGS) regs_dec<C::REGS_LOW>();
-        if (warp == C::WARP_TMA || (p.gather && warp > C::WARP_MMA)) {
+        if (warp == C::WARP_TMA || (c.fused && warp > C::WARP_MMA)) {
             // ------------------------------------------------------------ TMA producer
             // (with the fused packed path also warps 10 and 11: copy producers)
             const int nq = c.two ? 2 : 1;
             const int loads = 2 * n_all * C::UNITS;  // parts of K_0, V_0, K_1, V_1, ...
             int issued = 0;
             bool tail_issued = false;
-            if (p.gather) {
+            if (PAGED && copy_pages) {
+                // Paged K/V in small pages: warps 8, 10 and 11 (96 threads) copy rows with
+                // 16-byte cp.async into the swizzled layout; row r of a key tile is position
+                // pos of the sequence, read from its page; positions past the sequence end
+                // are zero-filled (no page is read for them). Q rows are plain token rows.
+                constexpr int CPB = SW / 16;
+                const int pw = (warp == C::WARP_TMA) ? 0 : warp - C::WARP_MMA;
+                const int32_t *bt = p.block_table + static_cast<int64_t>(blockIdx.z) * p.max_blocks;
+                bool bad_page = false;
+                // rows [pos0, pos0 + rows) x column blocks [b0, b0 + NB) into dst as [NB][rows][SW];
+                // `paged` selects the K/V pool (else the dense q rows of this sequence)
+                auto fill_rows = [&](auto nb_c, uint8_t *dst, const void *src, uint64_t *bar, int pos0, int rows,
+                                     int b0, bool paged) {
+                    constexpr int CPR = decltype(nb_c)::value * CPB;
+                    const uint32_t dst_u32 = smem_u32(dst);
+                    for (int g = pw; g * 32 < rows; g += 3) {
+                        const int pos = pos0 + g * 32 + lane;
+                        const bool valid = pos < seqlen;
+                        int64_t prow = 0;
+                        if (valid) {
+                            if (paged) {
+                                int pg = __ldg(bt + (pos >> p.page_shift));
+                                if (pg < 0 || pg >= p.num_pages) {
+                                    bad_page = true;
+                                    pg = 0;
+                                }
+                                prow = (static_cast<int64_t>(pg) << p.page_shift) + (pos & (p.page_size - 1));
+                            } else {
+                                prow = static_cast<int64_t>(seq_start) + pos;
+                            }
+                        }
+                        const uint8_t *srow = static_cast<const uint8_t *>(src) + b0 * SW;
+#pragma unroll 4
+                        for (int i = 0; i < CPR; ++i) {
+                            const int idx = i * 32 + lane;
+                            const int rr = idx / CPR, ch = idx % CPR;
+                            const int64_t pr = __shfl_sync(0xffffffffu, prow, rr);
+                            const bool ok_row = __shfl_sync(0xffffffffu, valid, rr);
+                            const int r = g * 32 + rr;
+                            const int blk = ch / CPB, cc = ch % CPB;
+                            const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
+                            cp_async_16_zfill(dst_u32 + blk * rows * SW + r * SW + ((cc ^ swz) << 4),
+                                              srow + (pr * p.H + h) * static_cast<int64_t>(D) * 2 + ch * 16,
+                                              ok_row ? 16u : 0u);
+                        }
+                    }
+                    cp_async_mbar_arrive(bar);
+                };
+                using AllBlk = std::integral_constant<int, C::NBLK>;
+                using KBlk = std::integral_constant<int, C::KBLK_PER_UNIT>;
+                for (int t = 0; t < nq; ++t)
+                    fill_rows(AllBlk{}, c.sQ + t * C::Q_BYTES, p.q, &c.q_full[t], q0 + t * BM, BM, 0, false);
+                for (int U = 0; U < loads; ++U) {
+                    const int stage = U % NS;
+                    if (U >= NS &&
+                        !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
+                        break;
+                    const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
+                    uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
+                    if (L & 1)
+                        fill_rows(AllBlk{}, dst, p.v, &c.kv_full[stage], j * BN + u * C::VROWS_PER_UNIT,
+                                  C::VROWS_PER_UNIT, 0, true);
+                    else
+                        fill_rows(KBlk{}, dst, p.k, &c.kv_full[stage], j * BN, BN, u * C::KBLK_PER_UNIT, true);
+                    issued = U + 1;
+                }
+                cp_async_wait_all();  // nothing of this thread is left in flight at exit
+                issued = 0;
+                if (bad_page) record_error(FA_ERR_INDEX, 151);
+            } else if (p.gather) {
                 // Fused packed path: warps 8, 10 and 11 (96 threads) copy every tile row from
                 // the padded tensor (row = padded row of the packed token; rows past the last
                 // token read row 0, which the masks then ignore) with 16-byte cp.async into the

@@ -94,6 +94,13 @@ __device__ __forceinline__ void cp_async_16(uint32_t smem_addr, const void *gptr
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr), "l"(gptr) : "memory");
 }
 
+// The same with `src_bytes` (0 or 16) read from gptr and the rest of the 16 bytes zero-filled:
+// src_bytes = 0 writes 16 zero bytes and reads nothing (gptr must still be a valid address).
+__device__ __forceinline__ void cp_async_16_zfill(uint32_t smem_addr, const void *gptr, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr), "l"(gptr), "r"(src_bytes)
+                 : "memory");
+}
+
 // Arrive on `bar` once every cp.async this thread issued so far has landed (the arrival is
 // counted in the barrier's expected count: .noinc).
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
