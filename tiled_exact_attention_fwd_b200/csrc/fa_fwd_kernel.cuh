@@ -947,9 +947,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             l = fmaf(l, alpha, rs);
             tmem_st_wait();
             if (jj > 0) {
-                // The previous PV is waited for on every step (it has normally finished long
-                // before), so this thread never falls two phases behind on pv_done.
-                if (!__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (jj - 1) & 1, c.abort_flag, c.lim, 310 + t))) {
+                // O must hold PV(j-1) before it is rescaled. With two tiles, PV_t(j-1) was
+                // issued before QK_t(j), and the commit behind s_full only fires once every
+                // earlier MMA of the issuing thread has completed, so it is done already. With
+                // one tile QK(j) precedes PV(j-1): wait for it (on every step, so this thread
+                // never falls two phases behind on pv_done). The final wait after the loop
+                // always targets the newest phase, which is correct either way.
+                if (!c.two &&
+                    !__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (jj - 1) & 1, c.abort_flag, c.lim, 310 + t))) {
                     ok = false;
                     break;
                 }
