@@ -40,7 +40,8 @@ import fa_inputs  # noqa: E402
 
 METRIC = "attention fwd TFLOPS and % of B200 tensor-core peak; varlen µs/call"
 WORKLOAD = "llm_causal_bf16"
-KERNEL_SOURCES = ["tiled_exact_attention_fwd_b200/csrc/fa_fwd_kernel.cuh", "tiled_exact_attention_fwd_b200/csrc/fa_ptx.cuh"]
+KERNEL_SOURCES = ["tiled_exact_attention_fwd_b200/csrc/fa_fwd_kernel.cuh", "tiled_exact_attention_fwd_b200/csrc/fa_ptx.cuh",
+                  "tiled_exact_attention_fwd_b200/csrc/fa_sync.cuh", "tiled_exact_attention_fwd_b200/csrc/fa_seq.cuh"]
 
 
 def kernel_source_hash() -> str:

@@ -114,6 +114,23 @@ FA_API fa_status fa_bwd(const void *q, const void *k, const void *v, const void 
                         int D, float scale, int causal, fa_dtype dtype, void *stream);
 
 /*
+ * Packed variable-length attention backward (the backward of fa_varlen_fwd): gradients of
+ * every sequence's attention, sequence s owning rows [cu_seqlens[s], cu_seqlens[s+1]).
+ *   q, k, v, out, dout   (total, H, D) packed inputs, output and output gradient.
+ *   lse                  (H, total) float32 from fa_varlen_fwd.
+ *   dq, dk, dv           (total, H, D) outputs; every element is written.
+ *   delta                (H, total) float32 caller-owned workspace (rowsum(dout * out)).
+ *   cu_seqlens, num_seqs, max_seqlen, total, scale, causal: as fa_varlen_fwd.
+ * D in {32, 64, 128}. Work is split into tiles of 128 consecutive packed tokens whatever
+ * sequences they hold. total == 0 is a successful no-op.
+ */
+FA_API fa_status fa_varlen_bwd(const void *q, const void *k, const void *v, const void *out,
+                               const void *dout, const float *lse, const int32_t *cu_seqlens,
+                               int num_seqs, int max_seqlen, int total, void *dq, void *dk, void *dv,
+                               float *delta, int H, int D, float scale, int causal, fa_dtype dtype,
+                               void *stream);
+
+/*
  * fa_bwd without the caller's delta workspace: the same computation and results, with the
  * workspace taken from a fixed device array that is part of the library (64 MiB, room for
  * B * H * S <= 2^24 rows; larger problems return FA_ERR_SHAPE before any launch). The pages

@@ -261,4 +261,4 @@ def pad(x: torch.Tensor, indices, batch: int, total_len: int) -> torch.Tensor:
 
 
 from .online_softmax import online_softmax_attention  # noqa: E402,F401
-from .backward import attention_backward, attention_backward_head  # noqa: E402,F401
+from .backward import attention_backward, attention_backward_head, attention_varlen_backward  # noqa: E402,F401

@@ -69,3 +69,21 @@ def attention_backward(q, k, v, dout, scale: Optional[float] = None, causal: boo
     for (b, h), (gq, gk, gv) in res.items():
         dq[b, :, h], dk[b, :, h], dv[b, :, h] = gq, gk, gv
     return dq, dk, dv
+
+
+def attention_varlen_backward(q, k, v, dout, cu_seqlens, scale: Optional[float] = None, causal: bool = False):
+    """Gradients of packed (total, H, D) attention: each sequence [cu[s], cu[s+1]) on its own
+    (page "IAW 模型 FA2 vs FA3 实测", section 1: the packed batch is attention within each
+    sequence), by attention_backward_head per (sequence, head). Returns float64 (total, H, D)."""
+    cu = [int(x) for x in (cu_seqlens.tolist() if isinstance(cu_seqlens, torch.Tensor) else cu_seqlens)]
+    total, H, D = q.shape
+    dq = np.zeros((total, H, D))
+    dk = np.zeros((total, H, D))
+    dv = np.zeros((total, H, D))
+    for s0, s1 in zip(cu[:-1], cu[1:]):
+        if s1 <= s0:
+            continue
+        for h in range(H):
+            gq, gk, gv = attention_backward_head(q[s0:s1, h], k[s0:s1, h], v[s0:s1, h], dout[s0:s1, h], scale, causal)
+            dq[s0:s1, h], dk[s0:s1, h], dv[s0:s1, h] = gq, gk, gv
+    return dq, dk, dv

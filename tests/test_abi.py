@@ -149,3 +149,22 @@ def test_bwd_validation(lib):
     assert call(0, FAKE + 8) == -5
     assert call(5, FAKE + 2) == -5
     assert call(9, FAKE + 2) == -5
+
+
+def test_varlen_bwd_validation(lib):
+    f = lib.fa_varlen_bwd
+    # q, k, v, out, dout, lse, cu, num_seqs, max_seqlen, total, dq, dk, dv, delta, H, D, scale, causal, dtype, st
+    ok = [FAKE] * 7 + [3, 64, 100] + [FAKE] * 4 + [2, 64, 0.0, 1, 1, None]
+
+    def call(i=None, val=None):
+        a = list(ok)
+        if i is not None:
+            a[i] = val
+        return f(*a)
+
+    assert call(9, 0) == 0      # no tokens: nothing to do
+    assert call(6, None) == -1
+    assert call(15, 256) == -4
+    assert call(8, 0) == -2
+    assert call(6, FAKE + 2) == -5
+    assert call(18, 4) == -3

@@ -87,3 +87,42 @@ def test_bwd_delta_workspace_is_rowsum(cuda_device):
     fa.fa_bwd(q, k, v, out, do, lse, delta=delta)
     ref = (out.double() * do.double()).sum(-1).permute(0, 2, 1)
     torch.testing.assert_close(delta.double(), ref, rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("D,dtype,causal", [(64, torch.bfloat16, True), (128, torch.float16, False),
+                                            (32, torch.bfloat16, False), (128, torch.bfloat16, True)])
+def test_varlen_bwd_matches_oracle(cuda_device, D, dtype, causal):
+    """Packed sequences of mixed lengths (shorter than, equal to and longer than a tile, and
+    empty), several sharing one 128-token tile."""
+    import tiled_exact_attention_fwd_b200 as fa
+    lengths = [5, 130, 0, 64, 1, 200, 63, 17]
+    H = 2
+    q, k, v, cu = fa_inputs.packed_qkv(lengths, H, D, dtype, seed=D)
+    total = int(cu[-1])
+    do = fa_inputs.normal((total, H, D), dtype, seed=D + 1)
+    dev = cuda_device
+    qd, kd, vd, dod, cud = (t.to(dev) for t in (q, k, v, do, cu))
+    out, lse = fa.fa_varlen_fwd(qd, kd, vd, cud, max(lengths), causal=causal)
+    dq, dk, dv = fa.fa_varlen_bwd(qd, kd, vd, out, dod, lse, cud, max(lengths), causal=causal)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status()[0] == 0
+    rq, rk, rv = oracle.attention_varlen_backward(q, k, v, do, cu, causal=causal)
+    for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        _close(name, g, r, dtype)
+
+
+@pytest.mark.gpu
+def test_varlen_bwd_single_sequence_equals_dense(cuda_device):
+    """One packed sequence spanning everything gives exactly the dense kernels' gradients."""
+    import tiled_exact_attention_fwd_b200 as fa
+    S, H, D = 300, 2, 64
+    q, k, v = (t.to(cuda_device) for t in fa_inputs.dense_qkv(1, S, H, D, torch.bfloat16, seed=5))
+    do = fa_inputs.normal((1, S, H, D), torch.bfloat16, seed=6).to(cuda_device)
+    out, lse = fa.fa_fwd(q, k, v, causal=True)
+    ref = fa.fa_bwd(q, k, v, out, do, lse, causal=True)
+    cu = torch.tensor([0, S], dtype=torch.int32, device=cuda_device)
+    got = fa.fa_varlen_bwd(q[0], k[0], v[0], out[0], do[0], lse[0].contiguous(), cu, S, causal=True)
+    torch.cuda.synchronize()
+    for g, r in zip(got, ref):
+        assert torch.equal(g.view(torch.int16), r[0].view(torch.int16))

@@ -88,3 +88,19 @@ def test_head_subset_matches_full():
     for (b, h), grads in part.items():
         for a, f in zip(grads, full):
             np.testing.assert_array_equal(a, f[b, :, h])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_backward_equals_per_sequence_dense(causal):
+    """The packed gradients are those of each sequence alone (zero-length sequences allowed)."""
+    lengths = [5, 0, 17, 1, 9]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    total, H, D = int(cu[-1]), 2, 8
+    q, k, v, g = (_rand((total, H, D), s) for s in (71, 72, 73, 74))
+    dq, dk, dv = oracle.attention_varlen_backward(q, k, v, g, cu, causal=causal)
+    for s0, s1 in zip(cu[:-1], cu[1:]):
+        if s1 == s0:
+            continue
+        ref = oracle.attention_backward(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1], g[None, s0:s1], causal=causal)
+        for a, r in zip((dq, dk, dv), ref):
+            np.testing.assert_array_equal(a[s0:s1], r[0])

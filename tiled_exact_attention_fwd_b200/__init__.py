@@ -50,6 +50,8 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_paged.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
         L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
         L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp]
+        L.fa_varlen_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, i32, i32, f32, i32, i32,
+                                    vp]
         L.fa_unpad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fa_pad.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fa_unpad_qkv.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp]
@@ -57,7 +59,7 @@ def lib() -> ctypes.CDLL:
                                            vp]
         L.fa_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.fa_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
-        for f in (L.fa_fwd, L.fa_fwd_paged, L.fa_bwd, L.fa_bwd_noalloc, L.fa_varlen_fwd, L.fa_varlen_fwd_padded, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad,
+        for f in (L.fa_fwd, L.fa_fwd_paged, L.fa_bwd, L.fa_bwd_noalloc, L.fa_varlen_bwd, L.fa_varlen_fwd, L.fa_varlen_fwd_padded, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad,
                   L.fa_device_status,
                   L.fa_selftest_bounded_wait):
             f.restype = ctypes.c_int
@@ -147,6 +149,29 @@ def fa_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                       _ptr(delta), B, H, S, D, float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q),
                       _stream(stream))
     _check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def fa_varlen_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
+                  lse: torch.Tensor, cu_seqlens: torch.Tensor, max_seqlen: int, scale: Optional[float] = None,
+                  causal: bool = False, stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Packed backward: (total, H, D) tensors, lse (H, total) from fa_varlen_fwd -> (dq, dk, dv)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse),
+                 ("cu_seqlens", cu_seqlens)):
+        _cuda_contig(n, t)
+    if q.dim() != 3 or any(t.shape != q.shape or t.dtype != q.dtype for t in (k, v, out, dout)):
+        raise ValueError("q, k, v, out, dout must share one (total, H, D) shape and dtype")
+    total, H, D = q.shape
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (H, total):
+        raise ValueError("lse must be float32 (H, total)")
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    delta = torch.empty((H, total), device=q.device, dtype=torch.float32)
+    st = lib().fa_varlen_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(cu_seqlens),
+                             cu_seqlens.numel() - 1, int(max_seqlen), total, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(delta),
+                             H, D, float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
+    _check(st, "fa_varlen_bwd")
     return dq, dk, dv
 
 

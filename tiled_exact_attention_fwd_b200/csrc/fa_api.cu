@@ -170,18 +170,16 @@ fa_status fa_fwd_paged(const void *q, const void *k_cache, const void *v_cache, 
                    &paging);
 }
 
-fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
-                 void *dq, void *dk, void *dv, float *delta, int B, int H, int S, int D, float scale, int causal,
-                 fa_dtype dtype, void *stream) {
-    if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !delta) return FA_ERR_NULL;
-    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
-    if (D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;  // dK and dV accumulators share TMEM
-    if (B <= 0 || H <= 0 || S <= 0) return FA_ERR_SHAPE;
+}  // extern "C"
+
+namespace {
+
+// Shared by the dense and packed backward entry points: N token rows; cu_seqlens null for
+// dense (B sequences of S) or the packed offsets (B = 1, S = N).
+fa_status run_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+                  void *dq, void *dk, void *dv, float *delta, const int32_t *cu_seqlens, int num_seqs, int B, int H,
+                  int S, int D, float scale, int causal, fa_dtype dtype, void *stream) {
     const int64_t N = static_cast<int64_t>(B) * S;
-    if (N > INT32_MAX || B > 65535 || (S + 127) / 128 > 65535) return FA_ERR_SHAPE;
-    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(dout, 16) ||
-        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(delta, 4))
-        return FA_ERR_ALIGN;
     const bool bf16 = dtype == FA_BF16;
     const int inner = fa::fwd_box_inner_elems(D);
     CUtensorMap tq, tk, tv, tdo;
@@ -200,11 +198,52 @@ fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, c
     p.B = B;
     p.H = H;
     p.seqlen = S;
+    p.cu_seqlens = cu_seqlens;
+    p.num_seqs = num_seqs;
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = wait_limit_ns();
     const cudaError_t e = fa::launch_bwd(D, bf16, causal != 0, tq, tk, tv, tdo, p, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+bool bwd_aligned(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+                 const void *dq, const void *dk, const void *dv, const float *delta) {
+    return aligned(q, 16) && aligned(k, 16) && aligned(v, 16) && aligned(out, 16) && aligned(dout, 16) &&
+           aligned(dq, 16) && aligned(dk, 16) && aligned(dv, 16) && aligned(lse, 4) && aligned(delta, 4);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+                 void *dq, void *dk, void *dv, float *delta, int B, int H, int S, int D, float scale, int causal,
+                 fa_dtype dtype, void *stream) {
+    if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !delta) return FA_ERR_NULL;
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;  // dK and dV accumulators share TMEM
+    if (B <= 0 || H <= 0 || S <= 0) return FA_ERR_SHAPE;
+    const int64_t N = static_cast<int64_t>(B) * S;
+    if (N > INT32_MAX || B > 65535 || (S + 127) / 128 > 65535) return FA_ERR_SHAPE;
+    if (!bwd_aligned(q, k, v, out, dout, lse, dq, dk, dv, delta)) return FA_ERR_ALIGN;
+    return run_bwd(q, k, v, out, dout, lse, dq, dk, dv, delta, nullptr, 0, B, H, S, D, scale, causal, dtype, stream);
+}
+
+fa_status fa_varlen_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
+                        const float *lse, const int32_t *cu_seqlens, int num_seqs, int max_seqlen, int total,
+                        void *dq, void *dk, void *dv, float *delta, int H, int D, float scale, int causal,
+                        fa_dtype dtype, void *stream) {
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;
+    if (num_seqs < 0 || total < 0 || max_seqlen < 0 || H <= 0) return FA_ERR_SHAPE;
+    if (total == 0 || num_seqs == 0) return FA_OK;  // no rows, nothing to launch
+    if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !delta || !cu_seqlens) return FA_ERR_NULL;
+    if (max_seqlen == 0) return FA_ERR_SHAPE;
+    if ((static_cast<int64_t>(total) + 127) / 128 > 65535) return FA_ERR_SHAPE;
+    if (!bwd_aligned(q, k, v, out, dout, lse, dq, dk, dv, delta) || !aligned(cu_seqlens, 4)) return FA_ERR_ALIGN;
+    return run_bwd(q, k, v, out, dout, lse, dq, dk, dv, delta, cu_seqlens, num_seqs, 1, H, total, D, scale, causal,
+                   dtype, stream);
 }
 
 fa_status fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *out, const void *dout,

@@ -30,6 +30,7 @@
 #include "fa.h"
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
+#include "fa_seq.cuh"
 #include "fa_sync.cuh"
 
 namespace fa {
@@ -133,20 +134,39 @@ __device__ __forceinline__ void store_row(uint32_t taddr, float mul, uint8_t *gr
 
 // DKDV: the CTA owns key tile j = blockIdx.y; fixed A0 = K_j, A1 = V_j; ring B0 = Q_i, B1 = dO_i.
 // !DKDV: the CTA owns query tile i (longest first); fixed A0 = Q_i, A1 = dO_i; ring B0 = K_j, B1 = V_j.
-template <int D, bool BF16, bool CAUSAL, bool DKDV>
+// PACKED: (total, H, D) tensors with cu_seqlens; tiles are 128 consecutive tokens whatever
+// sequences they hold (p.B = 1, p.seqlen = total), the streamed windows cover the tokens of
+// the owned tile's sequences, and every element is masked to its own sequence.
+template <int D, bool BF16, bool CAUSAL, bool DKDV, bool PACKED>
 __global__ void __launch_bounds__(BwdCfg<D>::NUM_THREADS, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const BwdParams p) {
     using C = BwdCfg<D>;
     constexpr int BM = C::BM;
-    const int h = blockIdx.x, b = blockIdx.z, S = p.seqlen;
+    const int h = blockIdx.x, b = blockIdx.z, S = p.seqlen;  // packed: S = total tokens
     const int ntiles = (S + BM - 1) / BM;
-    const int own = DKDV ? static_cast<int>(blockIdx.y) : ntiles - 1 - static_cast<int>(blockIdx.y);
-    // tiles streamed through the ring: [t0, t1)
-    const int t0 = (DKDV && CAUSAL) ? own : 0;
-    const int t1 = (!DKDV && CAUSAL) ? own + 1 : ntiles;
-    const int n = t1 - t0;
+    const int own = (DKDV || PACKED) ? static_cast<int>(blockIdx.y) : ntiles - 1 - static_cast<int>(blockIdx.y);
+    const int own_start = own * BM;  // position of the owned tile's first row
+    // Streamed windows t = 0..n-1 start at positions ws + t*BM.
+    int ws, n;
+    if constexpr (PACKED) {
+        const int lane_ = threadIdx.x & 31;
+        const int last = min(own_start + BM, S) - 1;
+        const int s_first = warp_seq_of_token(p.cu_seqlens, p.num_seqs, own_start, lane_);
+        const int s_last = warp_seq_of_token(p.cu_seqlens, p.num_seqs, last, lane_);
+        const int seq_lo = __ldg(p.cu_seqlens + s_first), seq_hi = __ldg(p.cu_seqlens + s_last + 1);
+        // dK/dV: queries of the tile's sequences (from the first key on, when causal);
+        // dQ: keys of the tile's sequences (up to the last query, when causal)
+        ws = (DKDV && CAUSAL) ? own_start : seq_lo;
+        const int we = (!DKDV && CAUSAL) ? min(seq_hi, last + 1) : seq_hi;
+        n = (we - ws + BM - 1) / BM;
+    } else {
+        const int t0 = (DKDV && CAUSAL) ? own : 0;
+        const int t1 = (!DKDV && CAUSAL) ? own + 1 : ntiles;
+        ws = t0 * BM;
+        n = t1 - t0;
+    }
     const int64_t row0 = static_cast<int64_t>(b) * S;  // first token row of this batch entry
 
     extern __shared__ uint8_t smem_raw[];
@@ -200,14 +220,14 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const CUtensorMap *fa0 = DKDV ? &tm_k : &tm_q, *fa1 = DKDV ? &tm_v : &tm_do;
             const CUtensorMap *rb0 = DKDV ? &tm_q : &tm_k, *rb1 = DKDV ? &tm_do : &tm_v;
             mbar_arrive_expect_tx(fix_full, 2 * C::TILE_BYTES);
-            load_tile<D>(fixA0, fa0, fix_full, h, static_cast<int>(row0 + own * BM), pol_fix);
-            load_tile<D>(fixA1, fa1, fix_full, h, static_cast<int>(row0 + own * BM), pol_fix);
+            load_tile<D>(fixA0, fa0, fix_full, h, static_cast<int>(row0 + own_start), pol_fix);
+            load_tile<D>(fixA1, fa1, fix_full, h, static_cast<int>(row0 + own_start), pol_fix);
             int issued = 0;
             for (int t = 0; t < n; ++t) {
                 const int s = t & 1;
                 if (t >= 2 && !wait_bounded(&ring_empty[s], ((t >> 1) - 1) & 1, abort_flag, lim, 400 + s)) break;
                 mbar_arrive_expect_tx(&ring_full[s], 2 * C::TILE_BYTES);
-                const int row = static_cast<int>(row0 + (t0 + t) * BM);
+                const int row = static_cast<int>(row0 + ws + t * BM);
                 load_tile<D>(ring_tile(s, 0), rb0, &ring_full[s], h, row, pol_ring);
                 load_tile<D>(ring_tile(s, 1), rb1, &ring_full[s], h, row, pol_ring);
                 issued = t + 1;
@@ -257,7 +277,17 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int quarter = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
         const int r = quarter * 32 + lane;                // TMEM lane = row of the owned tile
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        const int own_pos = own * BM + r;  // sequence position of this row (key or query)
+        const int own_pos = own_start + r;  // position of this row (key or query)
+        // the positions this row may pair with: its sequence (packed) or [0, S)
+        int row_lo = 0, row_hi = S;
+        if constexpr (PACKED) {
+            const int tok = min(own_pos, S - 1);
+            const int s0 = warp_seq_of_token(p.cu_seqlens, p.num_seqs, min(own_start + quarter * 32, S - 1), lane);
+            const int sq = lane_seq_of_token(p.cu_seqlens, p.num_seqs, s0, tok, lane);
+            row_lo = __ldg(p.cu_seqlens + sq);
+            row_hi = __ldg(p.cu_seqlens + sq + 1);
+            if (own_pos >= S) row_lo = row_hi = 0;  // past the last token: pairs with nothing
+        }
         const float sl2 = p.scale_log2;
         constexpr float kLog2e = 1.4426950408889634f;
         const int64_t stat_base = (static_cast<int64_t>(b) * p.H + h) * S;
@@ -275,13 +305,13 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const bool publisher = DKDV && half == 0;  // publishes the statistics of query column r
         float my_nl = 0.f, my_nd = 0.f;  // dQ: this row's statistics; dK/dV: prefetched column stats
         if (publisher) {
-            if (n > 0) query_stats(t0 * BM + r, my_nl, my_nd);
+            if (n > 0) query_stats(ws + r, my_nl, my_nd);
         } else if (!DKDV) {
             query_stats(own_pos, my_nl, my_nd);
         }
         // P (or P^T) and dZ for 32 columns starting at col0; MASK applies the causal diagonal
         // and (dQ) the keys past the sequence end.
-        auto chunk = [&](auto mask_c, int col0, const float *snl, const float *snd, int key_hi, bool diag) {
+        auto chunk = [&](auto mask_c, int col0, const float *snl, const float *snd, int w0) {
             constexpr bool MASK = decltype(mask_c)::value;
             uint32_t sv[32], dv[32];
             tmem_ld32(tmem + lane_base + C::COL_S + col0, sv);
@@ -308,10 +338,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 f2_split(x2, x0, x1);
                 float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                 if constexpr (MASK) {
-                    // key position > query position weighs 0 (dK/dV rows are keys and columns
-                    // queries, dQ the other way round); dQ: keys past the sequence end weigh 0
-                    if (DKDV ? (diag && r > col) : ((diag && col > r) || col >= key_hi)) p0 = 0.f;
-                    if (DKDV ? (diag && r > col + 1) : ((diag && col + 1 > r) || col + 1 >= key_hi)) p1 = 0.f;
+                    // a pair weighs 0 unless the column lies in the row's sequence (or [0, S))
+                    // and, when causal, the key position is not past the query position (dK/dV
+                    // rows are keys and columns queries, dQ the other way round)
+                    const int c0 = w0 + col, c1 = c0 + 1;
+                    if (c0 < row_lo || c0 >= row_hi || (CAUSAL && (DKDV ? c0 < own_pos : c0 > own_pos))) p0 = 0.f;
+                    if (c1 < row_lo || c1 >= row_hi || (CAUSAL && (DKDV ? c1 < own_pos : c1 > own_pos))) p1 = 0.f;
                 }
                 const uint64_t z2 = fmul2(f2(p0, p1), fadd2(f2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])),
                                                             f2(nd0, nd1)));
@@ -332,7 +364,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         };
         for (int t = 0; ok && t < n; ++t) {
-            const int other = t0 + t;  // the streamed tile (query tile for dK/dV, key tile for dQ)
+            const int w0 = ws + t * BM;  // position of the streamed window's first row
             const int slot = t & 1;
             const float *snl = stats + slot * 2 * BM, *snd = snl + BM;
             if (DKDV) {
@@ -341,25 +373,26 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     stats[slot * 2 * BM + r] = my_nl;
                     stats[slot * 2 * BM + BM + r] = my_nd;
                     mbar_arrive(&stats_ready[slot]);
-                    if (t + 1 < n) query_stats((other + 1) * BM + r, my_nl, my_nd);
+                    if (t + 1 < n) query_stats(w0 + BM + r, my_nl, my_nd);
                 }
                 if (!(ok = __all_sync(0xffffffffu, wait_bounded(&stats_ready[slot], (t >> 1) & 1, abort_flag, lim, 440))))
                     break;
             }
             if (!(ok = __all_sync(0xffffffffu, wait_bounded(s_full, t & 1, abort_flag, lim, 450)))) break;
             tc_fence_after_sync();
-            const int key_hi = DKDV ? BM : min(BM, S - other * BM);
-            const bool diag = CAUSAL && other == own;
-            const bool masked = diag || key_hi < BM;
+            // does any pair of this warp's rows with the window need a mask?
+            const bool row_partial = w0 < row_lo || w0 + BM > row_hi ||
+                                     (CAUSAL && (DKDV ? w0 < own_pos : w0 + BM - 1 > own_pos));
+            const bool masked = __any_sync(0xffffffffu, row_partial);
             // this thread's 64 columns: [64*half, 64*half + 64), two chunks; each chunk's
             // results are stored over columns this thread has already read
 #pragma unroll 1
             for (int c = 0; c < 2; ++c) {
                 const int col0 = half * 64 + c * 32;
                 if (masked)
-                    chunk(std::integral_constant<bool, true>{}, col0, snl, snd, key_hi, diag);
+                    chunk(std::integral_constant<bool, true>{}, col0, snl, snd, w0);
                 else
-                    chunk(std::integral_constant<bool, false>{}, col0, snl, snd, key_hi, diag);
+                    chunk(std::integral_constant<bool, false>{}, col0, snl, snd, w0);
             }
             tmem_st_wait();
             tc_fence_before_sync();
@@ -435,11 +468,11 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const void *out, const v
     }
 }
 
-template <int D, bool BF16, bool CAUSAL, bool DKDV>
+template <int D, bool BF16, bool CAUSAL, bool DKDV, bool PACKED>
 cudaError_t launch_bwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
                          const BwdParams &p, dim3 grid, cudaStream_t st) {
     using C = BwdCfg<D>;
-    auto kern = fa_bwd_kernel<D, BF16, CAUSAL, DKDV>;
+    auto kern = fa_bwd_kernel<D, BF16, CAUSAL, DKDV, PACKED>;
     static uint64_t attr_set_mask = 0;  // per-device shared-memory opt-in done
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -468,11 +501,18 @@ cudaError_t launch_bwd_d(bool causal, const CUtensorMap &tq, const CUtensorMap &
     if (e != cudaSuccess) return e;
     const int ntiles = (p.seqlen + 127) / 128;
     const dim3 grid(static_cast<unsigned>(p.H), static_cast<unsigned>(ntiles), static_cast<unsigned>(p.B));
-    e = causal ? launch_bwd_t<D, BF16, true, true>(tq, tk, tv, tdo, p, grid, st)
-               : launch_bwd_t<D, BF16, false, true>(tq, tk, tv, tdo, p, grid, st);
+    if (p.cu_seqlens) {
+        e = causal ? launch_bwd_t<D, BF16, true, true, true>(tq, tk, tv, tdo, p, grid, st)
+                   : launch_bwd_t<D, BF16, false, true, true>(tq, tk, tv, tdo, p, grid, st);
+        if (e != cudaSuccess) return e;
+        return causal ? launch_bwd_t<D, BF16, true, false, true>(tq, tk, tv, tdo, p, grid, st)
+                      : launch_bwd_t<D, BF16, false, false, true>(tq, tk, tv, tdo, p, grid, st);
+    }
+    e = causal ? launch_bwd_t<D, BF16, true, true, false>(tq, tk, tv, tdo, p, grid, st)
+               : launch_bwd_t<D, BF16, false, true, false>(tq, tk, tv, tdo, p, grid, st);
     if (e != cudaSuccess) return e;
-    return causal ? launch_bwd_t<D, BF16, true, false>(tq, tk, tv, tdo, p, grid, st)
-                  : launch_bwd_t<D, BF16, false, false>(tq, tk, tv, tdo, p, grid, st);
+    return causal ? launch_bwd_t<D, BF16, true, false, false>(tq, tk, tv, tdo, p, grid, st)
+                  : launch_bwd_t<D, BF16, false, false, false>(tq, tk, tv, tdo, p, grid, st);
 }
 
 }  // namespace

@@ -50,6 +50,7 @@
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
 #include "fa_sync.cuh"
+#include "fa_seq.cuh"
 
 namespace fa {
 
@@ -118,52 +119,6 @@ struct Cfg {
     // The MMA thread waits for K_{j+1} while V_j is still held: the ring needs both, plus a part.
     static_assert(NS >= 2 * UNITS + 1, "K/V ring too shallow");
 };
-
-// Sequence that packed token `tok` belongs to: the s with cu[s] <= tok < cu[s+1]
-// (binary search over the num_seqs + 1 offsets; empty sequences are skipped).
-__device__ __forceinline__ int seq_of_token(const int32_t *cu, int num_seqs, int tok) {
-    int lo = 0, hi = num_seqs;  // invariant: cu[lo] <= tok < cu[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(cu + mid) <= tok) lo = mid; else hi = mid;
-    }
-    return lo;
-}
-
-// seq_of_token for a token shared by the whole warp: 32 probes per dependent load.
-__device__ __forceinline__ int warp_seq_of_token(const int32_t *cu, int num_seqs, int tok, int lane) {
-    int lo = 0, hi = num_seqs;  // answer s in [lo, hi - 1]: the last s with cu[s] <= tok
-    while (hi - lo > 32) {
-        const int step = (hi - lo + 31) / 32;
-        const int p = lo + lane * step;
-        const bool le = p < hi && __ldg(cu + p) <= tok;
-        const int c = __popc(__ballot_sync(0xffffffffu, le));  // probes <= tok form a prefix (c >= 1)
-        const int new_lo = lo + (c - 1) * step;
-        hi = min(hi, lo + c * step);
-        lo = new_lo;
-    }
-    const int p = lo + lane;
-    const bool le = p < hi && __ldg(cu + p) <= tok;
-    return lo + __popc(__ballot_sync(0xffffffffu, le)) - 1;
-}
-
-// Sequence of each lane's token `tok` (tokens of one warp, >= cu[s0] where s0 is the sequence
-// of the warp's first token): one 32-wide load of cu[s0 + 1 ..] and a 5-step search over the
-// lanes; falls back to the plain search when the warp's tokens span more than 32 sequences.
-__device__ __forceinline__ int lane_seq_of_token(const int32_t *cu, int num_seqs, int s0, int tok, int lane) {
-    const int wi = s0 + 1 + lane;
-    const int w = (wi <= num_seqs) ? __ldg(cu + wi) : 0x7fffffff;
-    int lo = 0, hi = 32;  // count of window entries <= tok, in [lo, hi]
-#pragma unroll
-    for (int k = 0; k < 6; ++k) {
-        const int mid = (lo + hi + 1) >> 1;
-        const int v = __shfl_sync(0xffffffffu, w, (mid - 1) & 31);
-        if (mid <= hi && lo < hi) {
-            if (v <= tok) lo = mid; else hi = mid - 1;
-        }
-    }
-    return (lo < 32) ? s0 + lo : seq_of_token(cu, num_seqs, tok);
-}
 
 // Single-tile order of MMA steps: K0, K1, V0, K2, V1, ..., V_{n-1} (QK runs one tile ahead).
 __device__ __forceinline__ void decode_step(int idx, int n, bool &is_v, int &j) {

@@ -56,10 +56,12 @@ cudaError_t fwd_paged_take_device_error(int *code, int *where);
 // Attention backward (fa_bwd.cu): dQ, dK, dV from q, k, v, out, dout and the forward's LSE.
 struct BwdParams {
     const void *out, *dout;  // (B, S, H, D), read by the delta kernel
-    const float *lse;        // (B, H, S) from the forward
-    float *delta;            // (B, H, S) workspace: rowsum(dO * O)
+    const float *lse;        // (B, H, S) from the forward (packed: (H, total))
+    float *delta;            // (B, H, S) workspace: rowsum(dO * O) (packed: (H, total))
     void *dq, *dk, *dv;      // (B, S, H, D) gradients
-    int B, H, seqlen;
+    int B, H, seqlen;        // packed: B = 1, seqlen = total tokens
+    const int32_t *cu_seqlens;  // packed (total, H, D) tensors: sequence offsets (else null)
+    int num_seqs;
     float scale;             // softmax scale
     float scale_log2;        // scale * log2(e)
     uint64_t timeout_ns;     // bound of every pipeline wait
