@@ -1,6 +1,8 @@
 /*
  * fa.h -- C ABI of libfa: exact attention forward computed tile by tile on one
- * NVIDIA B200 (sm_100a), plus the unpad gather and pad scatter of the packed path.
+ * NVIDIA B200 (sm_100a), dense, packed and with paged K/V; the unpad gather and pad
+ * scatter of the packed path (also fused into the forward); and the backward pass by
+ * recomputation.
  *
  * Every entry point is asynchronous on the caller's CUDA stream, allocates no
  * device memory, never synchronises, and takes plain device pointers that the
@@ -22,9 +24,10 @@
  *   packed q, k, v, out : (total, H, D)        lse : (H, total)  float32
  *   lse is the natural log of sum_j exp(scale * q.k_j) over the keys the row sees.
  *
- * Supported: D in {32, 64, 128, 256}; q, k, v, out 16-byte aligned; lse 4-byte
- * aligned (may be NULL to skip it). Causal masking is aligned at the first token
- * of each sequence (query and key lengths are equal per sequence).
+ * Supported: D in {32, 64, 128, 256} (backward: 32, 64, 128); q, k, v, out 16-byte
+ * aligned; lse 4-byte aligned (may be NULL to skip it in the forward). Causal masking is
+ * aligned at the first token of each sequence (query and key lengths are equal per
+ * sequence). The header is plain C99.
  */
 #ifndef FA_H_
 #define FA_H_

@@ -19,12 +19,16 @@
 //   warps 0-7   two softmax warpgroups, warpgroup t for tile t; thread (warp w, lane l)
 //               owns row 32*(w%4)+l of its tile, the TMEM lane its warp may access. It
 //               reads its S row with tcgen05.ld, masks, updates (m, l) with exp2 of scores
-//               pre-multiplied by scale*log2(e), writes P (16-bit) over S in TMEM, and when
-//               its max grew by more than 2^8 rescales its O row in TMEM (lazy rescale:
-//               between rescales every exponent uses the same stale max, which the final
-//               1/l cancels exactly). At the end: O/l -> fp16/bf16 -> global, and the LSE.
+//               pre-multiplied by scale*log2(e), writes P (16-bit) over S in TMEM (D <= 64:
+//               into its own TMEM columns, so the next S can be computed meanwhile), and
+//               when its max grew by more than 2^8 rescales its O row in TMEM (lazy
+//               rescale: between rescales every exponent uses the same stale max, which the
+//               final 1/l cancels exactly). At the end: O/l -> fp16/bf16 -> global, and the
+//               LSE.
 //   warp 8      TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ... through an
-//               NS-stage shared-memory ring guarded by full/empty mbarriers.
+//               NS-stage shared-memory ring guarded by full/empty mbarriers. When tile
+//               rows must be gathered row by row (fused unpad, 16-row pages), warps 8, 10
+//               and 11 copy them with cp.async instead.
 //   warp 9      allocates TMEM; one thread issues every tcgen05.mma:
 //                 S_t = Q_t K_j^T   (A = Q_t, B = K_j, both K-major in SMEM, 128B swizzle)
 //                 O_t += P_t V_j    (A = P_t read from TMEM, B = V_j MN-major in SMEM)
