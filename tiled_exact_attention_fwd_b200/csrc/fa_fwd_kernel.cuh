@@ -554,49 +554,87 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // tile's barrier when they land, and the MMA thread fences the async proxy.
                 constexpr int CPB = SW / 16;  // 16-byte chunks per swizzle row (column block)
                 const int pw = (warp == C::WARP_TMA) ? 0 : warp - C::WARP_MMA;  // producer warp 0..2
-                // Copies rows [tok0, tok0 + rows) x column blocks [b0, b0 + NB) into dst laid out
-                // as [NB][rows][SW].
-                auto fill = [&](auto nb_c, uint8_t *dst, const void *src, uint64_t *bar, int tok0, int rows,
-                                int b0) {
+                // A job copies rows [tok0, tok0 + rows) x column blocks [b0, b0 + NB) into dst laid
+                // out as [NB][rows][SW]. Its 32-row groups go round-robin over the three warps (at
+                // most two groups per warp: rows <= 128); each warp first reads its groups' padded
+                // rows (one coalesced load per group) and then every lane issues 16-byte copies.
+                // The padded rows of the next job are read while this job's copies are issued,
+                // so the index loads never wait in line.
+                auto load_rows = [&](int tok0, int rows, int64_t (&pr)[2]) {
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const int g = pw + 3 * k;
+                        const int tok = tok0 + g * 32 + lane;
+                        int64_t r = (g * 32 < rows && tok >= 0 && tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
+                        if (r < 0 || r >= p.padded_rows) r = 0;  // never read outside q/k/v
+                        pr[k] = r;
+                    }
+                };
+                auto copy_rows = [&](auto nb_c, uint8_t *dst, const void *src, uint64_t *bar, int rows, int b0,
+                                     const int64_t (&pr)[2]) {
                     constexpr int CPR = decltype(nb_c)::value * CPB;  // chunks per row
                     const uint32_t dst_u32 = smem_u32(dst);
-                    // 32-row groups round-robin over the three warps: one coalesced load of the
-                    // group's padded rows, then every lane issues CPR 16-byte copies.
-                    for (int g = pw; g * 32 < rows; g += 3) {
-                        const int tok = tok0 + g * 32 + lane;
-                        int64_t prow = (tok >= 0 && tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
-                        if (prow < 0 || prow >= p.padded_rows) prow = 0;  // never read outside q/k/v
-                        const uint8_t *srow = static_cast<const uint8_t *>(src) + b0 * SW;
+                    const uint8_t *srow = static_cast<const uint8_t *>(src) + b0 * SW;
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const int g = pw + 3 * k;
+                        if (g * 32 >= rows) continue;
 #pragma unroll 4
                         for (int i = 0; i < CPR; ++i) {
                             const int idx = i * 32 + lane;
                             const int rr = idx / CPR, ch = idx % CPR;
-                            const int64_t pr = __shfl_sync(0xffffffffu, prow, rr);
+                            const int64_t prow = __shfl_sync(0xffffffffu, pr[k], rr);
                             const int r = g * 32 + rr;
                             const int blk = ch / CPB, cc = ch % CPB;
                             const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
                             cp_async_16(dst_u32 + blk * rows * SW + r * SW + ((cc ^ swz) << 4),
-                                        srow + (pr * p.H + h) * static_cast<int64_t>(D) * 2 + ch * 16);
+                                        srow + (prow * p.H + h) * static_cast<int64_t>(D) * 2 + ch * 16);
                         }
                     }
                     cp_async_mbar_arrive(bar);  // arrives once this thread's copies have landed
                 };
                 using AllBlk = std::integral_constant<int, C::NBLK>;
                 using KBlk = std::integral_constant<int, C::KBLK_PER_UNIT>;
-                for (int t = 0; t < nq; ++t)
-                    fill(AllBlk{}, c.sQ + t * C::Q_BYTES, p.q, &c.q_full[t], qbase + t * BM, BM, 0);
-                for (int U = 0; U < loads; ++U) {
-                    const int stage = U % NS;
+                // jobs 0..nq-1: query tiles; then one job per K/V ring part U = job - nq
+                const int njobs = nq + loads;
+                auto job_rows = [&](int J, int &tok0, int &rows) {
+                    if (J < nq) {
+                        tok0 = qbase + J * BM;
+                        rows = BM;
+                    } else {
+                        const int U = J - nq, L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
+                        tok0 = kvbase + j * BN + ((L & 1) ? u * C::VROWS_PER_UNIT : 0);
+                        rows = (L & 1) ? C::VROWS_PER_UNIT : BN;
+                    }
+                };
+                int64_t cur[2], nxt[2];
+                {
+                    int tok0, rows;
+                    job_rows(0, tok0, rows);
+                    load_rows(tok0, rows, nxt);
+                }
+                for (int J = 0; J < njobs; ++J) {
+                    cur[0] = nxt[0];
+                    cur[1] = nxt[1];
+                    if (J + 1 < njobs) {
+                        int tok0, rows;
+                        job_rows(J + 1, tok0, rows);
+                        load_rows(tok0, rows, nxt);
+                    }
+                    if (J < nq) {
+                        copy_rows(AllBlk{}, c.sQ + J * C::Q_BYTES, p.q, &c.q_full[J], BM, 0, cur);
+                        continue;
+                    }
+                    const int U = J - nq, stage = U % NS;
                     if (U >= NS &&
                         !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
                         break;
-                    const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
+                    const int L = U / C::UNITS, u = U % C::UNITS;
                     uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
                     if (L & 1)
-                        fill(AllBlk{}, dst, p.v, &c.kv_full[stage], kvbase + j * BN + u * C::VROWS_PER_UNIT,
-                             C::VROWS_PER_UNIT, 0);
+                        copy_rows(AllBlk{}, dst, p.v, &c.kv_full[stage], C::VROWS_PER_UNIT, 0, cur);
                     else
-                        fill(KBlk{}, dst, p.k, &c.kv_full[stage], kvbase + j * BN, BN, u * C::KBLK_PER_UNIT);
+                        copy_rows(KBlk{}, dst, p.k, &c.kv_full[stage], BN, u * C::KBLK_PER_UNIT, cur);
                     issued = U + 1;
                 }
                 cp_async_wait_all();  // nothing of this thread is left in flight at exit
