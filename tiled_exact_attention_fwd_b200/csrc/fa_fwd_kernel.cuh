@@ -28,7 +28,11 @@
 //   warp 8      TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ... through an
 //               NS-stage shared-memory ring guarded by full/empty mbarriers. When tile
 //               rows must be gathered row by row (fused unpad, 16-row pages), warps 8, 10
-//               and 11 copy them with cp.async instead.
+//               and 11 copy them with cp.async instead (fused unpad: each softmax warp
+//               copies its own Q rows, and warps 8, 10 and 11 clear the output's padding
+//               rows once their K/V copies are issued).
+//   epilogue    each softmax warp stages its 32 O rows in its tile's Q buffer (free once
+//               the tile's MMAs are done) and writes them out as whole rows.
 //   warp 9      allocates TMEM; one thread issues every tcgen05.mma:
 //                 S_t = Q_t K_j^T   (A = Q_t, B = K_j, both K-major in SMEM, 128B swizzle)
 //                 O_t += P_t V_j    (A = P_t read from TMEM, B = V_j MN-major in SMEM)
@@ -348,6 +352,43 @@ __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first
     return true;
 }
 
+// Fused packed path: padded rows of the 32-row groups g0 and g0 + 3 of a copy job over tokens
+// [tok0, tok0 + rows), one row per lane; rows past the job or the tokens, and indices outside
+// the padded tensor, read as row 0 (never outside q/k/v; the masks ignore such rows).
+__device__ __forceinline__ void fused_group_rows(const FwdParams &p, int tok0, int rows, int g0, int lane,
+                                                 int64_t (&pr)[2]) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int g = g0 + 3 * k;
+        const int tok = tok0 + g * 32 + lane;
+        int64_t r = (g * 32 < rows && tok >= 0 && tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
+        if (r < 0 || r >= p.padded_rows) r = 0;
+        pr[k] = r;
+    }
+}
+
+// Fused packed path: one warp copies the 32-row group g of a tile laid out [NB][rows][SW]
+// (the swizzled layout the TMA would produce) with 16-byte cp.async; tile row g*32 + i is
+// source row pr of lane i, whose column blocks [b0, b0 + NB) start at src + b0 * SW.
+template <int NB, int SW, int D>
+__device__ __forceinline__ void copy_group(uint32_t dst, int rows, int g, int64_t pr, const void *src, int b0,
+                                           int H, int h, int lane) {
+    constexpr int CPB = SW / 16;      // 16-byte chunks per swizzle row (column block)
+    constexpr int CPR = NB * CPB;     // chunks per tile row
+    const uint8_t *srow = static_cast<const uint8_t *>(src) + b0 * SW;
+#pragma unroll 4
+    for (int i = 0; i < CPR; ++i) {
+        const int idx = i * 32 + lane;
+        const int rr = idx / CPR, ch = idx % CPR;
+        const int64_t prow = __shfl_sync(0xffffffffu, pr, rr);
+        const int r = g * 32 + rr;
+        const int blk = ch / CPB, cc = ch % CPB;
+        const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
+        cp_async_16(dst + blk * rows * SW + r * SW + ((cc ^ swz) << 4),
+                    srow + (prow * H + h) * static_cast<int64_t>(D) * 2 + ch * 16);
+    }
+}
+
 // PAGED: K/V read through p.block_table (a separate instantiation, so the producer code of
 // the contiguous path stays as small as its register budget wants).
 template <int D, bool BF16, bool CAUSAL, bool PAGED>
@@ -383,17 +424,25 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (qbase >= p.total_tokens) return;
         two = (C::MAXQ == 2) && (qbase + BM < p.total_tokens);
         const int ln = threadIdx.x & 31;
-        const int s_first = warp_seq_of_token(p.cu_seqlens, p.num_seqs, qbase, ln);
-        kvbase = p.cu_seqlens[s_first];
+        // With fewer than 64 sequences every warp holds all of cu_seqlens (two entries per
+        // lane), so the lookups below are ballots and shuffles after one round of loads;
+        // otherwise each lookup is a search with dependent loads.
+        const CuWindow win(p.cu_seqlens, p.num_seqs, ln);
+        auto seq_of = [win, ln, &p](int tok) {
+            return win.ok ? win.seq(tok, ln) : warp_seq_of_token(p.cu_seqlens, p.num_seqs, tok, ln);
+        };
+        auto cu_at = [win, &p](int s) { return win.ok ? win.at(s) : p.cu_seqlens[s]; };
+        const int s_first = seq_of(qbase);
+        kvbase = cu_at(s_first);
         // keys of a tile end with its last row's sequence (or the causal limit)
         auto kv_end = [&](int tlast) {
-            const int s_last = warp_seq_of_token(p.cu_seqlens, p.num_seqs, tlast, ln);
-            return (CAUSAL ? min(p.cu_seqlens[s_last + 1], tlast + 1) : p.cu_seqlens[s_last + 1]) - kvbase;
+            const int s_last = seq_of(tlast);
+            return (CAUSAL ? min(cu_at(s_last + 1), tlast + 1) : cu_at(s_last + 1)) - kvbase;
         };
         kv_end_A = kv_end(min(qbase + BM, p.total_tokens) - 1);
         if (two) {
             kv_end_B = kv_end(min(qbase + 2 * BM, p.total_tokens) - 1);
-            kv_start_B = p.cu_seqlens[warp_seq_of_token(p.cu_seqlens, p.num_seqs, qbase + BM, ln)] - kvbase;
+            kv_start_B = cu_at(seq_of(qbase + BM)) - kvbase;
         }
     }
 
@@ -434,11 +483,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int pw = (warp == C::WARP_TMA) ? 0 : warp - C::WARP_MMA;  // copy producer warp 0..2 (8, 10, 11)
+    // Fused packed path: the copy warps read the padded rows of their groups of the first key
+    // part now, so that load overlaps the barrier and TMEM set-up.
+    int64_t first_rows[2] = {0, 0};
+    if (p.gather && (warp == C::WARP_TMA || warp > C::WARP_MMA)) fused_group_rows(p, kvbase, BN, pw, lane, first_rows);
 
     if (threadIdx.x == 0) {
         const int fill_arrivals = c.fused ? 96 : 1;  // copy producers: the 96 copy threads arrive
+        // fused packed path: a query tile is copied by the 128 threads of its softmax warpgroup
+        const int q_arrivals = p.gather ? 128 : fill_arrivals;
         for (int t = 0; t < 2; ++t) {
-            mbar_init(&c.q_full[t], fill_arrivals);
+            mbar_init(&c.q_full[t], q_arrivals);
             mbar_init(&c.s_full[t], 1);
             mbar_init(&c.p_full[t], 128);
             mbar_init(&c.pv_done[t], 1);
@@ -483,7 +539,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // pos of the sequence, read from its page; positions past the sequence end
                 // are zero-filled (no page is read for them). Q rows are plain token rows.
                 constexpr int CPB = SW / 16;
-                const int pw = (warp == C::WARP_TMA) ? 0 : warp - C::WARP_MMA;
                 const int32_t *bt = p.block_table + static_cast<int64_t>(blockIdx.z) * p.max_blocks;
                 bool bad_page = false;
                 // rows [pos0, pos0 + rows) x column blocks [b0, b0 + NB) into dst as [NB][rows][SW];
@@ -547,95 +602,99 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 issued = 0;
                 if (bad_page) record_error(FA_ERR_INDEX, 151);
             } else if (p.gather) {
-                // Fused packed path: warps 8, 10 and 11 (96 threads) copy every tile row from
-                // the padded tensor (row = padded row of the packed token; rows past the last
-                // token read row 0, which the masks then ignore) with 16-byte cp.async into the
-                // same swizzled layout the TMA would produce; each thread's copies arrive on the
-                // tile's barrier when they land, and the MMA thread fences the async proxy.
-                constexpr int CPB = SW / 16;  // 16-byte chunks per swizzle row (column block)
-                const int pw = (warp == C::WARP_TMA) ? 0 : warp - C::WARP_MMA;  // producer warp 0..2
-                // A job copies rows [tok0, tok0 + rows) x column blocks [b0, b0 + NB) into dst laid
-                // out as [NB][rows][SW]. Its 32-row groups go round-robin over the three warps (at
-                // most two groups per warp: rows <= 128); each warp first reads its groups' padded
-                // rows (one coalesced load per group) and then every lane issues 16-byte copies.
-                // The padded rows of the next job are read while this job's copies are issued,
-                // so the index loads never wait in line.
-                auto load_rows = [&](int tok0, int rows, int64_t (&pr)[2]) {
-#pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const int g = pw + 3 * k;
-                        const int tok = tok0 + g * 32 + lane;
-                        int64_t r = (g * 32 < rows && tok >= 0 && tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
-                        if (r < 0 || r >= p.padded_rows) r = 0;  // never read outside q/k/v
-                        pr[k] = r;
-                    }
+                // Fused packed path: warps 8, 10 and 11 (96 threads) copy every K/V row from the
+                // padded tensor (row = padded row of the packed token; rows past the last token
+                // read row 0, which the masks then ignore) with 16-byte cp.async into the same
+                // swizzled layout the TMA would produce; each thread's copies arrive on the part's
+                // barrier when they land, and the MMA thread fences the async proxy. (The softmax
+                // warps copy the query tiles.) The 32-row groups of the ring parts are dealt to
+                // the three warps in one running order (group G to warp G % 3), so each warp moves
+                // a third of the bytes and holds at most two groups of a part. A warp reads the
+                // padded rows of its next part's groups (one coalesced load per group) before it
+                // issues this part's copies, so index loads never wait in line.
+                auto part_rows = [&](int U, int &tok0, int &rows) {
+                    const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
+                    tok0 = kvbase + j * BN + ((L & 1) ? u * C::VROWS_PER_UNIT : 0);
+                    rows = (L & 1) ? C::VROWS_PER_UNIT : BN;
                 };
-                auto copy_rows = [&](auto nb_c, uint8_t *dst, const void *src, uint64_t *bar, int rows, int b0,
-                                     const int64_t (&pr)[2]) {
-                    constexpr int CPR = decltype(nb_c)::value * CPB;  // chunks per row
-                    const uint32_t dst_u32 = smem_u32(dst);
-                    const uint8_t *srow = static_cast<const uint8_t *>(src) + b0 * SW;
-#pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const int g = pw + 3 * k;
-                        if (g * 32 >= rows) continue;
-#pragma unroll 4
-                        for (int i = 0; i < CPR; ++i) {
-                            const int idx = i * 32 + lane;
-                            const int rr = idx / CPR, ch = idx % CPR;
-                            const int64_t prow = __shfl_sync(0xffffffffu, pr[k], rr);
-                            const int r = g * 32 + rr;
-                            const int blk = ch / CPB, cc = ch % CPB;
-                            const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
-                            cp_async_16(dst_u32 + blk * rows * SW + r * SW + ((cc ^ swz) << 4),
-                                        srow + (prow * p.H + h) * static_cast<int64_t>(D) * 2 + ch * 16);
-                        }
-                    }
-                    cp_async_mbar_arrive(bar);  // arrives once this thread's copies have landed
-                };
-                using AllBlk = std::integral_constant<int, C::NBLK>;
-                using KBlk = std::integral_constant<int, C::KBLK_PER_UNIT>;
-                // jobs 0..nq-1: query tiles; then one job per K/V ring part U = job - nq
-                const int njobs = nq + loads;
-                auto job_rows = [&](int J, int &tok0, int &rows) {
-                    if (J < nq) {
-                        tok0 = qbase + J * BM;
-                        rows = BM;
-                    } else {
-                        const int U = J - nq, L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
-                        tok0 = kvbase + j * BN + ((L & 1) ? u * C::VROWS_PER_UNIT : 0);
-                        rows = (L & 1) ? C::VROWS_PER_UNIT : BN;
-                    }
-                };
-                int64_t cur[2], nxt[2];
-                {
+                int64_t cur[2], nxt[2] = {first_rows[0], first_rows[1]};  // part 0's rows: read at set-up
+                int gU = 0;                                                // running index of part U's first group
+                for (int U = 0; U < loads; ++U) {
                     int tok0, rows;
-                    job_rows(0, tok0, rows);
-                    load_rows(tok0, rows, nxt);
-                }
-                for (int J = 0; J < njobs; ++J) {
+                    part_rows(U, tok0, rows);
+                    const int g0 = (pw + 3 - gU % 3) % 3;
+                    gU += rows / 32;
                     cur[0] = nxt[0];
                     cur[1] = nxt[1];
-                    if (J + 1 < njobs) {
-                        int tok0, rows;
-                        job_rows(J + 1, tok0, rows);
-                        load_rows(tok0, rows, nxt);
+                    if (U + 1 < loads) {
+                        int tok1, rows1;
+                        part_rows(U + 1, tok1, rows1);
+                        fused_group_rows(p, tok1, rows1, (pw + 3 - gU % 3) % 3, lane, nxt);
                     }
-                    if (J < nq) {
-                        copy_rows(AllBlk{}, c.sQ + J * C::Q_BYTES, p.q, &c.q_full[J], BM, 0, cur);
-                        continue;
-                    }
-                    const int U = J - nq, stage = U % NS;
+                    const int stage = U % NS;
                     if (U >= NS &&
                         !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
                         break;
-                    const int L = U / C::UNITS, u = U % C::UNITS;
-                    uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
-                    if (L & 1)
-                        copy_rows(AllBlk{}, dst, p.v, &c.kv_full[stage], C::VROWS_PER_UNIT, 0, cur);
-                    else
-                        copy_rows(KBlk{}, dst, p.k, &c.kv_full[stage], BN, u * C::KBLK_PER_UNIT, cur);
+                    const uint32_t dst = smem_u32(c.sKV + stage * C::UNIT_BYTES);
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const int g = g0 + 3 * k;
+                        if (g * 32 >= rows) continue;
+                        if ((U / C::UNITS) & 1)
+                            copy_group<C::NBLK, SW, D>(dst, rows, g, cur[k], p.v, 0, p.H, h, lane);
+                        else
+                            copy_group<C::KBLK_PER_UNIT, SW, D>(dst, rows, g, cur[k], p.k,
+                                                                (U % C::UNITS) * C::KBLK_PER_UNIT, p.H, h, lane);
+                    }
+                    cp_async_mbar_arrive(&c.kv_full[stage]);  // arrives once this thread's copies have landed
                     issued = U + 1;
+                }
+                if (!*c.abort_flag) {
+                    // Fused pad, while the attention runs: the packed tokens of this CTA go in
+                    // groups of 32 over the three warps; a group owns the padded rows from just
+                    // after the previous token's row up to its last token's row (through the end
+                    // of the tensor for the last token, from row 0 for the first). Of those, the
+                    // rows no token maps to become 0 (the others receive O). Candidates go 32 at
+                    // a time; the ones to clear are written whole, several rows per instruction.
+                    constexpr int RB = D * 2;                // bytes of one row of one head
+                    constexpr int CH = RB / 16;              // 16-byte chunks per row
+                    constexpr int LPR = CH < 32 ? CH : 32;  // lanes per row
+                    constexpr int RPI = 32 / LPR;            // rows per store instruction
+                    const int ch = lane % LPR;
+                    uint8_t *const zbase = static_cast<uint8_t *>(p.out) + static_cast<int64_t>(h) * RB + ch * 16;
+                    for (int gi = pw; gi < C::MAXQ * 4; gi += 3) {
+                        const int64_t tw0 = static_cast<int64_t>(qbase) + gi * 32;
+                        if (tw0 >= p.total_tokens) break;
+                        const int64_t tw1 = min(tw0 + 32, static_cast<int64_t>(p.total_tokens)) - 1;
+                        // padded rows of the group's tokens, sorted (lanes past the last token: +inf)
+                        const int64_t g_lane = (tw0 + lane <= tw1) ? __ldg(p.gather + tw0 + lane) : INT64_MAX;
+                        const int64_t lo_row = max(int64_t(0), (tw0 == 0) ? int64_t(0) : __ldg(p.gather + tw0 - 1) + 1);
+                        const int64_t hi_row =
+                            min(p.padded_rows, (tw1 == p.total_tokens - 1) ? p.padded_rows : __ldg(p.gather + tw1));
+                        for (int64_t base = lo_row; base < hi_row; base += 32) {
+                            const int64_t pr = base + lane;
+                            // is pr one of the 32 mapped rows? binary search over the lanes' sorted values
+                            int lo = 0;
+#pragma unroll
+                            for (int step = 16; step >= 1; step >>= 1) {
+                                const int64_t v = __shfl_sync(0xffffffffu, g_lane, lo + step - 1);
+                                if (v < pr) lo += step;
+                            }
+                            const bool mapped = __shfl_sync(0xffffffffu, g_lane, lo & 31) == pr;
+                            unsigned z = __ballot_sync(0xffffffffu, pr < hi_row && !mapped);  // rows to clear
+                            while (z) {
+                                int mine = -1;  // the candidate this lane's row slot takes
+#pragma unroll
+                                for (int sl = 0; sl < RPI; ++sl) {
+                                    const int bit = z ? __ffs(z) - 1 : -1;
+                                    z &= z - 1;
+                                    if (lane / LPR == sl) mine = bit;
+                                }
+                                if (mine >= 0)
+                                    *reinterpret_cast<uint4 *>(zbase + (base + mine) * p.H * RB) = make_uint4(0, 0, 0, 0);
+                            }
+                        }
+                    }
                 }
                 cp_async_wait_all();  // nothing of this thread is left in flight at exit
                 issued = 0;
@@ -808,6 +867,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         // This row's token and its visible keys [klo, khi), counted from kvbase.
         const int64_t tok = static_cast<int64_t>(qbase) + t * BM + r;
+        if (p.gather && (t == 0 || c.two)) {
+            // Fused packed path: each warp copies its own 32 rows of query tile t from their
+            // padded rows (rows past the last token read row 0); the warpgroup's 128 threads
+            // arrive on q_full[t] as their copies land.
+            int64_t pr = (tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
+            if (pr < 0 || pr >= p.padded_rows) pr = 0;  // never read outside q
+            copy_group<C::NBLK, SW, D>(smem_u32(c.sQ + t * C::Q_BYTES), BM, quarter, pr, p.q, 0, p.H, h, lane);
+            cp_async_mbar_arrive(&c.q_full[t]);
+        }
         int klo = 0, khi = 1;
         bool row_ok;
         if (!packed) {
@@ -986,8 +1054,17 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const float inv_l = 1.f / l;
             int64_t orow_idx = (p.gather && row_ok) ? __ldg(p.gather + tok) : tok;  // fused: padded row
             const bool store_ok = row_ok && (!p.gather || (orow_idx >= 0 && orow_idx < p.padded_rows));
-            uint4 *orow = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) +
-                                                    (orow_idx * p.H + h) * static_cast<int64_t>(D) * 2);
+            // O leaves through this tile's query buffer, unused now that every MMA of the tile
+            // has completed: each warp stages its 32 rows there (a lane writes its row, 16-byte
+            // chunk c of row r at chunk c ^ (r & 7), so eight lanes hit eight bank groups), then
+            // writes whole rows to global memory, consecutive lanes on consecutive 16 bytes.
+            constexpr int RB = D * 2;                // bytes of one row of one head
+            constexpr int CH = RB / 16;              // 16-byte chunks per row
+            constexpr int XM = (CH < 8 ? CH : 8) - 1;
+            constexpr int LPR = CH < 32 ? CH : 32;  // lanes per row in the global stores
+            constexpr int RPI = 32 / LPR;            // rows per store instruction
+            const uint32_t stage = smem_u32(c.sQ + t * C::Q_BYTES) + quarter * 32 * RB;
+            fence_proxy_async_smem();  // the tensor core's reads of Q come before these writes
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t o[32];
@@ -998,10 +1075,22 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     w[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-                if (store_ok) {
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        orow[cc * 4 + v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                for (int v4 = 0; v4 < 4; ++v4)
+                    st_shared_v4(stage + lane * RB + (((cc * 4 + v4) ^ (lane & XM)) << 4), w[4 * v4], w[4 * v4 + 1],
+                                 w[4 * v4 + 2], w[4 * v4 + 3]);
+            }
+            __syncwarp();
+            {
+                const int ch = lane % LPR;
+                uint8_t *const obase = static_cast<uint8_t *>(p.out) + static_cast<int64_t>(h) * RB + ch * 16;
+#pragma unroll 4
+                for (int r0 = 0; r0 < 32; r0 += RPI) {
+                    const int rr = r0 + lane / LPR;
+                    const int64_t orow_r = __shfl_sync(0xffffffffu, orow_idx, rr);
+                    const bool ok_r = __shfl_sync(0xffffffffu, store_ok, rr);
+                    const uint4 v = ld_shared_v4(stage + rr * RB + ((ch ^ (rr & XM)) << 4));
+                    if (ok_r) *reinterpret_cast<uint4 *>(obase + orow_r * p.H * RB) = v;
                 }
             }
             if (row_ok && p.lse) {
@@ -1010,41 +1099,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                           : (static_cast<int64_t>(blockIdx.z) * p.H + h) * p.seqlen + (tok - seq_start);
                 p.lse[li] = lse;
             }
-            if (p.gather) {
-                // Fused pad: this warp's 32 tokens own the padded rows from just after the
-                // previous token's row up to their last row (through the end of the tensor for
-                // the last token, from row 0 for the first); rows no token maps to become 0.
-                const int64_t tw0 = static_cast<int64_t>(qbase) + t * BM + quarter * 32;
-                if (tw0 < p.total_tokens) {
-                    const int64_t tw1 = min(tw0 + 32, static_cast<int64_t>(p.total_tokens)) - 1;
-                    // padded rows of this warp's tokens, sorted (lanes past the last token: +inf)
-                    const int64_t g_lane = (tw0 + lane <= tw1) ? __ldg(p.gather + tw0 + lane) : INT64_MAX;
-                    const int64_t lo_row = max(int64_t(0), (tw0 == 0) ? int64_t(0) : __ldg(p.gather + tw0 - 1) + 1);
-                    const int64_t hi_row =
-                        min(p.padded_rows, (tw1 == p.total_tokens - 1) ? p.padded_rows : __ldg(p.gather + tw1));
-                    constexpr int VEC = D * 2 / 16;  // 16-byte vectors per row of one head
-                    for (int64_t base = lo_row; base < hi_row; base += 32) {
-                        const int64_t pr = base + lane;
-                        // is pr one of the 32 mapped rows? binary search over the lanes' sorted values
-                        int lo = 0;
-#pragma unroll
-                        for (int step = 16; step >= 1; step >>= 1) {
-                            const int64_t v = __shfl_sync(0xffffffffu, g_lane, lo + step - 1);
-                            if (v < pr) lo += step;
-                        }
-                        const bool mapped = __shfl_sync(0xffffffffu, g_lane, lo & 31) == pr;
-                        if (pr < hi_row && !mapped) {
-                            uint4 *row = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) +
-                                                                   (pr * p.H + h) * static_cast<int64_t>(D) * 2);
-#pragma unroll
-                            for (int v4 = 0; v4 < VEC; ++v4) row[v4] = make_uint4(0, 0, 0, 0);
-                        }
-                    }
-                }
-            }
         }
     }
 
+    if (p.gather && warp < C::NUM_SOFTMAX_WARPS) cp_async_wait_all();  // the query copies (abort paths)
     tc_fence_before_sync();
     __syncthreads();
     if (warp == C::WARP_MMA) {

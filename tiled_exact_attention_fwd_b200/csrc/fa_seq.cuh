@@ -51,4 +51,30 @@ __device__ __forceinline__ int lane_seq_of_token(const int32_t *cu, int num_seqs
     return (lo < 32) ? s0 + lo : seq_of_token(cu, num_seqs, tok);
 }
 
+// cu[0 .. num_seqs] held by a warp, entries lane and 32 + lane of every lane, when
+// num_seqs < 64 (`ok`); then seq() and at() need no memory access. Every lane must take part
+// in each call, with the same arguments for at().
+struct CuWindow {
+    int v0, v1;  // cu[lane], cu[32 + lane] (INT32 max past cu[num_seqs])
+    int n;       // num_seqs
+    bool ok;
+    __device__ __forceinline__ CuWindow(const int32_t *cu, int num_seqs, int lane) : n(num_seqs) {
+        ok = num_seqs < 64;
+        v0 = (ok && lane <= num_seqs) ? __ldg(cu + lane) : 0x7fffffff;
+        v1 = (ok && 32 + lane <= num_seqs) ? __ldg(cu + 32 + lane) : 0x7fffffff;
+    }
+    // the last s < num_seqs with cu[s] <= tok (the entries <= tok form a prefix)
+    __device__ __forceinline__ int seq(int tok, int lane) const {
+        const unsigned a = __ballot_sync(0xffffffffu, lane < n && v0 <= tok);
+        const unsigned b = __ballot_sync(0xffffffffu, 32 + lane < n && v1 <= tok);
+        return __popc(a) + __popc(b) - 1;
+    }
+    // cu[s] for 0 <= s <= num_seqs
+    __device__ __forceinline__ int at(int s) const {
+        const int x = __shfl_sync(0xffffffffu, v0, s & 31);
+        const int y = __shfl_sync(0xffffffffu, v1, s & 31);
+        return s < 32 ? x : y;
+    }
+};
+
 }  // namespace fa
