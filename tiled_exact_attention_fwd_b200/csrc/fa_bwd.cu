@@ -9,11 +9,19 @@
 //
 // Two tcgen05 kernels, one template (no atomics, no accumulation workspace):
 //   dK/dV: a CTA owns one 128-row key tile j (K_j, V_j stay in shared memory) and streams the
-//          query tiles i >= j (causal) or all of them through a two-stage TMA ring:
-//            S^T  = K_j Q_i^T, dP^T = V_j dO_i^T        (SS MMAs, fp32 in TMEM)
-//            P^T, dZ^T (16-bit) over S^T, dP^T in TMEM  (4 elementwise warps, thread = key)
-//            dV  += P^T dO_i,  dK += dZ^T Q_i           (TS MMAs, A from TMEM)
-//   dQ:    a CTA owns one 128-row query tile i (Q_i, dO_i stay) and streams key tiles j <= i:
+//          query tiles i >= j (causal) or all of them through a two-stage TMA ring, each in
+//          two half-steps of 64 query rows:
+//            S^T  = K_j Q_i^T, dP^T = V_j dO_i^T        (SS MMAs, N = 64, fp32 in TMEM)
+//            P^T, dZ^T (16-bit) over S^T, dP^T in TMEM  (elementwise warps, thread = key)
+//            dV  += P^T dO_i,  dK += dZ^T Q_i           (TS MMAs, A from TMEM, K = 64)
+//          S^T and dP^T of consecutive half-steps alternate between two 128-column TMEM
+//          buffers, so the tensor core computes the next half-step's S^T and dP^T (and the
+//          previous one's accumulator updates) while the elementwise warps work on the
+//          current one: TMEM holds both buffers and the two accumulators (2 x 128 + 2 x D <=
+//          512 columns), which whole 128-row steps could not.
+//   dQ:    a CTA owns one 128-row query tile i (Q_i, dO_i stay) and streams key tiles j <= i
+//          in whole steps (an N = 64 MMA takes nearly as long as an N = 128 one, and the dQ
+//          kernel has one accumulator to overlap with, not two):
 //            S = Q_i K_j^T, dP = dO_i V_j^T;  dZ over S;  dQ += dZ K_j
 // Warps 0-7 do the elementwise work (two threads per TMEM lane = row, each on half of the
 // columns), warp 8 lane 0 issues the TMA loads, warp 9 allocates TMEM and lane 0 issues
@@ -54,17 +62,27 @@ struct BwdCfg {
     static constexpr int OFF_RING = 2 * TILE_BYTES;
     static constexpr int OFF_STAT = OFF_RING + 4 * TILE_BYTES;  // [slot][-lse*log2e | -delta][128]
     static constexpr int OFF_BAR = OFF_STAT + 2 * 2 * BM * 4;
-    // fix_full, ring_full[2], ring_empty[2], s_full, p_ready, done, drain, stats_ready[2]
-    static constexpr int NUM_BARS = 11;
+    // fix_full, ring_full[2], ring_empty[2], s_full[2], p_ready[2], done, drain, stats_ready[2]
+    static constexpr int NUM_BARS = 13;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int USED = OFF_MISC + 16;
     static constexpr int MIN_SMEM = 120 * 1024;  // one CTA (and one TMEM allocation) per SM
     static constexpr int SMEM_BYTES = (USED + 1024 > MIN_SMEM) ? USED + 1024 : MIN_SMEM;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr int COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
+    static constexpr int COL_ACC0 = 256, COL_ACC1 = 256 + D;  // accumulators
     static_assert(USED + 1024 <= 227 * 1024, "shared memory budget");
     static_assert(COL_ACC1 + D <= (int)TMEM_COLS, "TMEM budget (dK and dV accumulators)");
     static_assert(TILE_BYTES % 1024 == 0, "tile alignment");
+};
+
+// Steps of the streamed loop: STEP streamed rows each, S/dP buffers used in turn (buffer b at
+// TMEM column 128 b: S in [0, STEP), dP in [STEP, 2 STEP)).
+template <bool DKDV>
+struct BwdStep {
+    static constexpr int STEP = DKDV ? 64 : 128;  // streamed rows per step
+    static constexpr int NBUF = DKDV ? 2 : 1;     // S/dP buffers
+    static constexpr int PER_TILE = 128 / STEP;
+    static constexpr int COL_BUF = 128, COL_DP = STEP;
 };
 
 // Loads of one 128-row tile of a token-major (N, H, D) tensor: NBLK boxes side by side.
@@ -76,12 +94,13 @@ __device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *map, 
     for (int b = 0; b < C::NBLK; ++b) tma_load_3d(dst + b * C::BM * C::SW, map, bar, b * C::SWE, h, row, pol);
 }
 
-// D_out (+)= A B^T over the head dimension: A, B K-major 128-row tiles in shared memory.
-template <int D, bool BF16>
-__device__ __forceinline__ void mma_rows(uint32_t d_tmem, const uint8_t *a, const uint8_t *b) {
+// D_out = A B_u^T over the head dimension: A a K-major 128-row tile in shared memory, B_u rows
+// [STEP u, STEP u + STEP) of another (N = STEP).
+template <int D, bool BF16, int STEP>
+__device__ __forceinline__ void mma_rows_step(uint32_t d_tmem, const uint8_t *a, const uint8_t *b, int u) {
     using C = BwdCfg<D>;
-    constexpr uint32_t idesc = idesc_f16(C::BM, C::BM, BF16, false);
-    const uint32_t a0 = smem_u32(a), b0 = smem_u32(b);
+    constexpr uint32_t idesc = idesc_f16(C::BM, STEP, BF16, false);
+    const uint32_t a0 = smem_u32(a), b0 = smem_u32(b) + u * STEP * C::SW;
 #pragma unroll
     for (int k = 0; k < D / 16; ++k) {
         const uint32_t blk = (k * 32) / C::SW, off = (k * 32) % C::SW;
@@ -90,18 +109,20 @@ __device__ __forceinline__ void mma_rows(uint32_t d_tmem, const uint8_t *a, cons
     }
 }
 
-// D_out (+)= A_tmem B over 128 rows: A (128 x 128, 16-bit) in TMEM, B a 128-row tile read
-// MN-major (its D columns are the output columns). A's packed columns 0-31 (elements 0-63)
-// sit at a_tmem + [0, 32) and columns 32-63 at a_tmem + [64, 96): each half was written by
-// its own thread over the fp32 columns it had read.
-template <int D, bool BF16>
-__device__ __forceinline__ void mma_acc(uint32_t d_tmem, uint32_t a_tmem, const uint8_t *b, bool accumulate) {
+// D_out (+)= A_tmem B_u over STEP rows: A (128 x STEP, 16-bit) in TMEM, B_u rows
+// [STEP u, STEP u + STEP) of a 128-row tile read MN-major (its D columns are the output
+// columns). A's first STEP/2 elements sit packed at a_tmem + [0, STEP/4) and the others at
+// a_tmem + [STEP/2, 3 STEP/4): each half was written by its own thread over the fp32
+// columns it had read.
+template <int D, bool BF16, int STEP>
+__device__ __forceinline__ void mma_acc_step(uint32_t d_tmem, uint32_t a_tmem, const uint8_t *b, int u,
+                                             bool accumulate) {
     using C = BwdCfg<D>;
     constexpr uint32_t idesc = idesc_f16(C::BM, D, BF16, true);
-    const uint32_t b0 = smem_u32(b);
+    const uint32_t b0 = smem_u32(b) + u * STEP * C::SW;
 #pragma unroll
-    for (int k = 0; k < C::BM / 16; ++k)
-        umma_ts(d_tmem, a_tmem + k * 8 + (k >= 4 ? 32 : 0),
+    for (int k = 0; k < STEP / 16; ++k)
+        umma_ts(d_tmem, a_tmem + k * 8 + (k >= STEP / 32 ? STEP / 4 : 0),
                 smem_desc(b0 + k * 16 * C::SW, C::BM * C::SW, 8 * C::SW, C::LAYOUT), idesc,
                 (accumulate || k > 0) ? 1u : 0u);
 }
@@ -175,7 +196,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     float *stats = reinterpret_cast<float *>(smem + C::OFF_STAT);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *fix_full = bars, *ring_full = bars + 1, *ring_empty = bars + 3, *s_full = bars + 5,
-             *p_ready = bars + 6, *done = bars + 7, *drain = bars + 8, *stats_ready = bars + 9;
+             *p_ready = bars + 7, *done = bars + 9, *drain = bars + 10, *stats_ready = bars + 11;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     const uint64_t lim = p.timeout_ns;
@@ -188,9 +209,9 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_init(&ring_full[s], 1);
             mbar_init(&ring_empty[s], 1);
             mbar_init(&stats_ready[s], BM);  // the column-half-0 threads publish 128 columns
+            mbar_init(&s_full[s], 1);
+            mbar_init(&p_ready[s], C::NUM_EW);
         }
-        mbar_init(s_full, 1);
-        mbar_init(p_ready, C::NUM_EW);
         mbar_init(done, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -249,22 +270,44 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (lane == 0 && n > 0) {
             ok = wait_bounded(fix_full, 0, abort_flag, lim, 410);
             if (ok) tc_fence_after_sync();
-            for (int t = 0; ok && t < n; ++t) {
-                const int s = t & 1;
-                if (!(ok = wait_bounded(&ring_full[s], (t >> 1) & 1, abort_flag, lim, 420 + s))) break;
-                tc_fence_after_sync();
-                mma_rows<D, BF16>(tmem + C::COL_S, fixA0, ring_tile(s, 0));   // S (or S^T)
-                mma_rows<D, BF16>(tmem + C::COL_DP, fixA1, ring_tile(s, 1));  // dP (or dP^T)
-                umma_commit(s_full);
-                if (!(ok = wait_bounded(p_ready, t & 1, abort_flag, lim, 430))) break;
-                tc_fence_after_sync();
-                if (DKDV) {
-                    mma_acc<D, BF16>(tmem + C::COL_ACC0, tmem + C::COL_S, ring_tile(s, 1), t > 0);   // dV += P^T dO
-                    mma_acc<D, BF16>(tmem + C::COL_ACC1, tmem + C::COL_DP, ring_tile(s, 0), t > 0);  // dK += dZ^T Q
-                } else {
-                    mma_acc<D, BF16>(tmem + C::COL_ACC0, tmem + C::COL_S, ring_tile(s, 0), t > 0);   // dQ += dZ K
+            // Step k: streamed tile t = k / PER_TILE, rows [STEP u, STEP u + STEP) with
+            // u = k % PER_TILE, TMEM buffer k % NBUF. With two buffers the issue order is
+            // S/dP(k+1), then (once the elementwise warps are done with k) the accumulator
+            // updates of k; the tensor core runs them in that order, so S/dP(k+2) overwrite
+            // buffer k % 2 only after the updates of k have read it. With one buffer S/dP(k+1)
+            // follow the updates of k.
+            using St = BwdStep<DKDV>;
+            const int nk = n * St::PER_TILE;
+            auto issue_sdp = [&](int k) -> bool {
+                const int t = k / St::PER_TILE, u = k % St::PER_TILE, s = t & 1;
+                if (u == 0) {
+                    if (!wait_bounded(&ring_full[s], (t >> 1) & 1, abort_flag, lim, 420 + s)) return false;
+                    tc_fence_after_sync();
                 }
-                umma_commit(&ring_empty[s]);
+                const uint32_t buf = tmem + (k % St::NBUF) * St::COL_BUF;
+                mma_rows_step<D, BF16, St::STEP>(buf, fixA0, ring_tile(s, 0), u);               // S (or S^T)
+                mma_rows_step<D, BF16, St::STEP>(buf + St::COL_DP, fixA1, ring_tile(s, 1), u);  // dP (or dP^T)
+                umma_commit(&s_full[k % St::NBUF]);
+                return true;
+            };
+            if (ok) ok = issue_sdp(0);
+            for (int k = 0; ok && k < nk; ++k) {
+                if (St::NBUF == 2 && k + 1 < nk && !(ok = issue_sdp(k + 1))) break;
+                if (!(ok = wait_bounded(&p_ready[k % St::NBUF], (k / St::NBUF) & 1, abort_flag, lim,
+                                        430 + k % St::NBUF)))
+                    break;
+                tc_fence_after_sync();
+                const int t = k / St::PER_TILE, u = k % St::PER_TILE, s = t & 1;
+                const uint32_t buf = tmem + (k % St::NBUF) * St::COL_BUF;
+                if (DKDV) {
+                    mma_acc_step<D, BF16, St::STEP>(tmem + C::COL_ACC0, buf, ring_tile(s, 1), u, k > 0);  // dV += P^T dO
+                    mma_acc_step<D, BF16, St::STEP>(tmem + C::COL_ACC1, buf + St::COL_DP, ring_tile(s, 0), u,
+                                                    k > 0);  // dK += dZ^T Q
+                } else {
+                    mma_acc_step<D, BF16, St::STEP>(tmem + C::COL_ACC0, buf, ring_tile(s, 0), u, k > 0);  // dQ += dZ K
+                }
+                if (u == St::PER_TILE - 1) umma_commit(&ring_empty[s]);  // every step of tile t has read it
+                if (St::NBUF == 1 && k + 1 < nk && !(ok = issue_sdp(k + 1))) break;
             }
             if (ok) umma_commit(done);
             umma_commit(drain);  // every MMA issued above has finished once this arrives
@@ -309,13 +352,14 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         } else if (!DKDV) {
             query_stats(own_pos, my_nl, my_nd);
         }
-        // P (or P^T) and dZ for 32 columns starting at col0; MASK applies the causal diagonal
-        // and (dQ) the keys past the sequence end.
-        auto chunk = [&](auto mask_c, int col0, const float *snl, const float *snd, int w0) {
+        // P (or P^T) and dZ for the 32 columns [col0, col0 + 32) of TMEM buffer `buf`, whose
+        // column c is streamed position w0 + c; MASK applies the causal diagonal and the
+        // sequence bounds.
+        auto chunk = [&](auto mask_c, uint32_t buf, int col0, const float *snl, const float *snd, int w0) {
             constexpr bool MASK = decltype(mask_c)::value;
             uint32_t sv[32], dv[32];
-            tmem_ld32(tmem + lane_base + C::COL_S + col0, sv);
-            tmem_ld32(tmem + lane_base + C::COL_DP + col0, dv);
+            tmem_ld32(buf + lane_base + col0, sv);
+            tmem_ld32(buf + lane_base + BwdStep<DKDV>::COL_DP + col0, dv);
             tmem_ld_wait();
             tmem_reg_fence<32>(sv);
             tmem_reg_fence<32>(dv);
@@ -352,22 +396,24 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 pk[i] = pack2b<BF16>(p0, p1);
                 zk[i] = pack2b<BF16>(z0, z1);
             }
-            // packed columns of this half start at its own first column (32 * half packed
-            // columns further on for half 1), so neither thread of the row overwrites
-            // columns the other one has yet to read
-            const int pcol = col0 / 2 + 32 * half;
+            // packed columns of this thread start at its own first column (STEP/2 * half), so
+            // neither thread of the row overwrites columns the other one has yet to read
+            constexpr int HS = BwdStep<DKDV>::STEP / 2;  // columns per thread and step
+            const int pcol = half * HS + (col0 - half * HS) / 2;
             if (DKDV) {
-                tmem_st16(tmem + lane_base + C::COL_S + pcol, pk);   // P^T over S^T
-                tmem_st16(tmem + lane_base + C::COL_DP + pcol, zk);  // dZ^T over dP^T
+                tmem_st16(buf + lane_base + pcol, pk);                             // P^T over S^T
+                tmem_st16(buf + lane_base + BwdStep<DKDV>::COL_DP + pcol, zk);  // dZ^T over dP^T
             } else {
-                tmem_st16(tmem + lane_base + C::COL_S + pcol, zk);   // dZ over S
+                tmem_st16(buf + lane_base + pcol, zk);  // dZ over S
             }
         };
-        for (int t = 0; ok && t < n; ++t) {
-            const int w0 = ws + t * BM;  // position of the streamed window's first row
+        using St = BwdStep<DKDV>;
+        for (int k = 0; ok && k < n * St::PER_TILE; ++k) {
+            const int t = k / St::PER_TILE, u = k % St::PER_TILE;  // streamed tile, part
+            const int w0 = ws + t * BM + u * St::STEP;              // position of the step's first streamed row
             const int slot = t & 1;
-            const float *snl = stats + slot * 2 * BM, *snd = snl + BM;
-            if (DKDV) {
+            const float *snl = stats + slot * 2 * BM + u * St::STEP, *snd = snl + BM;
+            if (DKDV && u == 0) {
                 if (publisher) {
                     // publish this thread's query column statistics, prefetch the next tile's
                     stats[slot * 2 * BM + r] = my_nl;
@@ -378,25 +424,28 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (!(ok = __all_sync(0xffffffffu, wait_bounded(&stats_ready[slot], (t >> 1) & 1, abort_flag, lim, 440))))
                     break;
             }
-            if (!(ok = __all_sync(0xffffffffu, wait_bounded(s_full, t & 1, abort_flag, lim, 450)))) break;
+            if (!(ok = __all_sync(0xffffffffu, wait_bounded(&s_full[k % St::NBUF], (k / St::NBUF) & 1, abort_flag,
+                                                            lim, 450 + k % St::NBUF))))
+                break;
             tc_fence_after_sync();
-            // does any pair of this warp's rows with the window need a mask?
-            const bool row_partial = w0 < row_lo || w0 + BM > row_hi ||
-                                     (CAUSAL && (DKDV ? w0 < own_pos : w0 + BM - 1 > own_pos));
+            // does any pair of this warp's rows with the step's positions need a mask?
+            const bool row_partial = w0 < row_lo || w0 + St::STEP > row_hi ||
+                                     (CAUSAL && (DKDV ? w0 < own_pos : w0 + St::STEP - 1 > own_pos));
             const bool masked = __any_sync(0xffffffffu, row_partial);
-            // this thread's 64 columns: [64*half, 64*half + 64), two chunks; each chunk's
+            // this thread's STEP/2 columns [STEP/2 * half, ...) of the step, 32 at a time; the
             // results are stored over columns this thread has already read
+            const uint32_t buf = tmem + (k % St::NBUF) * St::COL_BUF;
 #pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-                const int col0 = half * 64 + c * 32;
+            for (int c = 0; c < St::STEP / 64; ++c) {
+                const int col0 = half * (St::STEP / 2) + c * 32;
                 if (masked)
-                    chunk(std::integral_constant<bool, true>{}, col0, snl, snd, w0);
+                    chunk(std::integral_constant<bool, true>{}, buf, col0, snl, snd, w0);
                 else
-                    chunk(std::integral_constant<bool, false>{}, col0, snl, snd, w0);
+                    chunk(std::integral_constant<bool, false>{}, buf, col0, snl, snd, w0);
             }
             tmem_st_wait();
             tc_fence_before_sync();
-            mbar_arrive(p_ready);
+            mbar_arrive(&p_ready[k % St::NBUF]);
         }
         if (ok && n > 0) ok = __all_sync(0xffffffffu, wait_bounded(done, 0, abort_flag, lim, 460));
         if (ok) {
