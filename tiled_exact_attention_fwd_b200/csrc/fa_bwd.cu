@@ -20,9 +20,13 @@
 //          current one: TMEM holds both buffers and the two accumulators (2 x 128 + 2 x D <=
 //          512 columns), which whole 128-row steps could not.
 //   dQ:    a CTA owns one 128-row query tile i (Q_i, dO_i stay) and streams key tiles j <= i
-//          in whole steps (an N = 64 MMA takes nearly as long as an N = 128 one, and the dQ
-//          kernel has one accumulator to overlap with, not two):
+//          in whole steps (an N = 64 MMA takes nearly as long as an N = 128 one):
 //            S = Q_i K_j^T, dP = dO_i V_j^T;  dZ over S;  dQ += dZ K_j
+//          S alternates between two TMEM buffers (2 x 128 + dP 128 + dQ D <= 512 columns):
+//          S_{j+1} is computed while the elementwise warps work on step j, and after them
+//          the tensor core runs dP_{j+1} first (the next step's last input), then dQ += dZ_j
+//          K_j and S_{j+2}. K and V stream through separate rings (three K slots: K_j is read
+//          from S_j until dQ's update two steps later; two V slots).
 // Warps 0-7 do the elementwise work (two threads per TMEM lane = row, each on half of the
 // columns), warp 8 lane 0 issues the TMA loads, warp 9 allocates TMEM and lane 0 issues
 // every MMA. Every wait is bounded.
@@ -56,33 +60,41 @@ struct BwdCfg {
     static constexpr int NUM_EW = 256;
     static constexpr int NUM_THREADS = NUM_EW + 64;
     static constexpr int WARP_TMA = 8, WARP_MMA = 9;
-    // shared memory: fixed tiles A0, A1; ring stages s = 0, 1 holding tiles B0, B1;
-    // per-column statistics (dK/dV kernel) in two slots; barriers; misc
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(TILE_BYTES % 1024 == 0, "tile alignment");
+};
+
+// Shared memory and TMEM of one kernel kind. Shared: fixed tiles A0, A1, then
+//   dK/dV: ring stages s = 0, 1 holding tiles B0 = Q_i, B1 = dO_i; per-column statistics in
+//          two slots;
+//   dQ:    K ring of three tiles, V ring of two;
+// then barriers and misc. Steps: STEP streamed rows each, S in TMEM buffer k % 2 (column
+// 128 (k % 2)); dP next to it (dK/dV: half-steps) or in its own columns (dQ); barriers for
+// S-ready / P-ready in NBAR sets used in turn.
+template <int D, bool DKDV>
+struct BwdKind {
+    using C = BwdCfg<D>;
+    static constexpr int STEP = DKDV ? 64 : 128;  // streamed rows per step
+    static constexpr int PER_TILE = 128 / STEP;
+    static constexpr int NBAR = DKDV ? 2 : 1;
+    static constexpr int COL_DP_DQ = 256;                         // dQ: dP columns
+    static constexpr int COL_ACC0 = DKDV ? 256 : 384;             // dV (dK/dV) or dQ
+    static constexpr int COL_ACC1 = 256 + D;                      // dK (dK/dV)
+    static constexpr int K_SLOTS = 3, V_SLOTS = 2;                // dQ rings
     static constexpr int OFF_FIX = 0;
-    static constexpr int OFF_RING = 2 * TILE_BYTES;
-    static constexpr int OFF_STAT = OFF_RING + 4 * TILE_BYTES;  // [slot][-lse*log2e | -delta][128]
-    static constexpr int OFF_BAR = OFF_STAT + 2 * 2 * BM * 4;
-    // fix_full, ring_full[2], ring_empty[2], s_full[2], p_ready[2], done, drain, stats_ready[2]
-    static constexpr int NUM_BARS = 13;
+    static constexpr int OFF_RING = 2 * C::TILE_BYTES;
+    static constexpr int RING_TILES = DKDV ? 4 : K_SLOTS + V_SLOTS;
+    static constexpr int OFF_STAT = OFF_RING + RING_TILES * C::TILE_BYTES;  // [slot][-lse*log2e | -delta][128]
+    static constexpr int OFF_BAR = OFF_STAT + (DKDV ? 2 * 2 * C::BM * 4 : 0);
+    // dK/dV: fix_full, ring_full[2], ring_empty[2], s_full[2], p_ready[2], done, drain, stats_ready[2]
+    // dQ:    fix_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, p_ready, done, drain
+    static constexpr int NUM_BARS = 16;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int USED = OFF_MISC + 16;
     static constexpr int MIN_SMEM = 120 * 1024;  // one CTA (and one TMEM allocation) per SM
     static constexpr int SMEM_BYTES = (USED + 1024 > MIN_SMEM) ? USED + 1024 : MIN_SMEM;
-    static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr int COL_ACC0 = 256, COL_ACC1 = 256 + D;  // accumulators
     static_assert(USED + 1024 <= 227 * 1024, "shared memory budget");
-    static_assert(COL_ACC1 + D <= (int)TMEM_COLS, "TMEM budget (dK and dV accumulators)");
-    static_assert(TILE_BYTES % 1024 == 0, "tile alignment");
-};
-
-// Steps of the streamed loop: STEP streamed rows each, S/dP buffers used in turn (buffer b at
-// TMEM column 128 b: S in [0, STEP), dP in [STEP, 2 STEP)).
-template <bool DKDV>
-struct BwdStep {
-    static constexpr int STEP = DKDV ? 64 : 128;  // streamed rows per step
-    static constexpr int NBUF = DKDV ? 2 : 1;     // S/dP buffers
-    static constexpr int PER_TILE = 128 / STEP;
-    static constexpr int COL_BUF = 128, COL_DP = STEP;
+    static_assert(DKDV ? (COL_ACC1 + D <= 512) : (COL_ACC0 + D <= 512), "TMEM budget");
 };
 
 // Loads of one 128-row tile of a token-major (N, H, D) tensor: NBLK boxes side by side.
@@ -164,6 +176,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const BwdParams p) {
     using C = BwdCfg<D>;
+    using Kd = BwdKind<D, DKDV>;
     constexpr int BM = C::BM;
     const int h = blockIdx.x, b = blockIdx.z, S = p.seqlen;  // packed: S = total tokens
     const int ntiles = (S + BM - 1) / BM;
@@ -192,25 +205,45 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *fixA0 = smem + C::OFF_FIX, *fixA1 = fixA0 + C::TILE_BYTES;
-    float *stats = reinterpret_cast<float *>(smem + C::OFF_STAT);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *fix_full = bars, *ring_full = bars + 1, *ring_empty = bars + 3, *s_full = bars + 5,
-             *p_ready = bars + 7, *done = bars + 9, *drain = bars + 10, *stats_ready = bars + 11;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    uint8_t *fixA0 = smem + Kd::OFF_FIX, *fixA1 = fixA0 + C::TILE_BYTES;
+    float *stats = reinterpret_cast<float *>(smem + Kd::OFF_STAT);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Kd::OFF_BAR);
+    uint64_t *fix_full = bars;
+    // dK/dV barriers
+    uint64_t *ring_full = bars + 1, *ring_empty = bars + 3, *stats_ready = bars + 11;
+    // dQ barriers
+    uint64_t *k_full = bars + 1, *k_empty = bars + 4, *v_full = bars + 7, *v_empty = bars + 9;
+    uint64_t *s_full = DKDV ? bars + 5 : bars + 11, *p_ready = DKDV ? bars + 7 : bars + 12;
+    uint64_t *done = DKDV ? bars + 9 : bars + 13, *drain = DKDV ? bars + 10 : bars + 14;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Kd::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Kd::OFF_MISC + 4);
     const uint64_t lim = p.timeout_ns;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    auto ring_tile = [&](int stage, int which) { return smem + C::OFF_RING + (2 * stage + which) * C::TILE_BYTES; };
+    auto ring_tile = [&](int stage, int which) { return smem + Kd::OFF_RING + (2 * stage + which) * C::TILE_BYTES; };
+    auto k_tile = [&](int slot) { return smem + Kd::OFF_RING + slot * C::TILE_BYTES; };
+    auto v_tile = [&](int slot) { return smem + Kd::OFF_RING + (Kd::K_SLOTS + slot) * C::TILE_BYTES; };
 
     if (threadIdx.x == 0) {
         mbar_init(fix_full, 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&ring_full[s], 1);
-            mbar_init(&ring_empty[s], 1);
-            mbar_init(&stats_ready[s], BM);  // the column-half-0 threads publish 128 columns
-            mbar_init(&s_full[s], 1);
-            mbar_init(&p_ready[s], C::NUM_EW);
+        if (DKDV) {
+            for (int s = 0; s < 2; ++s) {
+                mbar_init(&ring_full[s], 1);
+                mbar_init(&ring_empty[s], 1);
+                mbar_init(&stats_ready[s], BM);  // the column-half-0 threads publish 128 columns
+                mbar_init(&s_full[s], 1);
+                mbar_init(&p_ready[s], C::NUM_EW);
+            }
+        } else {
+            for (int s = 0; s < Kd::K_SLOTS; ++s) {
+                mbar_init(&k_full[s], 1);
+                mbar_init(&k_empty[s], 1);
+            }
+            for (int s = 0; s < Kd::V_SLOTS; ++s) {
+                mbar_init(&v_full[s], 1);
+                mbar_init(&v_empty[s], 1);
+            }
+            mbar_init(s_full, 1);
+            mbar_init(p_ready, C::NUM_EW);
         }
         mbar_init(done, 1);
         mbar_init(drain, 1);
@@ -243,25 +276,56 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_arrive_expect_tx(fix_full, 2 * C::TILE_BYTES);
             load_tile<D>(fixA0, fa0, fix_full, h, static_cast<int>(row0 + own_start), pol_fix);
             load_tile<D>(fixA1, fa1, fix_full, h, static_cast<int>(row0 + own_start), pol_fix);
-            int issued = 0;
-            for (int t = 0; t < n; ++t) {
-                const int s = t & 1;
-                if (t >= 2 && !wait_bounded(&ring_empty[s], ((t >> 1) - 1) & 1, abort_flag, lim, 400 + s)) break;
-                mbar_arrive_expect_tx(&ring_full[s], 2 * C::TILE_BYTES);
-                const int row = static_cast<int>(row0 + ws + t * BM);
-                load_tile<D>(ring_tile(s, 0), rb0, &ring_full[s], h, row, pol_ring);
-                load_tile<D>(ring_tile(s, 1), rb1, &ring_full[s], h, row, pol_ring);
-                issued = t + 1;
-            }
-            if (*abort_flag) {
-                // let the copies already issued land before shared memory goes away
-                const uint64_t g0 = global_timer_ns();
-                while (!mbar_try_wait(fix_full, 0) && global_timer_ns() - g0 < lim) {
+            // (bounded) wait for phase `ph` of `bar` before shared memory goes away
+            auto settle = [&](uint64_t *bar, uint32_t ph) {
+                const uint64_t g1 = global_timer_ns();
+                while (!mbar_try_wait(bar, ph) && global_timer_ns() - g1 < lim) {
                 }
-                for (int t = (issued > 2 ? issued - 2 : 0); t < issued; ++t) {
-                    const uint64_t g1 = global_timer_ns();
-                    while (!mbar_try_wait(&ring_full[t & 1], (t >> 1) & 1) && global_timer_ns() - g1 < lim) {
+            };
+            if constexpr (DKDV) {
+                int issued = 0;
+                for (int t = 0; t < n; ++t) {
+                    const int s = t & 1;
+                    if (t >= 2 && !wait_bounded(&ring_empty[s], ((t >> 1) - 1) & 1, abort_flag, lim, 400 + s)) break;
+                    mbar_arrive_expect_tx(&ring_full[s], 2 * C::TILE_BYTES);
+                    const int row = static_cast<int>(row0 + ws + t * BM);
+                    load_tile<D>(ring_tile(s, 0), rb0, &ring_full[s], h, row, pol_ring);
+                    load_tile<D>(ring_tile(s, 1), rb1, &ring_full[s], h, row, pol_ring);
+                    issued = t + 1;
+                }
+                if (*abort_flag) {
+                    // let the copies already issued land before shared memory goes away
+                    settle(fix_full, 0);
+                    for (int t = (issued > 2 ? issued - 2 : 0); t < issued; ++t) settle(&ring_full[t & 1], (t >> 1) & 1);
+                }
+            } else {
+                // K_t is first read two steps before V_t: order K_0, K_1, V_0, K_2, V_1, ...
+                int k_issued = 0, v_issued = 0;
+                for (int t = 0; t <= n; ++t) {
+                    if (t < n) {
+                        const int ks = t % Kd::K_SLOTS;
+                        if (t >= Kd::K_SLOTS &&
+                            !wait_bounded(&k_empty[ks], ((t / Kd::K_SLOTS) - 1) & 1, abort_flag, lim, 400 + ks))
+                            break;
+                        mbar_arrive_expect_tx(&k_full[ks], C::TILE_BYTES);
+                        load_tile<D>(k_tile(ks), rb0, &k_full[ks], h, static_cast<int>(row0 + ws + t * BM), pol_ring);
+                        k_issued = t + 1;
                     }
+                    if (t >= 1) {
+                        const int tv = t - 1, vs = tv & 1;
+                        if (tv >= Kd::V_SLOTS && !wait_bounded(&v_empty[vs], ((tv >> 1) - 1) & 1, abort_flag, lim, 404 + vs))
+                            break;
+                        mbar_arrive_expect_tx(&v_full[vs], C::TILE_BYTES);
+                        load_tile<D>(v_tile(vs), rb1, &v_full[vs], h, static_cast<int>(row0 + ws + tv * BM), pol_ring);
+                        v_issued = tv + 1;
+                    }
+                }
+                if (*abort_flag) {
+                    settle(fix_full, 0);
+                    for (int t = (k_issued > Kd::K_SLOTS ? k_issued - Kd::K_SLOTS : 0); t < k_issued; ++t)
+                        settle(&k_full[t % Kd::K_SLOTS], (t / Kd::K_SLOTS) & 1);
+                    for (int t = (v_issued > Kd::V_SLOTS ? v_issued - Kd::V_SLOTS : 0); t < v_issued; ++t)
+                        settle(&v_full[t & 1], (t >> 1) & 1);
                 }
             }
         }
@@ -270,44 +334,68 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (lane == 0 && n > 0) {
             ok = wait_bounded(fix_full, 0, abort_flag, lim, 410);
             if (ok) tc_fence_after_sync();
-            // Step k: streamed tile t = k / PER_TILE, rows [STEP u, STEP u + STEP) with
-            // u = k % PER_TILE, TMEM buffer k % NBUF. With two buffers the issue order is
-            // S/dP(k+1), then (once the elementwise warps are done with k) the accumulator
-            // updates of k; the tensor core runs them in that order, so S/dP(k+2) overwrite
-            // buffer k % 2 only after the updates of k have read it. With one buffer S/dP(k+1)
-            // follow the updates of k.
-            using St = BwdStep<DKDV>;
-            const int nk = n * St::PER_TILE;
-            auto issue_sdp = [&](int k) -> bool {
-                const int t = k / St::PER_TILE, u = k % St::PER_TILE, s = t & 1;
-                if (u == 0) {
-                    if (!wait_bounded(&ring_full[s], (t >> 1) & 1, abort_flag, lim, 420 + s)) return false;
+            if constexpr (DKDV) {
+                // Half-step k: streamed tile t = k / 2, rows [64 u, 64 u + 64) with u = k % 2,
+                // TMEM buffer k % 2. Issue order: S/dP(k+1), then (once the elementwise warps
+                // are done with k) the accumulator updates of k; the tensor core runs them in
+                // that order, so S/dP(k+2) overwrite buffer k % 2 only after the updates of k
+                // have read it.
+                const int nk = n * Kd::PER_TILE;
+                auto issue_sdp = [&](int k) -> bool {
+                    const int t = k / Kd::PER_TILE, u = k % Kd::PER_TILE, s = t & 1;
+                    if (u == 0) {
+                        if (!wait_bounded(&ring_full[s], (t >> 1) & 1, abort_flag, lim, 420 + s)) return false;
+                        tc_fence_after_sync();
+                    }
+                    const uint32_t buf = tmem + (k & 1) * 128;
+                    mma_rows_step<D, BF16, Kd::STEP>(buf, fixA0, ring_tile(s, 0), u);             // S^T
+                    mma_rows_step<D, BF16, Kd::STEP>(buf + Kd::STEP, fixA1, ring_tile(s, 1), u);  // dP^T
+                    umma_commit(&s_full[k & 1]);
+                    return true;
+                };
+                if (ok) ok = issue_sdp(0);
+                for (int k = 0; ok && k < nk; ++k) {
+                    if (k + 1 < nk && !(ok = issue_sdp(k + 1))) break;
+                    if (!(ok = wait_bounded(&p_ready[k & 1], (k >> 1) & 1, abort_flag, lim, 430 + (k & 1)))) break;
                     tc_fence_after_sync();
+                    const int t = k / Kd::PER_TILE, u = k % Kd::PER_TILE, s = t & 1;
+                    const uint32_t buf = tmem + (k & 1) * 128;
+                    mma_acc_step<D, BF16, Kd::STEP>(tmem + Kd::COL_ACC0, buf, ring_tile(s, 1), u, k > 0);  // dV += P^T dO
+                    mma_acc_step<D, BF16, Kd::STEP>(tmem + Kd::COL_ACC1, buf + Kd::STEP, ring_tile(s, 0), u,
+                                                    k > 0);                                        // dK += dZ^T Q
+                    if (u == Kd::PER_TILE - 1) umma_commit(&ring_empty[s]);  // both halves of tile t have read it
                 }
-                const uint32_t buf = tmem + (k % St::NBUF) * St::COL_BUF;
-                mma_rows_step<D, BF16, St::STEP>(buf, fixA0, ring_tile(s, 0), u);               // S (or S^T)
-                mma_rows_step<D, BF16, St::STEP>(buf + St::COL_DP, fixA1, ring_tile(s, 1), u);  // dP (or dP^T)
-                umma_commit(&s_full[k % St::NBUF]);
-                return true;
-            };
-            if (ok) ok = issue_sdp(0);
-            for (int k = 0; ok && k < nk; ++k) {
-                if (St::NBUF == 2 && k + 1 < nk && !(ok = issue_sdp(k + 1))) break;
-                if (!(ok = wait_bounded(&p_ready[k % St::NBUF], (k / St::NBUF) & 1, abort_flag, lim,
-                                        430 + k % St::NBUF)))
-                    break;
-                tc_fence_after_sync();
-                const int t = k / St::PER_TILE, u = k % St::PER_TILE, s = t & 1;
-                const uint32_t buf = tmem + (k % St::NBUF) * St::COL_BUF;
-                if (DKDV) {
-                    mma_acc_step<D, BF16, St::STEP>(tmem + C::COL_ACC0, buf, ring_tile(s, 1), u, k > 0);  // dV += P^T dO
-                    mma_acc_step<D, BF16, St::STEP>(tmem + C::COL_ACC1, buf + St::COL_DP, ring_tile(s, 0), u,
-                                                    k > 0);  // dK += dZ^T Q
-                } else {
-                    mma_acc_step<D, BF16, St::STEP>(tmem + C::COL_ACC0, buf, ring_tile(s, 0), u, k > 0);  // dQ += dZ K
+            } else {
+                // Step t: S_t in TMEM buffer t % 2, dP_t in its own columns. Issue order:
+                // S_0, dP_0, S_1; then per step t, once the elementwise warps are done with it:
+                // dP_{t+1}, dQ += dZ_t K_t, S_{t+2} (into buffer t % 2, after dQ has read dZ_t).
+                auto issue_s = [&](int t) -> bool {
+                    const int ks = t % Kd::K_SLOTS;
+                    if (!wait_bounded(&k_full[ks], (t / Kd::K_SLOTS) & 1, abort_flag, lim, 420 + ks)) return false;
+                    tc_fence_after_sync();
+                    mma_rows_step<D, BF16, 128>(tmem + (t & 1) * 128, fixA0, k_tile(ks), 0);  // S = Q K^T
+                    return true;
+                };
+                auto issue_dp = [&](int t) -> bool {
+                    const int vs = t & 1;
+                    if (!wait_bounded(&v_full[vs], (t >> 1) & 1, abort_flag, lim, 424 + vs)) return false;
+                    tc_fence_after_sync();
+                    mma_rows_step<D, BF16, 128>(tmem + Kd::COL_DP_DQ, fixA1, v_tile(vs), 0);  // dP = dO V^T
+                    umma_commit(&v_empty[vs]);
+                    umma_commit(s_full);  // step t's S and dP are done
+                    return true;
+                };
+                if (ok) ok = issue_s(0) && issue_dp(0);
+                if (ok && n > 1) ok = issue_s(1);
+                for (int t = 0; ok && t < n; ++t) {
+                    if (!(ok = wait_bounded(p_ready, t & 1, abort_flag, lim, 430))) break;
+                    tc_fence_after_sync();
+                    if (t + 1 < n && !(ok = issue_dp(t + 1))) break;
+                    mma_acc_step<D, BF16, 128>(tmem + Kd::COL_ACC0, tmem + (t & 1) * 128, k_tile(t % Kd::K_SLOTS), 0,
+                                               t > 0);  // dQ += dZ K
+                    umma_commit(&k_empty[t % Kd::K_SLOTS]);
+                    if (t + 2 < n && !(ok = issue_s(t + 2))) break;
                 }
-                if (u == St::PER_TILE - 1) umma_commit(&ring_empty[s]);  // every step of tile t has read it
-                if (St::NBUF == 1 && k + 1 < nk && !(ok = issue_sdp(k + 1))) break;
             }
             if (ok) umma_commit(done);
             umma_commit(drain);  // every MMA issued above has finished once this arrives
@@ -352,14 +440,15 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         } else if (!DKDV) {
             query_stats(own_pos, my_nl, my_nd);
         }
-        // P (or P^T) and dZ for the 32 columns [col0, col0 + 32) of TMEM buffer `buf`, whose
-        // column c is streamed position w0 + c; MASK applies the causal diagonal and the
-        // sequence bounds.
-        auto chunk = [&](auto mask_c, uint32_t buf, int col0, const float *snl, const float *snd, int w0) {
+        // P (or P^T) and dZ for the 32 columns [col0, col0 + 32) of the step (S at TMEM column
+        // s_col, dP at dp_col), column c being streamed position w0 + c; MASK applies the
+        // causal diagonal and the sequence bounds.
+        auto chunk = [&](auto mask_c, uint32_t s_col, uint32_t dp_col, int col0, const float *snl, const float *snd,
+                         int w0) {
             constexpr bool MASK = decltype(mask_c)::value;
             uint32_t sv[32], dv[32];
-            tmem_ld32(buf + lane_base + col0, sv);
-            tmem_ld32(buf + lane_base + BwdStep<DKDV>::COL_DP + col0, dv);
+            tmem_ld32(s_col + lane_base + col0, sv);
+            tmem_ld32(dp_col + lane_base + col0, dv);
             tmem_ld_wait();
             tmem_reg_fence<32>(sv);
             tmem_reg_fence<32>(dv);
@@ -398,21 +487,20 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             // packed columns of this thread start at its own first column (STEP/2 * half), so
             // neither thread of the row overwrites columns the other one has yet to read
-            constexpr int HS = BwdStep<DKDV>::STEP / 2;  // columns per thread and step
+            constexpr int HS = Kd::STEP / 2;  // columns per thread and step
             const int pcol = half * HS + (col0 - half * HS) / 2;
             if (DKDV) {
-                tmem_st16(buf + lane_base + pcol, pk);                             // P^T over S^T
-                tmem_st16(buf + lane_base + BwdStep<DKDV>::COL_DP + pcol, zk);  // dZ^T over dP^T
+                tmem_st16(s_col + lane_base + pcol, pk);   // P^T over S^T
+                tmem_st16(dp_col + lane_base + pcol, zk);  // dZ^T over dP^T
             } else {
-                tmem_st16(buf + lane_base + pcol, zk);  // dZ over S
+                tmem_st16(s_col + lane_base + pcol, zk);  // dZ over S
             }
         };
-        using St = BwdStep<DKDV>;
-        for (int k = 0; ok && k < n * St::PER_TILE; ++k) {
-            const int t = k / St::PER_TILE, u = k % St::PER_TILE;  // streamed tile, part
-            const int w0 = ws + t * BM + u * St::STEP;              // position of the step's first streamed row
+        for (int k = 0; ok && k < n * Kd::PER_TILE; ++k) {
+            const int t = k / Kd::PER_TILE, u = k % Kd::PER_TILE;  // streamed tile, part
+            const int w0 = ws + t * BM + u * Kd::STEP;              // position of the step's first streamed row
             const int slot = t & 1;
-            const float *snl = stats + slot * 2 * BM + u * St::STEP, *snd = snl + BM;
+            const float *snl = stats + slot * 2 * BM + u * Kd::STEP, *snd = snl + BM;
             if (DKDV && u == 0) {
                 if (publisher) {
                     // publish this thread's query column statistics, prefetch the next tile's
@@ -424,28 +512,30 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (!(ok = __all_sync(0xffffffffu, wait_bounded(&stats_ready[slot], (t >> 1) & 1, abort_flag, lim, 440))))
                     break;
             }
-            if (!(ok = __all_sync(0xffffffffu, wait_bounded(&s_full[k % St::NBUF], (k / St::NBUF) & 1, abort_flag,
-                                                            lim, 450 + k % St::NBUF))))
+            if (!(ok = __all_sync(0xffffffffu, wait_bounded(&s_full[k % Kd::NBAR], (k / Kd::NBAR) & 1, abort_flag,
+                                                            lim, 450 + k % Kd::NBAR))))
                 break;
             tc_fence_after_sync();
             // does any pair of this warp's rows with the step's positions need a mask?
-            const bool row_partial = w0 < row_lo || w0 + St::STEP > row_hi ||
-                                     (CAUSAL && (DKDV ? w0 < own_pos : w0 + St::STEP - 1 > own_pos));
+            const bool row_partial = w0 < row_lo || w0 + Kd::STEP > row_hi ||
+                                     (CAUSAL && (DKDV ? w0 < own_pos : w0 + Kd::STEP - 1 > own_pos));
             const bool masked = __any_sync(0xffffffffu, row_partial);
             // this thread's STEP/2 columns [STEP/2 * half, ...) of the step, 32 at a time; the
             // results are stored over columns this thread has already read
-            const uint32_t buf = tmem + (k % St::NBUF) * St::COL_BUF;
+            // S of step k in TMEM buffer k % 2; dP next to it (dK/dV) or in its own columns (dQ)
+            const uint32_t s_col = tmem + (k & 1) * 128;
+            const uint32_t dp_col = DKDV ? s_col + Kd::STEP : tmem + Kd::COL_DP_DQ;
 #pragma unroll 1
-            for (int c = 0; c < St::STEP / 64; ++c) {
-                const int col0 = half * (St::STEP / 2) + c * 32;
+            for (int c = 0; c < Kd::STEP / 64; ++c) {
+                const int col0 = half * (Kd::STEP / 2) + c * 32;
                 if (masked)
-                    chunk(std::integral_constant<bool, true>{}, buf, col0, snl, snd, w0);
+                    chunk(std::integral_constant<bool, true>{}, s_col, dp_col, col0, snl, snd, w0);
                 else
-                    chunk(std::integral_constant<bool, false>{}, buf, col0, snl, snd, w0);
+                    chunk(std::integral_constant<bool, false>{}, s_col, dp_col, col0, snl, snd, w0);
             }
             tmem_st_wait();
             tc_fence_before_sync();
-            mbar_arrive(&p_ready[k % St::NBUF]);
+            mbar_arrive(&p_ready[k % Kd::NBAR]);
         }
         if (ok && n > 0) ok = __all_sync(0xffffffffu, wait_bounded(done, 0, abort_flag, lim, 460));
         if (ok) {
@@ -453,12 +543,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const bool store = own_pos < S;
             const int64_t grow = (row0 + own_pos) * p.H + h;  // token row, head
             if (DKDV) {
-                store_row<D, BF16>(tmem + lane_base + C::COL_ACC0, 1.f, static_cast<uint8_t *>(p.dv) + grow * D * 2,
+                store_row<D, BF16>(tmem + lane_base + Kd::COL_ACC0, 1.f, static_cast<uint8_t *>(p.dv) + grow * D * 2,
                                    store, half);
-                store_row<D, BF16>(tmem + lane_base + C::COL_ACC1, p.scale, static_cast<uint8_t *>(p.dk) + grow * D * 2,
+                store_row<D, BF16>(tmem + lane_base + Kd::COL_ACC1, p.scale, static_cast<uint8_t *>(p.dk) + grow * D * 2,
                                    store, half);
             } else {
-                store_row<D, BF16>(tmem + lane_base + C::COL_ACC0, p.scale, static_cast<uint8_t *>(p.dq) + grow * D * 2,
+                store_row<D, BF16>(tmem + lane_base + Kd::COL_ACC0, p.scale, static_cast<uint8_t *>(p.dq) + grow * D * 2,
                                    store, half);
             }
         }
@@ -521,6 +611,7 @@ template <int D, bool BF16, bool CAUSAL, bool DKDV, bool PACKED>
 cudaError_t launch_bwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
                          const BwdParams &p, dim3 grid, cudaStream_t st) {
     using C = BwdCfg<D>;
+    using Kd = BwdKind<D, DKDV>;
     auto kern = fa_bwd_kernel<D, BF16, CAUSAL, DKDV, PACKED>;
     static uint64_t attr_set_mask = 0;  // per-device shared-memory opt-in done
     int dev = 0;
@@ -528,11 +619,11 @@ cudaError_t launch_bwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
     if (e != cudaSuccess) return e;
     const uint64_t bit = uint64_t(1) << (dev & 63);
     if (!(__atomic_load_n(&attr_set_mask, __ATOMIC_ACQUIRE) & bit)) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Kd::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         __atomic_fetch_or(&attr_set_mask, bit, __ATOMIC_RELEASE);
     }
-    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, tdo, p);
+    kern<<<grid, C::NUM_THREADS, Kd::SMEM_BYTES, st>>>(tq, tk, tv, tdo, p);
     return cudaGetLastError();
 }
 
