@@ -107,6 +107,19 @@ def varlen_case(lengths: Sequence[int], total_len: int, H: int, D: int,
     return VarlenCase(q, k, v, idx, cu, int(max(lengths) if lengths else 0), H, D)
 
 
+def right_padded_case(lengths: Sequence[int], slot: int, H: int, D: int,
+                      dtype: torch.dtype, seed: int = 0) -> VarlenCase:
+    """A (B, slot) batch with right padding, flattened to (1, B*slot, H, D): sequence b holds
+    rows [b*slot, b*slot + lengths[b]), so its valid positions form one consecutive run."""
+    if any(n > slot for n in lengths):
+        raise ValueError("a sequence is longer than its slot")
+    total_len = slot * len(lengths)
+    q, k, v = dense_qkv(1, total_len, H, D, dtype, seed)
+    idx = torch.tensor([b * slot + r for b, n in enumerate(lengths) for r in range(n)], dtype=torch.int64)
+    cu = cu_seqlens_from_lengths(lengths)
+    return VarlenCase(q, k, v, idx, cu, int(max(lengths) if lengths else 0), H, D)
+
+
 def packed_qkv(lengths: Sequence[int], H: int, D: int, dtype: torch.dtype, seed: int = 0):
     """Packed (total, H, D) q, k, v plus int32 cu_seqlens, with no padding step."""
     total = int(sum(lengths))

@@ -249,8 +249,10 @@ def test_workload_varlen_pipeline_all_rows():
 
 
 # ----------------------------------------------------------------------------- fused packed path
-def _fused_case(lengths, total_len, H, D, dtype, causal, seed):
-    case = fa_inputs.varlen_case(lengths, total_len, H, D, dtype, seed=seed)
+def _fused_case(lengths, total_len, H, D, dtype, causal, seed, case=None):
+    if case is None:
+        case = fa_inputs.varlen_case(lengths, total_len, H, D, dtype, seed=seed)
+    total_len = case.q_pad.shape[1]
     dev = torch.device("cuda:0")
     qp, kp, vp = case.q_pad.to(dev), case.k_pad.to(dev), case.v_pad.to(dev)
     idx, cu = case.indices.to(dev), case.cu_seqlens.to(dev)
@@ -279,6 +281,26 @@ def test_fused_padded_path(D, dtype, causal):
     flat = out.view(-1, 2, D)
     assert_o_close(flat[case.indices], O, dtype, "fused")
     assert_lse_close(lse, L, "fused")
+    mask = torch.ones(flat.shape[0], dtype=torch.bool)
+    mask[case.indices] = False
+    assert (flat[mask].view(torch.int16) == 0).all()
+
+
+@pytest.mark.parametrize("D,dtype", [(128, torch.bfloat16), (32, torch.float16), (256, torch.bfloat16)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fused_right_padded(D, dtype, causal):
+    """Right-padded batch: each sequence's rows form one run of consecutive padded rows, so
+    32-row groups inside a run move as TMA boxes and the others as per-row copies."""
+    lengths = [64, 97, 0, 32, 128, 5, 160, 33]
+    case = fa_inputs.right_padded_case(lengths, 160, 2, D, dtype, seed=D + 1)
+    case, out, lse, ref_pad, ref_lse = _fused_case(None, None, 2, D, dtype, causal, None, case=case)
+    assert torch.equal(out.view(torch.int16), ref_pad.view(torch.int16))
+    assert torch.equal(lse, ref_lse)
+    O, L = oracle.attention_varlen(oracle.unpad(case.q_pad, case.indices), oracle.unpad(case.k_pad, case.indices),
+                                   oracle.unpad(case.v_pad, case.indices), case.cu_seqlens, causal=causal)
+    flat = out.view(-1, 2, D)
+    assert_o_close(flat[case.indices], O, dtype, "fused right-padded")
+    assert_lse_close(lse, L, "fused right-padded")
     mask = torch.ones(flat.shape[0], dtype=torch.bool)
     mask[case.indices] = False
     assert (flat[mask].view(torch.int16) == 0).all()

@@ -82,11 +82,16 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     const bool bf16 = dtype == FA_BF16;
     const int inner = fa::fwd_box_inner_elems(D);
     CUtensorMap tq, tk, tv;
-    const int64_t map_rows = gather ? padded_rows : N;  // the fused path's copy threads do not use the maps
+    // fused path: maps over the padded tensors with 32-row boxes (one box per run of 32
+    // consecutive padded rows; other rows are copied by threads)
+    const int64_t map_rows = gather ? padded_rows : N;
     const int64_t kv_rows = paging ? static_cast<int64_t>(paging->num_pages) * paging->page_size : map_rows;
-    const int k_box = paging ? fa::fwd_paged_k_box_rows(D, paging->page_size) : fa::fwd_kv_tile_rows(D);
-    const int v_box = paging ? fa::fwd_paged_v_box_rows(D, paging->page_size) : fa::fwd_v_box_rows(D);
-    if (!encode_map(&tq, q, bf16, D, H, map_rows, inner, fa::fwd_tile_rows()) ||
+    const int q_box = gather ? fa::fwd_gather_run_rows() : fa::fwd_tile_rows();
+    const int k_box = paging ? fa::fwd_paged_k_box_rows(D, paging->page_size)
+                             : (gather ? fa::fwd_gather_run_rows() : fa::fwd_kv_tile_rows(D));
+    const int v_box = paging ? fa::fwd_paged_v_box_rows(D, paging->page_size)
+                             : (gather ? fa::fwd_gather_run_rows() : fa::fwd_v_box_rows(D));
+    if (!encode_map(&tq, q, bf16, D, H, map_rows, inner, q_box) ||
         !encode_map(&tk, k, bf16, D, H, kv_rows, inner, k_box) ||
         !encode_map(&tv, v, bf16, D, H, kv_rows, inner, v_box))
         return FA_ERR_CUDA;

@@ -51,6 +51,7 @@ int fwd_box_inner_elems(int D) { return (2 * D >= 128) ? 64 : D; }
 
 int fwd_kv_tile_rows(int D) { return 128; }
 int fwd_v_box_rows(int D) { return (D == 256) ? 64 : 128; }
+int fwd_gather_run_rows() { return 32; }
 int fwd_paged_k_box_rows(int D, int page_size) { return page_size < fwd_kv_tile_rows(D) ? page_size : fwd_kv_tile_rows(D); }
 int fwd_paged_v_box_rows(int D, int page_size) { return page_size < fwd_v_box_rows(D) ? page_size : fwd_v_box_rows(D); }
 

@@ -29,8 +29,9 @@
 //               NS-stage shared-memory ring guarded by full/empty mbarriers. When tile
 //               rows must be gathered row by row (fused unpad, 16-row pages), warps 8, 10
 //               and 11 copy them with cp.async instead (fused unpad: each softmax warp
-//               copies its own Q rows, and warps 8, 10 and 11 clear the output's padding
-//               rows once their K/V copies are issued).
+//               copies its own Q rows, 32-row runs of consecutive padded rows move as TMA
+//               boxes, and warps 8, 10 and 11 clear the output's padding rows once their
+//               K/V copies are issued).
 //   epilogue    each softmax warp stages its 32 O rows in its tile's Q buffer (free once
 //               the tile's MMAs are done) and writes them out as whole rows.
 //   warp 9      allocates TMEM; one thread issues every tcgen05.mma:
@@ -389,6 +390,27 @@ __device__ __forceinline__ void copy_group(uint32_t dst, int rows, int g, int64_
     }
 }
 
+// Fused packed path: the 32-row group g of a [NB][rows][SW] tile whose row g*32 + i comes from
+// padded row pr of lane i. When the 32 padded rows are consecutive (one sequence's tokens in
+// a right-padded batch) the group moves as NB TMA boxes of 32 rows, its bytes counted on
+// `bar` before this warp's arrivals; otherwise as 16-byte cp.async copies.
+template <int NB, int SW, int D>
+__device__ __forceinline__ void fetch_group(uint8_t *tile, int rows, int g, int64_t pr, const void *src,
+                                            const CUtensorMap *map, int b0, int H, int h, int lane, uint64_t *bar,
+                                            uint64_t pol) {
+    const int64_t pr0 = __shfl_sync(0xffffffffu, pr, 0);
+    if (__all_sync(0xffffffffu, pr == pr0 + lane)) {
+        if (lane == 0) {
+            mbar_expect_tx(bar, 32 * NB * SW);
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+                tma_load_3d(tile + (b * rows + g * 32) * SW, map, bar, (b0 + b) * (SW / 2), h, static_cast<int>(pr0), pol);
+        }
+    } else {
+        copy_group<NB, SW, D>(smem_u32(tile), rows, g, pr, src, b0, H, h, lane);
+    }
+}
+
 // PAGED: K/V read through p.block_table (a separate instantiation, so the producer code of
 // the contiguous path stays as small as its register budget wants).
 template <int D, bool BF16, bool CAUSAL, bool PAGED>
@@ -617,6 +639,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tok0 = kvbase + j * BN + ((L & 1) ? u * C::VROWS_PER_UNIT : 0);
                     rows = (L & 1) ? C::VROWS_PER_UNIT : BN;
                 };
+                const uint64_t pol_kv = l2_policy_evict_last();
                 int64_t cur[2], nxt[2] = {first_rows[0], first_rows[1]};  // part 0's rows: read at set-up
                 int gU = 0;                                                // running index of part U's first group
                 for (int U = 0; U < loads; ++U) {
@@ -635,16 +658,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     if (U >= NS &&
                         !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
                         break;
-                    const uint32_t dst = smem_u32(c.sKV + stage * C::UNIT_BYTES);
+                    uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
 #pragma unroll
                     for (int k = 0; k < 2; ++k) {
                         const int g = g0 + 3 * k;
                         if (g * 32 >= rows) continue;
                         if ((U / C::UNITS) & 1)
-                            copy_group<C::NBLK, SW, D>(dst, rows, g, cur[k], p.v, 0, p.H, h, lane);
+                            fetch_group<C::NBLK, SW, D>(dst, rows, g, cur[k], p.v, &tm_v, 0, p.H, h, lane,
+                                                        &c.kv_full[stage], pol_kv);
                         else
-                            copy_group<C::KBLK_PER_UNIT, SW, D>(dst, rows, g, cur[k], p.k,
-                                                                (U % C::UNITS) * C::KBLK_PER_UNIT, p.H, h, lane);
+                            fetch_group<C::KBLK_PER_UNIT, SW, D>(dst, rows, g, cur[k], p.k, &tm_k,
+                                                                 (U % C::UNITS) * C::KBLK_PER_UNIT, p.H, h, lane,
+                                                                 &c.kv_full[stage], pol_kv);
                     }
                     cp_async_mbar_arrive(&c.kv_full[stage]);  // arrives once this thread's copies have landed
                     issued = U + 1;
@@ -873,7 +898,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // arrive on q_full[t] as their copies land.
             int64_t pr = (tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
             if (pr < 0 || pr >= p.padded_rows) pr = 0;  // never read outside q
-            copy_group<C::NBLK, SW, D>(smem_u32(c.sQ + t * C::Q_BYTES), BM, quarter, pr, p.q, 0, p.H, h, lane);
+            fetch_group<C::NBLK, SW, D>(c.sQ + t * C::Q_BYTES, BM, quarter, pr, p.q, &tm_q, 0, p.H, h, lane,
+                                        &c.q_full[t], l2_policy_evict_first());
             cp_async_mbar_arrive(&c.q_full[t]);
         }
         int klo = 0, khi = 1;

@@ -46,6 +46,8 @@ int fwd_box_inner_elems(int D);
 int fwd_kv_tile_rows(int D);
 // Rows of one V box the producer copies (a V tile may move as several row parts).
 int fwd_v_box_rows(int D);
+// Fused packed path: rows of one TMA box (a run of consecutive padded rows).
+int fwd_gather_run_rows();
 // Paged K/V: rows per K box / V box for a page size (a box never crosses a page).
 int fwd_paged_k_box_rows(int D, int page_size);
 int fwd_paged_v_box_rows(int D, int page_size);
