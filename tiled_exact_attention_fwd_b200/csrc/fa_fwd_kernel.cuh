@@ -26,12 +26,12 @@
 //               final 1/l cancels exactly). At the end: O/l -> fp16/bf16 -> global, and the
 //               LSE.
 //   warp 8      TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ... through an
-//               NS-stage shared-memory ring guarded by full/empty mbarriers. When tile
-//               rows must be gathered row by row (fused unpad, 16-row pages), warps 8, 10
-//               and 11 copy them with cp.async instead (fused unpad: each softmax warp
-//               copies its own Q rows, 32-row runs of consecutive padded rows move as TMA
-//               boxes, and warps 8, 10 and 11 clear the output's padding rows once their
-//               K/V copies are issued).
+//               NS-stage shared-memory ring guarded by full/empty mbarriers. Fused unpad:
+//               warps 8, 10 and 11 copy the K/V rows with cp.async instead, each softmax
+//               warp copies its own Q rows, 32-row runs of consecutive padded rows move as
+//               TMA boxes, and warps 8, 10 and 11 clear the output's padding rows once their
+//               copies are issued. Pages under 64 rows: warp 8 moves Q and K by TMA while
+//               warps 10 and 11 copy V with cp.async.
 //   epilogue    each softmax warp stages its 32 O rows in its tile's Q buffer (free once
 //               the tile's MMAs are done) and writes them out as whole rows.
 //   warp 9      allocates TMEM; one thread issues every tcgen05.mma:
@@ -475,9 +475,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // after they land, so the MMA thread fences the async proxy after its waits. (The paged
     // path's zeroed page tails are fenced by the writing thread itself before it releases
     // the stage.)
-    // Paged K/V in 16-row pages: TMA boxes that small run at half the copy rate, so the fused
-    // path's copy threads fetch Q, K and V instead (the same fence applies).
-    const bool copy_pages = PAGED && p.page_size < 32;
+    // Paged K/V in pages under 64 rows: TMA boxes that small move too few bytes per SM, so
+    // the V parts go by cp.async copies beside the TMA's K parts (the same fence applies).
+    const bool copy_pages = PAGED && p.page_size < 64;
     c.fused = p.gather != nullptr || copy_pages;
     c.nA = (kv_end_A + BN - 1) / BN;
     c.nB = c.two ? (kv_end_B + BN - 1) / BN : 0;
@@ -512,9 +512,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (p.gather && (warp == C::WARP_TMA || warp > C::WARP_MMA)) fused_group_rows(p, kvbase, BN, pw, lane, first_rows);
 
     if (threadIdx.x == 0) {
-        const int fill_arrivals = c.fused ? 96 : 1;  // copy producers: the 96 copy threads arrive
-        // fused packed path: a query tile is copied by the 128 threads of its softmax warpgroup
-        const int q_arrivals = p.gather ? 128 : fill_arrivals;
+        // ring barriers: one arrival (the TMA lane's), or per copy thread: fused packed path 96
+        // (warps 8, 10, 11); pages under 64 rows 65 (the TMA lane + warps 10, 11). Query tiles: the
+        // TMA lane's, or the 128 threads of the softmax warpgroup (fused packed path).
+        const int fill_arrivals = p.gather ? 96 : (copy_pages ? 65 : 1);
+        const int q_arrivals = p.gather ? 128 : 1;
         for (int t = 0; t < 2; ++t) {
             mbar_init(&c.q_full[t], q_arrivals);
             mbar_init(&c.s_full[t], 1);
@@ -556,72 +558,99 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             int issued = 0;
             bool tail_issued = false;
             if (PAGED && copy_pages) {
-                // Paged K/V in small pages: warps 8, 10 and 11 (96 threads) copy rows with
-                // 16-byte cp.async into the swizzled layout; row r of a key tile is position
-                // pos of the sequence, read from its page; positions past the sequence end
-                // are zero-filled (no page is read for them). Q rows are plain token rows.
-                constexpr int CPB = SW / 16;
+                // Paged K/V in small pages: two engines share the bytes. Warp 8 (lane 0) moves
+                // the query tiles and the K parts by TMA, one box per page chunk (chunks wholly
+                // past the sequence end are boxes at a negative row: zeros); warps 10 and 11
+                // copy the V parts row by row with 16-byte cp.async into the swizzled layout,
+                // zero-filling positions past the sequence end (no page is read for them). A
+                // ring barrier takes 65 arrivals per part: the TMA lane's (with the K bytes, or
+                // a plain arrival on a V part) and one per copy thread (plain on a K part, or
+                // once its V copies have landed).
                 const int32_t *bt = p.block_table + static_cast<int64_t>(blockIdx.z) * p.max_blocks;
                 bool bad_page = false;
-                // rows [pos0, pos0 + rows) x column blocks [b0, b0 + NB) into dst as [NB][rows][SW];
-                // `paged` selects the K/V pool (else the dense q rows of this sequence)
-                auto fill_rows = [&](auto nb_c, uint8_t *dst, const void *src, uint64_t *bar, int pos0, int rows,
-                                     int b0, bool paged) {
-                    constexpr int CPR = decltype(nb_c)::value * CPB;
-                    const uint32_t dst_u32 = smem_u32(dst);
-                    for (int g = pw; g * 32 < rows; g += 3) {
-                        const int pos = pos0 + g * 32 + lane;
-                        const bool valid = pos < seqlen;
-                        int64_t prow = 0;
-                        if (valid) {
-                            if (paged) {
-                                int pg = __ldg(bt + (pos >> p.page_shift));
-                                if (pg < 0 || pg >= p.num_pages) {
-                                    bad_page = true;
-                                    pg = 0;
-                                }
-                                prow = (static_cast<int64_t>(pg) << p.page_shift) + (pos & (p.page_size - 1));
-                            } else {
-                                prow = static_cast<int64_t>(seq_start) + pos;
-                            }
+                auto page_row = [&](int pos) {  // physical row of key position pos (< seqlen)
+                    int pg = __ldg(bt + (pos >> p.page_shift));
+                    if (pg < 0 || pg >= p.num_pages) {
+                        bad_page = true;
+                        pg = 0;
+                    }
+                    return (static_cast<int64_t>(pg) << p.page_shift) + (pos & (p.page_size - 1));
+                };
+                if (warp == C::WARP_TMA) {
+                    if (lane == 0) {
+                        const uint64_t pol_q = l2_policy_evict_first();
+                        const uint64_t pol_kv = l2_policy_evict_last();
+                        for (int t = 0; t < nq; ++t) {
+                            mbar_arrive_expect_tx(&c.q_full[t], C::Q_BYTES);
+#pragma unroll
+                            for (int b = 0; b < C::NBLK; ++b)
+                                tma_load_3d(c.sQ + t * C::Q_BYTES + b * BM * SW, &tm_q, &c.q_full[t], b * C::SWE, h,
+                                            qbase + t * BM, pol_q);
                         }
-                        const uint8_t *srow = static_cast<const uint8_t *>(src) + b0 * SW;
-#pragma unroll 4
-                        for (int i = 0; i < CPR; ++i) {
-                            const int idx = i * 32 + lane;
-                            const int rr = idx / CPR, ch = idx % CPR;
-                            const int64_t pr = __shfl_sync(0xffffffffu, prow, rr);
-                            const bool ok_row = __shfl_sync(0xffffffffu, valid, rr);
-                            const int r = g * 32 + rr;
-                            const int blk = ch / CPB, cc = ch % CPB;
-                            const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
-                            cp_async_16_zfill(dst_u32 + blk * rows * SW + r * SW + ((cc ^ swz) << 4),
-                                              srow + (pr * p.H + h) * static_cast<int64_t>(D) * 2 + ch * 16,
-                                              ok_row ? 16u : 0u);
+                        const int box = min(p.page_size, BN);
+                        for (int U = 0; U < loads; ++U) {
+                            const int stage = U % NS;
+                            if (U >= NS &&
+                                !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
+                                break;
+                            const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
+                            if (L & 1) {
+                                mbar_arrive(&c.kv_full[stage]);  // V part: copied by warps 10 and 11
+                            } else {
+                                uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
+                                const int pos0 = j * BN;
+                                const int part_valid = seqlen - pos0;
+                                mbar_arrive_expect_tx(&c.kv_full[stage], C::UNIT_BYTES);
+                                for (int r = 0; r < BN; r += box) {
+                                    const int prow = (r < part_valid) ? static_cast<int>(page_row(pos0 + r)) : -box;
+                                    for (int b = 0; b < C::KBLK_PER_UNIT; ++b)
+                                        tma_load_3d(dst + (b * BN + r) * SW, &tm_k, &c.kv_full[stage],
+                                                    (u * C::KBLK_PER_UNIT + b) * C::SWE, h, prow, pol_kv);
+                                }
+                            }
+                            issued = U + 1;
                         }
                     }
-                    cp_async_mbar_arrive(bar);
-                };
-                using AllBlk = std::integral_constant<int, C::NBLK>;
-                using KBlk = std::integral_constant<int, C::KBLK_PER_UNIT>;
-                for (int t = 0; t < nq; ++t)
-                    fill_rows(AllBlk{}, c.sQ + t * C::Q_BYTES, p.q, &c.q_full[t], q0 + t * BM, BM, 0, false);
-                for (int U = 0; U < loads; ++U) {
-                    const int stage = U % NS;
-                    if (U >= NS &&
-                        !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
-                        break;
-                    const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
-                    uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
-                    if (L & 1)
-                        fill_rows(AllBlk{}, dst, p.v, &c.kv_full[stage], j * BN + u * C::VROWS_PER_UNIT,
-                                  C::VROWS_PER_UNIT, 0, true);
-                    else
-                        fill_rows(KBlk{}, dst, p.k, &c.kv_full[stage], j * BN, BN, u * C::KBLK_PER_UNIT, true);
-                    issued = U + 1;
+                } else {
+                    constexpr int CPB = SW / 16;
+                    constexpr int CPR = C::NBLK * CPB;  // 16-byte chunks per V row
+                    const int w = pw - 1;                // copy warp 0, 1
+                    for (int U = 0; U < loads; ++U) {
+                        const int stage = U % NS;
+                        if (U >= NS &&
+                            !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
+                            break;
+                        const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
+                        if (!(L & 1)) {
+                            mbar_arrive(&c.kv_full[stage]);  // K part: moved by the TMA
+                            continue;
+                        }
+                        // V part u of tile j: rows [pos0, pos0 + VROWS_PER_UNIT), every column block
+                        const int pos0 = j * BN + u * C::VROWS_PER_UNIT;
+                        const uint32_t dst_u32 = smem_u32(c.sKV + stage * C::UNIT_BYTES);
+                        for (int g = w; g * 32 < C::VROWS_PER_UNIT; g += 2) {
+                            const int pos = pos0 + g * 32 + lane;
+                            const bool valid = pos < seqlen;
+                            const int64_t prow = valid ? page_row(pos) : 0;
+#pragma unroll 4
+                            for (int i = 0; i < CPR; ++i) {
+                                const int idx = i * 32 + lane;
+                                const int rr = idx / CPR, ch = idx % CPR;
+                                const int64_t pr = __shfl_sync(0xffffffffu, prow, rr);
+                                const bool ok_row = __shfl_sync(0xffffffffu, valid, rr);
+                                const int r = g * 32 + rr;
+                                const int blk = ch / CPB, cc = ch % CPB;
+                                const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
+                                cp_async_16_zfill(dst_u32 + blk * C::VROWS_PER_UNIT * SW + r * SW + ((cc ^ swz) << 4),
+                                                  static_cast<const uint8_t *>(p.v) +
+                                                      (pr * p.H + h) * static_cast<int64_t>(D) * 2 + ch * 16,
+                                                  ok_row ? 16u : 0u);
+                            }
+                        }
+                        cp_async_mbar_arrive(&c.kv_full[stage]);  // arrives once this thread's copies have landed
+                    }
+                    cp_async_wait_all();  // nothing of this thread is left in flight at exit
                 }
-                cp_async_wait_all();  // nothing of this thread is left in flight at exit
-                issued = 0;
                 if (bad_page) record_error(FA_ERR_INDEX, 151);
             } else if (p.gather) {
                 // Fused packed path: warps 8, 10 and 11 (96 threads) copy every K/V row from the
