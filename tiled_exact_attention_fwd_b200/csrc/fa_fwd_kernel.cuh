@@ -104,9 +104,6 @@ struct Cfg {
     static_assert(!SPLIT_REGS || 128 * REGS_LOW + 256 * REGS_HIGH <= NUM_THREADS * LAUNCH_REGS, "register split");
     // Column pairs (out of every 4) whose exp2 runs on the FMA pipe instead of MUFU.
     static constexpr int EMU_PAIRS_OF_4 = 0;
-    // MMA descriptors as base + offset (measured: removes the D <= 64 kernels' spills, +2-4 %;
-    // at D = 128 the hoisted descriptors spill instead and the kernel loses 6 %)
-    static constexpr bool DESC_ADD = D <= 64;
     // shared memory map (offsets from a 1024-byte aligned base)
     static constexpr int SMEM_LIMIT = 227 * 1024;
     static constexpr int RESERVED = 1024 /*alignment*/ + 512 /*barriers, misc*/;
@@ -287,11 +284,11 @@ __device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first
         tc_fence_after_sync();
     }
     constexpr int UK = D / 16 / C::UNITS;  // k-steps per K part
-    const uint32_t q_addr = smem_u32(c.sQ + t * C::Q_BYTES);
-    // C::DESC_ADD: descriptors of the tile bases, to which a k-step adds its byte offset / 16
-    // (shared addresses stay below 2^18 bytes, so the 14-bit address field never carries);
-    // otherwise each k-step's descriptor is built from its address.
-    const uint64_t q_desc = smem_desc(q_addr, 16, 8 * SW, C::LAYOUT);
+    // Operand descriptors as 32-bit words: the low word of each tile base, to which a k-step
+    // adds its byte offset / 16, and the high word shared by Q and K (one add per operand
+    // and k-step keeps the single issuing thread's work per MMA short).
+    constexpr uint32_t dhi = smem_desc_hi(8 * SW, C::LAYOUT);
+    const uint32_t q_lo = smem_desc_lo(smem_u32(c.sQ + t * C::Q_BYTES), 16);
     const int b = c.buf(t, jj);
     const uint32_t d_tmem = c.tmem + b * BN;
 #pragma unroll
@@ -302,19 +299,14 @@ __device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first
             tc_fence_after_sync();
             if (c.fused) fence_proxy_async_smem();
         }
-        const uint32_t k_addr = smem_u32(c.sKV + stage * C::UNIT_BYTES);
-        const uint64_t k_desc = smem_desc(k_addr, 16, 8 * SW, C::LAYOUT);
+        const uint32_t k_lo = smem_desc_lo(smem_u32(c.sKV + stage * C::UNIT_BYTES), 16);
 #pragma unroll
         for (int kk = 0; kk < UK; ++kk) {
             const int k = u * UK + kk;
             const uint32_t blk = (k * 32) / SW, off = (k * 32) % SW;
             const uint32_t lb = blk - u * C::KBLK_PER_UNIT;  // column block inside the part
-            const uint32_t qo = blk * BM * SW + off, ko = lb * BN * SW + off;
-            if constexpr (C::DESC_ADD)
-                umma_ss(d_tmem, q_desc + (qo >> 4), k_desc + (ko >> 4), idesc, k > 0 ? 1u : 0u);
-            else
-                umma_ss(d_tmem, smem_desc(q_addr + qo, 16, 8 * SW, C::LAYOUT),
-                        smem_desc(k_addr + ko, 16, 8 * SW, C::LAYOUT), idesc, k > 0 ? 1u : 0u);
+            umma_ss_w(d_tmem, q_lo + ((blk * BM * SW + off) >> 4), k_lo + ((lb * BN * SW + off) >> 4), dhi, idesc,
+                      k > 0 ? 1u : 0u);
         }
         if (u + 1 < C::UNITS) {
             if (last_use) umma_commit(&c.kv_empty[stage]);  // release this part early
@@ -337,6 +329,7 @@ __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first
     if (!wait_bounded(&c.p_full[b], c.sphase(jj), c.abort_flag, c.lim, 210 + t)) return false;
     tc_fence_after_sync();
     constexpr int UV = BN / 16 / C::UNITS;  // k-steps per V part
+    constexpr uint32_t dhi = smem_desc_hi(8 * SW, C::LAYOUT);  // high descriptor word of V
     const uint32_t a_tmem = c.tmem + (c.dec ? C::P_COL + 64 * t : b * BN);
     const uint32_t o_tmem = c.tmem + C::O_COL + t * D;
 #pragma unroll
@@ -347,14 +340,11 @@ __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first
             tc_fence_after_sync();
             if (c.fused) fence_proxy_async_smem();
         }
-        const uint32_t v_addr = smem_u32(c.sKV + stage * C::UNIT_BYTES);
-        const uint64_t v_desc = smem_desc(v_addr, C::VROWS_PER_UNIT * SW, 8 * SW, C::LAYOUT);
+        const uint32_t v_lo = smem_desc_lo(smem_u32(c.sKV + stage * C::UNIT_BYTES), C::VROWS_PER_UNIT * SW);
 #pragma unroll
         for (int kk = 0; kk < UV; ++kk) {
             const int k = u * UV + kk;
-            const uint64_t bd = C::DESC_ADD ? v_desc + ((kk * 16 * SW) >> 4)
-                                            : smem_desc(v_addr + kk * 16 * SW, C::VROWS_PER_UNIT * SW, 8 * SW, C::LAYOUT);
-            umma_ts(o_tmem, a_tmem + k * 8, bd, idesc, (jj > 0 || k > 0) ? 1u : 0u);
+            umma_ts_w(o_tmem, a_tmem + k * 8, v_lo + ((kk * 16 * SW) >> 4), dhi, idesc, (jj > 0 || k > 0) ? 1u : 0u);
         }
         if (u + 1 < C::UNITS) {
             if (last_use) umma_commit(&c.kv_empty[stage]);
