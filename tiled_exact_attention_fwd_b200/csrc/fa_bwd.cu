@@ -112,12 +112,14 @@ template <int D, bool BF16, int STEP>
 __device__ __forceinline__ void mma_rows_step(uint32_t d_tmem, const uint8_t *a, const uint8_t *b, int u) {
     using C = BwdCfg<D>;
     constexpr uint32_t idesc = idesc_f16(C::BM, STEP, BF16, false);
-    const uint32_t a0 = smem_u32(a), b0 = smem_u32(b) + u * STEP * C::SW;
+    // descriptors as 32-bit words: a k-step adds its byte offset / 16 to the low word
+    constexpr uint32_t hi = smem_desc_hi(8 * C::SW, C::LAYOUT);
+    const uint32_t a_lo = smem_desc_lo(smem_u32(a), 16), b_lo = smem_desc_lo(smem_u32(b) + u * STEP * C::SW, 16);
 #pragma unroll
     for (int k = 0; k < D / 16; ++k) {
         const uint32_t blk = (k * 32) / C::SW, off = (k * 32) % C::SW;
-        umma_ss(d_tmem, smem_desc(a0 + blk * C::BM * C::SW + off, 16, 8 * C::SW, C::LAYOUT),
-                smem_desc(b0 + blk * C::BM * C::SW + off, 16, 8 * C::SW, C::LAYOUT), idesc, k > 0 ? 1u : 0u);
+        const uint32_t o = (blk * C::BM * C::SW + off) >> 4;
+        umma_ss_w(d_tmem, a_lo + o, b_lo + o, hi, idesc, k > 0 ? 1u : 0u);
     }
 }
 
@@ -131,12 +133,12 @@ __device__ __forceinline__ void mma_acc_step(uint32_t d_tmem, uint32_t a_tmem, c
                                              bool accumulate) {
     using C = BwdCfg<D>;
     constexpr uint32_t idesc = idesc_f16(C::BM, D, BF16, true);
-    const uint32_t b0 = smem_u32(b) + u * STEP * C::SW;
+    constexpr uint32_t hi = smem_desc_hi(8 * C::SW, C::LAYOUT);
+    const uint32_t b_lo = smem_desc_lo(smem_u32(b) + u * STEP * C::SW, C::BM * C::SW);
 #pragma unroll
     for (int k = 0; k < STEP / 16; ++k)
-        umma_ts(d_tmem, a_tmem + k * 8 + (k >= STEP / 32 ? STEP / 4 : 0),
-                smem_desc(b0 + k * 16 * C::SW, C::BM * C::SW, 8 * C::SW, C::LAYOUT), idesc,
-                (accumulate || k > 0) ? 1u : 0u);
+        umma_ts_w(d_tmem, a_tmem + k * 8 + (k >= STEP / 32 ? STEP / 4 : 0), b_lo + ((k * 16 * C::SW) >> 4), hi, idesc,
+                  (accumulate || k > 0) ? 1u : 0u);
 }
 
 template <bool BF16>
