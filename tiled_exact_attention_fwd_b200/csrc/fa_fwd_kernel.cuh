@@ -40,7 +40,9 @@
 //               in the ping-pong order QK_A0, QK_B0, PV_A0, QK_A1, PV_B0, QK_B1, ..., so the
 //               tensor core works on one tile while the other tile's softmax runs. With a
 //               single tile the two S buffers are used alternately by that tile instead
-//               (order QK_0, QK_1, PV_0, QK_2, PV_1, ...).
+//               (order QK_0, QK_1, PV_0, QK_2, PV_1, ...). A single issuing thread is slower
+//               than the tensor core unless each MMA costs it a few instructions, so the
+//               operand descriptors are kept as 32-bit words and a k-step adds its offset.
 //
 // Every pipeline wait is bounded: after `timeout_ns` the waiting thread records
 // FA_ERR_TIMEOUT in a device word, raises a CTA-wide abort flag, and all roles drain
@@ -551,11 +553,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     c.tmem = *tmem_slot;
 
     if (warp >= C::NUM_SOFTMAX_WARPS) {
-        // producer / MMA warpgroup (its two remaining warps idle)
+        // producer / MMA warpgroup (its two remaining warps idle unless they copy rows)
         if constexpr (C::SPLIT_REGS) regs_dec<C::REGS_LOW>();
         if (warp == C::WARP_TMA || (c.fused && warp > C::WARP_MMA)) {
             // ------------------------------------------------------------ TMA producer
-            // (with the fused packed path also warps 10 and 11: copy producers)
+            // (fused packed path and pages under 64 rows: warps 10 and 11 copy rows too)
             const int nq = c.two ? 2 : 1;
             const int loads = 2 * n_all * C::UNITS;  // parts of K_0, V_0, K_1, V_1, ...
             int issued = 0;
