@@ -74,8 +74,8 @@ FA_API fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, 
 
 /*
  * Dense attention forward with K and V in a paged pool (the PagedAttention layout that page
- * hwcomputing.csdn.net "FlashAttention 的加速玄学", section 5, recommends for long contexts;
- * the page gives no layout, so this one is the common block-table form). Same result as
+ * mooersco.com "FlashAttention 的“加速玄学”", section 5, recommends for long contexts; the
+ * page gives no layout, so this one is the common block-table form). Same result as
  * fa_fwd on the contiguous K/V that the block table describes.
  *   q            (B, S, H, D) queries, element type `dtype`.
  *   k_cache,
@@ -137,14 +137,18 @@ FA_API fa_status fa_varlen_bwd(const void *q, const void *k, const void *v, cons
  * fa_bwd without the caller's delta workspace: the same computation and results, with the
  * workspace taken from a fixed device array that is part of the library (64 MiB, room for
  * B * H * S <= 2^24 rows; larger problems return FA_ERR_SHAPE before any launch). The pages
- * have no counterpart to this entry point; it exists for callers that may not allocate
- * (nothing here calls cudaMalloc or any allocating routine).
- *   Set-up: the first call on each device looks the array's address up (this loads the
- *   library's module on that device); make that first call outside any stream capture. Later
- *   calls only launch kernels and may be captured into a CUDA graph.
+ * have no counterpart to this entry point. It is for callers that cannot allocate device
+ * memory at the point where they run the backward pass: a runtime whose caching allocator
+ * already owns the device's free memory (a cudaMalloc there fails or breaks the allocator's
+ * accounting), or an engine that plans all of its memory ahead of time and forbids
+ * allocation inside a step. Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+ *   Device: the array lives on every device that loads the library, until the process exits;
+ *   the call uses the copy on the current device, which must be the operands' device.
+ *   Set-up: the first call on each device looks the array's address up, which loads the
+ *   library's module on that device; make that first call before any stream capture.
  *   Nothing has to start at zero: every call overwrites the rows it reads.
- *   Calls that overlap in time (different streams, or concurrent graph nodes) share the one
- *   array and race; serialise them.
+ *   Calls that overlap on the GPU (different streams, or concurrent graph nodes) share the
+ *   one array and race; serialise them.
  * Arguments as fa_bwd, minus `delta`.
  */
 FA_API fa_status fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *out, const void *dout,
@@ -222,11 +226,15 @@ FA_API fa_status fa_pad(const void *x, const int64_t *indices, int64_t nnz, int6
                  int64_t row_bytes, void *out, void *stream);
 
 /*
- * Device-side status of earlier launches: synchronises the device, returns FA_OK or the
- * first FA_ERR_TIMEOUT / FA_ERR_INDEX recorded by a kernel since the last call, and
- * clears it. `where` (may be NULL) receives a kernel-specific location code.
+ * Device-side status of earlier launches: returns FA_OK or the first FA_ERR_TIMEOUT /
+ * FA_ERR_INDEX that a kernel of this library recorded on the current device since the last
+ * call, and clears it. `where` (may be NULL) receives a kernel-specific location code.
+ * One small kernel and one 8-byte copy run on `stream` (NULL = the legacy default stream),
+ * and the call then waits for that stream only: every launch queued on `stream` before the
+ * call is covered; work on other streams is covered once it has finished. Returns
+ * FA_ERR_CUDA if the stream reports an error (for example a fault of an earlier kernel).
  */
-FA_API fa_status fa_device_status(int *where);
+FA_API fa_status fa_device_status(int *where, void *stream);
 
 /*
  * Self-test of the bounded wait used by every pipeline wait in the attention kernel:

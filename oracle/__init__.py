@@ -150,7 +150,7 @@ def attention_dense(q, k, v, scale: Optional[float] = None, causal: bool = False
 def paged_to_contiguous(cache: torch.Tensor, block_table, S: int) -> torch.Tensor:
     """Key positions 0..S-1 of every batch entry read out of a page pool: (B, S, H, D).
 
-    Page hwcomputing.csdn.net "FlashAttention 的加速玄学", section 5, recommends PagedAttention
+    Page mooersco.com "FlashAttention 的“加速玄学”", section 5, recommends PagedAttention
     without giving a layout; the block-table reading is: position pos of entry b is row
     pos % page_size of page block_table[b][pos // page_size] of the (num_pages, page_size,
     H, D) pool. A plain copy, page by page.

@@ -168,3 +168,27 @@ def test_varlen_bwd_validation(lib):
     assert call(8, 0) == -2
     assert call(6, FAKE + 2) == -5
     assert call(18, 4) == -3
+
+
+# The Python binding checks every caller-given buffer before the library sees it (the C entry
+# points take sizes from q alone, so a smaller output would be written past its end).
+def test_binding_rejects_wrong_output_shapes():
+    import torch
+    q = torch.zeros((1, 8, 2, 64), dtype=torch.bfloat16)
+    lse = torch.zeros((1, 2, 8), dtype=torch.float32)
+    good = torch.zeros_like(q)
+    small = torch.zeros((1, 4, 2, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="dq"):
+        fa.fa_bwd_noalloc(q, q, q, q, q, lse, small, good, good)
+    with pytest.raises(ValueError, match="dv"):
+        fa.fa_bwd_noalloc(q, q, q, q, q, lse, good, good, good.float())
+    with pytest.raises(ValueError, match="lse"):
+        fa.fa_bwd_noalloc(q, q, q, q, q, lse[:, :1], good, good, good)
+    with pytest.raises(ValueError, match="shape and dtype"):
+        fa.fa_bwd_noalloc(q, small, q, q, q, lse, good, good, good)
+    with pytest.raises(ValueError, match="dk"):
+        fa.fa_bwd(q, q, q, q, q, lse, dk=small)
+    with pytest.raises(ValueError, match="delta"):
+        fa.fa_bwd(q, q, q, q, q, lse, delta=lse[:, :, :4])
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        fa.fa_bwd_noalloc(q, q, q, q, q, lse, good, good, good)

@@ -39,3 +39,17 @@ def test_out_of_range_index_is_reported_and_skipped():
     assert st == -8
     assert torch.equal(u[0].cpu(), x[0, 1].cpu())
     assert float(u[1].abs().sum()) == 0.0
+
+
+def test_status_waits_for_its_own_stream_only():
+    import time
+    a, b = torch.cuda.Stream(), torch.cuda.Stream()
+    fa.fa_device_status(stream=a)  # first call: looks the error words up
+    with torch.cuda.stream(b):
+        torch.cuda._sleep(1_000_000_000)  # about half a second of GPU time on stream b
+    t0 = time.perf_counter()
+    st, _ = fa.fa_device_status(stream=a)
+    dt = time.perf_counter() - t0
+    b.synchronize()
+    assert st == 0
+    assert dt < 0.2, f"status on stream a waited {dt:.3f} s for stream b"

@@ -1,4 +1,4 @@
-"""Paged K/V (the PagedAttention layout of page hwcomputing.csdn.net "FlashAttention 的加速玄学",
+"""Paged K/V (the PagedAttention layout of page mooersco.com "FlashAttention 的“加速玄学”",
 section 5; the block-table layout is this library's reading, the page gives none).
 
 CPU: the oracle's page gather returns the contiguous keys exactly, whatever the pools hold

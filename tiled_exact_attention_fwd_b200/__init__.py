@@ -57,7 +57,7 @@ def lib() -> ctypes.CDLL:
         L.fa_unpad_qkv.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp]
         L.fa_varlen_fwd_padded.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i64, vp, vp, i32, i32, f32, i32, i32,
                                            vp]
-        L.fa_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        L.fa_device_status.argtypes = [ctypes.POINTER(ctypes.c_int), vp]
         L.fa_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
         for f in (L.fa_fwd, L.fa_fwd_paged, L.fa_bwd, L.fa_bwd_noalloc, L.fa_varlen_bwd, L.fa_varlen_fwd, L.fa_varlen_fwd_padded, L.fa_unpad, L.fa_unpad_qkv, L.fa_pad,
                   L.fa_device_status,
@@ -103,6 +103,24 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _shape(name: str, t: torch.Tensor, shape, dtype) -> None:
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def _like(name: str, t: torch.Tensor, shape, dtype) -> None:
+    """A caller-given output or workspace: exactly `shape` and `dtype` (the library writes every
+    element of that shape, so a smaller buffer would be overrun), CUDA and contiguous."""
+    _shape(name, t, shape, dtype)
+    _cuda_contig(name, t)
+
+
+def _same_device(ref: torch.Tensor, *ts: Optional[torch.Tensor]) -> None:
+    for t in ts:
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"every tensor must be on {ref.device}; got one on {t.device}")
+
+
 def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torch.Tensor] = None,
            lse: Optional[torch.Tensor] = None, scale: Optional[float] = None, causal: bool = False,
            return_lse: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
@@ -114,13 +132,15 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torc
     B, S, H, D = q.shape
     if out is None:
         out = torch.empty_like(q)
-    _cuda_contig("out", out)
+    _like("out", out, q.shape, q.dtype)
     if return_lse and lse is None:
         lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
     if lse is not None:
-        _cuda_contig("lse", lse)
-    st = lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
-                      float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
+        _like("lse", lse, (B, H, S), torch.float32)
+    _same_device(q, k, v, out, lse)
+    with torch.cuda.device(q.device):
+        st = lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                          float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
     _check(st, "fa_fwd")
     return out, lse
 
@@ -131,23 +151,30 @@ def fa_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
            causal: bool = False, stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Dense backward: gradients (dq, dk, dv), each (B, S, H, D), of out = fa_fwd(q, k, v) given
     dout and the forward's lse (B, H, S). `delta` is an optional fp32 (B, H, S) workspace."""
-    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse)):
-        _cuda_contig(n, t)
     if q.dim() != 4 or any(t.shape != q.shape or t.dtype != q.dtype for t in (k, v, out, dout)):
         raise ValueError("q, k, v, out, dout must share one (B, S, H, D) shape and dtype")
     B, S, H, D = q.shape
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, S):
-        raise ValueError("lse must be float32 (B, H, S)")
+    _shape("lse", lse, (B, H, S), torch.float32)
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        if t is not None:
+            _shape(n, t, q.shape, q.dtype)
+    if delta is not None:
+        _shape("delta", delta, (B, H, S), torch.float32)
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse)):
+        _cuda_contig(n, t)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     if delta is None:
         delta = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
-    for n, t in (("dq", dq), ("dk", dk), ("dv", dv), ("delta", delta)):
-        _cuda_contig(n, t)
-    st = lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
-                      _ptr(delta), B, H, S, D, float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q),
-                      _stream(stream))
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _like(n, t, q.shape, q.dtype)
+    _like("delta", delta, (B, H, S), torch.float32)
+    _same_device(q, k, v, out, dout, lse, dq, dk, dv, delta)
+    with torch.cuda.device(q.device):
+        st = lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                          _ptr(dv), _ptr(delta), B, H, S, D, float(scale) if scale else 0.0, int(bool(causal)),
+                          _dtype_code(q), _stream(stream))
     _check(st, "fa_bwd")
     return dq, dk, dv
 
@@ -168,9 +195,12 @@ def fa_varlen_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.
         raise ValueError("cu_seqlens must be a 1-D int32 tensor")
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     delta = torch.empty((H, total), device=q.device, dtype=torch.float32)
-    st = lib().fa_varlen_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(cu_seqlens),
-                             cu_seqlens.numel() - 1, int(max_seqlen), total, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(delta),
-                             H, D, float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
+    _same_device(q, k, v, out, dout, lse, cu_seqlens)
+    with torch.cuda.device(q.device):
+        st = lib().fa_varlen_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(cu_seqlens),
+                                 cu_seqlens.numel() - 1, int(max_seqlen), total, _ptr(dq), _ptr(dk), _ptr(dv),
+                                 _ptr(delta), H, D, float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q),
+                                 _stream(stream))
     _check(st, "fa_varlen_bwd")
     return dq, dk, dv
 
@@ -179,14 +209,23 @@ def fa_bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch
                    lse: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor,
                    scale: Optional[float] = None, causal: bool = False, stream=None) -> None:
     """fa_bwd into caller-given dq, dk, dv with the library's fixed delta buffer (no
-    allocation by the library; concurrent calls share that buffer and must be serialised)."""
+    allocation by the library; concurrent calls share that buffer and must be serialised).
+    Every tensor is checked here, because the library takes B, H, S, D from q alone."""
+    if q.dim() != 4 or any(t.shape != q.shape or t.dtype != q.dtype for t in (k, v, out, dout)):
+        raise ValueError("q, k, v, out, dout must share one (B, S, H, D) shape and dtype")
+    B, S, H, D = q.shape
+    _shape("lse", lse, (B, H, S), torch.float32)
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _shape(n, t, q.shape, q.dtype)
     for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse), ("dq", dq),
                  ("dk", dk), ("dv", dv)):
         _cuda_contig(n, t)
-    B, S, H, D = q.shape
-    st = lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
-                              _ptr(dv), B, H, S, D, float(scale) if scale else 0.0, int(bool(causal)),
-                              _dtype_code(q), _stream(stream))
+    _same_device(q, k, v, out, dout, lse, dq, dk, dv)
+    # the fixed buffer is looked up on the current device: make it q's
+    with torch.cuda.device(q.device):
+        st = lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq),
+                                  _ptr(dk), _ptr(dv), B, H, S, D, float(scale) if scale else 0.0, int(bool(causal)),
+                                  _dtype_code(q), _stream(stream))
     _check(st, "fa_bwd_noalloc")
 
 
@@ -215,14 +254,16 @@ def fa_fwd_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, 
         raise ValueError("block_table must be an int32 (B, max_blocks_per_seq) tensor")
     if out is None:
         out = torch.empty_like(q)
-    _cuda_contig("out", out)
+    _like("out", out, q.shape, q.dtype)
     if return_lse and lse is None:
         lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
     if lse is not None:
-        _cuda_contig("lse", lse)
-    st = lib().fa_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
-                            page_size, num_pages, _ptr(out), _ptr(lse), B, H, S, D,
-                            float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
+        _like("lse", lse, (B, H, S), torch.float32)
+    _same_device(q, k_cache, v_cache, block_table, out, lse)
+    with torch.cuda.device(q.device):
+        st = lib().fa_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
+                                page_size, num_pages, _ptr(out), _ptr(lse), B, H, S, D,
+                                float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
     _check(st, "fa_fwd_paged")
     return out, lse
 
@@ -241,14 +282,16 @@ def fa_varlen_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens:
     total, H, D = q.shape
     if out is None:
         out = torch.empty_like(q)
-    _cuda_contig("out", out)
+    _like("out", out, q.shape, q.dtype)
     if return_lse and lse is None:
         lse = torch.empty((H, total), device=q.device, dtype=torch.float32)
     if lse is not None:
-        _cuda_contig("lse", lse)
-    st = lib().fa_varlen_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
-                             int(max_seqlen), total, _ptr(out), _ptr(lse), H, D,
-                             float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
+        _like("lse", lse, (H, total), torch.float32)
+    _same_device(q, k, v, cu_seqlens, out, lse)
+    with torch.cuda.device(q.device):
+        st = lib().fa_varlen_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                                 int(max_seqlen), total, _ptr(out), _ptr(lse), H, D,
+                                 float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
     _check(st, "fa_varlen_fwd")
     return out, lse
 
@@ -270,15 +313,17 @@ def fa_varlen_fwd_padded(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, indi
     total = indices.numel()
     if out is None:
         out = torch.empty_like(q)
-    _cuda_contig("out", out)
+    _like("out", out, q.shape, q.dtype)
     if return_lse and lse is None:
         lse = torch.empty((H, total), device=q.device, dtype=torch.float32)
     if lse is not None:
-        _cuda_contig("lse", lse)
-    st = lib().fa_varlen_fwd_padded(_ptr(q), _ptr(k), _ptr(v), _ptr(indices), _ptr(cu_seqlens),
-                                    cu_seqlens.numel() - 1, int(max_seqlen), total, padded_rows, _ptr(out), _ptr(lse),
-                                    H, D, float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q),
-                                    _stream(stream))
+        _like("lse", lse, (H, total), torch.float32)
+    _same_device(q, k, v, indices, cu_seqlens, out, lse)
+    with torch.cuda.device(q.device):
+        st = lib().fa_varlen_fwd_padded(_ptr(q), _ptr(k), _ptr(v), _ptr(indices), _ptr(cu_seqlens),
+                                        cu_seqlens.numel() - 1, int(max_seqlen), total, padded_rows, _ptr(out),
+                                        _ptr(lse), H, D, float(scale) if scale else 0.0, int(bool(causal)),
+                                        _dtype_code(q), _stream(stream))
     _check(st, "fa_varlen_fwd_padded")
     return out, lse
 
@@ -296,8 +341,10 @@ def fa_unpad(x: torch.Tensor, indices: torch.Tensor, out: Optional[torch.Tensor]
     nnz = indices.numel()
     if out is None:
         out = torch.empty((nnz, H, D), device=x.device, dtype=x.dtype)
-    _cuda_contig("out", out)
-    st = lib().fa_unpad(_ptr(x), _ptr(indices), nnz, total_rows, row_bytes, _ptr(out), _stream(stream))
+    _like("out", out, (nnz, H, D), x.dtype)
+    _same_device(x, indices, out)
+    with torch.cuda.device(x.device):
+        st = lib().fa_unpad(_ptr(x), _ptr(indices), nnz, total_rows, row_bytes, _ptr(out), _stream(stream))
     _check(st, "fa_unpad")
     return out
 
@@ -316,9 +363,12 @@ def fa_unpad_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, indices: tor
     if outs is None:
         outs = tuple(torch.empty((nnz, H, D), device=q.device, dtype=q.dtype) for _ in range(3))
     for i, o in enumerate(outs):
-        _cuda_contig(f"outs[{i}]", o)
-    st = lib().fa_unpad_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(indices), nnz, q.numel() // (H * D),
-                            H * D * q.element_size(), _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), _stream(stream))
+        _like(f"outs[{i}]", o, (nnz, H, D), q.dtype)
+    _same_device(q, k, v, indices, *outs)
+    with torch.cuda.device(q.device):
+        st = lib().fa_unpad_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(indices), nnz, q.numel() // (H * D),
+                                H * D * q.element_size(), _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]),
+                                _stream(stream))
     _check(st, "fa_unpad_qkv")
     return outs
 
@@ -331,19 +381,29 @@ def fa_pad(x: torch.Tensor, indices: torch.Tensor, batch: int, total_len: int,
     if indices.dtype != torch.int64:
         raise ValueError("indices must be int64")
     nnz, H, D = x.shape
+    if indices.numel() != nnz:
+        raise ValueError("indices must hold one entry per row of x")
     if out is None:
         out = torch.empty((batch, total_len, H, D), device=x.device, dtype=x.dtype)
-    _cuda_contig("out", out)
-    st = lib().fa_pad(_ptr(x), _ptr(indices), nnz, batch * total_len, H * D * x.element_size(), _ptr(out),
-                      _stream(stream))
+    _like("out", out, (batch, total_len, H, D), x.dtype)
+    _same_device(x, indices, out)
+    with torch.cuda.device(x.device):
+        st = lib().fa_pad(_ptr(x), _ptr(indices), nnz, batch * total_len, H * D * x.element_size(), _ptr(out),
+                          _stream(stream))
     _check(st, "fa_pad")
     return out
 
 
-def fa_device_status() -> Tuple[int, int]:
-    """(status, where) recorded by kernels since the last call (synchronises the device)."""
+def fa_device_status(stream=None, device=None) -> Tuple[int, int]:
+    """(status, where) recorded by kernels on the device since the last call. Waits for `stream`
+    only (default: the current stream of `device`, default the current device)."""
     where = ctypes.c_int(0)
-    st = lib().fa_device_status(ctypes.byref(where))
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if isinstance(stream, torch.cuda.Stream):
+        dev = stream.device
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream(dev).cuda_stream if stream is None else _stream(stream)
+        st = lib().fa_device_status(ctypes.byref(where), s)
     return st, where.value
 
 

@@ -1,6 +1,7 @@
 // fa_api.cu -- the C ABI declared in include/fa.h: argument validation, TMA tensor-map
 // encoding and kernel dispatch. No entry point allocates, synchronises (except
-// fa_device_status, whose job it is) or touches host copies of tensor data.
+// fa_device_status, which waits for the caller's stream) or touches host copies of tensor
+// data.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -50,6 +51,23 @@ uint64_t wait_limit_ns() {
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Streaming multiprocessors of the current device (looked up once per device).
+int sm_count() {
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return -1;
+    if (dev >= 64) {
+        int n = 0;
+        return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? n : -1;
+    }
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return -1;
+        cached[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
 
 bool head_dim_ok(int D) { return D == 32 || D == 64 || D == 128 || D == 256; }
 
@@ -119,15 +137,24 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     p.num_pages = paging ? paging->num_pages : 0;
     const int rows = fa::fwd_tile_rows();
     dim3 grid;
+    p.batch = num_seqs;
+    p.npairs = 0;
+    p.num_items = 0;
     if (cu_seqlens) {
         // packed: one CTA per tiles_per_cta x 128 consecutive tokens of the packed tensor
         const int64_t span = static_cast<int64_t>(rows) * fa::fwd_tiles_per_cta(D);
         grid = dim3(static_cast<unsigned>(H), static_cast<unsigned>((N + span - 1) / span), 1);
     } else {
+        // dense: persistent, one CTA per SM (at most one per work item)
         const int qtiles = (seqlen + rows - 1) / rows;
         const int per_cta = fa::fwd_tiles_per_cta(D);
-        grid = dim3(static_cast<unsigned>(H), static_cast<unsigned>((qtiles + per_cta - 1) / per_cta),
-                    static_cast<unsigned>(num_seqs));
+        p.npairs = (qtiles + per_cta - 1) / per_cta;
+        const int64_t items = static_cast<int64_t>(num_seqs) * H * p.npairs;
+        if (items > INT32_MAX) return FA_ERR_SHAPE;
+        p.num_items = static_cast<int>(items);
+        const int sms = sm_count();
+        if (sms <= 0) return FA_ERR_CUDA;
+        grid = dim3(static_cast<unsigned>(p.num_items < sms ? p.num_items : sms), 1, 1);
     }
     const cudaError_t e = paging ? fa::launch_fwd_paged(D, bf16, causal != 0, tq, tk, tv, p, grid,
                                                         static_cast<cudaStream_t>(stream))
@@ -216,6 +243,29 @@ bool bwd_aligned(const void *q, const void *k, const void *v, const void *out, c
                  const void *dq, const void *dk, const void *dv, const float *delta) {
     return aligned(q, 16) && aligned(k, 16) && aligned(v, 16) && aligned(out, 16) && aligned(dout, 16) &&
            aligned(dq, 16) && aligned(dk, 16) && aligned(dv, 16) && aligned(lse, 4) && aligned(delta, 4);
+}
+
+// The error words of the kernel families (one per compilation unit), read and cleared in one
+// launch on the caller's stream; the first nonzero code wins.
+constexpr int kErrorWords = 4;
+struct ErrorWords {
+    int *code[kErrorWords];
+    int *where[kErrorWords];
+};
+
+__device__ int g_status_out[2];
+
+__global__ void status_collect_kernel(ErrorWords w) {
+    int code = 0, where = 0;
+    for (int i = 0; i < kErrorWords; ++i) {
+        const int c = atomicExch(w.code[i], 0), wh = atomicExch(w.where[i], 0);
+        if (c != 0 && code == 0) {
+            code = c;
+            where = wh;
+        }
+    }
+    g_status_out[0] = code;
+    g_status_out[1] = where;
 }
 
 }  // namespace
@@ -342,21 +392,24 @@ fa_status fa_pad(const void *x, const int64_t *indices, int64_t nnz, int64_t tot
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-fa_status fa_device_status(int *where) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
-    // every kernel family keeps its own word; all are read (and so cleared), the first set wins
-    int code[4] = {0, 0, 0, 0}, w[4] = {0, 0, 0, 0};
-    if (fa::fwd_take_device_error(&code[0], &w[0]) != cudaSuccess) return FA_ERR_CUDA;
-    if (fa::fwd_paged_take_device_error(&code[1], &w[1]) != cudaSuccess) return FA_ERR_CUDA;
-    if (fa::bwd_take_device_error(&code[2], &w[2]) != cudaSuccess) return FA_ERR_CUDA;
-    if (fa::pad_take_device_error(&code[3], &w[3]) != cudaSuccess) return FA_ERR_CUDA;
-    for (int i = 0; i < 4; ++i)
-        if (code[i]) {
-            if (where) *where = w[i];
-            return static_cast<fa_status>(code[i]);
-        }
-    if (where) *where = 0;
-    return FA_OK;
+fa_status fa_device_status(int *where, void *stream) {
+    // every kernel family keeps its own word; one kernel on the caller's stream reads and
+    // clears them all, one copy brings the result back, and only that stream is waited for
+    ErrorWords w;
+    if (fa::fwd_error_addrs(&w.code[0], &w.where[0]) != cudaSuccess ||
+        fa::fwd_paged_error_addrs(&w.code[1], &w.where[1]) != cudaSuccess ||
+        fa::bwd_error_addrs(&w.code[2], &w.where[2]) != cudaSuccess ||
+        fa::pad_error_addrs(&w.code[3], &w.where[3]) != cudaSuccess)
+        return FA_ERR_CUDA;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    status_collect_kernel<<<1, 1, 0, st>>>(w);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    int res[2] = {0, 0};
+    if (cudaMemcpyFromSymbolAsync(res, g_status_out, sizeof(res), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return FA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return FA_ERR_CUDA;
+    if (where) *where = res[1];
+    return static_cast<fa_status>(res[0]);
 }
 
 fa_status fa_selftest_bounded_wait(uint64_t limit_ns, void *stream) {

@@ -672,6 +672,6 @@ cudaError_t launch_bwd(int D, bool bf16, bool causal, const CUtensorMap &tq, con
     }
 }
 
-cudaError_t bwd_take_device_error(int *code, int *where) { return take_device_error(code, where); }
+cudaError_t bwd_error_addrs(int **code, int **where) { return device_error_addrs(code, where); }
 
 }  // namespace fa

@@ -1,6 +1,6 @@
 // fa_fwd.cu -- the attention forward over contiguous K/V (dense and packed sequences, and the
-// fused packed path): instantiations of the kernel in fa_fwd_kernel.cuh, the bounded-wait
-// self-test, and the host-side tile geometry shared with fa_api.cu.
+// fused packed path): instantiations of the kernel in fa_fwd_kernel.cuh (dense persistent and
+// packed), the bounded-wait self-test, and the host-side tile geometry shared with fa_api.cu.
 #include "fa_fwd_kernel.cuh"
 
 namespace fa {
@@ -21,8 +21,11 @@ __global__ void fa_selftest_wait_kernel(uint64_t limit_ns) {
 template <int D, bool BF16>
 static cudaError_t launch_c(bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
                             const CUtensorMap &tv, const FwdParams &p, dim3 grid, cudaStream_t st) {
-    return causal ? launch_t<D, BF16, true, false>(tq, tk, tv, p, grid, st)
-                  : launch_t<D, BF16, false, false>(tq, tk, tv, p, grid, st);
+    if (p.cu_seqlens)
+        return causal ? launch_t<D, BF16, true, false, true>(tq, tk, tv, p, grid, st)
+                      : launch_t<D, BF16, false, false, true>(tq, tk, tv, p, grid, st);
+    return causal ? launch_t<D, BF16, true, false, false>(tq, tk, tv, p, grid, st)
+                  : launch_t<D, BF16, false, false, false>(tq, tk, tv, p, grid, st);
 }
 
 template <int D>
@@ -60,6 +63,6 @@ cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t fwd_take_device_error(int *code, int *where) { return take_device_error(code, where); }
+cudaError_t fwd_error_addrs(int **code, int **where) { return device_error_addrs(code, where); }
 
 }  // namespace fa

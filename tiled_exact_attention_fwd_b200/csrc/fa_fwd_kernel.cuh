@@ -34,15 +34,16 @@
 //               warps 10 and 11 copy V with cp.async.
 //   epilogue    each softmax warp stages its 32 O rows in its tile's Q buffer (free once
 //               the tile's MMAs are done) and writes them out as whole rows.
-//   warp 9      allocates TMEM; one thread issues every tcgen05.mma:
+//   warp 9      allocates TMEM and issues every tcgen05.mma (the whole warp runs the loop and
+//               waits; elect.sync picks the lane that issues each MMA and commit):
 //                 S_t = Q_t K_j^T   (A = Q_t, B = K_j, both K-major in SMEM, 128B swizzle)
 //                 O_t += P_t V_j    (A = P_t read from TMEM, B = V_j MN-major in SMEM)
 //               in the ping-pong order QK_A0, QK_B0, PV_A0, QK_A1, PV_B0, QK_B1, ..., so the
 //               tensor core works on one tile while the other tile's softmax runs. With a
 //               single tile the two S buffers are used alternately by that tile instead
-//               (order QK_0, QK_1, PV_0, QK_2, PV_1, ...). A single issuing thread is slower
-//               than the tensor core unless each MMA costs it a few instructions, so the
-//               operand descriptors are kept as 32-bit words and a k-step adds its offset.
+//               (order QK_0, QK_1, PV_0, QK_2, PV_1, ...). The issuing lane is slower than the
+//               tensor core unless each MMA costs it a few instructions, so the operand
+//               descriptors are kept as 32-bit words and a k-step adds its offset.
 //
 // Every pipeline wait is bounded: after `timeout_ns` the waiting thread records
 // FA_ERR_TIMEOUT in a device word, raises a CTA-wide abort flag, and all roles drain
@@ -96,14 +97,19 @@ struct Cfg {
     // A full last warpgroup (two idle warps) so that per-warpgroup register limits apply.
     static constexpr int NUM_THREADS = 32 * (NUM_SOFTMAX_WARPS + 4);
     // Register split (two query tiles): 384 threads launch with LAUNCH_REGS each; the
-    // producer/MMA warpgroup drops to REGS_LOW and the softmax warpgroups rise to REGS_HIGH.
+    // producer/MMA warpgroup drops to regs_low and the softmax warpgroups rise to regs_high.
+    // The persistent (dense) kernel keeps more state in its producer and MMA loops than the
+    // packed one, so it moves 8 registers per softmax thread over to them.
     // The host refuses to launch unless the pool covers the split (it would otherwise wait).
     static constexpr int LAUNCH_REGS = 168;
-    static constexpr int REGS_LOW = 56;
-    static constexpr int REGS_HIGH = 224;
+    static constexpr int regs_low(bool packed) { return packed ? 56 : 72; }
+    static constexpr int regs_high(bool packed) { return packed ? 224 : 216; }
 
     static constexpr bool SPLIT_REGS = (MAXQ == 2);
-    static_assert(!SPLIT_REGS || 128 * REGS_LOW + 256 * REGS_HIGH <= NUM_THREADS * LAUNCH_REGS, "register split");
+    static_assert(!SPLIT_REGS || 128 * regs_low(true) + 256 * regs_high(true) <= NUM_THREADS * LAUNCH_REGS,
+                  "register split");
+    static_assert(!SPLIT_REGS || 128 * regs_low(false) + 256 * regs_high(false) <= NUM_THREADS * LAUNCH_REGS,
+                  "register split");
     // Column pairs (out of every 4) whose exp2 runs on the FMA pipe instead of MUFU.
     static constexpr int EMU_PAIRS_OF_4 = 0;
     // shared memory map (offsets from a 1024-byte aligned base)
@@ -114,8 +120,8 @@ struct Cfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = MAXQ * Q_BYTES;
     static constexpr int OFF_BAR = OFF_KV + NS * UNIT_BYTES;
-    // q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], drain, s_free[2], tail
-    static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1 + 2 + 1;
+    // q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], drain, s_free[2], tail, q_free[2]
+    static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1 + 2 + 1 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // TMEM address, abort flag
     static constexpr int USED = OFF_MISC + 16;
     // More than half of the SM's shared memory, so exactly one CTA (and one 512-column
@@ -244,60 +250,163 @@ __device__ __forceinline__ float softmax_row_to_regs(const uint32_t *sr, float c
     return lo + hi;
 }
 
-// Shared state of one CTA: shared-memory buffers, barriers, TMEM base and the plan.
+// Shared state of one CTA: shared-memory buffers, barriers, TMEM base, the current work item,
+// and running counts that carry every barrier's phase from one work item to the next (a CTA
+// of the dense path runs several items one after another).
 template <int D>
 struct Cta {
     using C = Cfg<D>;
     uint8_t *sQ, *sKV;
-    uint64_t *q_full, *kv_full, *kv_empty, *s_full, *p_full, *pv_done, *drain, *s_free;
-    uint64_t *tail;  // paged K/V: the one V part that straddles the sequence end lands here first
+    uint64_t *q_full, *kv_full, *kv_empty, *s_full, *p_full, *pv_done, *drain, *s_free, *q_free;
+    uint64_t *tail;  // paged K/V: the V part that straddles a sequence end lands here first
     volatile int *abort_flag;
     uint32_t tmem;
     uint64_t lim;
-    // Tile A visits key tiles [0, nA), tile B [jB0, nB) (nB = 0 when B is absent); key tile j
-    // covers tokens kvbase + [j*BN, (j+1)*BN). In dense sequences jB0 = 0; in packed ones
-    // B may begin a later sequence. Always jB0 <= nA <= nB, so the two ranges leave no gap.
+    bool dec;     // separate P buffers (Cfg::DECOUPLED)
+    bool single;  // one query tile per CTA (Cfg::MAXQ == 1): its S alternates between two buffers
+    bool fused;   // Q/K/V tiles written by threads (cp.async), not TMA: fence before the MMA reads them
+    // The current work item: query tiles A (and B) of head h; their rows are tokens qbase + t*128
+    // + r, keys are addressed from token kvbase. Dense: batch entry b, rows from position q0 of
+    // the sequence that starts at token seq_start. Tile A visits key tiles [0, nA), tile B
+    // [jB0, nB) (nB = jB0 = 0 when B is absent); key tile j covers tokens kvbase + [j*BN,
+    // (j+1)*BN). In dense sequences jB0 = 0; in packed ones B may begin a later sequence. Always
+    // jB0 <= nA <= nB when B is present, so the two ranges leave no gap.
+    int h, b, q0, seq_start, seqlen, qbase, kvbase;
     int nA, nB, jB0;
+    bool two;  // tile B present
+    // Items done so far: K/V ring parts loaded (u0), key steps of tile t (g0(t)), Q_t loads (nq(t)).
+    // Scalars, not arrays: an array indexed by the runtime tile index would put the whole
+    // struct in local memory.
+    int u0, g0a, g0b, nqa, nqb;
+    __device__ __forceinline__ int g0(int t) const { return t ? g0b : g0a; }
+    __device__ __forceinline__ int nq(int t) const { return t ? nqb : nqa; }
     __device__ __forceinline__ int j0(int t) const { return t ? jB0 : 0; }
+    __device__ __forceinline__ int steps(int t) const { return t ? nB - jB0 : nA; }
     __device__ __forceinline__ bool uses(int t, int j) const { return t ? (j >= jB0 && j < nB) : (j < nA); }
-    bool two;      // two query tiles (ping-pong) or one (S double-buffered)
-    bool dec;      // two tiles with separate P buffers (Cfg::DECOUPLED)
-    bool fused;    // Q/K/V tiles written by threads (cp.async), not TMA: fence before the MMA reads them
-    // S/P buffer and barrier phase used by tile t at key step j
-    __device__ __forceinline__ int buf(int t, int j) const { return two ? t : (j & 1); }
-    __device__ __forceinline__ uint32_t sphase(int j) const { return two ? (j & 1) : ((j >> 1) & 1); }
+    __device__ __forceinline__ int loads() const { return 2 * max(nA, nB) * C::UNITS; }  // ring parts of the item
+    // S/P buffer of tile t at its running key step gs, and that buffer's barrier phase
+    __device__ __forceinline__ int buf(int t, int gs) const { return single ? (gs & 1) : t; }
+    __device__ __forceinline__ uint32_t sphase(int gs) const { return single ? ((gs >> 1) & 1) : (gs & 1); }
+    __device__ __forceinline__ void advance() {
+        u0 += loads();
+        g0a += nA;
+        g0b += nB - jB0;
+        nqa += 1;
+        nqb += two ? 1 : 0;
+    }
 };
 
-// One MMA step of the issuing thread. Returns false when a wait gave up.
+// The dense work items: (batch entry, head, group of MAXQ query tiles), B*H*npairs in all. Causal
+// items are ordered longest first (query-tile group descending); otherwise the groups of one
+// (batch entry, head) are consecutive, so CTAs that run at the same time share its K/V in L2.
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void set_dense_item(Cta<D> &c, const FwdParams &p, int w) {
+    using C = Cfg<D>;
+    const int bh_count = p.batch * p.H;
+    int pair, bh;
+    if (CAUSAL) {
+        pair = p.npairs - 1 - w / bh_count;
+        bh = w % bh_count;
+    } else {
+        pair = w % p.npairs;
+        bh = w / p.npairs;
+    }
+    c.b = bh / p.H;
+    c.h = bh % p.H;
+    c.seqlen = p.seqlen;
+    c.seq_start = c.b * p.seqlen;
+    c.q0 = pair * C::MAXQ * C::BM;
+    c.two = (C::MAXQ == 2) && (c.q0 + C::BM < p.seqlen);
+    c.qbase = c.seq_start + c.q0;
+    c.kvbase = c.seq_start;
+    const int end_a = CAUSAL ? min(p.seqlen, c.q0 + C::BM) : p.seqlen;
+    const int end_b = CAUSAL ? min(p.seqlen, c.q0 + 2 * C::BM) : p.seqlen;
+    c.nA = (end_a + C::BN - 1) / C::BN;
+    c.nB = c.two ? (end_b + C::BN - 1) / C::BN : 0;
+    c.jB0 = 0;
+}
+
+// Work item of round r for CTA `cta` of G: a snake over the item order (forward in even rounds,
+// backward in odd ones), so that with longest-first items every CTA gets a similar total.
+__device__ __forceinline__ int item_of_round(int r, int G, int cta) { return r * G + ((r & 1) ? G - 1 - cta : cta); }
+
+// Head, batch entry, first query position and first query token of this CTA's item at round r
+// (which must exist), derived afresh: packed inputs from the block index, dense ones as
+// set_dense_item does. Keeps these out of the registers that live through an item's key steps.
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void item_coords(const FwdParams &p, int r, bool persistent, int &h, int &b, int &q0,
+                                            int &qbase) {
+    using C = Cfg<D>;
+    if (!persistent) {
+        h = blockIdx.x;
+        b = 0;
+        q0 = 0;
+        qbase = blockIdx.y * C::MAXQ * C::BM;
+        return;
+    }
+    const int w = item_of_round(r, gridDim.x, blockIdx.x);
+    const int bh_count = p.batch * p.H;
+    const int pair = CAUSAL ? p.npairs - 1 - w / bh_count : w % p.npairs;
+    const int bh = CAUSAL ? w % bh_count : w / p.npairs;
+    b = bh / p.H;
+    h = bh % p.H;
+    q0 = pair * C::MAXQ * C::BM;
+    qbase = b * p.seqlen + q0;
+}
+
+// Moves to this CTA's next work item at round r or later (r is advanced past rounds without
+// one); false once there is none. Packed inputs: the one item set up front, at round 0. Called
+// again with the same r it sets the same item.
+template <int D, bool CAUSAL>
+__device__ __forceinline__ bool next_item(Cta<D> &c, const FwdParams &p, int &r, bool persistent) {
+    if (!persistent) return r == 0;
+    const int G = gridDim.x, cta = blockIdx.x;
+    for (;; ++r) {
+        if (r * G >= p.num_items) return false;
+        const int w = item_of_round(r, G, cta);
+        if (w < p.num_items) {
+            set_dense_item<D, CAUSAL>(c, p, w);
+            return true;
+        }
+    }
+}
+
+// S_t = Q_t K_j^T for key tile j (tile-local step jj = j - j0(t)); after the tile's last QK of
+// the item, q_free[t] fires once the MMAs reading Q_t are done. Returns false when a wait gave up.
 template <int D, bool BF16>
-// S_t = Q_t K_j^T for key tile j (tile-local step jj = j - j0(t)).
 __device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first_use, bool last_use) {
     using C = Cfg<D>;
     constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
     constexpr uint32_t idesc = idesc_f16(BM, BN, BF16, false);
     const int jj = j - c.j0(t);
+    const int gs = c.g0(t) + jj;  // running key step of tile t
     if (jj == 0) {
-        if (!wait_bounded(&c.q_full[t], 0, c.abort_flag, c.lim, 200 + t)) return false;
+        if (!__all_sync(0xffffffffu, wait_bounded(&c.q_full[t], c.nq(t) & 1, c.abort_flag, c.lim, 200 + t)))
+            return false;
         tc_fence_after_sync();
         if (c.fused) fence_proxy_async_smem();
-    } else if (c.dec) {
+    }
+    if (c.dec && gs > 0) {
         // S_t is overwritten: the softmax warps must have read the previous S_t
-        if (!wait_bounded(&c.s_free[t], (jj - 1) & 1, c.abort_flag, c.lim, 240 + t)) return false;
+        if (!__all_sync(0xffffffffu, wait_bounded(&c.s_free[t], (gs - 1) & 1, c.abort_flag, c.lim, 240 + t)))
+            return false;
         tc_fence_after_sync();
     }
     constexpr int UK = D / 16 / C::UNITS;  // k-steps per K part
     // Operand descriptors as 32-bit words: the low word of each tile base, to which a k-step
     // adds its byte offset / 16, and the high word shared by Q and K (one add per operand
-    // and k-step keeps the single issuing thread's work per MMA short).
+    // and k-step keeps the issuing lane's work per MMA short).
     constexpr uint32_t dhi = smem_desc_hi(8 * SW, C::LAYOUT);
     const uint32_t q_lo = smem_desc_lo(smem_u32(c.sQ + t * C::Q_BYTES), 16);
-    const int b = c.buf(t, jj);
+    const int b = c.buf(t, gs);
     const uint32_t d_tmem = c.tmem + b * BN;
 #pragma unroll
     for (int u = 0; u < C::UNITS; ++u) {
-        const int U = 2 * j * C::UNITS + u, stage = U % NS;  // ring part holding K_j part u
+        const int U = c.u0 + 2 * j * C::UNITS + u, stage = U % NS;  // ring part holding K_j part u
         if (first_use) {
-            if (!wait_bounded(&c.kv_full[stage], (U / NS) & 1, c.abort_flag, c.lim, 220 + stage)) return false;
+            if (!__all_sync(0xffffffffu,
+                            wait_bounded(&c.kv_full[stage], (U / NS) & 1, c.abort_flag, c.lim, 220 + stage)))
+                return false;
             tc_fence_after_sync();
             if (c.fused) fence_proxy_async_smem();
         }
@@ -307,28 +416,31 @@ __device__ __forceinline__ bool mma_qk(const Cta<D> &c, int t, int j, bool first
             const int k = u * UK + kk;
             const uint32_t blk = (k * 32) / SW, off = (k * 32) % SW;
             const uint32_t lb = blk - u * C::KBLK_PER_UNIT;  // column block inside the part
-            umma_ss_w(d_tmem, q_lo + ((blk * BM * SW + off) >> 4), k_lo + ((lb * BN * SW + off) >> 4), dhi, idesc,
-                      k > 0 ? 1u : 0u);
+            umma_ss_elect(d_tmem, q_lo + ((blk * BM * SW + off) >> 4), k_lo + ((lb * BN * SW + off) >> 4), dhi, idesc,
+                          k > 0 ? 1u : 0u);
         }
         if (u + 1 < C::UNITS) {
-            if (last_use) umma_commit(&c.kv_empty[stage]);  // release this part early
+            if (last_use) umma_commit_elect(&c.kv_empty[stage]);  // release this part early
         } else {
-            umma_commit(&c.s_full[b]);  // the softmax waits on S first
-            if (last_use) umma_commit(&c.kv_empty[stage]);
+            umma_commit_elect(&c.s_full[b]);  // the softmax waits on S first
+            if (last_use) umma_commit_elect(&c.kv_empty[stage]);
         }
     }
+    if (jj == c.steps(t) - 1) umma_commit_elect(&c.q_free[t]);  // Q_t may be reloaded for the next item
     return true;
 }
 
-template <int D, bool BF16>
 // O_t += P_t V_j for key tile j (tile-local step jj = j - j0(t)).
+template <int D, bool BF16>
 __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first_use, bool last_use) {
     using C = Cfg<D>;
     constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
     constexpr uint32_t idesc = idesc_f16(BM, D, BF16, true);
     const int jj = j - c.j0(t);
-    const int b = c.buf(t, jj);
-    if (!wait_bounded(&c.p_full[b], c.sphase(jj), c.abort_flag, c.lim, 210 + t)) return false;
+    const int gs = c.g0(t) + jj;
+    const int b = c.buf(t, gs);
+    if (!__all_sync(0xffffffffu, wait_bounded(&c.p_full[b], c.sphase(gs), c.abort_flag, c.lim, 210 + t)))
+        return false;
     tc_fence_after_sync();
     constexpr int UV = BN / 16 / C::UNITS;  // k-steps per V part
     constexpr uint32_t dhi = smem_desc_hi(8 * SW, C::LAYOUT);  // high descriptor word of V
@@ -336,9 +448,11 @@ __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first
     const uint32_t o_tmem = c.tmem + C::O_COL + t * D;
 #pragma unroll
     for (int u = 0; u < C::UNITS; ++u) {
-        const int U = (2 * j + 1) * C::UNITS + u, stage = U % NS;  // ring part holding V_j part u
+        const int U = c.u0 + (2 * j + 1) * C::UNITS + u, stage = U % NS;  // ring part holding V_j part u
         if (first_use) {
-            if (!wait_bounded(&c.kv_full[stage], (U / NS) & 1, c.abort_flag, c.lim, 230 + stage)) return false;
+            if (!__all_sync(0xffffffffu,
+                            wait_bounded(&c.kv_full[stage], (U / NS) & 1, c.abort_flag, c.lim, 230 + stage)))
+                return false;
             tc_fence_after_sync();
             if (c.fused) fence_proxy_async_smem();
         }
@@ -346,13 +460,14 @@ __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first
 #pragma unroll
         for (int kk = 0; kk < UV; ++kk) {
             const int k = u * UV + kk;
-            umma_ts_w(o_tmem, a_tmem + k * 8, v_lo + ((kk * 16 * SW) >> 4), dhi, idesc, (jj > 0 || k > 0) ? 1u : 0u);
+            umma_ts_elect(o_tmem, a_tmem + k * 8, v_lo + ((kk * 16 * SW) >> 4), dhi, idesc,
+                          (jj > 0 || k > 0) ? 1u : 0u);
         }
         if (u + 1 < C::UNITS) {
-            if (last_use) umma_commit(&c.kv_empty[stage]);
+            if (last_use) umma_commit_elect(&c.kv_empty[stage]);
         } else {
-            umma_commit(&c.pv_done[t]);
-            if (last_use) umma_commit(&c.kv_empty[stage]);
+            umma_commit_elect(&c.pv_done[t]);
+            if (last_use) umma_commit_elect(&c.kv_empty[stage]);
         }
     }
     return true;
@@ -417,39 +532,43 @@ __device__ __forceinline__ void fetch_group(uint8_t *tile, int rows, int g, int6
 }
 
 // PAGED: K/V read through p.block_table (a separate instantiation, so the producer code of
-// the contiguous path stays as small as its register budget wants).
-template <int D, bool BF16, bool CAUSAL, bool PAGED>
+// the contiguous path stays as small as its register budget wants). PACKED: packed sequences
+// (cu_seqlens); a separate instantiation too, so that neither path's state takes registers in
+// the other's loops.
+//
+// Dense inputs run persistently: the grid has one CTA per SM (at most one per work item), and
+// each CTA takes its work items in rounds (item_of_round). Every role loops over the same items;
+// the producer loads an item's Q tiles as soon as the previous item's QKs on them are done, so
+// the next item's loads and first QKs overlap the current item's last steps and epilogue.
+// Packed inputs launch one CTA per 256 consecutive tokens (one item per CTA).
+template <int D, bool BF16, bool CAUSAL, bool PAGED, bool PACKED>
 __global__ void __launch_bounds__(Cfg<D>::NUM_THREADS, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     using C = Cfg<D>;
     constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
 
-    const int h = blockIdx.x;
-    // Rows of the CTA are tokens qbase + t*128 + r; keys are addressed from token kvbase.
-    //  dense : blockIdx.z is the batch entry; the CTA owns query tiles `pair` (two of them
-    //          when MAXQ = 2) of that sequence, longest (causal) tiles launched first.
-    //  packed: the CTA owns the 128 consecutive packed tokens of tile blockIdx.y, whatever
-    //          sequences they belong to; its keys are the union of those sequences' keys
-    //          (the device walks cu_seqlens), and each row is masked to its own sequence.
-    const bool packed = p.cu_seqlens != nullptr;
-    int seq_start = 0, seqlen = 0, q0 = 0, qbase, kvbase, kv_end_A, kv_end_B = 0, kv_start_B = 0;
-    bool two = false;
-    if (!packed) {
-        const int pair = gridDim.y - 1 - blockIdx.y;
-        seq_start = blockIdx.z * p.seqlen;
-        seqlen = p.seqlen;
-        q0 = pair * C::MAXQ * BM;
-        if (q0 >= seqlen) return;  // uniform over the CTA, before any barrier exists
-        two = (C::MAXQ == 2) && (q0 + BM < seqlen);
-        qbase = seq_start + q0;
-        kvbase = seq_start;
-        kv_end_A = CAUSAL ? min(seqlen, q0 + BM) : seqlen;
-        if (two) kv_end_B = CAUSAL ? min(seqlen, q0 + 2 * BM) : seqlen;
-    } else {
-        qbase = blockIdx.y * C::MAXQ * BM;
-        if (qbase >= p.total_tokens) return;
-        two = (C::MAXQ == 2) && (qbase + BM < p.total_tokens);
+    static_assert(!(PAGED && PACKED), "paged K/V is for dense queries");
+    constexpr bool packed = PACKED;  // the host launches PACKED exactly when p.cu_seqlens is set
+    constexpr bool persistent = !packed;
+    Cta<D> c;
+    c.dec = C::DECOUPLED;
+    c.single = C::MAXQ == 1;
+    c.u0 = 0;
+    c.g0a = c.g0b = 0;
+    c.nqa = c.nqb = 0;
+    if (packed) {
+        // The CTA owns the 128 * MAXQ consecutive packed tokens of tile blockIdx.y, whatever
+        // sequences they belong to; its keys are the union of those sequences' keys (the device
+        // walks cu_seqlens), and each row is masked to its own sequence.
+        c.h = blockIdx.x;
+        c.b = 0;
+        c.q0 = 0;
+        c.seq_start = 0;
+        c.seqlen = 0;
+        c.qbase = blockIdx.y * C::MAXQ * BM;
+        if (c.qbase >= p.total_tokens) return;  // uniform over the CTA, before any barrier exists
+        c.two = (C::MAXQ == 2) && (c.qbase + BM < p.total_tokens);
         const int ln = threadIdx.x & 31;
         // With fewer than 64 sequences every warp holds all of cu_seqlens (two entries per
         // lane), so the lookups below are ballots and shuffles after one round of loads;
@@ -459,23 +578,22 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             return win.ok ? win.seq(tok, ln) : warp_seq_of_token(p.cu_seqlens, p.num_seqs, tok, ln);
         };
         auto cu_at = [win, &p](int s) { return win.ok ? win.at(s) : p.cu_seqlens[s]; };
-        const int s_first = seq_of(qbase);
-        kvbase = cu_at(s_first);
+        const int s_first = seq_of(c.qbase);
+        c.kvbase = cu_at(s_first);
         // keys of a tile end with its last row's sequence (or the causal limit)
         auto kv_end = [&](int tlast) {
             const int s_last = seq_of(tlast);
-            return (CAUSAL ? min(cu_at(s_last + 1), tlast + 1) : cu_at(s_last + 1)) - kvbase;
+            return (CAUSAL ? min(cu_at(s_last + 1), tlast + 1) : cu_at(s_last + 1)) - c.kvbase;
         };
-        kv_end_A = kv_end(min(qbase + BM, p.total_tokens) - 1);
-        if (two) {
-            kv_end_B = kv_end(min(qbase + 2 * BM, p.total_tokens) - 1);
-            kv_start_B = cu_at(seq_of(qbase + BM)) - kvbase;
+        const int end_a = kv_end(min(c.qbase + BM, p.total_tokens) - 1);
+        c.nA = (end_a + BN - 1) / BN;
+        c.nB = c.jB0 = 0;
+        if (c.two) {
+            const int end_b = kv_end(min(c.qbase + 2 * BM, p.total_tokens) - 1);
+            c.nB = (end_b + BN - 1) / BN;
+            c.jB0 = (cu_at(seq_of(c.qbase + BM)) - c.kvbase) / BN;
         }
     }
-
-    Cta<D> c;
-    c.two = two;
-    c.dec = C::DECOUPLED && c.two;
     // Fused path: stage contents are written by cp.async copies, whose writer cannot fence
     // after they land, so the MMA thread fences the async proxy after its waits. (The paged
     // path's zeroed page tails are fenced by the writing thread itself before it releases
@@ -484,10 +602,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // the V parts go by cp.async copies beside the TMA's K parts (the same fence applies).
     const bool copy_pages = PAGED && p.page_size < 64;
     c.fused = p.gather != nullptr || copy_pages;
-    c.nA = (kv_end_A + BN - 1) / BN;
-    c.nB = c.two ? (kv_end_B + BN - 1) / BN : 0;
-    c.jB0 = c.two ? kv_start_B / BN : 0;
-    const int n_all = max(c.nA, c.nB);  // key tiles this CTA loads
+    // Separate P buffers and no copy warps: the MMAs are issued by two warps, warp 9 the
+    // QKs and warp 10 the PVs, so that a tile's next S is computed as soon as its S buffer has
+    // been read, never held up behind the other tile's PV (which waits for that tile's P).
+    const bool split_issue = c.dec && !c.fused;
+    // Every role runs `for (int rd = 0; next_item(...); ++rd) { ...; c.advance(); }` over this
+    // CTA's work items (dense: the rounds of item_of_round; packed: the one item set above),
+    // leaving the loop early when a wait gives up.
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -504,6 +625,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     c.drain = c.pv_done + 2;
     c.s_free = c.drain + 1;
     c.tail = c.s_free + 2;
+    c.q_free = c.tail + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     c.abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     c.lim = p.timeout_ns;
@@ -514,7 +636,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // Fused packed path: the copy warps read the padded rows of their groups of the first key
     // part now, so that load overlaps the barrier and TMEM set-up.
     int64_t first_rows[2] = {0, 0};
-    if (p.gather && (warp == C::WARP_TMA || warp > C::WARP_MMA)) fused_group_rows(p, kvbase, BN, pw, lane, first_rows);
+    if (p.gather && (warp == C::WARP_TMA || warp > C::WARP_MMA)) fused_group_rows(p, c.kvbase, BN, pw, lane, first_rows);
 
     if (threadIdx.x == 0) {
         // ring barriers: one arrival (the TMA lane's), or per copy thread: fused packed path 96
@@ -528,12 +650,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_init(&c.p_full[t], 128);
             mbar_init(&c.pv_done[t], 1);
             mbar_init(&c.s_free[t], 4);  // one arrival per softmax warp
+            mbar_init(&c.q_free[t], 1);
         }
         for (int s = 0; s < NS; ++s) {
             mbar_init(&c.kv_full[s], fill_arrivals);
             mbar_init(&c.kv_empty[s], 1);
         }
-        mbar_init(c.drain, 1);
+        mbar_init(c.drain, split_issue ? 2 : 1);  // one commit per issuing warp
         mbar_init(c.tail, 1);
         *c.abort_flag = 0;
         fence_mbar_init();
@@ -553,15 +676,42 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     c.tmem = *tmem_slot;
 
     if (warp >= C::NUM_SOFTMAX_WARPS) {
-        // producer / MMA warpgroup (its two remaining warps idle unless they copy rows)
-        if constexpr (C::SPLIT_REGS) regs_dec<C::REGS_LOW>();
+        // producer / MMA warpgroup (its remaining warps idle unless they copy rows or issue PVs)
+        if constexpr (C::SPLIT_REGS) regs_dec<C::regs_low(PACKED)>();
         if (warp == C::WARP_TMA || (c.fused && warp > C::WARP_MMA)) {
-            // ------------------------------------------------------------ TMA producer
+            // ------------------------------------------------------------ producer
             // (fused packed path and pages under 64 rows: warps 10 and 11 copy rows too)
-            const int nq = c.two ? 2 : 1;
-            const int loads = 2 * n_all * C::UNITS;  // parts of K_0, V_0, K_1, V_1, ...
-            int issued = 0;
-            bool tail_issued = false;
+            int issued = 0;                  // ring parts issued (running count)
+            int q_issued_a = 0, q_issued_b = 0;  // Q_A, Q_B loads issued (running counts)
+            int tail_uses = 0;               // paged: parts that went through `tail` (running count)
+            int tail_pending = -1;           // phase of a `tail` use whose wait was cut short
+            bool bad_page = false;           // reported once, after the loads
+            const uint64_t pol_q = l2_policy_evict_first();
+            const uint64_t pol_kv = l2_policy_evict_last();
+            // Q_t of the current item into its buffer, once the previous item's QKs on it are done.
+            auto load_q = [&](int t) -> bool {
+                if (c.nq(t) > 0 && !wait_bounded(&c.q_free[t], (c.nq(t) - 1) & 1, c.abort_flag, c.lim, 110 + t))
+                    return false;
+                mbar_arrive_expect_tx(&c.q_full[t], C::Q_BYTES);
+#pragma unroll
+                for (int b = 0; b < C::NBLK; ++b)
+                    tma_load_3d(c.sQ + t * C::Q_BYTES + b * BM * SW, &tm_q, &c.q_full[t], b * C::SWE, c.h,
+                                c.qbase + t * BM, pol_q);
+                (t ? q_issued_b : q_issued_a) = c.nq(t) + 1;
+                return true;
+            };
+            // Physical row of key position pos (< seqlen) of the item's batch entry. A page index
+            // outside the pool is reported and replaced by page 0 (the result is then wrong, but
+            // nothing outside the pool is read).
+            auto page_row = [&](int pos) -> int64_t {
+                const int32_t *bt = p.block_table + static_cast<int64_t>(c.b) * p.max_blocks;
+                int pg = __ldg(bt + (pos >> p.page_shift));
+                if (pg < 0 || pg >= p.num_pages) {
+                    bad_page = true;
+                    pg = 0;
+                }
+                return (static_cast<int64_t>(pg) << p.page_shift) + (pos & (p.page_size - 1));
+            };
             if (PAGED && copy_pages) {
                 // Paged K/V in small pages: two engines share the bytes. Warp 8 (lane 0) moves
                 // the query tiles and the K parts by TMA, one box per page chunk (chunks wholly
@@ -571,109 +721,111 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // ring barrier takes 65 arrivals per part: the TMA lane's (with the K bytes, or
                 // a plain arrival on a V part) and one per copy thread (plain on a K part, or
                 // once its V copies have landed).
-                const int32_t *bt = p.block_table + static_cast<int64_t>(blockIdx.z) * p.max_blocks;
-                bool bad_page = false;
-                auto page_row = [&](int pos) {  // physical row of key position pos (< seqlen)
-                    int pg = __ldg(bt + (pos >> p.page_shift));
-                    if (pg < 0 || pg >= p.num_pages) {
-                        bad_page = true;
-                        pg = 0;
-                    }
-                    return (static_cast<int64_t>(pg) << p.page_shift) + (pos & (p.page_size - 1));
-                };
                 if (warp == C::WARP_TMA) {
                     if (lane == 0) {
-                        const uint64_t pol_q = l2_policy_evict_first();
-                        const uint64_t pol_kv = l2_policy_evict_last();
-                        for (int t = 0; t < nq; ++t) {
-                            mbar_arrive_expect_tx(&c.q_full[t], C::Q_BYTES);
-#pragma unroll
-                            for (int b = 0; b < C::NBLK; ++b)
-                                tma_load_3d(c.sQ + t * C::Q_BYTES + b * BM * SW, &tm_q, &c.q_full[t], b * C::SWE, h,
-                                            qbase + t * BM, pol_q);
-                        }
                         const int box = min(p.page_size, BN);
-                        for (int U = 0; U < loads; ++U) {
-                            const int stage = U % NS;
-                            if (U >= NS &&
-                                !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
-                                break;
-                            const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
-                            if (L & 1) {
-                                mbar_arrive(&c.kv_full[stage]);  // V part: copied by warps 10 and 11
-                            } else {
-                                uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
-                                const int pos0 = j * BN;
-                                const int part_valid = seqlen - pos0;
-                                mbar_arrive_expect_tx(&c.kv_full[stage], C::UNIT_BYTES);
-                                for (int r = 0; r < BN; r += box) {
-                                    const int prow = (r < part_valid) ? static_cast<int>(page_row(pos0 + r)) : -box;
-                                    for (int b = 0; b < C::KBLK_PER_UNIT; ++b)
-                                        tma_load_3d(dst + (b * BN + r) * SW, &tm_k, &c.kv_full[stage],
-                                                    (u * C::KBLK_PER_UNIT + b) * C::SWE, h, prow, pol_kv);
+                        bool ok = true;
+                        for (int rd = 0; ok && next_item<D, CAUSAL>(c, p, rd, persistent); ++rd) {
+                            ok = load_q(0);
+                            const int loads = c.loads();
+                            for (int L = 0; ok && L < loads; ++L) {
+                                if (L == C::UNITS && c.two && !load_q(1)) {
+                                    ok = false;
+                                    break;
                                 }
+                                const int U = c.u0 + L, stage = U % NS;
+                                if (U >= NS && !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag,
+                                                             c.lim, 100 + stage)) {
+                                    ok = false;
+                                    break;
+                                }
+                                const int Lk = L / C::UNITS, u = L % C::UNITS, j = Lk >> 1;
+                                if (Lk & 1) {
+                                    mbar_arrive(&c.kv_full[stage]);  // V part: copied by warps 10 and 11
+                                } else {
+                                    uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
+                                    const int pos0 = j * BN;
+                                    const int part_valid = c.seqlen - pos0;
+                                    mbar_arrive_expect_tx(&c.kv_full[stage], C::UNIT_BYTES);
+                                    for (int r = 0; r < BN; r += box) {
+                                        const int prow = (r < part_valid) ? static_cast<int>(page_row(pos0 + r)) : -box;
+                                        for (int b = 0; b < C::KBLK_PER_UNIT; ++b)
+                                            tma_load_3d(dst + (b * BN + r) * SW, &tm_k, &c.kv_full[stage],
+                                                        (u * C::KBLK_PER_UNIT + b) * C::SWE, c.h, prow, pol_kv);
+                                    }
+                                }
+                                issued = U + 1;
                             }
-                            issued = U + 1;
+                            c.advance();
                         }
                     }
                 } else {
                     constexpr int CPB = SW / 16;
                     constexpr int CPR = C::NBLK * CPB;  // 16-byte chunks per V row
                     const int w = pw - 1;                // copy warp 0, 1
-                    for (int U = 0; U < loads; ++U) {
-                        const int stage = U % NS;
-                        if (U >= NS &&
-                            !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
-                            break;
-                        const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
-                        if (!(L & 1)) {
-                            mbar_arrive(&c.kv_full[stage]);  // K part: moved by the TMA
-                            continue;
-                        }
-                        // V part u of tile j: rows [pos0, pos0 + VROWS_PER_UNIT), every column block
-                        const int pos0 = j * BN + u * C::VROWS_PER_UNIT;
-                        const uint32_t dst_u32 = smem_u32(c.sKV + stage * C::UNIT_BYTES);
-                        for (int g = w; g * 32 < C::VROWS_PER_UNIT; g += 2) {
-                            const int pos = pos0 + g * 32 + lane;
-                            const bool valid = pos < seqlen;
-                            const int64_t prow = valid ? page_row(pos) : 0;
-#pragma unroll 4
-                            for (int i = 0; i < CPR; ++i) {
-                                const int idx = i * 32 + lane;
-                                const int rr = idx / CPR, ch = idx % CPR;
-                                const int64_t pr = __shfl_sync(0xffffffffu, prow, rr);
-                                const bool ok_row = __shfl_sync(0xffffffffu, valid, rr);
-                                const int r = g * 32 + rr;
-                                const int blk = ch / CPB, cc = ch % CPB;
-                                const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
-                                cp_async_16_zfill(dst_u32 + blk * C::VROWS_PER_UNIT * SW + r * SW + ((cc ^ swz) << 4),
-                                                  static_cast<const uint8_t *>(p.v) +
-                                                      (pr * p.H + h) * static_cast<int64_t>(D) * 2 + ch * 16,
-                                                  ok_row ? 16u : 0u);
+                    bool ok = true;
+                    for (int rd = 0; ok && next_item<D, CAUSAL>(c, p, rd, persistent); ++rd) {
+                        const int loads = c.loads();
+                        for (int L = 0; L < loads; ++L) {
+                            const int U = c.u0 + L, stage = U % NS;
+                            if (U >= NS && !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag,
+                                                         c.lim, 100 + stage)) {
+                                ok = false;
+                                break;
                             }
+                            const int Lk = L / C::UNITS, u = L % C::UNITS, j = Lk >> 1;
+                            if (!(Lk & 1)) {
+                                mbar_arrive(&c.kv_full[stage]);  // K part: moved by the TMA
+                                continue;
+                            }
+                            // V part u of tile j: rows [pos0, pos0 + VROWS_PER_UNIT), every column block
+                            const int pos0 = j * BN + u * C::VROWS_PER_UNIT;
+                            const uint32_t dst_u32 = smem_u32(c.sKV + stage * C::UNIT_BYTES);
+                            for (int g = w; g * 32 < C::VROWS_PER_UNIT; g += 2) {
+                                const int pos = pos0 + g * 32 + lane;
+                                const bool valid = pos < c.seqlen;
+                                const int64_t prow = valid ? page_row(pos) : 0;
+#pragma unroll 4
+                                for (int i = 0; i < CPR; ++i) {
+                                    const int idx = i * 32 + lane;
+                                    const int rr = idx / CPR, ch = idx % CPR;
+                                    const int64_t pr = __shfl_sync(0xffffffffu, prow, rr);
+                                    const bool ok_row = __shfl_sync(0xffffffffu, valid, rr);
+                                    const int r = g * 32 + rr;
+                                    const int blk = ch / CPB, cc = ch % CPB;
+                                    const int swz = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
+                                    cp_async_16_zfill(dst_u32 + blk * C::VROWS_PER_UNIT * SW + r * SW + ((cc ^ swz) << 4),
+                                                      static_cast<const uint8_t *>(p.v) +
+                                                          (pr * p.H + c.h) * static_cast<int64_t>(D) * 2 + ch * 16,
+                                                      ok_row ? 16u : 0u);
+                                }
+                            }
+                            cp_async_mbar_arrive(&c.kv_full[stage]);  // arrives once this thread's copies have landed
                         }
-                        cp_async_mbar_arrive(&c.kv_full[stage]);  // arrives once this thread's copies have landed
+                        c.advance();
                     }
                     cp_async_wait_all();  // nothing of this thread is left in flight at exit
                 }
                 if (bad_page) record_error(FA_ERR_INDEX, 151);
             } else if (p.gather) {
-                // Fused packed path: warps 8, 10 and 11 (96 threads) copy every K/V row from the
-                // padded tensor (row = padded row of the packed token; rows past the last token
-                // read row 0, which the masks then ignore) with 16-byte cp.async into the same
-                // swizzled layout the TMA would produce; each thread's copies arrive on the part's
-                // barrier when they land, and the MMA thread fences the async proxy. (The softmax
-                // warps copy the query tiles.) The 32-row groups of the ring parts are dealt to
-                // the three warps in one running order (group G to warp G % 3), so each warp moves
-                // a third of the bytes and holds at most two groups of a part. A warp reads the
-                // padded rows of its next part's groups (one coalesced load per group) before it
-                // issues this part's copies, so index loads never wait in line.
+                // Fused packed path (one work item): warps 8, 10 and 11 (96 threads) copy every K/V
+                // row from the padded tensor (row = padded row of the packed token; rows past the
+                // last token read row 0, which the masks then ignore) with 16-byte cp.async into
+                // the same swizzled layout the TMA would produce; each thread's copies arrive on
+                // the part's barrier when they land, and the MMA thread fences the async proxy.
+                // (The softmax warps copy the query tiles.) The 32-row groups of the ring parts
+                // are dealt to the three warps in one running order (group G to warp G % 3), so
+                // each warp moves a third of the bytes and holds at most two groups of a part. A
+                // warp reads the padded rows of its next part's groups (one coalesced load per
+                // group) before it issues this part's copies, so index loads never wait in line.
+                q_issued_a = 1;
+                q_issued_b = c.two ? 1 : 0;
                 auto part_rows = [&](int U, int &tok0, int &rows) {
                     const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
-                    tok0 = kvbase + j * BN + ((L & 1) ? u * C::VROWS_PER_UNIT : 0);
+                    tok0 = c.kvbase + j * BN + ((L & 1) ? u * C::VROWS_PER_UNIT : 0);
                     rows = (L & 1) ? C::VROWS_PER_UNIT : BN;
                 };
-                const uint64_t pol_kv = l2_policy_evict_last();
+                const int loads = c.loads();
                 int64_t cur[2], nxt[2] = {first_rows[0], first_rows[1]};  // part 0's rows: read at set-up
                 int gU = 0;                                                // running index of part U's first group
                 for (int U = 0; U < loads; ++U) {
@@ -698,11 +850,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         const int g = g0 + 3 * k;
                         if (g * 32 >= rows) continue;
                         if ((U / C::UNITS) & 1)
-                            fetch_group<C::NBLK, SW, D>(dst, rows, g, cur[k], p.v, &tm_v, 0, p.H, h, lane,
+                            fetch_group<C::NBLK, SW, D>(dst, rows, g, cur[k], p.v, &tm_v, 0, p.H, c.h, lane,
                                                         &c.kv_full[stage], pol_kv);
                         else
                             fetch_group<C::KBLK_PER_UNIT, SW, D>(dst, rows, g, cur[k], p.k, &tm_k,
-                                                                 (U % C::UNITS) * C::KBLK_PER_UNIT, p.H, h, lane,
+                                                                 (U % C::UNITS) * C::KBLK_PER_UNIT, p.H, c.h, lane,
                                                                  &c.kv_full[stage], pol_kv);
                     }
                     cp_async_mbar_arrive(&c.kv_full[stage]);  // arrives once this thread's copies have landed
@@ -720,9 +872,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     constexpr int LPR = CH < 32 ? CH : 32;  // lanes per row
                     constexpr int RPI = 32 / LPR;            // rows per store instruction
                     const int ch = lane % LPR;
-                    uint8_t *const zbase = static_cast<uint8_t *>(p.out) + static_cast<int64_t>(h) * RB + ch * 16;
+                    uint8_t *const zbase = static_cast<uint8_t *>(p.out) + static_cast<int64_t>(c.h) * RB + ch * 16;
                     for (int gi = pw; gi < C::MAXQ * 4; gi += 3) {
-                        const int64_t tw0 = static_cast<int64_t>(qbase) + gi * 32;
+                        const int64_t tw0 = static_cast<int64_t>(c.qbase) + gi * 32;
                         if (tw0 >= p.total_tokens) break;
                         const int64_t tw1 = min(tw0 + 32, static_cast<int64_t>(p.total_tokens)) - 1;
                         // padded rows of the group's tokens, sorted (lanes past the last token: +inf)
@@ -758,102 +910,102 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 cp_async_wait_all();  // nothing of this thread is left in flight at exit
                 issued = 0;
             } else if (lane == 0) {
-                const uint64_t pol_q = l2_policy_evict_first();
-                const uint64_t pol_kv = l2_policy_evict_last();
-                for (int t = 0; t < nq; ++t) {
-                    mbar_arrive_expect_tx(&c.q_full[t], C::Q_BYTES);
-#pragma unroll
-                    for (int b = 0; b < C::NBLK; ++b)
-                        tma_load_3d(c.sQ + t * C::Q_BYTES + b * BM * SW, &tm_q, &c.q_full[t], b * C::SWE, h,
-                                    qbase + t * BM, pol_q);
-                }
-                // Paged K/V: physical row of key position pos (< seqlen) of this batch entry. A
-                // page index outside the pool is reported and replaced by page 0 (the result is
-                // then wrong, but nothing outside the pool is read).
-                const int32_t *bt = PAGED ? p.block_table + static_cast<int64_t>(blockIdx.z) * p.max_blocks : nullptr;
-                bool bad_page = false;  // reported once, after the loads
-                auto paged_row = [&](int pos) {
-                    int pg = __ldg(bt + (pos >> p.page_shift));
-                    if (pg < 0 || pg >= p.num_pages) {
-                        bad_page = true;
-                        pg = 0;
-                    }
-                    return (pg << p.page_shift) + (pos & (p.page_size - 1));
-                };
-                for (int U = 0; U < loads; ++U) {
-                    const int stage = U % NS;
-                    if (U >= NS &&
-                        !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage))
-                        break;
-                    const int L = U / C::UNITS, u = U % C::UNITS, j = L >> 1;
-                    uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
-                    if constexpr (PAGED) {
-                        // One box per (column block, page-sized row chunk) of the part. Rows of a
-                        // sequence's last page past its end hold whatever the pool holds there:
-                        // for K they are masked (their scores become -inf), but in V a NaN would
-                        // survive P = 0, so the V part that straddles the end lands on `tail`
-                        // first, its stray rows are zeroed, and only then is the stage released.
-                        const bool is_v = L & 1;
-                        const int rows = is_v ? C::VROWS_PER_UNIT : BN;
-                        const int box = min(p.page_size, rows);
-                        const int pos0 = j * BN + (is_v ? u * C::VROWS_PER_UNIT : 0);
-                        const int part_valid = p.seqlen - pos0;  // rows of the part inside the sequence
-                        const bool straddles = is_v && part_valid > 0 && part_valid < rows && part_valid % box != 0;
-                        uint64_t *bar = straddles ? c.tail : &c.kv_full[stage];
-                        tail_issued |= straddles;
-                        mbar_arrive_expect_tx(bar, C::UNIT_BYTES);
-                        for (int r = 0; r < rows; r += box) {
-                            // a chunk wholly past the sequence end (its table entry need not
-                            // exist) is a box at a negative row: all fill value (zeros)
-                            const int prow = (r < part_valid) ? paged_row(pos0 + r) : -box;
-                            if (is_v) {
-                                for (int b = 0; b < C::NBLK; ++b)
-                                    tma_load_3d(dst + (b * C::VROWS_PER_UNIT + r) * SW, &tm_v, bar, b * C::SWE, h,
-                                                prow, pol_kv);
-                            } else {
-                                for (int b = 0; b < C::KBLK_PER_UNIT; ++b)
-                                    tma_load_3d(dst + (b * BN + r) * SW, &tm_k, bar, (u * C::KBLK_PER_UNIT + b) * C::SWE,
-                                                h, prow, pol_kv);
-                            }
+                bool ok = true;
+                for (int rd = 0; ok && next_item<D, CAUSAL>(c, p, rd, persistent); ++rd) {
+                    ok = load_q(0);
+                    const int loads = c.loads();
+                    for (int L = 0; ok && L < loads; ++L) {
+                        if (L == C::UNITS && c.two && !load_q(1)) {
+                            ok = false;
+                            break;
                         }
-                        if (straddles) {
-                            // at most one such part per CTA (the last V tile): phase 0 of `tail`
-                            if (!wait_bounded(c.tail, 0, c.abort_flag, c.lim, 160)) break;
-                            const int r1 = min(rows, (part_valid + box - 1) / box * box);  // end of the ragged chunk
-                            for (int b = 0; b < C::NBLK; ++b)
-                                for (int r = part_valid; r < r1; ++r) {
-                                    uint4 *row = reinterpret_cast<uint4 *>(dst + (b * C::VROWS_PER_UNIT + r) * SW);
-#pragma unroll
-                                    for (int i = 0; i < SW / 16; ++i) row[i] = make_uint4(0u, 0u, 0u, 0u);
+                        const int U = c.u0 + L, stage = U % NS;
+                        if (U >= NS &&
+                            !wait_bounded(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag, c.lim, 100 + stage)) {
+                            ok = false;
+                            break;
+                        }
+                        const int Lk = L / C::UNITS, u = L % C::UNITS, j = Lk >> 1;
+                        uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
+                        if constexpr (PAGED) {
+                            // One box per (column block, page-sized row chunk) of the part. Rows of a
+                            // sequence's last page past its end hold whatever the pool holds there:
+                            // for K they are masked (their scores become -inf), but in V a NaN would
+                            // survive P = 0, so the V part that straddles the end lands on `tail`
+                            // first, its stray rows are zeroed, and only then is the stage released.
+                            const bool is_v = Lk & 1;
+                            const int rows = is_v ? C::VROWS_PER_UNIT : BN;
+                            const int box = min(p.page_size, rows);
+                            const int pos0 = j * BN + (is_v ? u * C::VROWS_PER_UNIT : 0);
+                            const int part_valid = c.seqlen - pos0;  // rows of the part inside the sequence
+                            const bool straddles = is_v && part_valid > 0 && part_valid < rows && part_valid % box != 0;
+                            uint64_t *bar = straddles ? c.tail : &c.kv_full[stage];
+                            mbar_arrive_expect_tx(bar, C::UNIT_BYTES);
+                            for (int r = 0; r < rows; r += box) {
+                                // a chunk wholly past the sequence end (its table entry need not
+                                // exist) is a box at a negative row: all fill value (zeros)
+                                const int prow = (r < part_valid) ? static_cast<int>(page_row(pos0 + r)) : -box;
+                                if (is_v) {
+                                    for (int b = 0; b < C::NBLK; ++b)
+                                        tma_load_3d(dst + (b * C::VROWS_PER_UNIT + r) * SW, &tm_v, bar, b * C::SWE,
+                                                    c.h, prow, pol_kv);
+                                } else {
+                                    for (int b = 0; b < C::KBLK_PER_UNIT; ++b)
+                                        tma_load_3d(dst + (b * BN + r) * SW, &tm_k, bar,
+                                                    (u * C::KBLK_PER_UNIT + b) * C::SWE, c.h, prow, pol_kv);
                                 }
-                            fence_proxy_async_smem();  // the zeros, before the tensor core reads them
-                            mbar_arrive(&c.kv_full[stage]);
-                        }
-                    } else {
-                        mbar_arrive_expect_tx(&c.kv_full[stage], C::UNIT_BYTES);
-                        if (L & 1) {
-                            // V part u: rows [u*VROWS_PER_UNIT, ...) of the tile, every column block
+                            }
+                            if (straddles) {
+                                // at most one such part per item (its last V tile); `tail` phases
+                                // count those parts over the items
+                                if (!wait_bounded(c.tail, tail_uses & 1, c.abort_flag, c.lim, 160)) {
+                                    tail_pending = tail_uses & 1;
+                                    ok = false;
+                                    break;
+                                }
+                                ++tail_uses;
+                                tail_pending = -1;
+                                const int r1 = min(rows, (part_valid + box - 1) / box * box);  // end of the ragged chunk
+                                for (int b = 0; b < C::NBLK; ++b)
+                                    for (int r = part_valid; r < r1; ++r) {
+                                        uint4 *row = reinterpret_cast<uint4 *>(dst + (b * C::VROWS_PER_UNIT + r) * SW);
 #pragma unroll
-                            for (int b = 0; b < C::NBLK; ++b)
-                                tma_load_3d(dst + b * C::VROWS_PER_UNIT * SW, &tm_v, &c.kv_full[stage], b * C::SWE,
-                                            h, kvbase + j * BN + u * C::VROWS_PER_UNIT, pol_kv);
+                                        for (int i = 0; i < SW / 16; ++i) row[i] = make_uint4(0u, 0u, 0u, 0u);
+                                    }
+                                fence_proxy_async_smem();  // the zeros, before the tensor core reads them
+                                mbar_arrive(&c.kv_full[stage]);
+                            }
+                            issued = U + 1;
                         } else {
-                            // K part u: column blocks [u*KBLK_PER_UNIT, ...) of every tile row
+                            mbar_arrive_expect_tx(&c.kv_full[stage], C::UNIT_BYTES);
+                            if (Lk & 1) {
+                                // V part u: rows [u*VROWS_PER_UNIT, ...) of the tile, every column block
 #pragma unroll
-                            for (int b = 0; b < C::KBLK_PER_UNIT; ++b)
-                                tma_load_3d(dst + b * BN * SW, &tm_k, &c.kv_full[stage],
-                                            (u * C::KBLK_PER_UNIT + b) * C::SWE, h, kvbase + j * BN, pol_kv);
+                                for (int b = 0; b < C::NBLK; ++b)
+                                    tma_load_3d(dst + b * C::VROWS_PER_UNIT * SW, &tm_v, &c.kv_full[stage],
+                                                b * C::SWE, c.h, c.kvbase + j * BN + u * C::VROWS_PER_UNIT, pol_kv);
+                            } else {
+                                // K part u: column blocks [u*KBLK_PER_UNIT, ...) of every tile row
+#pragma unroll
+                                for (int b = 0; b < C::KBLK_PER_UNIT; ++b)
+                                    tma_load_3d(dst + b * BN * SW, &tm_k, &c.kv_full[stage],
+                                                (u * C::KBLK_PER_UNIT + b) * C::SWE, c.h, c.kvbase + j * BN, pol_kv);
+                            }
+                            issued = U + 1;
                         }
                     }
-                    issued = U + 1;
+                    c.advance();
                 }
                 if (PAGED && bad_page) record_error(FA_ERR_INDEX, 150);
             }
             if (warp == C::WARP_TMA && lane == 0 && *c.abort_flag) {
                 // Let the copies already issued land before the CTA's shared memory goes away.
-                for (int t = 0; t < nq; ++t) {
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const int qi = t ? q_issued_b : q_issued_a;
+                    if (qi == 0) continue;
                     const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(&c.q_full[t], 0) && global_timer_ns() - t0 < c.lim) {
+                    while (!mbar_try_wait(&c.q_full[t], (qi - 1) & 1) && global_timer_ns() - t0 < c.lim) {
                     }
                 }
                 for (int U = (issued > NS ? issued - NS : 0); U < issued; ++U) {
@@ -862,17 +1014,20 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     while (!mbar_try_wait(&c.kv_full[stage], (U / NS) & 1) && global_timer_ns() - t0 < c.lim) {
                     }
                 }
-                if (tail_issued) {
+                if (tail_pending >= 0) {
                     const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(c.tail, 0) && global_timer_ns() - t0 < c.lim) {
+                    while (!mbar_try_wait(c.tail, tail_pending) && global_timer_ns() - t0 < c.lim) {
                     }
                 }
             }
-        } else if (warp == C::WARP_MMA) {
-            // ------------------------------------------------------------ MMA issuer
-            if (lane == 0) {
-                bool ok = true;
-                if (!c.two) {
+        } else if (warp == C::WARP_MMA || (split_issue && warp == C::WARP_MMA + 1)) {
+            // ------------------------------------------------------------ MMA issuer(s)
+            bool ok = true;
+            const bool qk = !split_issue || warp == C::WARP_MMA;
+            const bool pv = !split_issue || warp != C::WARP_MMA;
+            for (int rd = 0; ok && next_item<D, CAUSAL>(c, p, rd, persistent); ++rd) {
+                const int nl = max(c.nA, c.nB);  // key tiles of the item
+                if (c.single) {
                     const int n = c.nA;
                     for (int idx = 0; ok && idx < 2 * n; ++idx) {
                         bool is_v;
@@ -883,24 +1038,24 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 } else if (c.dec) {
                     // Separate P buffers: QK_t(j+1) only waits until the softmax warps have read
                     // S_t(j), so it runs while they compute P_t(j). Order per key tile j:
-                    // QK_A(j+1), QK_B(j+1), PV_A(j), PV_B(j), each when that tile uses key tile j.
-                    const int nB = c.nB;
-                    if (c.uses(0, 0)) ok = mma_qk<D, BF16>(c, 0, 0, true, !c.uses(1, 0));
-                    if (ok && c.uses(1, 0)) ok = mma_qk<D, BF16>(c, 1, 0, !c.uses(0, 0), true);
-                    for (int j = 0; ok && j < nB; ++j) {
+                    // QK_A(j+1), QK_B(j+1), PV_A(j), PV_B(j), each when that tile uses key tile j;
+                    // with two issuing warps each keeps its own half of that order (a key tile
+                    // is released by the QK warp, a value tile by the PV warp).
+                    if (qk && c.uses(0, 0)) ok = mma_qk<D, BF16>(c, 0, 0, true, !c.uses(1, 0));
+                    if (qk && ok && c.uses(1, 0)) ok = mma_qk<D, BF16>(c, 1, 0, !c.uses(0, 0), true);
+                    for (int j = 0; ok && j < nl; ++j) {
                         const bool a1 = c.uses(0, j + 1), b1 = c.uses(1, j + 1), a0 = c.uses(0, j), b0 = c.uses(1, j);
-                        if (a1) ok = mma_qk<D, BF16>(c, 0, j + 1, true, !b1);
-                        if (ok && b1) ok = mma_qk<D, BF16>(c, 1, j + 1, !a1, true);
-                        if (ok && a0) ok = mma_pv<D, BF16>(c, 0, j, true, !b0);
-                        if (ok && b0) ok = mma_pv<D, BF16>(c, 1, j, !a0, true);
+                        if (qk && a1) ok = mma_qk<D, BF16>(c, 0, j + 1, true, !b1);
+                        if (qk && ok && b1) ok = mma_qk<D, BF16>(c, 1, j + 1, !a1, true);
+                        if (pv && ok && a0) ok = mma_pv<D, BF16>(c, 0, j, true, !b0);
+                        if (pv && ok && b0) ok = mma_pv<D, BF16>(c, 1, j, !a0, true);
                     }
                 } else {
                     // Ping-pong over key tiles j: PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j). A key or
                     // value tile is waited for at its first use and released after its last.
-                    const int nB = c.nB;
                     if (c.uses(0, 0)) ok = mma_qk<D, BF16>(c, 0, 0, true, !c.uses(1, 0));
                     if (ok && c.uses(1, 0)) ok = mma_qk<D, BF16>(c, 1, 0, !c.uses(0, 0), true);
-                    for (int j = 1; ok && j <= nB; ++j) {
+                    for (int j = 1; ok && j <= nl; ++j) {
                         const bool ap = c.uses(0, j - 1), bp = c.uses(1, j - 1), ac = c.uses(0, j), bc = c.uses(1, j);
                         if (ap) ok = mma_pv<D, BF16>(c, 0, j - 1, true, !bp);
                         if (ok && ac) ok = mma_qk<D, BF16>(c, 0, j, true, !bc);
@@ -908,255 +1063,301 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         if (ok && bc) ok = mma_qk<D, BF16>(c, 1, j, !ac, true);
                     }
                 }
-                // Every MMA issued above has finished once `drain` completes.
-                umma_commit(c.drain);
-                const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(c.drain, 0) && global_timer_ns() - t0 < c.lim) {
-                }
+                c.advance();
             }
-    }
+            // Every MMA issued above has finished once `drain` completes.
+            umma_commit_elect(c.drain);
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(c.drain, 0) && global_timer_ns() - t0 < c.lim) {
+            }
+        }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        if constexpr (C::SPLIT_REGS) regs_inc<C::REGS_HIGH>();
+        if constexpr (C::SPLIT_REGS) regs_inc<C::regs_high(PACKED)>();
         const int t = warp >> 2;                      // query tile of this warpgroup
-        const int n = t ? c.nB - c.jB0 : c.nA;  // key tiles this warpgroup visits
-        const int j0 = c.j0(t);
         const int quarter = warp & 3;                 // TMEM lanes this warp may access
         const int r = quarter * 32 + lane;            // row of the tile == TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        // This row's token and its visible keys [klo, khi), counted from kvbase.
-        const int64_t tok = static_cast<int64_t>(qbase) + t * BM + r;
-        if (p.gather && (t == 0 || c.two)) {
-            // Fused packed path: each warp copies its own 32 rows of query tile t from their
-            // padded rows (rows past the last token read row 0); the warpgroup's 128 threads
-            // arrive on q_full[t] as their copies land.
-            int64_t pr = (tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
-            if (pr < 0 || pr >= p.padded_rows) pr = 0;  // never read outside q
-            fetch_group<C::NBLK, SW, D>(c.sQ + t * C::Q_BYTES, BM, quarter, pr, p.q, &tm_q, 0, p.H, h, lane,
-                                        &c.q_full[t], l2_policy_evict_first());
-            cp_async_mbar_arrive(&c.q_full[t]);
-        }
-        int klo = 0, khi = 1;
-        bool row_ok;
-        if (!packed) {
-            const int row_pos = q0 + t * BM + r;  // position inside the sequence
-            row_ok = row_pos < seqlen;
-            khi = CAUSAL ? min(seqlen, row_pos + 1) : seqlen;
-        } else {
-            row_ok = tok < p.total_tokens;
-            const int tw0 = qbase + t * BM + quarter * 32;  // this warp's first token
-            int s_lane = 0;
-            if (tw0 < p.total_tokens) {  // warp-uniform
-                const int s_w = warp_seq_of_token(p.cu_seqlens, p.num_seqs, tw0, lane);
-                s_lane = lane_seq_of_token(p.cu_seqlens, p.num_seqs, s_w,
-                                           static_cast<int>(min(tok, static_cast<int64_t>(p.total_tokens - 1))), lane);
-            }
-            if (row_ok) {
-                const int s_r = s_lane;
-                klo = p.cu_seqlens[s_r] - kvbase;
-                khi = (CAUSAL ? min(p.cu_seqlens[s_r + 1], static_cast<int>(tok) + 1) : p.cu_seqlens[s_r + 1]) - kvbase;
-            }
-        }
         const uint32_t o_col = C::O_COL + t * D;
         const float sc = p.scale_log2;
-        float m = -INFINITY;  // running max of scaled scores, log2 units (possibly stale)
-        float l = 0.f;        // running sum of 2^(s*sc - m)
-        bool ok = n > 0;
-        if (c.dec) {
-            // Separate P buffer: S_t is released right after it is read, so QK_t(j+1) overlaps
-            // this step's exponentials; P_t(j) is written once PV_t(j-1) has consumed P_t(j-1).
-            const uint32_t p_addr = c.tmem + lane_base + C::P_COL + 64 * t;
-            for (int jj = 0; jj < n; ++jj) {
-                const int j = j0 + jj;  // key tile
-                if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[t], jj & 1, c.abort_flag, c.lim, 330 + t))) {
-                    ok = false;
-                    break;
+        bool ok = true;
+        // Only the round and this tile's running key-step count stay live across an item's key
+        // steps (the softmax warps are at their register limit there); the item is looked up
+        // again for the epilogue.
+        int gbase = 0;
+        for (int rd = 0; ok && next_item<D, CAUSAL>(c, p, rd, persistent); ++rd) {
+            const int n = c.steps(t);  // key tiles this warpgroup visits in the item
+            if (n <= 0) continue;      // tile absent
+            const int j0 = c.j0(t);
+            // This row's token and its visible keys [klo, khi), counted from kvbase.
+            const int64_t tok = static_cast<int64_t>(c.qbase) + t * BM + r;
+            if (p.gather) {
+                // Fused packed path: each warp copies its own 32 rows of query tile t from their
+                // padded rows (rows past the last token read row 0); the warpgroup's 128 threads
+                // arrive on q_full[t] as their copies land.
+                int64_t pr = (tok < p.total_tokens) ? __ldg(p.gather + tok) : 0;
+                if (pr < 0 || pr >= p.padded_rows) pr = 0;  // never read outside q
+                fetch_group<C::NBLK, SW, D>(c.sQ + t * C::Q_BYTES, BM, quarter, pr, p.q, &tm_q, 0, p.H, c.h, lane,
+                                            &c.q_full[t], l2_policy_evict_first());
+                cp_async_mbar_arrive(&c.q_full[t]);
+            }
+            int klo = 0, khi = 1;
+            bool row_ok;
+            if (!packed) {
+                const int row_pos = c.q0 + t * BM + r;  // position inside the sequence
+                row_ok = row_pos < c.seqlen;
+                khi = CAUSAL ? min(c.seqlen, row_pos + 1) : c.seqlen;
+            } else {
+                row_ok = tok < p.total_tokens;
+                const int tw0 = c.qbase + t * BM + quarter * 32;  // this warp's first token
+                int s_lane = 0;
+                if (tw0 < p.total_tokens) {  // warp-uniform
+                    const int s_w = warp_seq_of_token(p.cu_seqlens, p.num_seqs, tw0, lane);
+                    s_lane = lane_seq_of_token(p.cu_seqlens, p.num_seqs, s_w,
+                                               static_cast<int>(min(tok, static_cast<int64_t>(p.total_tokens - 1))), lane);
                 }
-                tc_fence_after_sync();
-                uint32_t sr[BN];
-#pragma unroll
-                for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(c.tmem + lane_base + t * BN + cc * 32, sr + cc * 32);
-                tmem_ld_wait();
-                tmem_reg_fence<BN>(sr);
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&c.s_free[t]);
-                const int lo = klo - j * BN, hi = khi - j * BN;  // visible columns of this tile
-                const bool need_mask = __any_sync(0xffffffffu, lo > 0 || hi < BN);
-                if (need_mask) {
-#pragma unroll
-                    for (int i = 0; i < BN; ++i)
-                        if (i < lo || i >= hi) sr[i] = __float_as_uint(-INFINITY);
+                if (row_ok) {
+                    const int s_r = s_lane;
+                    klo = p.cu_seqlens[s_r] - c.kvbase;
+                    khi = (CAUSAL ? min(p.cu_seqlens[s_r + 1], static_cast<int>(tok) + 1) : p.cu_seqlens[s_r + 1]) -
+                          c.kvbase;
                 }
-                const float m_cand = row_max<BN>(sr) * sc;
-                const bool grow = m_cand > m + 8.0f;
-                float alpha = 1.f;
-                if (grow) {
-                    alpha = ex2_approx(m - m_cand);
-                    m = m_cand;
-                }
-                const bool warp_grow = __any_sync(0xffffffffu, grow);
-                uint32_t pk[BN / 2];
-                // a packed row may not have met any visible key yet (m = -inf): its P is 0
-                const float neg_m = (m == -INFINITY) ? 0.f : -m;
-                const float rs = need_mask ? softmax_row_to_regs<BN, BF16, 0>(sr, sc, neg_m, pk)
-                                           : softmax_row_to_regs<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, pk);
-                l = fmaf(l, alpha, rs);
-                if (jj > 0) {
-                    if (!__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (jj - 1) & 1, c.abort_flag, c.lim, 340 + t))) {
+            }
+            float m = -INFINITY;  // running max of scaled scores, log2 units (possibly stale)
+            float l = 0.f;        // running sum of 2^(s*sc - m)
+            if (c.dec) {
+                // Separate P buffer: S_t is released right after it is read, so QK_t(j+1) overlaps
+                // this step's exponentials; P_t(j) is written once PV_t(j-1) has consumed P_t(j-1)
+                // (at an item's first step, the previous item's epilogue has waited for its last PV).
+                const uint32_t p_addr = c.tmem + lane_base + C::P_COL + 64 * t;
+                for (int jj = 0; jj < n; ++jj) {
+                    const int j = j0 + jj;       // key tile
+                    const int gs = gbase + jj;  // running key step of this tile
+                    if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[t], gs & 1, c.abort_flag, c.lim, 330 + t))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    if (warp_grow) {
-                        const uint64_t a2 = f2(alpha, alpha);
-#pragma unroll 1
-                        for (int cc = 0; cc < D / 32; ++cc) {
-                            uint32_t o[32];
-                            tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
-                            tmem_ld_wait();
-                            tmem_reg_fence<32>(o);
+                    uint32_t sr[BN];
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                float lo, hi;
-                                f2_split(fmul2(f2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), lo, hi);
-                                o[2 * i] = __float_as_uint(lo);
-                                o[2 * i + 1] = __float_as_uint(hi);
+                    for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(c.tmem + lane_base + t * BN + cc * 32, sr + cc * 32);
+                    tmem_ld_wait();
+                    tmem_reg_fence<BN>(sr);
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&c.s_free[t]);
+                    const int lo = klo - j * BN, hi = khi - j * BN;  // visible columns of this tile
+                    const bool need_mask = __any_sync(0xffffffffu, lo > 0 || hi < BN);
+                    if (need_mask) {
+#pragma unroll
+                        for (int i = 0; i < BN; ++i)
+                            if (i < lo || i >= hi) sr[i] = __float_as_uint(-INFINITY);
+                    }
+                    const float m_cand = row_max<BN>(sr) * sc;
+                    const bool grow = m_cand > m + 8.0f;
+                    float alpha = 1.f;
+                    if (grow) {
+                        alpha = ex2_approx(m - m_cand);
+                        m = m_cand;
+                    }
+                    const bool warp_grow = __any_sync(0xffffffffu, grow);
+                    uint32_t pk[BN / 2];
+                    // a packed row may not have met any visible key yet (m = -inf): its P is 0
+                    const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                    const float rs = need_mask ? softmax_row_to_regs<BN, BF16, 0>(sr, sc, neg_m, pk)
+                                               : softmax_row_to_regs<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, pk);
+                    l = fmaf(l, alpha, rs);
+                    if (jj > 0) {
+                        if (!__all_sync(0xffffffffu,
+                                        wait_bounded(&c.pv_done[t], (gs - 1) & 1, c.abort_flag, c.lim, 340 + t))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        if (warp_grow) {
+                            const uint64_t a2 = f2(alpha, alpha);
+#pragma unroll 1
+                            for (int cc = 0; cc < D / 32; ++cc) {
+                                uint32_t o[32];
+                                tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
+                                tmem_ld_wait();
+                                tmem_reg_fence<32>(o);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) {
+                                    float lo, hi;
+                                    f2_split(fmul2(f2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), lo, hi);
+                                    o[2 * i] = __float_as_uint(lo);
+                                    o[2 * i + 1] = __float_as_uint(hi);
+                                }
+                                tmem_st32(c.tmem + lane_base + o_col + cc * 32, o);
                             }
-                            tmem_st32(c.tmem + lane_base + o_col + cc * 32, o);
                         }
                     }
-                }
 #pragma unroll
-                for (int cc = 0; cc < BN / 64; ++cc) tmem_st32(p_addr + cc * 32, pk + cc * 32);
-                tmem_st_wait();
-                tc_fence_before_sync();
-                mbar_arrive(&c.p_full[t]);
-            }
-        } else
-        for (int jj = 0; jj < n; ++jj) {
-            const int j = j0 + jj;  // key tile
-            const int b = c.buf(t, jj);
-            if (!__all_sync(0xffffffffu, wait_bounded(&c.s_full[b], c.sphase(jj), c.abort_flag, c.lim, 300 + t))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after_sync();
-            uint32_t sr[BN];
-#pragma unroll
-            for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(c.tmem + lane_base + b * BN + cc * 32, sr + cc * 32);
-            tmem_ld_wait();
-            tmem_reg_fence<BN>(sr);
-            const int lo = klo - j * BN, hi = khi - j * BN;  // visible columns of this tile
-            const bool need_mask = __any_sync(0xffffffffu, lo > 0 || hi < BN);
-            if (need_mask) {
-#pragma unroll
-                for (int i = 0; i < BN; ++i)
-                    if (i < lo || i >= hi) sr[i] = __float_as_uint(-INFINITY);
-            }
-            const float mx = row_max<BN>(sr);
-            const float m_cand = mx * sc;
-            const bool grow = m_cand > m + 8.0f;
-            float alpha = 1.f;
-            if (grow) {
-                alpha = ex2_approx(m - m_cand);
-                m = m_cand;
-            }
-            const bool warp_grow = __any_sync(0xffffffffu, grow);
-            // P = 2^(s*sc - m): written back to TMEM over S, 64 columns at a time.
-            // a packed row may not have met any visible key yet (m = -inf): its P is 0
-            const float neg_m = (m == -INFINITY) ? 0.f : -m;
-            const uint32_t p_addr = c.tmem + lane_base + b * BN;
-            const float rs = need_mask ? softmax_chunk_store<BN, BF16, 0>(sr, sc, neg_m, p_addr)  // -inf -> exactly 0
-                                       : softmax_chunk_store<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, p_addr);
-            l = fmaf(l, alpha, rs);
-            tmem_st_wait();
-            if (jj > 0) {
-                // O must hold PV(j-1) before it is rescaled. With two tiles, PV_t(j-1) was
-                // issued before QK_t(j), and the commit behind s_full only fires once every
-                // earlier MMA of the issuing thread has completed, so it is done already. With
-                // one tile QK(j) precedes PV(j-1): wait for it (on every step, so this thread
-                // never falls two phases behind on pv_done). The final wait after the loop
-                // always targets the newest phase, which is correct either way.
-                if (!c.two &&
-                    !__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (jj - 1) & 1, c.abort_flag, c.lim, 310 + t))) {
-                    ok = false;
-                    break;
-                }
-                if (warp_grow) {
-                    // O holds sum_{j' < j} P_j' V_j'; bring it to the new running max.
-                    tc_fence_after_sync();
-#pragma unroll 1
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
-                        tmem_ld_wait();
-                        tmem_reg_fence<32>(o);
-                        const uint64_t a2 = f2(alpha, alpha);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float lo, hi;
-                            f2_split(fmul2(f2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), lo, hi);
-                            o[2 * i] = __float_as_uint(lo);
-                            o[2 * i + 1] = __float_as_uint(hi);
-                        }
-                        tmem_st32(c.tmem + lane_base + o_col + cc * 32, o);
-                    }
+                    for (int cc = 0; cc < BN / 64; ++cc) tmem_st32(p_addr + cc * 32, pk + cc * 32);
                     tmem_st_wait();
+                    tc_fence_before_sync();
+                    mbar_arrive(&c.p_full[t]);
                 }
-            }
-            tc_fence_before_sync();
-            mbar_arrive(&c.p_full[b]);
-        }
-        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (n - 1) & 1, c.abort_flag, c.lim, 320 + t));
-        if (ok) {
-            tc_fence_after_sync();
-            const float inv_l = 1.f / l;
-            int64_t orow_idx = (p.gather && row_ok) ? __ldg(p.gather + tok) : tok;  // fused: padded row
-            const bool store_ok = row_ok && (!p.gather || (orow_idx >= 0 && orow_idx < p.padded_rows));
-            // O leaves through this tile's query buffer, unused now that every MMA of the tile
-            // has completed: each warp stages its 32 rows there (a lane writes its row, 16-byte
-            // chunk c of row r at chunk c ^ (r & 7), so eight lanes hit eight bank groups), then
-            // writes whole rows to global memory, consecutive lanes on consecutive 16 bytes.
-            constexpr int RB = D * 2;                // bytes of one row of one head
-            constexpr int CH = RB / 16;              // 16-byte chunks per row
-            constexpr int XM = (CH < 8 ? CH : 8) - 1;
-            constexpr int LPR = CH < 32 ? CH : 32;  // lanes per row in the global stores
-            constexpr int RPI = 32 / LPR;            // rows per store instruction
-            const uint32_t stage = smem_u32(c.sQ + t * C::Q_BYTES) + quarter * 32 * RB;
-            fence_proxy_async_smem();  // the tensor core's reads of Q come before these writes
+            } else {
+                for (int jj = 0; jj < n; ++jj) {
+                    const int j = j0 + jj;       // key tile
+                    const int gs = gbase + jj;  // running key step of this tile
+                    const int b = c.buf(t, gs);
+                    if (!__all_sync(0xffffffffu,
+                                    wait_bounded(&c.s_full[b], c.sphase(gs), c.abort_flag, c.lim, 300 + t))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    uint32_t sr[BN];
+#pragma unroll
+                    for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(c.tmem + lane_base + b * BN + cc * 32, sr + cc * 32);
+                    tmem_ld_wait();
+                    tmem_reg_fence<BN>(sr);
+                    const int lo = klo - j * BN, hi = khi - j * BN;  // visible columns of this tile
+                    const bool need_mask = __any_sync(0xffffffffu, lo > 0 || hi < BN);
+                    if (need_mask) {
+#pragma unroll
+                        for (int i = 0; i < BN; ++i)
+                            if (i < lo || i >= hi) sr[i] = __float_as_uint(-INFINITY);
+                    }
+                    const float mx = row_max<BN>(sr);
+                    const float m_cand = mx * sc;
+                    const bool grow = m_cand > m + 8.0f;
+                    float alpha = 1.f;
+                    if (grow) {
+                        alpha = ex2_approx(m - m_cand);
+                        m = m_cand;
+                    }
+                    const bool warp_grow = __any_sync(0xffffffffu, grow);
+                    // P = 2^(s*sc - m): written back to TMEM over S, 64 columns at a time.
+                    // a packed row may not have met any visible key yet (m = -inf): its P is 0
+                    const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                    const uint32_t p_addr = c.tmem + lane_base + b * BN;
+                    const float rs = need_mask
+                                         ? softmax_chunk_store<BN, BF16, 0>(sr, sc, neg_m, p_addr)  // -inf -> exactly 0
+                                         : softmax_chunk_store<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, p_addr);
+                    l = fmaf(l, alpha, rs);
+                    tmem_st_wait();
+                    if (jj > 0) {
+                        // O must hold PV(j-1) before it is rescaled. With two tiles, PV_t(j-1) was
+                        // issued before QK_t(j), and the commit behind s_full only fires once every
+                        // earlier MMA of the issuing thread has completed, so it is done already. With
+                        // one tile QK(j) precedes PV(j-1): wait for it (on every step, so this thread
+                        // never falls two phases behind on pv_done). The final wait after the loop
+                        // always targets the newest phase, which is correct either way.
+                        if (c.single && !__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (gs - 1) & 1,
+                                                                              c.abort_flag, c.lim, 310 + t))) {
+                            ok = false;
+                            break;
+                        }
+                        if (warp_grow) {
+                            // O holds sum_{j' < j} P_j' V_j'; bring it to the new running max.
+                            tc_fence_after_sync();
 #pragma unroll 1
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t o[32];
-                tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
-                tmem_ld_wait();
-                tmem_reg_fence<32>(o);
-                uint32_t w[16];
+                            for (int cc = 0; cc < D / 32; ++cc) {
+                                uint32_t o[32];
+                                tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
+                                tmem_ld_wait();
+                                tmem_reg_fence<32>(o);
+                                const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    w[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-#pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4)
-                    st_shared_v4(stage + lane * RB + (((cc * 4 + v4) ^ (lane & XM)) << 4), w[4 * v4], w[4 * v4 + 1],
-                                 w[4 * v4 + 2], w[4 * v4 + 3]);
-            }
-            __syncwarp();
-            {
-                const int ch = lane % LPR;
-                uint8_t *const obase = static_cast<uint8_t *>(p.out) + static_cast<int64_t>(h) * RB + ch * 16;
-#pragma unroll 4
-                for (int r0 = 0; r0 < 32; r0 += RPI) {
-                    const int rr = r0 + lane / LPR;
-                    const int64_t orow_r = __shfl_sync(0xffffffffu, orow_idx, rr);
-                    const bool ok_r = __shfl_sync(0xffffffffu, store_ok, rr);
-                    const uint4 v = ld_shared_v4(stage + rr * RB + ((ch ^ (rr & XM)) << 4));
-                    if (ok_r) *reinterpret_cast<uint4 *>(obase + orow_r * p.H * RB) = v;
+                                for (int i = 0; i < 16; ++i) {
+                                    float lo, hi;
+                                    f2_split(fmul2(f2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), lo, hi);
+                                    o[2 * i] = __float_as_uint(lo);
+                                    o[2 * i + 1] = __float_as_uint(hi);
+                                }
+                                tmem_st32(c.tmem + lane_base + o_col + cc * 32, o);
+                            }
+                            tmem_st_wait();
+                        }
+                    }
+                    tc_fence_before_sync();
+                    mbar_arrive(&c.p_full[b]);
                 }
             }
-            if (row_ok && p.lse) {
+            if (ok)
+                ok = __all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (gbase + n - 1) & 1, c.abort_flag, c.lim, 320 + t));
+            if (!ok) break;
+            gbase += n;
+            tc_fence_after_sync();
+            // the item's coordinates again, computed afresh rather than carried through the key steps
+            int eh, eb, eq0, eqbase;
+            item_coords<D, CAUSAL>(p, rd, persistent, eh, eb, eq0, eqbase);
+            const int64_t otok = static_cast<int64_t>(eqbase) + t * BM + r;
+            const bool orow_ok = packed ? otok < p.total_tokens : (eq0 + t * BM + r < p.seqlen);
+            const float inv_l = 1.f / l;
+            constexpr int RB = D * 2;  // bytes of one row of one head
+            if (persistent) {
+                // Each thread writes its own row straight from registers (16-byte stores): the
+                // tile's query buffer may already hold the next item's Q.
+                uint8_t *const orow = static_cast<uint8_t *>(p.out) + (otok * p.H + eh) * RB;
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
+                    tmem_ld_wait();
+                    tmem_reg_fence<32>(o);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        w[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+                    if (orow_ok) {
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            *reinterpret_cast<uint4 *>(orow + cc * 64 + v4 * 16) =
+                                make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                    }
+                }
+            } else {
+                int64_t orow_idx = (p.gather && orow_ok) ? __ldg(p.gather + otok) : otok;  // fused: padded row
+                const bool store_ok = orow_ok && (!p.gather || (orow_idx >= 0 && orow_idx < p.padded_rows));
+                // O leaves through this tile's query buffer, unused now that every MMA of the tile
+                // has completed (one work item per CTA here): each warp stages its 32 rows there (a
+                // lane writes its row, 16-byte chunk c of row r at chunk c ^ (r & 7), so eight
+                // lanes hit eight bank groups), then writes whole rows to global memory,
+                // consecutive lanes on consecutive 16 bytes.
+                constexpr int CH = RB / 16;              // 16-byte chunks per row
+                constexpr int XM = (CH < 8 ? CH : 8) - 1;
+                constexpr int LPR = CH < 32 ? CH : 32;  // lanes per row in the global stores
+                constexpr int RPI = 32 / LPR;            // rows per store instruction
+                const uint32_t stage = smem_u32(c.sQ + t * C::Q_BYTES) + quarter * 32 * RB;
+                fence_proxy_async_smem();  // the tensor core's reads of Q come before these writes
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
+                    tmem_ld_wait();
+                    tmem_reg_fence<32>(o);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        w[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        st_shared_v4(stage + lane * RB + (((cc * 4 + v4) ^ (lane & XM)) << 4), w[4 * v4], w[4 * v4 + 1],
+                                     w[4 * v4 + 2], w[4 * v4 + 3]);
+                }
+                __syncwarp();
+                {
+                    const int ch = lane % LPR;
+                    uint8_t *const obase = static_cast<uint8_t *>(p.out) + static_cast<int64_t>(eh) * RB + ch * 16;
+#pragma unroll 4
+                    for (int r0 = 0; r0 < 32; r0 += RPI) {
+                        const int rr = r0 + lane / LPR;
+                        const int64_t orow_r = __shfl_sync(0xffffffffu, orow_idx, rr);
+                        const bool ok_r = __shfl_sync(0xffffffffu, store_ok, rr);
+                        const uint4 v = ld_shared_v4(stage + rr * RB + ((ch ^ (rr & XM)) << 4));
+                        if (ok_r) *reinterpret_cast<uint4 *>(obase + orow_r * p.H * RB) = v;
+                    }
+                }
+            }
+            if (orow_ok && p.lse) {
                 const float lse = m * 0.6931471805599453f + logf(l);
-                const int64_t li = packed ? static_cast<int64_t>(h) * p.total_tokens + tok
-                                          : (static_cast<int64_t>(blockIdx.z) * p.H + h) * p.seqlen + (tok - seq_start);
+                const int64_t li = packed ? static_cast<int64_t>(eh) * p.total_tokens + otok
+                                          : (static_cast<int64_t>(eb) * p.H + eh) * p.seqlen + (eq0 + t * BM + r);
                 p.lse[li] = lse;
             }
         }
@@ -1172,11 +1373,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 }
 
 // ------------------------------------------------------------------ host launchers
-template <int D, bool BF16, bool CAUSAL, bool PAGED>
+template <int D, bool BF16, bool CAUSAL, bool PAGED, bool PACKED>
 static cudaError_t launch_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             const FwdParams &p, dim3 grid, cudaStream_t st) {
     using C = Cfg<D>;
-    auto kern = fa_fwd_kernel<D, BF16, CAUSAL, PAGED>;
+    auto kern = fa_fwd_kernel<D, BF16, CAUSAL, PAGED, PACKED>;
     // The shared-memory opt-in is a per-device function attribute; setting it twice is harmless.
     static uint64_t attr_set_mask = 0;
     int dev = 0;
@@ -1189,7 +1390,7 @@ static cudaError_t launch_t(const CUtensorMap &tq, const CUtensorMap &tk, const 
             cudaFuncAttributes fa_attr;
             e = cudaFuncGetAttributes(&fa_attr, kern);
             if (e != cudaSuccess) return e;
-            if (fa_attr.numRegs * C::NUM_THREADS < 128 * C::REGS_LOW + 256 * C::REGS_HIGH)
+            if (fa_attr.numRegs * C::NUM_THREADS < 128 * C::regs_low(PACKED) + 256 * C::regs_high(PACKED))
                 return cudaErrorInvalidConfiguration;
         }
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);

@@ -7,8 +7,8 @@ namespace fa {
 template <int D, bool BF16>
 static cudaError_t launch_paged_c(bool causal, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const FwdParams &p, dim3 grid, cudaStream_t st) {
-    return causal ? launch_t<D, BF16, true, true>(tq, tk, tv, p, grid, st)
-                  : launch_t<D, BF16, false, true>(tq, tk, tv, p, grid, st);
+    return causal ? launch_t<D, BF16, true, true, false>(tq, tk, tv, p, grid, st)
+                  : launch_t<D, BF16, false, true, false>(tq, tk, tv, p, grid, st);
 }
 
 template <int D>
@@ -29,6 +29,6 @@ cudaError_t launch_fwd_paged(int D, bool bf16, bool causal, const CUtensorMap &t
     }
 }
 
-cudaError_t fwd_paged_take_device_error(int *code, int *where) { return take_device_error(code, where); }
+cudaError_t fwd_paged_error_addrs(int **code, int **where) { return device_error_addrs(code, where); }
 
 }  // namespace fa

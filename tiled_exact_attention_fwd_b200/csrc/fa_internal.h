@@ -30,11 +30,15 @@ struct FwdParams {
     int page_size;   // a power of two
     int page_shift;  // log2(page_size)
     int num_pages;
+    // Dense inputs (persistent grid): batch entries, groups of fwd_tiles_per_cta(D) query tiles
+    // per sequence, and work items batch * H * npairs.
+    int batch, npairs, num_items;
 };
 
-// Attention forward. Dense: grid (H, ceil(ceil(S / 128) / tiles_per_cta), B), a CTA owns
-// fwd_tiles_per_cta(D) consecutive 128-row query tiles of one sequence. Packed: grid
-// (H, ceil(total / (128 * tiles_per_cta)), 1), a CTA owns that many consecutive packed tokens.
+// Attention forward. Dense: a persistent grid of min(num_items, SMs) CTAs; a work item is
+// fwd_tiles_per_cta(D) consecutive 128-row query tiles of one head of one sequence. Packed:
+// grid (H, ceil(total / (128 * tiles_per_cta)), 1), a CTA owns that many consecutive packed
+// tokens.
 cudaError_t launch_fwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
                        const CUtensorMap &tv, const FwdParams &p, dim3 grid, cudaStream_t st);
 // The same with p.block_table set (paged K/V; maps tk/tv cover the page pools).
@@ -52,8 +56,9 @@ int fwd_gather_run_rows();
 int fwd_paged_k_box_rows(int D, int page_size);
 int fwd_paged_v_box_rows(int D, int page_size);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t st);
-cudaError_t fwd_take_device_error(int *code, int *where);
-cudaError_t fwd_paged_take_device_error(int *code, int *where);
+// Device addresses of each kernel family's error word (code, location) on the current device.
+cudaError_t fwd_error_addrs(int **code, int **where);
+cudaError_t fwd_paged_error_addrs(int **code, int **where);
 
 // Attention backward (fa_bwd.cu): dQ, dK, dV from q, k, v, out, dout and the forward's LSE.
 struct BwdParams {
@@ -71,7 +76,7 @@ struct BwdParams {
 // tq, tk, tv, tdo: TMA maps of q, k, v, dout as for the forward (128-row boxes).
 cudaError_t launch_bwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
                        const CUtensorMap &tv, const CUtensorMap &tdo, const BwdParams &p, cudaStream_t st);
-cudaError_t bwd_take_device_error(int *code, int *where);
+cudaError_t bwd_error_addrs(int **code, int **where);
 // The fixed delta buffer of fa_bwd_noalloc: kNoallocDeltaFloats floats (64 MiB) in device
 // memory that belongs to the library's module image; its address on the current device.
 constexpr int64_t kNoallocDeltaFloats = int64_t(1) << 24;
@@ -84,6 +89,6 @@ cudaError_t launch_unpad3(const void *const x[3], const int64_t *indices, int64_
                           int64_t row_bytes, void *const out[3], cudaStream_t st);
 cudaError_t launch_pad(const void *x, const int64_t *indices, int64_t nnz, int64_t total_rows,
                        int64_t row_bytes, void *out, cudaStream_t st);
-cudaError_t pad_take_device_error(int *code, int *where);
+cudaError_t pad_error_addrs(int **code, int **where);
 
 }  // namespace fa

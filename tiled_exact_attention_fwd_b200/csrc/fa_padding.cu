@@ -227,15 +227,10 @@ cudaError_t launch_pad(const void *x, const int64_t *indices, int64_t nnz, int64
     return cudaGetLastError();
 }
 
-cudaError_t pad_take_device_error(int *code, int *where) {
-    int zero = 0;
-    cudaError_t e = cudaMemcpyFromSymbol(code, g_pad_err_code, sizeof(int));
+cudaError_t pad_error_addrs(int **code, int **where) {
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(code), g_pad_err_code);
     if (e != cudaSuccess) return e;
-    e = cudaMemcpyFromSymbol(where, g_pad_err_where, sizeof(int));
-    if (e != cudaSuccess) return e;
-    e = cudaMemcpyToSymbol(g_pad_err_code, &zero, sizeof(int));
-    if (e != cudaSuccess) return e;
-    return cudaMemcpyToSymbol(g_pad_err_where, &zero, sizeof(int));
+    return cudaGetSymbolAddress(reinterpret_cast<void **>(where), g_pad_err_where);
 }
 
 }  // namespace fa

@@ -1,6 +1,7 @@
 // fa_sync.cuh -- the device error word and the bounded mbarrier wait shared by the kernels.
 // Each compilation unit that includes this header gets its own error word (static device
-// variables); take_device_error reads and clears the word of the unit that calls it.
+// variables); device_error_addrs gives its device addresses, which the status query reads
+// and clears on the caller's stream.
 #pragma once
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -36,16 +37,11 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
     }
 }
 
-// Reads and clears this compilation unit's error word.
-static cudaError_t take_device_error(int *code, int *where) {
-    int zero = 0;
-    cudaError_t e = cudaMemcpyFromSymbol(code, g_err_code, sizeof(int));
+// Device addresses (on the current device) of this compilation unit's error word.
+static cudaError_t device_error_addrs(int **code, int **where) {
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(code), g_err_code);
     if (e != cudaSuccess) return e;
-    e = cudaMemcpyFromSymbol(where, g_err_where, sizeof(int));
-    if (e != cudaSuccess) return e;
-    e = cudaMemcpyToSymbol(g_err_code, &zero, sizeof(int));
-    if (e != cudaSuccess) return e;
-    return cudaMemcpyToSymbol(g_err_where, &zero, sizeof(int));
+    return cudaGetSymbolAddress(reinterpret_cast<void **>(where), g_err_where);
 }
 
 }  // namespace fa
