@@ -14,9 +14,15 @@ Also reported on the same line:
   roofline     tensor-bound: achieved TFLOPS of the attention kernel vs the measured bf16 peak.
   cpu_baseline the float64 CPU oracle on a bounded sample of the same workload.
 
-Launch: `python bench.py [--gpus N --steps K --warmup W]`; for N > 1 under
-torch.distributed.run, every rank runs the same per-GPU workload (weak scaling, no
-collective on the data path) and the time is the max over ranks.
+  configs      every workload of the pages (small dense, packed 32x64, ViT, the causal 8192
+               case, the head-dim sweep at 4096): time per call or TFLOPS, and each one's
+               roofline: tensor-bound (FLOPs / measured bf16 peak) or exp-bound (one exp2 per
+               visible score / MUFU rate of 16 per clock per SM at the sampled SM clock).
+
+Launch: `python bench.py [--gpus N --steps K --warmup W]`. With N > 1 and no torchrun
+environment, bench.py starts itself under torch.distributed.run with N local ranks; every
+rank runs the same per-GPU workload (replicas: weak scaling, no collective on the data path)
+and the time is the max over ranks.
 `--impl reference` times the float64 CPU oracle (the only reference this path has).
 """
 from __future__ import annotations
@@ -26,7 +32,9 @@ import hashlib
 import json
 import math
 import os
+import socket
 import statistics
+import subprocess
 import sys
 import threading
 import time
@@ -83,7 +91,7 @@ def recorded_traffic(kernel: str):
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML every ~10 ms while running."""
+    """Samples SM clock and throttle reasons through NVML every ~2 ms while running."""
 
     REASONS = {
         0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
@@ -116,7 +124,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(0.002)
 
     def __enter__(self):
         if self._ok:
@@ -132,8 +140,11 @@ class ClockSampler:
     def summary(self):
         if not self._ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        bins = {}
+        for mhz in self.samples:
+            bins[str(int(mhz) // 15 * 15)] = bins.get(str(int(mhz) // 15 * 15), 0) + 1
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "mhz_bins_15": bins}
 
 
 def dist_info():
@@ -303,6 +314,10 @@ def run_ours(args):
     d2h = hosts[0][0].numel() * hosts[0][0].element_size() + hosts[0][1].numel() * 4
     del sets[1:]
 
+    # the other legs run under a second clock sampler (their timings use its median clock)
+    legs_sampler = ClockSampler(device.index)
+    legs_sampler.__enter__()
+
     # ---- the backward pass of the same problem (recomputation from the saved LSE)
     backward = run_backward_leg(fa, device, stream, q, k, v, out, lse, causal, args.warmup, rank)
 
@@ -314,8 +329,15 @@ def run_ours(args):
     padding = run_padding_hbm_leg(fa, device, stream, 20)
     del qp, kp, vp, hosts
 
+    # ---- every workload of the pages, each against its own roofline
+    main_clocks = sampler.summary()
+    mhz = main_clocks.get("sm_mhz") or main_clocks.get("sm_max_mhz") or 1965.0
+    configs = run_configs_leg(fa, device, stream, args.warmup, float(mhz), ms_local, varlen)
+    legs_sampler.__exit__()
+
     peak_burst, peak_bw, peak_kind, peak_sust = load_peaks()
-    clocks = sampler.summary()
+    clocks = main_clocks
+    clocks["other_legs"] = legs_sampler.summary()
     timed_ms = ms_local * args.steps
     long_region = timed_ms > BURST_WINDOW_MS or "sw_power_cap" in clocks.get("reasons", [])
     peak_tf = peak_sust if long_region else peak_burst
@@ -339,6 +361,7 @@ def run_ours(args):
                      "frac_vs_sustained": round(kernel_tflops / peak_sust, 4),
                      "kernel": "fa_fwd_kernel<128,bf16,causal>",
                      "traffic": recorded_traffic("fa_fwd_kernel_d128_bf16_causal")},
+        "configs": configs,
         "varlen": varlen,
         "paged": paged,
         "backward": backward,
@@ -433,8 +456,13 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
     ku, vu, ou = torch.empty_like(qu), torch.empty_like(qu), torch.empty_like(qu)
     lse = torch.empty((H, case.nnz), device=device, dtype=torch.float32)
     out_pad = torch.empty_like(qp)
-    # L2 flush buffer (2x L2) written between timed calls: the inputs here are L2-sized
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    # L2 flush between timed calls (the inputs here are L2-sized): a reduction READS a 2x-L2
+    # buffer, so L2 is left holding clean lines and no timed kernel pays for write-backs.
+    flush = torch.ones(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    flush_out = torch.empty((), dtype=torch.int64, device=device)
+
+    def flush_l2():
+        torch.sum(flush, dtype=torch.int64, out=flush_out)
 
     def call():
         fa.fa_unpad_qkv(qp, kp, vp, idx, outs=(qu, ku, vu), stream=stream)
@@ -450,8 +478,8 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
     for it in range(iters):
         # keep the GPU busy while the host queues the whole call, so the events time the
         # kernels and not the host's launch gaps
+        flush_l2()
         torch.cuda._sleep(400000)
-        flush.fill_(it & 0xFF)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
         ev[0].record(stream)
         fa.fa_unpad_qkv(qp, kp, vp, idx, outs=(qu, ku, vu), stream=stream)
@@ -468,8 +496,8 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
     # the same path as one launch (unpad and pad folded into the attention kernel)
     fused = []
     for it in range(iters):
+        flush_l2()
         torch.cuda._sleep(400000)
-        flush.fill_(it & 0xFF)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         fa.fa_varlen_fwd_padded(qp, kp, vp, idx, cu, case.max_seqlen, out=out_pad, lse=lse, stream=stream)
@@ -480,7 +508,8 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
     us = statistics.median(fused)
     us3 = statistics.median(whole)
     return {"value": round(us, 2), "unit": "us/call",
-            "stat": f"median of {iters}, L2 flushed before each call, launches queued ahead (GPU time)",
+            "stat": f"median of {iters}, L2 flushed before each call by reading a 256 MiB buffer (no dirty "
+                    f"lines left), launches queued ahead (GPU time)",
             "config": "32 seqs x 64 tokens, H=16 D=128 bf16, padded (1,4096,16,128), non-causal; "
                       "fa_varlen_fwd_padded (unpad + attention + pad in one launch)",
             "gpu_launches_per_call": 1,
@@ -524,6 +553,79 @@ def run_padding_hbm_leg(fa, device, stream, iters):
         res[name] = {"us": round(us, 2), "bytes": nbytes, "achieved_gbs": round(gbs, 1), "peak_gbs": peak_bw,
                      "frac": round(gbs / peak_bw, 4), "peak_kind": f"{peak_kind} HBM copy"}
     res["config"] = "(1, 262144, 16, 128) bf16 padded (1 GiB), 131072 valid rows; inputs larger than L2"
+    return res
+
+
+# MUFU exp2 throughput of one SM per clock (sm_100, measured by a probe kernel: 16 results per
+# clock for ex2.approx.f32 and for the packed f16x2 / bf16x2 forms alike).
+MUFU_EXP2_PER_CLK_SM = 16
+NUM_SMS = 148
+
+
+def attention_exps(B: int, H: int, S: int, causal: bool) -> float:
+    """One exp2 per visible score: S*S per (batch, head), S*(S+1)/2 when causal."""
+    return float(B * H * (S * (S + 1) // 2 if causal else S * S))
+
+
+def config_roofline(flops: float, exps: float, seconds: float, peak_tf: float, sm_mhz: float) -> dict:
+    """Tensor time (FLOPs / peak) against exp time (exps / MUFU rate at the sampled clock): the
+    larger is the bound; frac = that bound's time / the measured time."""
+    t_mma = flops / (peak_tf * 1e12)
+    t_exp = exps / (MUFU_EXP2_PER_CLK_SM * NUM_SMS * sm_mhz * 1e6)
+    bound = "tensor" if t_mma >= t_exp else "exp (MUFU)"
+    return {"bound": bound, "t_mma_us": round(t_mma * 1e6, 1), "t_exp_us": round(t_exp * 1e6, 1),
+            "frac": round(max(t_mma, t_exp) / seconds, 4), "mufu_clock_mhz": round(sm_mhz, 0)}
+
+
+def run_configs_leg(fa, device, stream, warmup, sm_mhz, main_ms, varlen):
+    """Every workload of the pages on this GPU. Dense ones: fa_fwd, 20 launches after warm-up
+    (the small fp16 case: 200 back-to-back calls, microseconds per call); inputs are larger
+    than L2 except for the small case, whose point is the per-call latency."""
+    peak_burst, peak_bw, _, _ = load_peaks()
+    res = {}
+    for name in ("dense_fp16_small", "vit_bf16", "llm_causal_bf16", "hdim_sweep_fp16_d32", "hdim_sweep_fp16_d64",
+                 "hdim_sweep_fp16_d128", "hdim_sweep_fp16_d256"):
+        w = fa_inputs.WORKLOADS[name]
+        B, S, H, D, causal = w["B"], w["S"], w["H"], w["D"], w["causal"]
+        flops = fa.attention_flops(B, H, S, S, D, causal)
+        exps = attention_exps(B, H, S, causal)
+        entry = {"shape": f"B{B} H{H} S{S} D{D} {w['dtype']}{' causal' if causal else ''}"}
+        if name == "llm_causal_bf16":
+            ms = main_ms  # the main timed region above
+            entry["source"] = "main timed region"
+        else:
+            q, k, v = (t.to(device) for t in fa_inputs.dense_qkv(B, S, H, D, fa_inputs.DTYPES[w["dtype"]], seed=0))
+            out = torch.empty_like(q)
+            lse = torch.empty((B, H, S), device=device, dtype=torch.float32)
+            n = 200 if name == "dense_fp16_small" else 20
+            for _ in range(max(warmup, 3)):
+                fa.fa_fwd(q, k, v, out=out, lse=lse, causal=causal, stream=stream)
+            torch.cuda.synchronize(device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                fa.fa_fwd(q, k, v, out=out, lse=lse, causal=causal, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            ms = e0.elapsed_time(e1) / n
+            entry["launches"] = n
+            del q, k, v, out, lse
+        entry["ms"] = round(ms, 4)
+        entry["tflops"] = round(flops / (ms * 1e-3) / 1e12, 1)
+        if name == "dense_fp16_small":
+            entry["us_per_call"] = round(ms * 1e3, 2)
+            entry["bound"] = "launch latency (8.4 MFLOP per call; the pages' small case)"
+        else:
+            entry.update(config_roofline(flops, exps, ms * 1e-3, peak_burst, sm_mhz))
+        res[name] = entry
+    v = varlen
+    res["varlen_bf16_32x64"] = {"shape": "32 x 64 tokens, H16 D128 bf16, padded (1, 4096, 16, 128)",
+                                "us_per_call": v["value"], "path": "fa_varlen_fwd_padded (one launch)",
+                                "three_launch_us_per_call": v["three_launch_path"]["value"],
+                                "bound": "latency (the inputs sit in L2); see varlen"}
+    st, where = fa.fa_device_status(stream=stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} at {where} after the configs leg")
     return res
 
 
@@ -589,6 +691,46 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+def launch_local_ranks(n: int) -> int:
+    """Runs this script again under torch.distributed.run with n local ranks (one per GPU, every
+    rank on the same workload) and returns its exit code; rank 0 prints the JSON line."""
+    sk = socket.socket()
+    sk.bind(("127.0.0.1", 0))
+    port = sk.getsockname()[1]
+    sk.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
+def run_cpu_stub(args):
+    """The N-rank plumbing without a GPU: CPU ranks over gloo, each step a small CPU matmul,
+    the time the max over ranks. A test of the launcher and the rank logic, not a measurement."""
+    import datetime
+
+    import torch.distributed as dist
+    ws, rank, _ = dist_info()
+    if ws > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    a = torch.randn(128, 128)
+    for _ in range(args.warmup):
+        a @ a
+    if ws > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        a @ a
+    ms = max_over_ranks((time.perf_counter() - t0) / args.steps * 1e3, ws, torch.device("cpu"))
+    if ws > 1:
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "value": None, "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
+                          "warmup": args.warmup, "ms_per_step": round(ms, 4), "scaling": "weak",
+                          "stub": "CPU ranks over gloo: a test of the launcher, not a measurement"}), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -601,10 +743,16 @@ def main():
     ap.add_argument("--only-backward", action="store_true", help="run the backward leg only (for profiling)")
     ap.add_argument("--all-configs", action="store_true",
                     help="print one informational line per workload (dense/causal/head-dim sweep)")
+    ap.add_argument("--cpu-stub", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # N GPUs of this node: one process per GPU under torch.distributed.run
+        sys.exit(launch_local_ranks(args.gpus))
+    if args.cpu_stub:
+        run_cpu_stub(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.all_configs:
         run_all_configs(args)

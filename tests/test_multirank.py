@@ -53,3 +53,21 @@ def test_single_rank_defaults(monkeypatch):
         monkeypatch.delenv(k, raising=False)
     assert bench.dist_info() == (1, 0, 0)
     assert bench.max_over_ranks(3.25, 1, torch.device("cpu")) == 3.25
+
+
+def test_bench_launches_n_ranks_on_cpu():
+    """`bench.py --gpus 2` (no torchrun environment) starts itself under torch.distributed.run
+    with two ranks; the gloo stand-in for the GPU step checks the launcher and the rank logic."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR",
+                                                             "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--cpu-stub", "--steps", "3",
+                        "--warmup", "3"], capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    rec = json.loads(lines[0])
+    assert rec["n_gpus"] == 2 and rec["steps"] == 3 and rec["scaling"] == "weak"

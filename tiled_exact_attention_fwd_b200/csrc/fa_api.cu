@@ -138,6 +138,7 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     const int rows = fa::fwd_tile_rows();
     dim3 grid;
     p.batch = num_seqs;
+    p.out_align32 = (reinterpret_cast<uintptr_t>(out) % 32) == 0;
     p.npairs = 0;
     p.num_items = 0;
     if (cu_seqlens) {

@@ -28,8 +28,9 @@
 //          K_j and S_{j+2}. K and V stream through separate rings (three K slots: K_j is read
 //          from S_j until dQ's update two steps later; two V slots).
 // Warps 0-7 do the elementwise work (two threads per TMEM lane = row, each on half of the
-// columns), warp 8 lane 0 issues the TMA loads, warp 9 allocates TMEM and lane 0 issues
-// every MMA. Every wait is bounded.
+// columns), warp 8 lane 0 issues the TMA loads, warp 9 allocates TMEM and issues every MMA
+// (the whole warp runs the loop and waits; elect.sync picks the lane that issues each MMA and
+// commit). Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -119,7 +120,7 @@ __device__ __forceinline__ void mma_rows_step(uint32_t d_tmem, const uint8_t *a,
     for (int k = 0; k < D / 16; ++k) {
         const uint32_t blk = (k * 32) / C::SW, off = (k * 32) % C::SW;
         const uint32_t o = (blk * C::BM * C::SW + off) >> 4;
-        umma_ss_w(d_tmem, a_lo + o, b_lo + o, hi, idesc, k > 0 ? 1u : 0u);
+        umma_ss_elect(d_tmem, a_lo + o, b_lo + o, hi, idesc, k > 0 ? 1u : 0u);
     }
 }
 
@@ -137,8 +138,8 @@ __device__ __forceinline__ void mma_acc_step(uint32_t d_tmem, uint32_t a_tmem, c
     const uint32_t b_lo = smem_desc_lo(smem_u32(b) + u * STEP * C::SW, C::BM * C::SW);
 #pragma unroll
     for (int k = 0; k < STEP / 16; ++k)
-        umma_ts_w(d_tmem, a_tmem + k * 8 + (k >= STEP / 32 ? STEP / 4 : 0), b_lo + ((k * 16 * C::SW) >> 4), hi, idesc,
-                  (accumulate || k > 0) ? 1u : 0u);
+        umma_ts_elect(d_tmem, a_tmem + k * 8 + (k >= STEP / 32 ? STEP / 4 : 0), b_lo + ((k * 16 * C::SW) >> 4), hi,
+                      idesc, (accumulate || k > 0) ? 1u : 0u);
 }
 
 template <bool BF16>
@@ -333,8 +334,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
     } else if (warp == C::WARP_MMA) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && n > 0) {
-            ok = wait_bounded(fix_full, 0, abort_flag, lim, 410);
+        // (every wait below is taken by the whole warp: __all_sync keeps its control flow converged)
+        auto wait_all = [&](uint64_t *bar, uint32_t ph, int where) {
+            return __all_sync(0xffffffffu, wait_bounded(bar, ph, abort_flag, lim, where));
+        };
+        if (n > 0) {
+            ok = wait_all(fix_full, 0, 410);
             if (ok) tc_fence_after_sync();
             if constexpr (DKDV) {
                 // Half-step k: streamed tile t = k / 2, rows [64 u, 64 u + 64) with u = k % 2,
@@ -346,26 +351,26 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 auto issue_sdp = [&](int k) -> bool {
                     const int t = k / Kd::PER_TILE, u = k % Kd::PER_TILE, s = t & 1;
                     if (u == 0) {
-                        if (!wait_bounded(&ring_full[s], (t >> 1) & 1, abort_flag, lim, 420 + s)) return false;
+                        if (!wait_all(&ring_full[s], (t >> 1) & 1, 420 + s)) return false;
                         tc_fence_after_sync();
                     }
                     const uint32_t buf = tmem + (k & 1) * 128;
                     mma_rows_step<D, BF16, Kd::STEP>(buf, fixA0, ring_tile(s, 0), u);             // S^T
                     mma_rows_step<D, BF16, Kd::STEP>(buf + Kd::STEP, fixA1, ring_tile(s, 1), u);  // dP^T
-                    umma_commit(&s_full[k & 1]);
+                    umma_commit_elect(&s_full[k & 1]);
                     return true;
                 };
                 if (ok) ok = issue_sdp(0);
                 for (int k = 0; ok && k < nk; ++k) {
                     if (k + 1 < nk && !(ok = issue_sdp(k + 1))) break;
-                    if (!(ok = wait_bounded(&p_ready[k & 1], (k >> 1) & 1, abort_flag, lim, 430 + (k & 1)))) break;
+                    if (!(ok = wait_all(&p_ready[k & 1], (k >> 1) & 1, 430 + (k & 1)))) break;
                     tc_fence_after_sync();
                     const int t = k / Kd::PER_TILE, u = k % Kd::PER_TILE, s = t & 1;
                     const uint32_t buf = tmem + (k & 1) * 128;
                     mma_acc_step<D, BF16, Kd::STEP>(tmem + Kd::COL_ACC0, buf, ring_tile(s, 1), u, k > 0);  // dV += P^T dO
                     mma_acc_step<D, BF16, Kd::STEP>(tmem + Kd::COL_ACC1, buf + Kd::STEP, ring_tile(s, 0), u,
                                                     k > 0);                                        // dK += dZ^T Q
-                    if (u == Kd::PER_TILE - 1) umma_commit(&ring_empty[s]);  // both halves of tile t have read it
+                    if (u == Kd::PER_TILE - 1) umma_commit_elect(&ring_empty[s]);  // both halves of tile t have read it
                 }
             } else {
                 // Step t: S_t in TMEM buffer t % 2, dP_t in its own columns. Issue order:
@@ -373,34 +378,34 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // dP_{t+1}, dQ += dZ_t K_t, S_{t+2} (into buffer t % 2, after dQ has read dZ_t).
                 auto issue_s = [&](int t) -> bool {
                     const int ks = t % Kd::K_SLOTS;
-                    if (!wait_bounded(&k_full[ks], (t / Kd::K_SLOTS) & 1, abort_flag, lim, 420 + ks)) return false;
+                    if (!wait_all(&k_full[ks], (t / Kd::K_SLOTS) & 1, 420 + ks)) return false;
                     tc_fence_after_sync();
                     mma_rows_step<D, BF16, 128>(tmem + (t & 1) * 128, fixA0, k_tile(ks), 0);  // S = Q K^T
                     return true;
                 };
                 auto issue_dp = [&](int t) -> bool {
                     const int vs = t & 1;
-                    if (!wait_bounded(&v_full[vs], (t >> 1) & 1, abort_flag, lim, 424 + vs)) return false;
+                    if (!wait_all(&v_full[vs], (t >> 1) & 1, 424 + vs)) return false;
                     tc_fence_after_sync();
                     mma_rows_step<D, BF16, 128>(tmem + Kd::COL_DP_DQ, fixA1, v_tile(vs), 0);  // dP = dO V^T
-                    umma_commit(&v_empty[vs]);
-                    umma_commit(s_full);  // step t's S and dP are done
+                    umma_commit_elect(&v_empty[vs]);
+                    umma_commit_elect(s_full);  // step t's S and dP are done
                     return true;
                 };
                 if (ok) ok = issue_s(0) && issue_dp(0);
                 if (ok && n > 1) ok = issue_s(1);
                 for (int t = 0; ok && t < n; ++t) {
-                    if (!(ok = wait_bounded(p_ready, t & 1, abort_flag, lim, 430))) break;
+                    if (!(ok = wait_all(p_ready, t & 1, 430))) break;
                     tc_fence_after_sync();
                     if (t + 1 < n && !(ok = issue_dp(t + 1))) break;
                     mma_acc_step<D, BF16, 128>(tmem + Kd::COL_ACC0, tmem + (t & 1) * 128, k_tile(t % Kd::K_SLOTS), 0,
                                                t > 0);  // dQ += dZ K
-                    umma_commit(&k_empty[t % Kd::K_SLOTS]);
+                    umma_commit_elect(&k_empty[t % Kd::K_SLOTS]);
                     if (t + 2 < n && !(ok = issue_s(t + 2))) break;
                 }
             }
-            if (ok) umma_commit(done);
-            umma_commit(drain);  // every MMA issued above has finished once this arrives
+            if (ok) umma_commit_elect(done);
+            umma_commit_elect(drain);  // every MMA issued above has finished once this arrives
             const uint64_t g0 = global_timer_ns();
             while (!mbar_try_wait(drain, 0) && global_timer_ns() - g0 < lim) {
             }

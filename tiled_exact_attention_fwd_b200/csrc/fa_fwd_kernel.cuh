@@ -110,8 +110,6 @@ struct Cfg {
                   "register split");
     static_assert(!SPLIT_REGS || 128 * regs_low(false) + 256 * regs_high(false) <= NUM_THREADS * LAUNCH_REGS,
                   "register split");
-    // Column pairs (out of every 4) whose exp2 runs on the FMA pipe instead of MUFU.
-    static constexpr int EMU_PAIRS_OF_4 = 0;
     // shared memory map (offsets from a 1024-byte aligned base)
     static constexpr int SMEM_LIMIT = 227 * 1024;
     static constexpr int RESERVED = 1024 /*alignment*/ + 512 /*barriers, misc*/;
@@ -150,31 +148,6 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return BF16 ? pack2_bf16(lo, hi) : pack2_f16(lo, hi);
 }
 
-// 2^x for a pair of scores, evaluated on the FMA pipe instead of the MUFU unit. Cody-Waite
-// style reduction x = n + f with n = round(x) taken from the 1.5*2^23 shifter and f in
-// [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted with the Remez algorithm for minimax
-// relative error (7.5e-5, below the 2^-11 rounding of the 16-bit P it feeds;
-// gen_exp2_poly.py); 2^n is added to the exponent field. The float arithmetic runs two
-// lanes at a time (add/fma .f32x2). Inputs below -126 are clamped (the result is then ~1e-38
-// instead of a smaller number, irrelevant next to the row sum, which is at least 1); it is
-// only used on tiles without masked (-inf) scores.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float &y1) {
-    constexpr float c3 = 5.517166853e-02f, c2 = 2.426111251e-01f, c1 = 6.932609677e-01f, c0 = 9.999280572e-01f;
-    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-    const uint64_t x2 = f2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-    const uint64_t t2 = fadd2(x2, f2(kShift, kShift));
-    const uint64_t n2 = fadd2(t2, f2(-kShift, -kShift));
-    const uint64_t r2 = ffma2(n2, f2(-1.0f, -1.0f), x2);  // x - n, exact
-    uint64_t p2 = ffma2(f2(c3, c3), r2, f2(c2, c2));
-    p2 = ffma2(p2, r2, f2(c1, c1));
-    p2 = ffma2(p2, r2, f2(c0, c0));
-    float t0, t1, p0, p1;
-    f2_split(t2, t0, t1);
-    f2_split(p2, p0, p1);
-    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 // Maximum of an S row held in registers: 8 independent chains of three-input maxima.
 template <int BN>
 __device__ __forceinline__ float row_max(const uint32_t *sr) {
@@ -189,10 +162,10 @@ __device__ __forceinline__ float row_max(const uint32_t *sr) {
 }
 
 // For each 64-column chunk of an S row (in registers): p = 2^(s*c + neg_m) (scaling done two
-// lanes at a time with fma.f32x2), row sum in four fp32x2 partial sums, pairs packed to
-// 16 bits and the chunk stored to TMEM at p_addr. Of every 4 column pairs, EMU use
-// exp2_poly, the rest the MUFU ex2. Returns the row sum of this tile.
-template <int BN, bool BF16, int EMU>
+// lanes at a time with fma.f32x2, exp2 on the MUFU unit), row sum in four fp32x2 partial sums,
+// pairs packed to 16 bits and the chunk stored to TMEM at p_addr. Returns the row sum of this
+// tile.
+template <int BN, bool BF16>
 __device__ __forceinline__ float softmax_chunk_store(const uint32_t *sr, float c, float neg_m, uint32_t p_addr) {
     const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
     uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
@@ -205,13 +178,7 @@ __device__ __forceinline__ float softmax_chunk_store(const uint32_t *sr, float c
             const uint64_t x2 = ffma2(f2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, nm2);
             float x0, x1;
             f2_split(x2, x0, x1);
-            float p0, p1;
-            if ((i & 3) >= 4 - EMU) {
-                exp2_poly2(x0, x1, p0, p1);
-            } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-            }
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             acc[i & 3] = fadd2(acc[i & 3], f2(p0, p1));
             pk[i] = pack2<BF16>(p0, p1);
         }
@@ -225,7 +192,7 @@ __device__ __forceinline__ float softmax_chunk_store(const uint32_t *sr, float c
 
 // A whole S row (in registers) to packed 16-bit P in registers pk[BN/2]:
 // p = 2^(s*c + neg_m), scaling two lanes at a time; returns the row sum.
-template <int BN, bool BF16, int EMU>
+template <int BN, bool BF16>
 __device__ __forceinline__ float softmax_row_to_regs(const uint32_t *sr, float c, float neg_m, uint32_t *pk) {
     const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
     uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
@@ -234,13 +201,7 @@ __device__ __forceinline__ float softmax_row_to_regs(const uint32_t *sr, float c
         const uint64_t x2 = ffma2(f2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, nm2);
         float x0, x1;
         f2_split(x2, x0, x1);
-        float p0, p1;
-        if ((i & 3) >= 4 - EMU) {
-            exp2_poly2(x0, x1, p0, p1);
-        } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-        }
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
         acc[i & 3] = fadd2(acc[i & 3], f2(p0, p1));
         pk[i] = pack2<BF16>(p0, p1);
     }
@@ -1164,8 +1125,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     uint32_t pk[BN / 2];
                     // a packed row may not have met any visible key yet (m = -inf): its P is 0
                     const float neg_m = (m == -INFINITY) ? 0.f : -m;
-                    const float rs = need_mask ? softmax_row_to_regs<BN, BF16, 0>(sr, sc, neg_m, pk)
-                                               : softmax_row_to_regs<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, pk);
+                    const float rs = softmax_row_to_regs<BN, BF16>(sr, sc, neg_m, pk);  // -inf -> exactly 0
                     l = fmaf(l, alpha, rs);
                     if (jj > 0) {
                         if (!__all_sync(0xffffffffu,
@@ -1235,9 +1195,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     // a packed row may not have met any visible key yet (m = -inf): its P is 0
                     const float neg_m = (m == -INFINITY) ? 0.f : -m;
                     const uint32_t p_addr = c.tmem + lane_base + b * BN;
-                    const float rs = need_mask
-                                         ? softmax_chunk_store<BN, BF16, 0>(sr, sc, neg_m, p_addr)  // -inf -> exactly 0
-                                         : softmax_chunk_store<BN, BF16, C::EMU_PAIRS_OF_4>(sr, sc, neg_m, p_addr);
+                    const float rs = softmax_chunk_store<BN, BF16>(sr, sc, neg_m, p_addr);  // -inf -> exactly 0
                     l = fmaf(l, alpha, rs);
                     tmem_st_wait();
                     if (jj > 0) {
@@ -1291,24 +1249,37 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const float inv_l = 1.f / l;
             constexpr int RB = D * 2;  // bytes of one row of one head
             if (persistent) {
-                // Each thread writes its own row straight from registers (16-byte stores): the
-                // tile's query buffer may already hold the next item's Q.
+                // Each thread writes its own row straight from registers: the tile's query buffer
+                // may already hold the next item's Q. Up to 128 columns of O come out of TMEM per
+                // wait, and each lane stores 32 bytes at a time (whole sectors) when out allows.
                 uint8_t *const orow = static_cast<uint8_t *>(p.out) + (otok * p.H + eh) * RB;
+                constexpr int CW = (C::MAXQ == 1) ? 64 : (D < 128 ? D : 128);  // O columns per TMEM wave
 #pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t o[32];
-                    tmem_ld32(c.tmem + lane_base + o_col + cc * 32, o);
-                    tmem_ld_wait();
-                    tmem_reg_fence<32>(o);
-                    uint32_t w[16];
+                for (int c0 = 0; c0 < D; c0 += CW) {
+                    uint32_t o[CW];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
+                    for (int cc = 0; cc < CW / 32; ++cc) tmem_ld32(c.tmem + lane_base + o_col + c0 + cc * 32, o + cc * 32);
+                    tmem_ld_wait();
+                    tmem_reg_fence<CW>(o);
+                    uint32_t w[CW / 2];
+#pragma unroll
+                    for (int i = 0; i < CW / 2; ++i)
                         w[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
                     if (orow_ok) {
+                        if (p.out_align32) {
 #pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4)
-                            *reinterpret_cast<uint4 *>(orow + cc * 64 + v4 * 16) =
-                                make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                            for (int v = 0; v < CW / 16; ++v)
+                                asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                                                 orow + c0 * 2 + v * 32),
+                                             "r"(w[8 * v]), "r"(w[8 * v + 1]), "r"(w[8 * v + 2]), "r"(w[8 * v + 3]),
+                                             "r"(w[8 * v + 4]), "r"(w[8 * v + 5]), "r"(w[8 * v + 6]), "r"(w[8 * v + 7])
+                                             : "memory");
+                        } else {
+#pragma unroll
+                            for (int v4 = 0; v4 < CW / 8; ++v4)
+                                *reinterpret_cast<uint4 *>(orow + c0 * 2 + v4 * 16) =
+                                    make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                        }
                     }
                 }
             } else {

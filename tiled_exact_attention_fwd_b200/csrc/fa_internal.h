@@ -33,6 +33,7 @@ struct FwdParams {
     // Dense inputs (persistent grid): batch entries, groups of fwd_tiles_per_cta(D) query tiles
     // per sequence, and work items batch * H * npairs.
     int batch, npairs, num_items;
+    int out_align32;  // out is 32-byte aligned (the persistent epilogue then stores 32 bytes per lane)
 };
 
 // Attention forward. Dense: a persistent grid of min(num_items, SMs) CTAs; a work item is

@@ -174,57 +174,13 @@ __device__ __forceinline__ void tc_fence_after_sync() {
 }
 
 // ------------------------------------------------------------------ tcgen05: MMA
-// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (fp16/bf16 in, fp32 accumulate).
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem desc]; A is K-major in TMEM (row m in lane m, two
-// 16-bit elements per 32-bit column).
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrive once on `bar` when every tcgen05 operation this thread issued so far completes.
-// The same two MMAs with each 64-bit shared-memory descriptor given as its low and high
-// 32-bit words (see smem_desc_lo / smem_desc_hi): a k-step then changes one 32-bit add.
-__device__ __forceinline__ void umma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-        "mov.b64 da, {%1, %3};\n\t"
-        "mov.b64 db, {%2, %3};\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void umma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
-                                          uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
-        "mov.b64 db, {%2, %3};\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// The same MMAs and commit for a whole warp in converged control flow: elect.sync picks one
-// lane to issue, so the loop around them (waits, descriptor arithmetic) stays warp-uniform
-// and its values can live in uniform registers, which the tensor-core instructions read.
+// D[tmem] (+)= A * B, kind::f16 (fp16/bf16 in, fp32 accumulate), issued by a whole warp in
+// converged control flow: elect.sync picks one lane to issue, so the loop around the MMAs
+// (waits, descriptor arithmetic) stays warp-uniform and its values can live in uniform
+// registers, which the tensor-core instructions read. Each 64-bit shared-memory descriptor is
+// given as its low and high 32-bit words (see smem_desc_lo / smem_desc_hi): a k-step then
+// changes one 32-bit add.
+// A from shared memory (descriptor words a_lo/hi), B from shared memory (b_lo/hi).
 __device__ __forceinline__ void umma_ss_elect(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc,
                                           uint32_t accumulate) {
     asm volatile(
@@ -237,6 +193,8 @@ __device__ __forceinline__ void umma_ss_elect(uint32_t d_tmem, uint32_t a_lo, ui
         "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// A from TMEM (K-major: row m in lane m, two 16-bit elements per 32-bit column), B from
+// shared memory.
 __device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
                                           uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -248,17 +206,12 @@ __device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, 
         "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// Arrive once on `bar` when every tcgen05 operation the electing lane issued so far completes.
 __device__ __forceinline__ void umma_commit_elect(uint64_t *bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\t"
         "elect.sync rx|e, 0xffffffff;\n\t"
         "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             smem_u32(bar))
         : "memory");
 }
@@ -319,29 +272,19 @@ __device__ __forceinline__ void tmem_reg_fence(uint32_t *r) {
 }
 
 // ------------------------------------------------------------------ UMMA descriptors
-// Shared-memory matrix descriptor (sm_100 layout): start address, leading and stride
-// byte offsets (all >> 4), version 1 at bits 46-47, swizzle mode at bits 61-63.
+// Swizzle modes of a shared-memory matrix descriptor (bits 61-63).
 enum : uint32_t { kLayoutSw128 = 2, kLayoutSw64 = 4, kLayoutSw32 = 6 };
 
-// Low / high 32-bit words of smem_desc(saddr, lbo_bytes, sbo_bytes, layout). The address
-// field is the low 14 bits: adding (offset >> 4) to the low word moves the start address
-// as long as saddr + offset stays below 2^18 bytes (always true for shared memory).
+// Low / high 32-bit words of a shared-memory matrix descriptor (sm_100 layout): start address,
+// leading and stride byte offsets (all >> 4), version 1 at bits 46-47, swizzle mode at bits
+// 61-63. The address field is the low 14 bits: adding (offset >> 4) to the low word moves the
+// start address as long as saddr + offset stays below 2^18 bytes (always true for shared
+// memory).
 __device__ __forceinline__ uint32_t smem_desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
     return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
 }
 __host__ __device__ constexpr uint32_t smem_desc_hi(uint32_t sbo_bytes, uint32_t layout) {
     return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | ((layout & 0x7u) << 29);
-}
-
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes,
-                                              uint32_t sbo_bytes, uint32_t layout) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-    d |= static_cast<uint64_t>(1) << 46;
-    d |= static_cast<uint64_t>(layout & 0x7u) << 61;
-    return d;
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, A and B both fp16 or both bf16,
