@@ -462,7 +462,7 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
     flush_out = torch.empty((), dtype=torch.int64, device=device)
 
     def flush_l2():
-        torch.sum(flush, dtype=torch.int64, out=flush_out)
+        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_out)
 
     def call():
         fa.fa_unpad_qkv(qp, kp, vp, idx, outs=(qu, ku, vu), stream=stream)
@@ -524,21 +524,26 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
 def run_padding_hbm_leg(fa, device, stream, iters):
     """unpad / pad GB/s on the packed structure scaled past L2: (1, 262144, 16, 128) bf16 = 1 GiB
     padded, half the positions valid. Algorithmic bytes: unpad reads and writes nnz rows plus the
-    indices; pad reads nnz rows and the indices and writes every one of the total rows."""
+    indices; pad reads nnz rows and the indices and writes every one of the total rows; unpad_qkv
+    gathers the same rows from three distinct 1 GiB tensors in one launch."""
     _, peak_bw, peak_kind, _ = load_peaks()
     L, H, D = 262144, 16, 128
     nnz = L // 2
     g = torch.Generator(device="cpu")
     g.manual_seed(5)
     x = torch.randn((1, L, H, D), generator=g, dtype=torch.float32).to(torch.bfloat16).to(device)
+    xk, xv = torch.empty_like(x).copy_(x), torch.empty_like(x).copy_(x)  # distinct buffers for the q, k, v gather
     idx = fa_inputs.valid_indices(L, nnz, seed=6).to(device)
     u = torch.empty((nnz, H, D), device=device, dtype=torch.bfloat16)
+    uk, uv = torch.empty_like(u), torch.empty_like(u)
     out = torch.empty_like(x)
     row = H * D * 2
     res = {}
     for name, fn, nbytes in (
             ("unpad", lambda: fa.fa_unpad(x, idx, out=u, stream=stream), 2 * nnz * row + 8 * nnz),
-            ("pad", lambda: fa.fa_pad(u, idx, 1, L, out=out, stream=stream), nnz * row + L * row + 8 * nnz)):
+            ("pad", lambda: fa.fa_pad(u, idx, 1, L, out=out, stream=stream), nnz * row + L * row + 8 * nnz),
+            ("unpad_qkv", lambda: fa.fa_unpad_qkv(x, xk, xv, idx, outs=(u, uk, uv), stream=stream),
+             3 * 2 * nnz * row + 8 * nnz)):
         for _ in range(3):
             fn()
         torch.cuda.synchronize(device)
@@ -552,7 +557,8 @@ def run_padding_hbm_leg(fa, device, stream, iters):
         gbs = nbytes / (us * 1e-6) / 1e9
         res[name] = {"us": round(us, 2), "bytes": nbytes, "achieved_gbs": round(gbs, 1), "peak_gbs": peak_bw,
                      "frac": round(gbs / peak_bw, 4), "peak_kind": f"{peak_kind} HBM copy"}
-    res["config"] = "(1, 262144, 16, 128) bf16 padded (1 GiB), 131072 valid rows; inputs larger than L2"
+    res["config"] = ("(1, 262144, 16, 128) bf16 padded (1 GiB; three of them for unpad_qkv), 131072 valid rows; "
+                     "inputs larger than L2")
     return res
 
 
