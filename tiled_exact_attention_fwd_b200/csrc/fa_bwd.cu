@@ -168,7 +168,10 @@ __device__ __forceinline__ void store_row(uint32_t taddr, float mul, uint8_t *gr
     }
 }
 
-// DKDV: the CTA owns key tile j = blockIdx.y; fixed A0 = K_j, A1 = V_j; ring B0 = Q_i, B1 = dO_i.
+// Heads per group in the order the backward CTAs are dealt out (see fa_bwd_kernel).
+constexpr int BWD_HEAD_GROUP = 8;
+
+// DKDV: the CTA owns key tile j; fixed A0 = K_j, A1 = V_j; ring B0 = Q_i, B1 = dO_i.
 // !DKDV: the CTA owns query tile i (longest first); fixed A0 = Q_i, A1 = dO_i; ring B0 = K_j, B1 = V_j.
 // PACKED: (total, H, D) tensors with cu_seqlens; tiles are 128 consecutive tokens whatever
 // sequences they hold (p.B = 1, p.seqlen = total), the streamed windows cover the tokens of
@@ -181,9 +184,21 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     using C = BwdCfg<D>;
     using Kd = BwdKind<D, DKDV>;
     constexpr int BM = C::BM;
-    const int h = blockIdx.x, b = blockIdx.z, S = p.seqlen;  // packed: S = total tokens
+    const int b = blockIdx.z, S = p.seqlen;  // packed: S = total tokens
     const int ntiles = (S + BM - 1) / BM;
-    const int own = (DKDV || PACKED) ? static_cast<int>(blockIdx.y) : ntiles - 1 - static_cast<int>(blockIdx.y);
+    // Blocks start in linear order (x fastest), so the (head, tile) pairs are dealt in groups of
+    // BWD_HEAD_GROUP heads, tile by tile inside a group (longest work first): the CTAs resident at
+    // a time stream the tensors of a few heads, which then stay in L2, instead of those of all.
+    int h, tile;
+    {
+        const int lin = static_cast<int>(blockIdx.x) + p.H * static_cast<int>(blockIdx.y);
+        const int g0 = (lin / (BWD_HEAD_GROUP * ntiles)) * BWD_HEAD_GROUP;  // first head of the group
+        const int gsize = min(BWD_HEAD_GROUP, p.H - g0);
+        const int idx = lin - g0 * ntiles;
+        tile = idx / gsize;
+        h = g0 + idx % gsize;
+    }
+    const int own = (DKDV || PACKED) ? tile : ntiles - 1 - tile;
     const int own_start = own * BM;  // position of the owned tile's first row
     // Streamed windows t = 0..n-1 start at positions ws + t*BM.
     int ws, n;
