@@ -1,8 +1,9 @@
 """The dense forward's persistent grid (one CTA per SM running several work items) against the
 float64 oracle, on shapes chosen to stress it (needs a B200): many more items than SMs, items
 whose second query tile is absent (an odd number of 128-row tiles) mixed with full ones in the
-same CTA, every head dim, causal and not, paged K/V, and an output buffer that is 16- but not
-32-byte aligned (the epilogue's narrower store path)."""
+same CTA, every head dim, causal and not, paged K/V, an output buffer that is 16- but not
+32-byte aligned (the epilogue's narrower store path), and causal problems large enough that
+the items are dealt in groups of heads."""
 import numpy as np
 import pytest
 import torch
@@ -73,3 +74,31 @@ def test_output_16_byte_aligned(causal):
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
     assert bool((buf[:8] == 7.0).all()) and bool((buf[8 + n:] == 7.0).all())
+
+
+@pytest.mark.parametrize("B,H", [(1, 36), (2, 18)])
+def test_head_groups_match_single_heads(B, H):
+    """Causal S8192 D128 with 36 (batch entry, head) pairs: their K/V (144 MB) exceeds what the
+    kernel keeps in L2, so the items are dealt in groups of heads (8, 8, 8, 8 and a partial 4,
+    crossing batch entries when B = 2). Each pair's output and LSE must equal, bit for bit, those
+    of a call on that pair alone (one group); rows of one pair are checked against the oracle."""
+    S, D, dtype = 8192, 128, torch.bfloat16
+    dev = torch.device("cuda:0")
+    q, k, v = (t.to(dev) for t in fa_inputs.dense_qkv(B, S, H, D, dtype, seed=5))
+    out, lse = fa.fa_fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    for bh in [0, 7, 8, 15, 16, 31, 32, 35]:
+        b, h = divmod(bh, H)
+        qs, ks, vs = (t[b:b + 1, :, h:h + 1].contiguous() for t in (q, k, v))
+        o1, l1 = fa.fa_fwd(qs, ks, vs, causal=True)
+        torch.cuda.synchronize()
+        assert torch.equal(out[b:b + 1, :, h:h + 1], o1), f"output of pair {bh}"
+        assert torch.equal(lse[b:b + 1, h:h + 1], l1), f"LSE of pair {bh}"
+    # one pair's rows against the oracle (that head alone, float64 on the CPU)
+    b, h = divmod(33, H)
+    qh, kh, vh = (t[b:b + 1, :, h:h + 1].cpu() for t in (q, k, v))
+    idx = np.array([0, 1, 127, 128, 4095, 8000, 8191])
+    rows = np.stack([np.zeros_like(idx), np.zeros_like(idx), idx], axis=1)
+    O, L = oracle.attention_dense(qh, kh, vh, causal=True, rows=rows)
+    assert_o_close(out[b, idx, h].cpu(), O, dtype, "sampled rows")
+    assert_lse_close(lse[b, h, idx].cpu(), L, "sampled rows")

@@ -141,6 +141,7 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     p.out_align32 = (reinterpret_cast<uintptr_t>(out) % 32) == 0;
     p.npairs = 0;
     p.num_items = 0;
+    p.head_group = p.num_groups = p.group_rounds = 0;
     if (cu_seqlens) {
         // packed: one CTA per tiles_per_cta x 128 consecutive tokens of the packed tensor
         const int64_t span = static_cast<int64_t>(rows) * fa::fwd_tiles_per_cta(D);
@@ -156,6 +157,21 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
         const int sms = sm_count();
         if (sms <= 0) return FA_ERR_CUDA;
         grid = dim3(static_cast<unsigned>(p.num_items < sms ? p.num_items : sms), 1, 1);
+        // Causal items run longest first across all heads; when the K/V of all (batch entry,
+        // head) pairs exceeds 64 MB (half of L2), they are dealt in groups of heads whose K/V
+        // takes ~32 MB, each group at least 1.5 rounds of the grid (so the rounds stay balanced).
+        const int bh = num_seqs * H, G = static_cast<int>(grid.x);
+        int hg = bh;
+        const double per_bh = static_cast<double>(seqlen) * D * 4.0;  // K and V bytes of one pair
+        if (causal && per_bh * bh > 64.0 * 1024 * 1024) {
+            hg = static_cast<int>(32.0 * 1024 * 1024 / per_bh);
+            if (hg < 1) hg = 1;
+            while (hg < bh && 2LL * hg * p.npairs < 3LL * G) hg *= 2;
+            if (hg > bh) hg = bh;
+        }
+        p.head_group = hg;
+        p.num_groups = (bh + hg - 1) / hg;
+        p.group_rounds = static_cast<int>((static_cast<int64_t>(hg) * p.npairs + G - 1) / G);
     }
     const cudaError_t e = paging ? fa::launch_fwd_paged(D, bf16, causal != 0, tq, tk, tv, p, grid,
                                                         static_cast<cudaStream_t>(stream))

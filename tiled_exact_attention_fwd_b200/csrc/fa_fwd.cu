@@ -24,8 +24,10 @@ static cudaError_t launch_c(bool causal, const CUtensorMap &tq, const CUtensorMa
     if (p.cu_seqlens)
         return causal ? launch_t<D, BF16, true, false, true>(tq, tk, tv, p, grid, st)
                       : launch_t<D, BF16, false, false, true>(tq, tk, tv, p, grid, st);
-    return causal ? launch_t<D, BF16, true, false, false>(tq, tk, tv, p, grid, st)
-                  : launch_t<D, BF16, false, false, false>(tq, tk, tv, p, grid, st);
+    if (causal)
+        return p.num_groups > 1 ? launch_t<D, BF16, true, false, false, true>(tq, tk, tv, p, grid, st)
+                                : launch_t<D, BF16, true, false, false>(tq, tk, tv, p, grid, st);
+    return launch_t<D, BF16, false, false, false>(tq, tk, tv, p, grid, st);
 }
 
 template <int D>

@@ -257,21 +257,50 @@ struct Cta {
     }
 };
 
-// The dense work items: (batch entry, head, group of MAXQ query tiles), B*H*npairs in all. Causal
-// items are ordered longest first (query-tile group descending); otherwise the groups of one
-// (batch entry, head) are consecutive, so CTAs that run at the same time share its K/V in L2.
-template <int D, bool CAUSAL>
-__device__ __forceinline__ void set_dense_item(Cta<D> &c, const FwdParams &p, int w) {
-    using C = Cfg<D>;
-    const int bh_count = p.batch * p.H;
-    int pair, bh;
-    if (CAUSAL) {
-        pair = p.npairs - 1 - w / bh_count;
-        bh = w % bh_count;
-    } else {
-        pair = w % p.npairs;
-        bh = w / p.npairs;
+// The dense work items: (batch entry, head, group of MAXQ query tiles), B*H*npairs in all, dealt
+// to the G CTAs in rounds of one item each. The (batch entry, head) pairs form p.num_groups groups
+// of p.head_group, each taking p.group_rounds rounds. Inside a group, causal items go longest
+// first (query-tile group descending, all heads of the group at each step) and non-causal ones
+// head by head (the groups of one head consecutive, so CTAs running together share its K/V in
+// L2). Each round runs forward or backward over the CTAs (a snake, so that with longest-first
+// items every CTA gets a similar total), and each group starts the snake a quarter of the grid
+// further on. Returns false when CTA `cta` has no item in round rd. GROUPED: more than one group
+// (a separate instantiation: the single-group arithmetic, which every role runs at every item,
+// stays as short as it can be).
+template <bool CAUSAL, bool GROUPED>
+__device__ __forceinline__ bool dense_item_at(const FwdParams &p, int rd, int G, int cta, int &pair, int &bh) {
+    if (!GROUPED) {
+        const int w = rd * G + ((rd & 1) ? G - 1 - cta : cta);
+        if (w >= p.num_items) return false;
+        if (CAUSAL) {
+            const int bhc = p.batch * p.H, q = w / bhc;
+            pair = p.npairs - 1 - q;
+            bh = w - q * bhc;
+        } else {
+            bh = w / p.npairs;
+            pair = w - bh * p.npairs;
+        }
+        return true;
     }
+    const int g = rd / p.group_rounds, r = rd - g * p.group_rounds;
+    const int g0 = g * p.head_group;
+    const int gb = min(p.head_group, p.batch * p.H - g0);  // pairs in this group
+    const int slot = (cta + g * (G / 4)) % G;
+    const int within = r * G + ((r & 1) ? G - 1 - slot : slot);
+    if (within >= gb * p.npairs) return false;
+    if (CAUSAL) {
+        pair = p.npairs - 1 - within / gb;
+        bh = g0 + within % gb;
+    } else {
+        pair = within % p.npairs;
+        bh = g0 + within / p.npairs;
+    }
+    return true;
+}
+
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void set_dense_item(Cta<D> &c, const FwdParams &p, int pair, int bh) {
+    using C = Cfg<D>;
     c.b = bh / p.H;
     c.h = bh % p.H;
     c.seqlen = p.seqlen;
@@ -287,14 +316,10 @@ __device__ __forceinline__ void set_dense_item(Cta<D> &c, const FwdParams &p, in
     c.jB0 = 0;
 }
 
-// Work item of round r for CTA `cta` of G: a snake over the item order (forward in even rounds,
-// backward in odd ones), so that with longest-first items every CTA gets a similar total.
-__device__ __forceinline__ int item_of_round(int r, int G, int cta) { return r * G + ((r & 1) ? G - 1 - cta : cta); }
-
 // Head, batch entry, first query position and first query token of this CTA's item at round r
 // (which must exist), derived afresh: packed inputs from the block index, dense ones as
-// set_dense_item does. Keeps these out of the registers that live through an item's key steps.
-template <int D, bool CAUSAL>
+// dense_item_at does. Keeps these out of the registers that live through an item's key steps.
+template <int D, bool CAUSAL, bool GROUPED>
 __device__ __forceinline__ void item_coords(const FwdParams &p, int r, bool persistent, int &h, int &b, int &q0,
                                             int &qbase) {
     using C = Cfg<D>;
@@ -305,10 +330,8 @@ __device__ __forceinline__ void item_coords(const FwdParams &p, int r, bool pers
         qbase = blockIdx.y * C::MAXQ * C::BM;
         return;
     }
-    const int w = item_of_round(r, gridDim.x, blockIdx.x);
-    const int bh_count = p.batch * p.H;
-    const int pair = CAUSAL ? p.npairs - 1 - w / bh_count : w % p.npairs;
-    const int bh = CAUSAL ? w % bh_count : w / p.npairs;
+    int pair = 0, bh = 0;
+    dense_item_at<CAUSAL, GROUPED>(p, r, gridDim.x, blockIdx.x, pair, bh);
     b = bh / p.H;
     h = bh % p.H;
     q0 = pair * C::MAXQ * C::BM;
@@ -318,18 +341,19 @@ __device__ __forceinline__ void item_coords(const FwdParams &p, int r, bool pers
 // Moves to this CTA's next work item at round r or later (r is advanced past rounds without
 // one); false once there is none. Packed inputs: the one item set up front, at round 0. Called
 // again with the same r it sets the same item.
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool GROUPED>
 __device__ __forceinline__ bool next_item(Cta<D> &c, const FwdParams &p, int &r, bool persistent) {
     if (!persistent) return r == 0;
     const int G = gridDim.x, cta = blockIdx.x;
-    for (;; ++r) {
-        if (r * G >= p.num_items) return false;
-        const int w = item_of_round(r, G, cta);
-        if (w < p.num_items) {
-            set_dense_item<D, CAUSAL>(c, p, w);
+    const int rounds = p.num_groups * p.group_rounds;
+    for (; r < rounds; ++r) {
+        int pair, bh;
+        if (dense_item_at<CAUSAL, GROUPED>(p, r, G, cta, pair, bh)) {
+            set_dense_item<D, CAUSAL>(c, p, pair, bh);
             return true;
         }
     }
+    return false;
 }
 
 // S_t = Q_t K_j^T for key tile j (tile-local step jj = j - j0(t)); after the tile's last QK of
@@ -498,11 +522,11 @@ __device__ __forceinline__ void fetch_group(uint8_t *tile, int rows, int g, int6
 // the other's loops.
 //
 // Dense inputs run persistently: the grid has one CTA per SM (at most one per work item), and
-// each CTA takes its work items in rounds (item_of_round). Every role loops over the same items;
+// each CTA takes its work items in rounds (dense_item_at). Every role loops over the same items;
 // the producer loads an item's Q tiles as soon as the previous item's QKs on them are done, so
 // the next item's loads and first QKs overlap the current item's last steps and epilogue.
 // Packed inputs launch one CTA per 256 consecutive tokens (one item per CTA).
-template <int D, bool BF16, bool CAUSAL, bool PAGED, bool PACKED>
+template <int D, bool BF16, bool CAUSAL, bool PAGED, bool PACKED, bool GROUPED>
 __global__ void __launch_bounds__(Cfg<D>::NUM_THREADS, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -510,6 +534,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
 
     static_assert(!(PAGED && PACKED), "paged K/V is for dense queries");
+    static_assert(!GROUPED || (CAUSAL && !PACKED), "head groups order dense causal items");
     constexpr bool packed = PACKED;  // the host launches PACKED exactly when p.cu_seqlens is set
     constexpr bool persistent = !packed;
     Cta<D> c;
@@ -568,7 +593,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // been read, never held up behind the other tile's PV (which waits for that tile's P).
     const bool split_issue = c.dec && !c.fused;
     // Every role runs `for (int rd = 0; next_item(...); ++rd) { ...; c.advance(); }` over this
-    // CTA's work items (dense: the rounds of item_of_round; packed: the one item set above),
+    // CTA's work items (dense: the rounds of dense_item_at; packed: the one item set above),
     // leaving the loop early when a wait gives up.
 
     extern __shared__ uint8_t smem_raw[];
@@ -686,7 +711,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     if (lane == 0) {
                         const int box = min(p.page_size, BN);
                         bool ok = true;
-                        for (int rd = 0; ok && next_item<D, CAUSAL>(c, p, rd, persistent); ++rd) {
+                        for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED>(c, p, rd, persistent); ++rd) {
                             ok = load_q(0);
                             const int loads = c.loads();
                             for (int L = 0; ok && L < loads; ++L) {
@@ -725,7 +750,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     constexpr int CPR = C::NBLK * CPB;  // 16-byte chunks per V row
                     const int w = pw - 1;                // copy warp 0, 1
                     bool ok = true;
-                    for (int rd = 0; ok && next_item<D, CAUSAL>(c, p, rd, persistent); ++rd) {
+                    for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED>(c, p, rd, persistent); ++rd) {
                         const int loads = c.loads();
                         for (int L = 0; L < loads; ++L) {
                             const int U = c.u0 + L, stage = U % NS;
@@ -872,7 +897,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 issued = 0;
             } else if (lane == 0) {
                 bool ok = true;
-                for (int rd = 0; ok && next_item<D, CAUSAL>(c, p, rd, persistent); ++rd) {
+                for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED>(c, p, rd, persistent); ++rd) {
                     ok = load_q(0);
                     const int loads = c.loads();
                     for (int L = 0; ok && L < loads; ++L) {
@@ -986,7 +1011,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             bool ok = true;
             const bool qk = !split_issue || warp == C::WARP_MMA;
             const bool pv = !split_issue || warp != C::WARP_MMA;
-            for (int rd = 0; ok && next_item<D, CAUSAL>(c, p, rd, persistent); ++rd) {
+            for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED>(c, p, rd, persistent); ++rd) {
                 const int nl = max(c.nA, c.nB);  // key tiles of the item
                 if (c.single) {
                     const int n = c.nA;
@@ -1046,7 +1071,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // steps (the softmax warps are at their register limit there); the item is looked up
         // again for the epilogue.
         int gbase = 0;
-        for (int rd = 0; ok && next_item<D, CAUSAL>(c, p, rd, persistent); ++rd) {
+        for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED>(c, p, rd, persistent); ++rd) {
             const int n = c.steps(t);  // key tiles this warpgroup visits in the item
             if (n <= 0) continue;      // tile absent
             const int j0 = c.j0(t);
@@ -1243,7 +1268,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tc_fence_after_sync();
             // the item's coordinates again, computed afresh rather than carried through the key steps
             int eh, eb, eq0, eqbase;
-            item_coords<D, CAUSAL>(p, rd, persistent, eh, eb, eq0, eqbase);
+            item_coords<D, CAUSAL, GROUPED>(p, rd, persistent, eh, eb, eq0, eqbase);
             const int64_t otok = static_cast<int64_t>(eqbase) + t * BM + r;
             const bool orow_ok = packed ? otok < p.total_tokens : (eq0 + t * BM + r < p.seqlen);
             const float inv_l = 1.f / l;
@@ -1344,11 +1369,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 }
 
 // ------------------------------------------------------------------ host launchers
-template <int D, bool BF16, bool CAUSAL, bool PAGED, bool PACKED>
+template <int D, bool BF16, bool CAUSAL, bool PAGED, bool PACKED, bool GROUPED = false>
 static cudaError_t launch_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             const FwdParams &p, dim3 grid, cudaStream_t st) {
     using C = Cfg<D>;
-    auto kern = fa_fwd_kernel<D, BF16, CAUSAL, PAGED, PACKED>;
+    auto kern = fa_fwd_kernel<D, BF16, CAUSAL, PAGED, PACKED, GROUPED>;
     // The shared-memory opt-in is a per-device function attribute; setting it twice is harmless.
     static uint64_t attr_set_mask = 0;
     int dev = 0;

@@ -7,8 +7,10 @@ namespace fa {
 template <int D, bool BF16>
 static cudaError_t launch_paged_c(bool causal, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const FwdParams &p, dim3 grid, cudaStream_t st) {
-    return causal ? launch_t<D, BF16, true, true, false>(tq, tk, tv, p, grid, st)
-                  : launch_t<D, BF16, false, true, false>(tq, tk, tv, p, grid, st);
+    if (causal)
+        return p.num_groups > 1 ? launch_t<D, BF16, true, true, false, true>(tq, tk, tv, p, grid, st)
+                                : launch_t<D, BF16, true, true, false>(tq, tk, tv, p, grid, st);
+    return launch_t<D, BF16, false, true, false>(tq, tk, tv, p, grid, st);
 }
 
 template <int D>

@@ -33,6 +33,10 @@ struct FwdParams {
     // Dense inputs (persistent grid): batch entries, groups of fwd_tiles_per_cta(D) query tiles
     // per sequence, and work items batch * H * npairs.
     int batch, npairs, num_items;
+    // The items are dealt in groups of head_group (batch entry, head) pairs (num_groups groups,
+    // group_rounds rounds of one item per CTA each), so that the CTAs running at a time read the
+    // K/V of a few heads; head_group = batch * H (one group) unless K/V would not fit in L2.
+    int head_group, num_groups, group_rounds;
     int out_align32;  // out is 32-byte aligned (the persistent epilogue then stores 32 bytes per lane)
 };
 
