@@ -615,6 +615,25 @@ def run_configs_leg(fa, device, stream, warmup, sm_mhz, main_ms, varlen):
             torch.cuda.synchronize(device)
             ms = e0.elapsed_time(e1) / n
             entry["launches"] = n
+            if name == "dense_fp16_small":
+                # The same n calls captured in one CUDA graph and replayed: the per-call time
+                # without the host's launch path (what a caller replaying a graph sees).
+                side = torch.cuda.Stream(device)
+                side.wait_stream(torch.cuda.current_stream(device))
+                with torch.cuda.stream(side):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=side):
+                        for _ in range(n):
+                            fa.fa_fwd(q, k, v, out=out, lse=lse, causal=causal)
+                torch.cuda.current_stream(device).wait_stream(side)
+                g.replay()
+                torch.cuda.synchronize(device)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                torch.cuda.synchronize(device)
+                entry["graph_us_per_call"] = round(e0.elapsed_time(e1) / n * 1e3, 2)
+                del g
             del q, k, v, out, lse
         entry["ms"] = round(ms, 4)
         entry["tflops"] = round(flops / (ms * 1e-3) / 1e12, 1)

@@ -13,6 +13,7 @@ built, every call raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from typing import Optional, Tuple
@@ -115,6 +116,14 @@ def _like(name: str, t: torch.Tensor, shape, dtype) -> None:
     _cuda_contig(name, t)
 
 
+def _on_device(t: torch.Tensor):
+    """The operands' device made current for the call (a no-op context when it already is, which
+    keeps the per-call host cost of small problems down)."""
+    if t.get_device() == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(t.device)
+
+
 def _same_device(ref: torch.Tensor, *ts: Optional[torch.Tensor]) -> None:
     for t in ts:
         if t is not None and t.device != ref.device:
@@ -138,7 +147,7 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torc
     if lse is not None:
         _like("lse", lse, (B, H, S), torch.float32)
     _same_device(q, k, v, out, lse)
-    with torch.cuda.device(q.device):
+    with _on_device(q):
         st = lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
                           float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
     _check(st, "fa_fwd")
@@ -171,7 +180,7 @@ def fa_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
         _like(n, t, q.shape, q.dtype)
     _like("delta", delta, (B, H, S), torch.float32)
     _same_device(q, k, v, out, dout, lse, dq, dk, dv, delta)
-    with torch.cuda.device(q.device):
+    with _on_device(q):
         st = lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                           _ptr(dv), _ptr(delta), B, H, S, D, float(scale) if scale else 0.0, int(bool(causal)),
                           _dtype_code(q), _stream(stream))
@@ -196,7 +205,7 @@ def fa_varlen_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     delta = torch.empty((H, total), device=q.device, dtype=torch.float32)
     _same_device(q, k, v, out, dout, lse, cu_seqlens)
-    with torch.cuda.device(q.device):
+    with _on_device(q):
         st = lib().fa_varlen_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(cu_seqlens),
                                  cu_seqlens.numel() - 1, int(max_seqlen), total, _ptr(dq), _ptr(dk), _ptr(dv),
                                  _ptr(delta), H, D, float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q),
@@ -222,7 +231,7 @@ def fa_bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch
         _cuda_contig(n, t)
     _same_device(q, k, v, out, dout, lse, dq, dk, dv)
     # the fixed buffer is looked up on the current device: make it q's
-    with torch.cuda.device(q.device):
+    with _on_device(q):
         st = lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq),
                                   _ptr(dk), _ptr(dv), B, H, S, D, float(scale) if scale else 0.0, int(bool(causal)),
                                   _dtype_code(q), _stream(stream))
@@ -260,7 +269,7 @@ def fa_fwd_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, 
     if lse is not None:
         _like("lse", lse, (B, H, S), torch.float32)
     _same_device(q, k_cache, v_cache, block_table, out, lse)
-    with torch.cuda.device(q.device):
+    with _on_device(q):
         st = lib().fa_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
                                 page_size, num_pages, _ptr(out), _ptr(lse), B, H, S, D,
                                 float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
@@ -288,7 +297,7 @@ def fa_varlen_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens:
     if lse is not None:
         _like("lse", lse, (H, total), torch.float32)
     _same_device(q, k, v, cu_seqlens, out, lse)
-    with torch.cuda.device(q.device):
+    with _on_device(q):
         st = lib().fa_varlen_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
                                  int(max_seqlen), total, _ptr(out), _ptr(lse), H, D,
                                  float(scale) if scale else 0.0, int(bool(causal)), _dtype_code(q), _stream(stream))
@@ -319,7 +328,7 @@ def fa_varlen_fwd_padded(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, indi
     if lse is not None:
         _like("lse", lse, (H, total), torch.float32)
     _same_device(q, k, v, indices, cu_seqlens, out, lse)
-    with torch.cuda.device(q.device):
+    with _on_device(q):
         st = lib().fa_varlen_fwd_padded(_ptr(q), _ptr(k), _ptr(v), _ptr(indices), _ptr(cu_seqlens),
                                         cu_seqlens.numel() - 1, int(max_seqlen), total, padded_rows, _ptr(out),
                                         _ptr(lse), H, D, float(scale) if scale else 0.0, int(bool(causal)),
@@ -343,7 +352,7 @@ def fa_unpad(x: torch.Tensor, indices: torch.Tensor, out: Optional[torch.Tensor]
         out = torch.empty((nnz, H, D), device=x.device, dtype=x.dtype)
     _like("out", out, (nnz, H, D), x.dtype)
     _same_device(x, indices, out)
-    with torch.cuda.device(x.device):
+    with _on_device(x):
         st = lib().fa_unpad(_ptr(x), _ptr(indices), nnz, total_rows, row_bytes, _ptr(out), _stream(stream))
     _check(st, "fa_unpad")
     return out
@@ -365,7 +374,7 @@ def fa_unpad_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, indices: tor
     for i, o in enumerate(outs):
         _like(f"outs[{i}]", o, (nnz, H, D), q.dtype)
     _same_device(q, k, v, indices, *outs)
-    with torch.cuda.device(q.device):
+    with _on_device(q):
         st = lib().fa_unpad_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(indices), nnz, q.numel() // (H * D),
                                 H * D * q.element_size(), _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]),
                                 _stream(stream))
@@ -387,7 +396,7 @@ def fa_pad(x: torch.Tensor, indices: torch.Tensor, batch: int, total_len: int,
         out = torch.empty((batch, total_len, H, D), device=x.device, dtype=x.dtype)
     _like("out", out, (batch, total_len, H, D), x.dtype)
     _same_device(x, indices, out)
-    with torch.cuda.device(x.device):
+    with _on_device(x):
         st = lib().fa_pad(_ptr(x), _ptr(indices), nnz, batch * total_len, H * D * x.element_size(), _ptr(out),
                           _stream(stream))
     _check(st, "fa_pad")
