@@ -105,10 +105,12 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     const int64_t map_rows = gather ? padded_rows : N;
     const int64_t kv_rows = paging ? static_cast<int64_t>(paging->num_pages) * paging->page_size : map_rows;
     const int q_box = gather ? fa::fwd_gather_run_rows() : fa::fwd_tile_rows();
+    // dense D = 256 runs in CTA pairs: each CTA loads 64 key rows of K_j and 128 columns of V_j
+    const bool pair = fa::fwd_pair_mode(D) && !paging && !cu_seqlens;
     const int k_box = paging ? fa::fwd_paged_k_box_rows(D, paging->page_size)
-                             : (gather ? fa::fwd_gather_run_rows() : fa::fwd_kv_tile_rows(D));
+                             : (gather ? fa::fwd_gather_run_rows() : (pair ? 64 : fa::fwd_kv_tile_rows(D)));
     const int v_box = paging ? fa::fwd_paged_v_box_rows(D, paging->page_size)
-                             : (gather ? fa::fwd_gather_run_rows() : fa::fwd_v_box_rows(D));
+                             : (gather ? fa::fwd_gather_run_rows() : (pair ? 128 : fa::fwd_v_box_rows(D)));
     if (!encode_map(&tq, q, bf16, D, H, map_rows, inner, q_box) ||
         !encode_map(&tk, k, bf16, D, H, kv_rows, inner, k_box) ||
         !encode_map(&tv, v, bf16, D, H, kv_rows, inner, v_box))
@@ -149,21 +151,26 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
     } else {
         // dense: persistent, one CTA per SM (at most one per work item)
         const int qtiles = (seqlen + rows - 1) / rows;
-        const int per_cta = fa::fwd_tiles_per_cta(D);
+        const int per_cta = pair ? 2 : fa::fwd_tiles_per_cta(D);  // query tiles per work item
         p.npairs = (qtiles + per_cta - 1) / per_cta;
         const int64_t items = static_cast<int64_t>(num_seqs) * H * p.npairs;
         if (items > INT32_MAX) return FA_ERR_SHAPE;
         p.num_items = static_cast<int>(items);
         const int sms = sm_count();
         if (sms <= 0) return FA_ERR_CUDA;
-        grid = dim3(static_cast<unsigned>(p.num_items < sms ? p.num_items : sms), 1, 1);
+        if (pair) {
+            const int clusters = sms / 2;  // CTA pairs: one cluster of two per two SMs
+            grid = dim3(2u * static_cast<unsigned>(p.num_items < clusters ? p.num_items : clusters), 1, 1);
+        } else {
+            grid = dim3(static_cast<unsigned>(p.num_items < sms ? p.num_items : sms), 1, 1);
+        }
         // Causal items run longest first across all heads; when the K/V of all (batch entry,
         // head) pairs exceeds 64 MB (half of L2), they are dealt in groups of heads whose K/V
         // takes ~32 MB, each group at least 1.5 rounds of the grid (so the rounds stay balanced).
-        const int bh = num_seqs * H, G = static_cast<int>(grid.x);
+        const int bh = num_seqs * H, G = static_cast<int>(pair ? grid.x / 2 : grid.x);
         int hg = bh;
         const double per_bh = static_cast<double>(seqlen) * D * 4.0;  // K and V bytes of one pair
-        if (causal && per_bh * bh > 64.0 * 1024 * 1024) {
+        if (causal && !pair && per_bh * bh > 64.0 * 1024 * 1024) {
             hg = static_cast<int>(32.0 * 1024 * 1024 / per_bh);
             if (hg < 1) hg = 1;
             while (hg < bh && 2LL * hg * p.npairs < 3LL * G) hg *= 2;

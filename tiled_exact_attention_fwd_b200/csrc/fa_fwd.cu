@@ -52,6 +52,8 @@ int fwd_tile_rows() { return 128; }
 
 int fwd_tiles_per_cta(int D) { return (D == 256) ? 1 : 2; }
 
+bool fwd_pair_mode(int D) { return D == 256; }
+
 int fwd_box_inner_elems(int D) { return (2 * D >= 128) ? 64 : D; }
 
 int fwd_kv_tile_rows(int D) { return 128; }

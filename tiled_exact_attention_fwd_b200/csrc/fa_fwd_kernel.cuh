@@ -118,8 +118,9 @@ struct Cfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = MAXQ * Q_BYTES;
     static constexpr int OFF_BAR = OFF_KV + NS * UNIT_BYTES;
-    // q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], drain, s_free[2], tail, q_free[2]
-    static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1 + 2 + 1 + 2;
+    // q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], drain, s_free[2], tail, q_free[2],
+    // q_peer, kv_peer[NS] (CTA pairs: the other CTA's copies have landed)
+    static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1 + 2 + 1 + 2 + 1 + NS;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // TMEM address, abort flag
     static constexpr int USED = OFF_MISC + 16;
     // More than half of the SM's shared memory, so exactly one CTA (and one 512-column
@@ -220,12 +221,15 @@ struct Cta {
     uint8_t *sQ, *sKV;
     uint64_t *q_full, *kv_full, *kv_empty, *s_full, *p_full, *pv_done, *drain, *s_free, *q_free;
     uint64_t *tail;  // paged K/V: the V part that straddles a sequence end lands here first
+    uint64_t *q_peer, *kv_peer;  // CTA pairs (CTA 0): the other CTA's Q tile / ring part has landed
     volatile int *abort_flag;
     uint32_t tmem;
     uint64_t lim;
     bool dec;     // separate P buffers (Cfg::DECOUPLED)
     bool single;  // one query tile per CTA (Cfg::MAXQ == 1): its S alternates between two buffers
     bool fused;   // Q/K/V tiles written by threads (cp.async), not TMA: fence before the MMA reads them
+    bool pair;    // one query tile in each CTA of a 2-CTA cluster, whose MMAs CTA 0 issues for both
+    uint32_t rank;  // rank of this CTA in its pair
     // The current work item: query tiles A (and B) of head h; their rows are tokens qbase + t*128
     // + r, keys are addressed from token kvbase. Dense: batch entry b, rows from position q0 of
     // the sequence that starts at token seq_start. Tile A visits key tiles [0, nA), tile B
@@ -244,7 +248,8 @@ struct Cta {
     __device__ __forceinline__ int j0(int t) const { return t ? jB0 : 0; }
     __device__ __forceinline__ int steps(int t) const { return t ? nB - jB0 : nA; }
     __device__ __forceinline__ bool uses(int t, int j) const { return t ? (j >= jB0 && j < nB) : (j < nA); }
-    __device__ __forceinline__ int loads() const { return 2 * max(nA, nB) * C::UNITS; }  // ring parts of the item
+    // ring parts of the item (CTA pairs: half of K_j, then half of V_j, one part each)
+    __device__ __forceinline__ int loads() const { return pair ? 2 * nA : 2 * max(nA, nB) * C::UNITS; }
     // S/P buffer of tile t at its running key step gs, and that buffer's barrier phase
     __device__ __forceinline__ int buf(int t, int gs) const { return single ? (gs & 1) : t; }
     __device__ __forceinline__ uint32_t sphase(int gs) const { return single ? ((gs >> 1) & 1) : (gs & 1); }
@@ -298,18 +303,21 @@ __device__ __forceinline__ bool dense_item_at(const FwdParams &p, int rd, int G,
     return true;
 }
 
-template <int D, bool CAUSAL>
+// PAIR: item `pair` is query tiles 2*pair (CTA 0) and 2*pair + 1 (CTA 1) of the head, run as
+// one 256-row tile; both CTAs visit the key tiles of the longer one (CTA 0's rows mask the
+// last one away when causal).
+template <int D, bool CAUSAL, bool PAIR = false>
 __device__ __forceinline__ void set_dense_item(Cta<D> &c, const FwdParams &p, int pair, int bh) {
     using C = Cfg<D>;
     c.b = bh / p.H;
     c.h = bh % p.H;
     c.seqlen = p.seqlen;
     c.seq_start = c.b * p.seqlen;
-    c.q0 = pair * C::MAXQ * C::BM;
+    c.q0 = PAIR ? (2 * pair + static_cast<int>(c.rank)) * C::BM : pair * C::MAXQ * C::BM;
     c.two = (C::MAXQ == 2) && (c.q0 + C::BM < p.seqlen);
     c.qbase = c.seq_start + c.q0;
     c.kvbase = c.seq_start;
-    const int end_a = CAUSAL ? min(p.seqlen, c.q0 + C::BM) : p.seqlen;
+    const int end_a = CAUSAL ? min(p.seqlen, (PAIR ? (2 * pair + 2) * C::BM : c.q0 + C::BM)) : p.seqlen;
     const int end_b = CAUSAL ? min(p.seqlen, c.q0 + 2 * C::BM) : p.seqlen;
     c.nA = (end_a + C::BN - 1) / C::BN;
     c.nB = c.two ? (end_b + C::BN - 1) / C::BN : 0;
@@ -319,7 +327,7 @@ __device__ __forceinline__ void set_dense_item(Cta<D> &c, const FwdParams &p, in
 // Head, batch entry, first query position and first query token of this CTA's item at round r
 // (which must exist), derived afresh: packed inputs from the block index, dense ones as
 // dense_item_at does. Keeps these out of the registers that live through an item's key steps.
-template <int D, bool CAUSAL, bool GROUPED>
+template <int D, bool CAUSAL, bool GROUPED, bool PAIR = false>
 __device__ __forceinline__ void item_coords(const FwdParams &p, int r, bool persistent, int &h, int &b, int &q0,
                                             int &qbase) {
     using C = Cfg<D>;
@@ -331,25 +339,30 @@ __device__ __forceinline__ void item_coords(const FwdParams &p, int r, bool pers
         return;
     }
     int pair = 0, bh = 0;
-    dense_item_at<CAUSAL, GROUPED>(p, r, gridDim.x, blockIdx.x, pair, bh);
+    if (PAIR)
+        dense_item_at<CAUSAL, GROUPED>(p, r, gridDim.x >> 1, blockIdx.x >> 1, pair, bh);
+    else
+        dense_item_at<CAUSAL, GROUPED>(p, r, gridDim.x, blockIdx.x, pair, bh);
     b = bh / p.H;
     h = bh % p.H;
-    q0 = pair * C::MAXQ * C::BM;
+    q0 = PAIR ? (2 * pair + static_cast<int>(cluster_ctarank())) * C::BM : pair * C::MAXQ * C::BM;
     qbase = b * p.seqlen + q0;
 }
 
 // Moves to this CTA's next work item at round r or later (r is advanced past rounds without
 // one); false once there is none. Packed inputs: the one item set up front, at round 0. Called
 // again with the same r it sets the same item.
-template <int D, bool CAUSAL, bool GROUPED>
+template <int D, bool CAUSAL, bool GROUPED, bool PAIR = false>
 __device__ __forceinline__ bool next_item(Cta<D> &c, const FwdParams &p, int &r, bool persistent) {
     if (!persistent) return r == 0;
-    const int G = gridDim.x, cta = blockIdx.x;
+    // pairs: the rounds deal items to the clusters of two CTAs
+    const int G = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+    const int cta = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     const int rounds = p.num_groups * p.group_rounds;
     for (; r < rounds; ++r) {
         int pair, bh;
         if (dense_item_at<CAUSAL, GROUPED>(p, r, G, cta, pair, bh)) {
-            set_dense_item<D, CAUSAL>(c, p, pair, bh);
+            set_dense_item<D, CAUSAL, PAIR>(c, p, pair, bh);
             return true;
         }
     }
@@ -458,6 +471,76 @@ __device__ __forceinline__ bool mma_pv(const Cta<D> &c, int t, int j, bool first
     return true;
 }
 
+// CTA pairs: a bounded wait taken by the whole MMA warp, cluster scope.
+template <int D>
+__device__ __forceinline__ bool pair_wait(const Cta<D> &c, uint64_t *bar, uint32_t parity, int where) {
+    return __all_sync(0xffffffffu, wait_bounded_cluster(bar, parity, c.abort_flag, c.lim, where));
+}
+// CTA pairs: arrive on `bar` (same offset) in both CTAs once the pair MMAs issued so far complete.
+__device__ __forceinline__ void pair_commit(uint64_t *bar) {
+    umma_commit_pair_elect(smem_u32(bar));
+    umma_commit_pair_elect(mapa_shared(bar, 1));
+}
+
+// CTA pairs, issued by CTA 0: S = Q K_j^T for the pair's 256 query rows (M = 256; CTA 0's query
+// tile is rows 0-127, CTA 1's rows 128-255; N = 128 keys, rows [0, 64) of key tile j in CTA 0's
+// ring part and [64, 128) in CTA 1's; K = D). The tile's S lands in each CTA's TMEM.
+template <int D, bool BF16>
+__device__ __forceinline__ bool mma_qk_pair(const Cta<D> &c, int j) {
+    using C = Cfg<D>;
+    constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
+    constexpr uint32_t idesc = idesc_f16(2 * BM, BN, BF16, false);
+    const int gs = c.g0(0) + j;
+    if (j == 0) {
+        if (!pair_wait(c, &c.q_full[0], c.nq(0) & 1, 200) || !pair_wait(c, c.q_peer, c.nq(0) & 1, 201)) return false;
+    }
+    const int U = c.u0 + 2 * j, stage = U % NS;  // ring part holding this CTA's half of K_j
+    if (!pair_wait(c, &c.kv_full[stage], (U / NS) & 1, 220 + stage) ||
+        !pair_wait(c, &c.kv_peer[stage], (U / NS) & 1, 230 + stage))
+        return false;
+    tc_fence_after_sync();
+    constexpr uint32_t dhi = smem_desc_hi(8 * SW, C::LAYOUT);
+    const uint32_t q_lo = smem_desc_lo(smem_u32(c.sQ), 16);
+    const uint32_t k_lo = smem_desc_lo(smem_u32(c.sKV + stage * C::UNIT_BYTES), 16);
+    const int b = gs & 1;  // S buffer
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+        const uint32_t blk = (k * 32) / SW, off = (k * 32) % SW;  // column block of 64, byte offset inside
+        umma_ss_pair_elect(c.tmem + b * BN, q_lo + ((blk * BM * SW + off) >> 4),
+                           k_lo + ((blk * (BN / 2) * SW + off) >> 4), dhi, idesc, k > 0 ? 1u : 0u);
+    }
+    pair_commit(&c.s_full[b]);
+    pair_commit(&c.kv_empty[stage]);
+    if (j == c.nA - 1) pair_commit(&c.q_free[0]);  // the Q tiles may be reloaded for the next item
+    return true;
+}
+
+// CTA pairs, issued by CTA 0: O += P V_j (M = 256, A = each CTA's P in its TMEM; N = D, columns
+// [0, 128) of V_j in CTA 0's ring part and [128, 256) in CTA 1's, MN-major; K = 128 keys).
+template <int D, bool BF16>
+__device__ __forceinline__ bool mma_pv_pair(const Cta<D> &c, int j) {
+    using C = Cfg<D>;
+    constexpr int BM = C::BM, BN = C::BN, SW = C::SW, NS = C::NS;
+    constexpr uint32_t idesc = idesc_f16(2 * BM, D, BF16, true);
+    const int gs = c.g0(0) + j;
+    const int b = gs & 1;
+    if (!pair_wait(c, &c.p_full[b], (gs >> 1) & 1, 210)) return false;
+    const int U = c.u0 + 2 * j + 1, stage = U % NS;  // ring part holding this CTA's half of V_j
+    if (!pair_wait(c, &c.kv_full[stage], (U / NS) & 1, 220 + stage) ||
+        !pair_wait(c, &c.kv_peer[stage], (U / NS) & 1, 230 + stage))
+        return false;
+    tc_fence_after_sync();
+    constexpr uint32_t dhi = smem_desc_hi(8 * SW, C::LAYOUT);
+    const uint32_t v_lo = smem_desc_lo(smem_u32(c.sKV + stage * C::UNIT_BYTES), BN * SW);
+#pragma unroll
+    for (int k = 0; k < BN / 16; ++k)
+        umma_ts_pair_elect(c.tmem + C::O_COL, c.tmem + b * BN + k * 8, v_lo + ((k * 16 * SW) >> 4), dhi, idesc,
+                           (j > 0 || k > 0) ? 1u : 0u);
+    pair_commit(&c.pv_done[0]);
+    pair_commit(&c.kv_empty[stage]);
+    return true;
+}
+
 // Fused packed path: padded rows of the 32-row groups g0 and g0 + 3 of a copy job over tokens
 // [tok0, tok0 + rows), one row per lane; rows past the job or the tokens, and indices outside
 // the padded tensor, read as row 0 (never outside q/k/v; the masks ignore such rows).
@@ -537,9 +620,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     static_assert(!GROUPED || (CAUSAL && !PACKED), "head groups order dense causal items");
     constexpr bool packed = PACKED;  // the host launches PACKED exactly when p.cu_seqlens is set
     constexpr bool persistent = !packed;
+    // Dense D = 256 runs in 2-CTA clusters (the host launches them so): the pair's two query tiles
+    // share every K/V tile, each CTA loading half of it, and CTA 0 issues M = 256 MMAs for both.
+    constexpr bool PAIR = (D == 256) && !PAGED && !PACKED;
     Cta<D> c;
     c.dec = C::DECOUPLED;
     c.single = C::MAXQ == 1;
+    c.pair = PAIR;
+    c.rank = PAIR ? cluster_ctarank() : 0u;
     c.u0 = 0;
     c.g0a = c.g0b = 0;
     c.nqa = c.nqb = 0;
@@ -612,6 +700,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     c.s_free = c.drain + 1;
     c.tail = c.s_free + 2;
     c.q_free = c.tail + 1;
+    c.q_peer = c.q_free + 2;
+    c.kv_peer = c.q_peer + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     c.abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     c.lim = p.timeout_ns;
@@ -633,7 +723,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int t = 0; t < 2; ++t) {
             mbar_init(&c.q_full[t], q_arrivals);
             mbar_init(&c.s_full[t], 1);
-            mbar_init(&c.p_full[t], 128);
+            mbar_init(&c.p_full[t], PAIR ? 256 : 128);  // pairs: CTA 0's barrier takes both CTAs' rows
             mbar_init(&c.pv_done[t], 1);
             mbar_init(&c.s_free[t], 4);  // one arrival per softmax warp
             mbar_init(&c.q_free[t], 1);
@@ -643,6 +733,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_init(&c.kv_empty[s], 1);
         }
         mbar_init(c.drain, split_issue ? 2 : 1);  // one commit per issuing warp
+        mbar_init(c.q_peer, 1);
+        for (int s = 0; s < NS; ++s) mbar_init(&c.kv_peer[s], 1);
         mbar_init(c.tail, 1);
         *c.abort_flag = 0;
         fence_mbar_init();
@@ -653,11 +745,17 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tma_prefetch_desc(&tm_v);
     }
     if (warp == C::WARP_MMA) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before_sync();
     __syncthreads();
+    if (PAIR) cluster_sync();  // both CTAs' barriers exist before either arrives on the other's
     tc_fence_after_sync();
     c.tmem = *tmem_slot;
 
@@ -711,7 +809,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     if (lane == 0) {
                         const int box = min(p.page_size, BN);
                         bool ok = true;
-                        for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED>(c, p, rd, persistent); ++rd) {
+                        for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
                             ok = load_q(0);
                             const int loads = c.loads();
                             for (int L = 0; ok && L < loads; ++L) {
@@ -750,7 +848,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     constexpr int CPR = C::NBLK * CPB;  // 16-byte chunks per V row
                     const int w = pw - 1;                // copy warp 0, 1
                     bool ok = true;
-                    for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED>(c, p, rd, persistent); ++rd) {
+                    for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
                         const int loads = c.loads();
                         for (int L = 0; L < loads; ++L) {
                             const int U = c.u0 + L, stage = U % NS;
@@ -895,9 +993,51 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
                 cp_async_wait_all();  // nothing of this thread is left in flight at exit
                 issued = 0;
+            } else if (PAIR && lane == 0) {
+                // CTA pairs: this CTA's query tile, then for each key tile j its half of K_j (key
+                // rows [64 * rank, +64), all of D) and its half of V_j (columns [128 * rank, +128)),
+                // each on this CTA's own barriers (CTA 1's reporter warp passes them on to CTA 0). The
+                // ring slots and Q buffer are released by CTA 0's MMA commits.
+                bool ok = true;
+                for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
+                    if (c.nq(0) > 0 && !wait_bounded_cluster(&c.q_free[0], (c.nq(0) - 1) & 1, c.abort_flag, c.lim, 110)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&c.q_full[0], C::Q_BYTES);
+#pragma unroll
+                    for (int b = 0; b < C::NBLK; ++b)
+                        tma_load_3d(c.sQ + b * BM * SW, &tm_q, &c.q_full[0], b * C::SWE, c.h, c.qbase, pol_q);
+                    q_issued_a = c.nq(0) + 1;
+                    const int loads = c.loads();
+                    for (int L = 0; ok && L < loads; ++L) {
+                        const int U = c.u0 + L, stage = U % NS, j = L >> 1;
+                        if (U >= NS && !wait_bounded_cluster(&c.kv_empty[stage], ((U / NS) - 1) & 1, c.abort_flag,
+                                                             c.lim, 100 + stage)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *dst = c.sKV + stage * C::UNIT_BYTES;
+                        mbar_arrive_expect_tx(&c.kv_full[stage], C::UNIT_BYTES);
+                        if (!(L & 1)) {
+#pragma unroll
+                            for (int b = 0; b < C::NBLK; ++b)
+                                tma_load_3d(dst + b * (BN / 2) * SW, &tm_k, &c.kv_full[stage], b * C::SWE, c.h,
+                                            c.kvbase + j * BN + static_cast<int>(c.rank) * (BN / 2), pol_kv);
+                        } else {
+#pragma unroll
+                            for (int b = 0; b < C::NBLK / 2; ++b)
+                                tma_load_3d(dst + b * BN * SW, &tm_v, &c.kv_full[stage],
+                                            (static_cast<int>(c.rank) * (C::NBLK / 2) + b) * C::SWE, c.h, c.kvbase + j * BN,
+                                            pol_kv);
+                        }
+                        issued = U + 1;
+                    }
+                    c.advance();
+                }
             } else if (lane == 0) {
                 bool ok = true;
-                for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED>(c, p, rd, persistent); ++rd) {
+                for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
                     ok = load_q(0);
                     const int loads = c.loads();
                     for (int L = 0; ok && L < loads; ++L) {
@@ -1006,12 +1146,50 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                 }
             }
+        } else if (PAIR && warp == C::WARP_MMA + 1 && c.rank == 1) {
+            // ------------------------------------------------------------ pair reporter (CTA 1)
+            // Each of this CTA's Q tiles and ring parts, once landed, is reported to CTA 0
+            // (q_peer, kv_peer), whose MMAs read it.
+            if (lane == 0) {
+                bool ok = true;
+                const uint32_t q_peer0 = mapa_shared(c.q_peer, 0);
+                for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
+                    if (!(ok = wait_bounded(&c.q_full[0], c.nq(0) & 1, c.abort_flag, c.lim, 120))) break;
+                    mbar_arrive_cluster(q_peer0);
+                    const int loads = c.loads();
+                    for (int L = 0; ok && L < loads; ++L) {
+                        const int U = c.u0 + L, stage = U % NS;
+                        if (!(ok = wait_bounded(&c.kv_full[stage], (U / NS) & 1, c.abort_flag, c.lim, 125))) break;
+                        mbar_arrive_cluster(mapa_shared(&c.kv_peer[stage], 0));
+                    }
+                    c.advance();
+                }
+            }
+        } else if (PAIR && warp == C::WARP_MMA) {
+            // ------------------------------------------------------------ pair MMA issuer (CTA 0)
+            bool ok = true;
+            if (c.rank == 0) {
+                for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
+                    const int n = c.nA;
+                    for (int idx = 0; ok && idx < 2 * n; ++idx) {
+                        bool is_v;
+                        int j;
+                        decode_step(idx, n, is_v, j);
+                        ok = is_v ? mma_pv_pair<D, BF16>(c, j) : mma_qk_pair<D, BF16>(c, j);
+                    }
+                    c.advance();
+                }
+                umma_commit_pair_elect(smem_u32(c.drain));
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(c.drain, 0) && global_timer_ns() - t0 < c.lim) {
+                }
+            }
         } else if (warp == C::WARP_MMA || (split_issue && warp == C::WARP_MMA + 1)) {
             // ------------------------------------------------------------ MMA issuer(s)
             bool ok = true;
             const bool qk = !split_issue || warp == C::WARP_MMA;
             const bool pv = !split_issue || warp != C::WARP_MMA;
-            for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED>(c, p, rd, persistent); ++rd) {
+            for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
                 const int nl = max(c.nA, c.nB);  // key tiles of the item
                 if (c.single) {
                     const int n = c.nA;
@@ -1060,6 +1238,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     } else {
         // ------------------------------------------------------------ softmax + epilogue
         if constexpr (C::SPLIT_REGS) regs_inc<C::regs_high(PACKED)>();
+        // pairs: S, P and O barriers are completed by CTA 0's MMA commits (cluster scope)
+        auto swait = [&](uint64_t *bar, uint32_t ph, int where) {
+            return PAIR ? wait_bounded_cluster(bar, ph, c.abort_flag, c.lim, where)
+                        : wait_bounded(bar, ph, c.abort_flag, c.lim, where);
+        };
         const int t = warp >> 2;                      // query tile of this warpgroup
         const int quarter = warp & 3;                 // TMEM lanes this warp may access
         const int r = quarter * 32 + lane;            // row of the tile == TMEM lane
@@ -1071,7 +1254,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // steps (the softmax warps are at their register limit there); the item is looked up
         // again for the epilogue.
         int gbase = 0;
-        for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED>(c, p, rd, persistent); ++rd) {
+        for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
             const int n = c.steps(t);  // key tiles this warpgroup visits in the item
             if (n <= 0) continue;      // tile absent
             const int j0 = c.j0(t);
@@ -1190,7 +1373,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const int gs = gbase + jj;  // running key step of this tile
                     const int b = c.buf(t, gs);
                     if (!__all_sync(0xffffffffu,
-                                    wait_bounded(&c.s_full[b], c.sphase(gs), c.abort_flag, c.lim, 300 + t))) {
+                                    swait(&c.s_full[b], c.sphase(gs), 300 + t))) {
                         ok = false;
                         break;
                     }
@@ -1230,8 +1413,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         // one tile QK(j) precedes PV(j-1): wait for it (on every step, so this thread
                         // never falls two phases behind on pv_done). The final wait after the loop
                         // always targets the newest phase, which is correct either way.
-                        if (c.single && !__all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (gs - 1) & 1,
-                                                                              c.abort_flag, c.lim, 310 + t))) {
+                        if (c.single && !__all_sync(0xffffffffu, swait(&c.pv_done[t], (gs - 1) & 1, 310 + t))) {
                             ok = false;
                             break;
                         }
@@ -1258,17 +1440,20 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         }
                     }
                     tc_fence_before_sync();
-                    mbar_arrive(&c.p_full[b]);
+                    if (PAIR && c.rank != 0)
+                        mbar_arrive_cluster(mapa_shared(&c.p_full[b], 0));  // CTA 0's MMA warp takes the pair's P
+                    else
+                        mbar_arrive(&c.p_full[b]);
                 }
             }
             if (ok)
-                ok = __all_sync(0xffffffffu, wait_bounded(&c.pv_done[t], (gbase + n - 1) & 1, c.abort_flag, c.lim, 320 + t));
+                ok = __all_sync(0xffffffffu, swait(&c.pv_done[t], (gbase + n - 1) & 1, 320 + t));
             if (!ok) break;
             gbase += n;
             tc_fence_after_sync();
             // the item's coordinates again, computed afresh rather than carried through the key steps
             int eh, eb, eq0, eqbase;
-            item_coords<D, CAUSAL, GROUPED>(p, rd, persistent, eh, eb, eq0, eqbase);
+            item_coords<D, CAUSAL, GROUPED, PAIR>(p, rd, persistent, eh, eb, eq0, eqbase);
             const int64_t otok = static_cast<int64_t>(eqbase) + t * BM + r;
             const bool orow_ok = packed ? otok < p.total_tokens : (eq0 + t * BM + r < p.seqlen);
             const float inv_l = 1.f / l;
@@ -1362,9 +1547,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (p.gather && warp < C::NUM_SOFTMAX_WARPS) cp_async_wait_all();  // the query copies (abort paths)
     tc_fence_before_sync();
     __syncthreads();
+    // pairs: neither CTA leaves (and frees shared memory or TMEM) while the other's MMAs, which
+    // read both CTAs' tiles, or its arrivals may still be running
+    if (PAIR) cluster_sync();
     if (warp == C::WARP_MMA) {
         tc_fence_after_sync();
-        tmem_dealloc(c.tmem, C::TMEM_COLS);
+        if (PAIR)
+            tmem_dealloc_pair(c.tmem, C::TMEM_COLS);
+        else
+            tmem_dealloc(c.tmem, C::TMEM_COLS);
     }
 }
 
@@ -1392,6 +1583,24 @@ static cudaError_t launch_t(const CUtensorMap &tq, const CUtensorMap &tk, const 
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         __atomic_fetch_or(&attr_set_mask, bit, __ATOMIC_RELEASE);
+    }
+    if constexpr (D == 256 && !PAGED && !PACKED) {
+        // CTA pairs: clusters of two CTAs along x (the grid is an even number of CTAs)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
     }
     kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
     return cudaGetLastError();

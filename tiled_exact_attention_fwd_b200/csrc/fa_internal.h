@@ -51,6 +51,9 @@ cudaError_t launch_fwd_paged(int D, bool bf16, bool causal, const CUtensorMap &t
                              const CUtensorMap &tv, const FwdParams &p, dim3 grid, cudaStream_t st);
 int fwd_tile_rows();
 int fwd_tiles_per_cta(int D);
+// Dense (not paged, not packed) inputs of head dim D run in 2-CTA clusters: each work item is two
+// consecutive query tiles, one per CTA, and the grid is twice the number of clusters.
+bool fwd_pair_mode(int D);
 int fwd_box_inner_elems(int D);
 int fwd_kv_tile_rows(int D);
 // Rows of one V box the producer copies (a V tile may move as several row parts).

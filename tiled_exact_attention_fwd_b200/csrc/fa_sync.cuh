@@ -37,6 +37,26 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
     }
 }
 
+// The same with cluster-scope acquire, for barriers that the other CTA of a pair (its threads
+// or its MMA commits) completes.
+__device__ __forceinline__ bool wait_bounded_cluster(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                     uint64_t limit_ns, int where) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+#pragma unroll 1
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((it & 31u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > limit_ns) {
+                *abort_flag = 1;
+                record_error(FA_ERR_TIMEOUT, where);
+                return false;
+            }
+        }
+    }
+}
+
 // Device addresses (on the current device) of this compilation unit's error word.
 static cudaError_t device_error_addrs(int **code, int **where) {
     cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(code), g_err_code);
