@@ -24,7 +24,7 @@
  *   packed q, k, v, out : (total, H, D)        lse : (H, total)  float32
  *   lse is the natural log of sum_j exp(scale * q.k_j) over the keys the row sees.
  *
- * Supported: D in {32, 64, 128, 256} (backward: 32, 64, 128); q, k, v, out 16-byte
+ * Supported: D in {32, 64, 128, 256} (forward and backward); q, k, v, out 16-byte
  * aligned; lse 4-byte aligned (may be NULL to skip it in the forward). Causal masking is
  * aligned at the first token of each sequence (query and key lengths are equal per
  * sequence). The header is plain C99.
@@ -109,8 +109,9 @@ FA_API fa_status fa_fwd_paged(const void *q, const void *k_cache, const void *v_
  *   delta          (B, H, S) float32 caller-owned workspace; on return it holds
  *                  rowsum(dout * out), the per-row term of the softmax derivative.
  *   scale          <= 0 selects 1/sqrt(D); must be the value the forward used.
- * D in {32, 64, 128} (the dK and dV accumulators of a 128-key tile share TMEM; D = 256 is
- * FA_ERR_HEADDIM). Three launches on `stream` (delta, dK/dV, dQ); nothing is allocated.
+ * D in {32, 64, 128, 256}. Launches on `stream`: delta, then dK/dV and dQ (D <= 128, where
+ * the dK and dV accumulators of a 128-key tile fit in TMEM side by side) or dV, dK and dQ
+ * (D = 256, one accumulator per kernel); nothing is allocated.
  */
 FA_API fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
                         const float *lse, void *dq, void *dk, void *dv, float *delta, int B, int H, int S,
@@ -124,7 +125,7 @@ FA_API fa_status fa_bwd(const void *q, const void *k, const void *v, const void 
  *   dq, dk, dv           (total, H, D) outputs; every element is written.
  *   delta                (H, total) float32 caller-owned workspace (rowsum(dout * out)).
  *   cu_seqlens, num_seqs, max_seqlen, total, scale, causal: as fa_varlen_fwd.
- * D in {32, 64, 128}. Work is split into tiles of 128 consecutive packed tokens whatever
+ * D in {32, 64, 128, 256}. Work is split into tiles of 128 consecutive packed tokens whatever
  * sequences they hold. total == 0 is a successful no-op.
  */
 FA_API fa_status fa_varlen_bwd(const void *q, const void *k, const void *v, const void *out,

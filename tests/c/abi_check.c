@@ -31,8 +31,8 @@ int main(void) {
            FA_ERR_SHAPE, "fa_varlen_fwd_padded total > padded_rows");
     expect(fa_fwd_paged(f, f, f, cu, 3, 24, 10, f, NULL, 2, 4, 130, 128, 0.f, 0, FA_BF16, NULL), FA_ERR_SHAPE,
            "fa_fwd_paged page 24");
-    expect(fa_bwd(f, f, f, f, f, lse, f, f, f, (float *)f, 1, 2, 128, 256, 0.f, 1, FA_BF16, NULL), FA_ERR_HEADDIM,
-           "fa_bwd D=256");
+    expect(fa_bwd(f, f, f, f, f, lse, f, f, f, (float *)f, 1, 2, 128, 96, 0.f, 1, FA_BF16, NULL), FA_ERR_HEADDIM,
+           "fa_bwd D=96");
     expect(fa_varlen_bwd(f, f, f, f, f, lse, cu, 3, 64, 0, f, f, f, (float *)f, 2, 64, 0.f, 1, FA_BF16, NULL), FA_OK,
            "fa_varlen_bwd empty");
     expect(fa_bwd_noalloc(f, f, f, f, f, lse, f, f, f, 1, 128, 131073, 128, 0.f, 1, FA_BF16, NULL), FA_ERR_SHAPE,

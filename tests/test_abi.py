@@ -141,7 +141,7 @@ def test_bwd_validation(lib):
 
     for i in range(10):
         assert call(i, None) == -1, i
-    assert call(13, 256) == -4   # dK and dV accumulators would not fit in TMEM
+    assert call(13, 48) == -4
     assert call(13, 96) == -4
     assert call(16, 3) == -3
     assert call(10, 0) == -2
@@ -164,7 +164,7 @@ def test_varlen_bwd_validation(lib):
 
     assert call(9, 0) == 0      # no tokens: nothing to do
     assert call(6, None) == -1
-    assert call(15, 256) == -4
+    assert call(15, 48) == -4
     assert call(8, 0) == -2
     assert call(6, FAKE + 2) == -5
     assert call(18, 4) == -3

@@ -43,7 +43,7 @@ def _run(B, S, H, D, dtype, causal, seed, dev):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("D", [32, 64, 128])
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("causal", [False, True])
 def test_bwd_matches_oracle(cuda_device, D, dtype, causal):
@@ -62,6 +62,30 @@ def test_bwd_edge_lengths(cuda_device, S):
     rq, rk, rv = oracle.attention_backward(q, k, v, do, causal=True)
     for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
         _close(name, g, r, torch.bfloat16)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("S", [1, 64, 65, 129, 192])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_d256_edge_lengths(cuda_device, S, causal):
+    """D = 256 streams 64-row half tiles: one key, exactly one half tile, one half tile plus one
+    row, a tile plus one row, a tile and a half."""
+    (q, k, v, do), (dq, dk, dv) = _run(1, S, 2, 256, torch.float16, causal, seed=S + 1, dev=cuda_device)
+    rq, rk, rv = oracle.attention_backward(q, k, v, do, causal=causal)
+    for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        _close(name, g, r, torch.float16)
+
+
+@pytest.mark.gpu
+def test_bwd_d256_long_causal_sampled_heads(cuda_device):
+    """B1 H16 S2048 D256 causal bf16 (16 query tiles, 32 half-tile steps), two heads checked
+    against the oracle over every row."""
+    B, S, H, D = 1, 2048, 16, 256
+    (q, k, v, do), (dq, dk, dv) = _run(B, S, H, D, torch.bfloat16, True, seed=11, dev=cuda_device)
+    ref = oracle.attention_backward(q, k, v, do, causal=True, heads=[(0, 0), (0, 13)])
+    for (b, h), (rq, rk, rv) in ref.items():
+        for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+            _close(f"{name}[h={h}]", g[b, :, h], r, torch.bfloat16)
 
 
 @pytest.mark.gpu
@@ -91,7 +115,8 @@ def test_bwd_delta_workspace_is_rowsum(cuda_device):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("D,dtype,causal", [(64, torch.bfloat16, True), (128, torch.float16, False),
-                                            (32, torch.bfloat16, False), (128, torch.bfloat16, True)])
+                                            (32, torch.bfloat16, False), (128, torch.bfloat16, True),
+                                            (256, torch.bfloat16, True), (256, torch.float16, False)])
 def test_varlen_bwd_matches_oracle(cuda_device, D, dtype, causal):
     """Packed sequences of mixed lengths (shorter than, equal to and longer than a tile, and
     empty), several sharing one 128-token tile."""
@@ -113,10 +138,11 @@ def test_varlen_bwd_matches_oracle(cuda_device, D, dtype, causal):
 
 
 @pytest.mark.gpu
-def test_varlen_bwd_single_sequence_equals_dense(cuda_device):
+@pytest.mark.parametrize("D", [64, 256])
+def test_varlen_bwd_single_sequence_equals_dense(cuda_device, D):
     """One packed sequence spanning everything gives exactly the dense kernels' gradients."""
     import tiled_exact_attention_fwd_b200 as fa
-    S, H, D = 300, 2, 64
+    S, H = 300, 2
     q, k, v = (t.to(cuda_device) for t in fa_inputs.dense_qkv(1, S, H, D, torch.bfloat16, seed=5))
     do = fa_inputs.normal((1, S, H, D), torch.bfloat16, seed=6).to(cuda_device)
     out, lse = fa.fa_fwd(q, k, v, causal=True)

@@ -16,7 +16,7 @@ def test_oversize_problem_is_refused_before_any_launch():
     # B * H * S = 2^24 + 128 rows > the 2^24-float buffer
     assert L.fa_bwd_noalloc(*([FAKE] * 9), 1, 128, 131073, 128, 0.0, 1, 1, None) == -2
     assert L.fa_bwd_noalloc(None, *([FAKE] * 8), 1, 1, 128, 128, 0.0, 1, 1, None) == -1
-    assert L.fa_bwd_noalloc(*([FAKE] * 9), 1, 1, 128, 256, 0.0, 1, 1, None) == -4
+    assert L.fa_bwd_noalloc(*([FAKE] * 9), 1, 1, 128, 96, 0.0, 1, 1, None) == -4
 
 
 @pytest.mark.gpu

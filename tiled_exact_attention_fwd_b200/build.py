@@ -18,7 +18,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libfa.so")
-SOURCES = ["fa_fwd.cu", "fa_fwd_paged.cu", "fa_bwd.cu", "fa_bwd_noalloc.cu", "fa_padding.cu", "fa_api.cu"]
+SOURCES = ["fa_fwd.cu", "fa_fwd_paged.cu", "fa_bwd.cu", "fa_bwd256.cu", "fa_bwd_noalloc.cu", "fa_padding.cu",
+           "fa_api.cu"]
 HEADERS = ["fa_fwd_kernel.cuh", "fa_sync.cuh", "fa_seq.cuh", "fa_ptx.cuh", "fa_internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

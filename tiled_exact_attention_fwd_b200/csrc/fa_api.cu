@@ -239,8 +239,9 @@ fa_status run_bwd(const void *q, const void *k, const void *v, const void *out, 
     const bool bf16 = dtype == FA_BF16;
     const int inner = fa::fwd_box_inner_elems(D);
     CUtensorMap tq, tk, tv, tdo;
-    if (!encode_map(&tq, q, bf16, D, H, N, inner, 128) || !encode_map(&tk, k, bf16, D, H, N, inner, 128) ||
-        !encode_map(&tv, v, bf16, D, H, N, inner, 128) || !encode_map(&tdo, dout, bf16, D, H, N, inner, 128))
+    const int box_rows = (D == 256) ? 64 : 128;  // D = 256 streams 64-row half tiles
+    if (!encode_map(&tq, q, bf16, D, H, N, inner, box_rows) || !encode_map(&tk, k, bf16, D, H, N, inner, box_rows) ||
+        !encode_map(&tv, v, bf16, D, H, N, inner, box_rows) || !encode_map(&tdo, dout, bf16, D, H, N, inner, box_rows))
         return FA_ERR_CUDA;
     if (!(scale > 0.f)) scale = 1.0f / sqrtf(static_cast<float>(D));
     fa::BwdParams p;
@@ -271,7 +272,7 @@ bool bwd_aligned(const void *q, const void *k, const void *v, const void *out, c
 
 // The error words of the kernel families (one per compilation unit), read and cleared in one
 // launch on the caller's stream; the first nonzero code wins.
-constexpr int kErrorWords = 4;
+constexpr int kErrorWords = 5;
 struct ErrorWords {
     int *code[kErrorWords];
     int *where[kErrorWords];
@@ -301,7 +302,7 @@ fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, c
                  fa_dtype dtype, void *stream) {
     if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !delta) return FA_ERR_NULL;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
-    if (D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;  // dK and dV accumulators share TMEM
+    if (!head_dim_ok(D)) return FA_ERR_HEADDIM;
     if (B <= 0 || H <= 0 || S <= 0) return FA_ERR_SHAPE;
     const int64_t N = static_cast<int64_t>(B) * S;
     if (N > INT32_MAX || B > 65535 || (S + 127) / 128 > 65535) return FA_ERR_SHAPE;
@@ -314,7 +315,7 @@ fa_status fa_varlen_bwd(const void *q, const void *k, const void *v, const void 
                         void *dq, void *dk, void *dv, float *delta, int H, int D, float scale, int causal,
                         fa_dtype dtype, void *stream) {
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
-    if (D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;
+    if (!head_dim_ok(D)) return FA_ERR_HEADDIM;
     if (num_seqs < 0 || total < 0 || max_seqlen < 0 || H <= 0) return FA_ERR_SHAPE;
     if (total == 0 || num_seqs == 0) return FA_OK;  // no rows, nothing to launch
     if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !delta || !cu_seqlens) return FA_ERR_NULL;
@@ -332,7 +333,7 @@ fa_status fa_bwd_noalloc(const void *q, const void *k, const void *v, const void
     if (B > 0 && H > 0 && S > 0 && static_cast<int64_t>(B) * H * S > fa::kNoallocDeltaFloats) return FA_ERR_SHAPE;
     if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv) return FA_ERR_NULL;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
-    if (D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;
+    if (!head_dim_ok(D)) return FA_ERR_HEADDIM;
     if (B <= 0 || H <= 0 || S <= 0) return FA_ERR_SHAPE;
     float *delta = nullptr;
     if (fa::noalloc_delta_buffer(&delta) != cudaSuccess) return FA_ERR_CUDA;
@@ -423,7 +424,8 @@ fa_status fa_device_status(int *where, void *stream) {
     if (fa::fwd_error_addrs(&w.code[0], &w.where[0]) != cudaSuccess ||
         fa::fwd_paged_error_addrs(&w.code[1], &w.where[1]) != cudaSuccess ||
         fa::bwd_error_addrs(&w.code[2], &w.where[2]) != cudaSuccess ||
-        fa::pad_error_addrs(&w.code[3], &w.where[3]) != cudaSuccess)
+        fa::pad_error_addrs(&w.code[3], &w.where[3]) != cudaSuccess ||
+        fa::bwd256_error_addrs(&w.code[4], &w.where[4]) != cudaSuccess)
         return FA_ERR_CUDA;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
     status_collect_kernel<<<1, 1, 0, st>>>(w);

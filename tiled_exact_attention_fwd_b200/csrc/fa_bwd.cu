@@ -650,8 +650,7 @@ cudaError_t launch_bwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
 }
 
 template <int D, bool BF16>
-cudaError_t launch_bwd_d(bool causal, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                         const CUtensorMap &tdo, const BwdParams &p, cudaStream_t st) {
+cudaError_t launch_delta(const BwdParams &p, cudaStream_t st) {
     const int rows = p.B * p.seqlen;
     const int64_t items = static_cast<int64_t>(rows) * p.H;
     const int threads = 256;
@@ -659,7 +658,13 @@ cudaError_t launch_bwd_d(bool causal, const CUtensorMap &tq, const CUtensorMap &
     if (blocks > 148 * 16) blocks = 148 * 16;
     bwd_delta_kernel<D, BF16><<<static_cast<unsigned>(blocks), threads, 0, st>>>(p.out, p.dout, p.delta, rows, p.H,
                                                                                  p.seqlen);
-    cudaError_t e = cudaGetLastError();
+    return cudaGetLastError();
+}
+
+template <int D, bool BF16>
+cudaError_t launch_bwd_d(bool causal, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                         const CUtensorMap &tdo, const BwdParams &p, cudaStream_t st) {
+    cudaError_t e = launch_delta<D, BF16>(p, st);
     if (e != cudaSuccess) return e;
     const int ntiles = (p.seqlen + 127) / 128;
     const dim3 grid(static_cast<unsigned>(p.H), static_cast<unsigned>(ntiles), static_cast<unsigned>(p.B));
@@ -688,6 +693,11 @@ cudaError_t launch_bwd(int D, bool bf16, bool causal, const CUtensorMap &tq, con
                              : launch_bwd_d<64, false>(causal, tq, tk, tv, tdo, p, st);
         case 128: return bf16 ? launch_bwd_d<128, true>(causal, tq, tk, tv, tdo, p, st)
                               : launch_bwd_d<128, false>(causal, tq, tk, tv, tdo, p, st);
+        case 256: {
+            const cudaError_t e = bf16 ? launch_delta<256, true>(p, st) : launch_delta<256, false>(p, st);
+            if (e != cudaSuccess) return e;
+            return launch_bwd256(bf16, causal, tq, tk, tv, tdo, p, st);
+        }
         default: return cudaErrorInvalidValue;
     }
 }

@@ -81,10 +81,15 @@ struct BwdParams {
     float scale_log2;        // scale * log2(e)
     uint64_t timeout_ns;     // bound of every pipeline wait
 };
-// tq, tk, tv, tdo: TMA maps of q, k, v, dout as for the forward (128-row boxes).
+// tq, tk, tv, tdo: TMA maps of q, k, v, dout as for the forward (128-row boxes; 64 at D = 256).
 cudaError_t launch_bwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
                        const CUtensorMap &tv, const CUtensorMap &tdo, const BwdParams &p, cudaStream_t st);
 cudaError_t bwd_error_addrs(int **code, int **where);
+// D = 256 (fa_bwd256.cu): dV, dK and dQ kernels after the delta kernel; tq, tk, tv, tdo with
+// 64-row boxes.
+cudaError_t launch_bwd256(bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                          const CUtensorMap &tdo, const BwdParams &p, cudaStream_t st);
+cudaError_t bwd256_error_addrs(int **code, int **where);
 // The fixed delta buffer of fa_bwd_noalloc: kNoallocDeltaFloats floats (64 MiB) in device
 // memory that belongs to the library's module image; its address on the current device.
 constexpr int64_t kNoallocDeltaFloats = int64_t(1) << 24;
