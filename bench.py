@@ -402,6 +402,34 @@ def run_backward_leg(fa, device, stream, q, k, v, out, lse, causal, warmup, rank
     delta = torch.empty((B, H, S), device=device, dtype=torch.float32)
     fa.fa_fwd(q, k, v, out=out, lse=lse, causal=causal, stream=stream)
 
+    ms = _time_bwd(fa, device, stream, q, k, v, out, do, lse, dq, dk, dv, delta, causal, warmup, iters)
+    flops = fa.attention_bwd_flops(B, H, S, D, causal)
+    peak_burst, _, _, _ = load_peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    res = {"what": "fa_bwd (delta, dK/dV and dQ kernels) on the main workload; FLOPs = 2.5x the forward's "
+                   "(five S x S x D products; the dQ kernel recomputes two of them, not counted)",
+           "ms": round(ms, 4), "tflops": round(tf, 1), "frac_vs_burst": round(tf / peak_burst, 4),
+           "launches": 3 * iters}
+    # the largest head dim of the head-dim sweep (page "FlashAttention性能调优：block_size和head_dim怎么选？",
+    # head_dim measurements at seq_len 4096)
+    B2, S2, H2, D2 = 1, 4096, 16, 256
+    q2, k2, v2 = (t.to(device) for t in fa_inputs.dense_qkv(B2, S2, H2, D2, torch.float16, seed=rank + 200))
+    do2 = fa_inputs.normal((B2, S2, H2, D2), torch.float16, seed=rank + 300).to(device)
+    out2, lse2 = fa.fa_fwd(q2, k2, v2, causal=True, stream=stream)
+    g2 = [torch.empty_like(q2) for _ in range(3)]
+    delta2 = torch.empty((B2, H2, S2), device=device, dtype=torch.float32)
+    ms2 = _time_bwd(fa, device, stream, q2, k2, v2, out2, do2, lse2, *g2, delta2, True, warmup, iters)
+    tf2 = fa.attention_bwd_flops(B2, H2, S2, D2, True) / (ms2 * 1e-3) / 1e12
+    res["hdim256"] = {"what": "fa_bwd at B1 H16 S4096 D256 causal fp16 (delta, dV, dK and dQ kernels: one "
+                              "accumulator per kernel at D = 256); FLOPs = 2.5x the forward's (the kernels "
+                              "compute eight S x S x D products, three recomputed and not counted)",
+                      "ms": round(ms2, 4), "tflops": round(tf2, 1), "frac_vs_burst": round(tf2 / peak_burst, 4),
+                      "launches": 4 * iters}
+    return res
+
+
+def _time_bwd(fa, device, stream, q, k, v, out, do, lse, dq, dk, dv, delta, causal, warmup, iters):
+    """Mean ms of one fa_bwd call over `iters` back-to-back calls (CUDA events on `stream`)."""
     def call():
         fa.fa_bwd(q, k, v, out, do, lse, dq=dq, dk=dk, dv=dv, delta=delta, causal=causal, stream=stream)
 
@@ -414,17 +442,10 @@ def run_backward_leg(fa, device, stream, q, k, v, out, lse, causal, warmup, rank
         call()
     e1.record(stream)
     torch.cuda.synchronize(device)
-    ms = e0.elapsed_time(e1) / iters
-    flops = fa.attention_bwd_flops(B, H, S, D, causal)
     st, where = fa.fa_device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} at {where} after the backward leg")
-    peak_burst, _, _, _ = load_peaks()
-    tf = flops / (ms * 1e-3) / 1e12
-    return {"what": "fa_bwd (delta, dK/dV and dQ kernels) on the main workload; FLOPs = 2.5x the forward's "
-                    "(five S x S x D products; the dQ kernel recomputes two of them, not counted)",
-            "ms": round(ms, 4), "tflops": round(tf, 1), "frac_vs_burst": round(tf / peak_burst, 4),
-            "launches": 3 * iters}
+    return e0.elapsed_time(e1) / iters
 
 
 def run_paged_leg(fa, device, stream, q, k_h, v_h, causal, flops, warmup, rank, iters=20):
