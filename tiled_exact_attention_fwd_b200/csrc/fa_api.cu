@@ -117,6 +117,7 @@ fa_status run_fwd(const void *q, const void *k, const void *v, void *out, float 
         return FA_ERR_CUDA;
     if (!(scale > 0.f)) scale = 1.0f / sqrtf(static_cast<float>(D));
     fa::FwdParams p;
+    p.queue = nullptr;  // set by the launcher where the item queue applies
     p.out = out;
     p.lse = lse;
     p.cu_seqlens = cu_seqlens;

@@ -1,9 +1,18 @@
 // fa_fwd.cu -- the attention forward over contiguous K/V (dense and packed sequences, and the
 // fused packed path): instantiations of the kernel in fa_fwd_kernel.cuh (dense persistent and
 // packed), the bounded-wait self-test, and the host-side tile geometry shared with fa_api.cu.
+#include <atomic>
+
 #include "fa_fwd_kernel.cuh"
 
 namespace fa {
+
+// Counters of the dense item queue, {next item index, CTAs done} per slot (zero while no launch
+// uses them: the last CTA of a launch zeroes its slot). Each launch takes the next slot, so
+// launches in flight at the same time on other streams use other counters.
+constexpr int kQueueSlots = 64;
+static __device__ int g_item_queue[2 * kQueueSlots];
+static std::atomic<unsigned> g_queue_seq{0};
 
 // One CTA waits on a barrier that nothing completes; the bounded wait must give up.
 __global__ void fa_selftest_wait_kernel(uint64_t limit_ns) {
@@ -38,7 +47,18 @@ static cudaError_t launch_d(bool bf16, bool causal, const CUtensorMap &tq, const
 }
 
 cudaError_t launch_fwd(int D, bool bf16, bool causal, const CUtensorMap &tq, const CUtensorMap &tk,
-                       const CUtensorMap &tv, const FwdParams &p, dim3 grid, cudaStream_t st) {
+                       const CUtensorMap &tv, const FwdParams &p_in, dim3 grid, cudaStream_t st) {
+    FwdParams p = p_in;
+    p.queue = nullptr;
+    // Dense non-causal inputs over more than one round of the persistent grid take their items
+    // from a queue (causal items and the CTA pairs of D = 256 keep the static rounds).
+    if (!p.cu_seqlens && !causal && D != 256 && p.num_items > static_cast<int>(grid.x)) {
+        void *base = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&base, g_item_queue);  // on the current device
+        if (e != cudaSuccess) return e;
+        const unsigned slot = g_queue_seq.fetch_add(1u, std::memory_order_relaxed) % kQueueSlots;
+        p.queue = static_cast<int *>(base) + 2 * slot;
+    }
     switch (D) {
         case 32: return launch_d<32>(bf16, causal, tq, tk, tv, p, grid, st);
         case 64: return launch_d<64>(bf16, causal, tq, tk, tv, p, grid, st);

@@ -119,10 +119,14 @@ struct Cfg {
     static constexpr int OFF_KV = MAXQ * Q_BYTES;
     static constexpr int OFF_BAR = OFF_KV + NS * UNIT_BYTES;
     // q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], drain, s_free[2], tail, q_free[2],
-    // q_peer, kv_peer[NS] (CTA pairs: the other CTA's copies have landed)
-    static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1 + 2 + 1 + 2 + 1 + NS;
-    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // TMEM address, abort flag
-    static constexpr int USED = OFF_MISC + 16;
+    // q_peer, kv_peer[NS] (CTA pairs: the other CTA's copies have landed), item_full[QSLOTS],
+    // item_empty[QSLOTS] (the item queue's ring)
+    static constexpr int QSLOTS = 4;
+    static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1 + 2 + 1 + 2 + 1 + NS + 2 * QSLOTS;
+    // TMEM address, abort flag, the item queue's ring (QSLOTS item indices) and one more word
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int MISC_BYTES = 8 + 4 * QSLOTS + 8;
+    static constexpr int USED = OFF_MISC + MISC_BYTES;
     // More than half of the SM's shared memory, so exactly one CTA (and one 512-column
     // TMEM allocation) lives on an SM.
     static constexpr int MIN_SMEM = 120 * 1024;
@@ -130,7 +134,7 @@ struct Cfg {
     static_assert(NS >= 3, "K/V ring too shallow");
     static_assert(O_COL + MAXQ * D <= TMEM_COLS, "TMEM budget");
     static_assert(USED + 1024 <= SMEM_LIMIT, "shared memory budget");
-    static_assert(NUM_BARS * 8 + 16 <= 512, "barrier area");
+    static_assert(NUM_BARS * 8 + MISC_BYTES <= 512, "barrier area");
     static_assert(Q_BYTES % 1024 == 0 && UNIT_BYTES % 1024 == 0, "tile alignment");
     // The MMA thread waits for K_{j+1} while V_j is still held: the ring needs both, plus a part.
     static_assert(NS >= 2 * UNITS + 1, "K/V ring too shallow");
@@ -222,6 +226,8 @@ struct Cta {
     uint64_t *q_full, *kv_full, *kv_empty, *s_full, *p_full, *pv_done, *drain, *s_free, *q_free;
     uint64_t *tail;  // paged K/V: the V part that straddles a sequence end lands here first
     uint64_t *q_peer, *kv_peer;  // CTA pairs (CTA 0): the other CTA's Q tile / ring part has landed
+    uint64_t *item_full, *item_empty;  // item queue: a ring slot holds this CTA's next item / is free again
+    volatile int *items;               // item queue: the ring of item indices (-1: no more items)
     volatile int *abort_flag;
     uint32_t tmem;
     uint64_t lim;
@@ -367,6 +373,83 @@ __device__ __forceinline__ bool next_item(Cta<D> &c, const FwdParams &p, int &r,
         }
     }
     return false;
+}
+
+// ------------------------------------------------------------------ item queue
+// Dense non-causal inputs over more than one round (contiguous K/V, D <= 128) take their items
+// from a counter in global memory instead of round by round: item index w runs over the order
+// the rounds use, and a CTA that finishes early takes the next index, so CTAs that run faster
+// than others (their place on the chip, the L2 slices they read) end together. (All items
+// have the same length there; causal items keep the rounds, which deal their mixed lengths
+// more evenly.) The producer's TMA lane takes the indices (atomicAdd, one item
+// ahead, so the round trip overlaps an item) and puts each into a ring of QSLOTS slots in
+// shared memory (item_full); the MMA and softmax warps read it from there and free the slot
+// (item_empty, one arrival per warp) when they move on to their next item.
+
+// (query-tile group, batch-entry-and-head) of item index w, in the rounds' order.
+template <bool CAUSAL, bool GROUPED>
+__device__ __forceinline__ void dense_item_of(const FwdParams &p, int w, int &pair, int &bh) {
+    if (!GROUPED) {
+        if (CAUSAL) {
+            const int bhc = p.batch * p.H, q = w / bhc;
+            pair = p.npairs - 1 - q;
+            bh = w - q * bhc;
+        } else {
+            bh = w / p.npairs;
+            pair = w - bh * p.npairs;
+        }
+        return;
+    }
+    const int per = p.head_group * p.npairs;  // items of a whole group
+    const int g = w / per, within = w - g * per;
+    const int g0 = g * p.head_group;
+    const int gb = min(p.head_group, p.batch * p.H - g0);  // (batch entry, head) pairs of group g
+    pair = p.npairs - 1 - within / gb;                     // head groups are causal only
+    bh = g0 + within % gb;
+}
+
+// A reading warp's n-th item (whole warp): frees the slot of item n - 1, then waits for slot
+// n % QSLOTS. False at the end of the items or when the wait gave up.
+template <int D, bool CAUSAL, bool GROUPED>
+__device__ __forceinline__ bool take_item(Cta<D> &c, const FwdParams &p, int n) {
+    using C = Cfg<D>;
+    if (n > 0) {
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(&c.item_empty[(n - 1) % C::QSLOTS]);
+    }
+    if (!wait_bounded(&c.item_full[n % C::QSLOTS], (n / C::QSLOTS) & 1, c.abort_flag, c.lim, 170)) return false;
+    const int w = c.items[n % C::QSLOTS];
+    if (w < 0) return false;
+    int pair, bh;
+    dense_item_of<CAUSAL, GROUPED>(p, w, pair, bh);
+    set_dense_item<D, CAUSAL>(c, p, pair, bh);
+    return true;
+}
+
+// The producer's TMA lane: publishes this CTA's n-th item (index wa for even n, wb for odd n,
+// taken one item earlier) and takes the index after next in its place.
+template <int D, bool CAUSAL, bool GROUPED>
+__device__ __forceinline__ bool fetch_item(Cta<D> &c, const FwdParams &p, int n, int &wa, int &wb) {
+    using C = Cfg<D>;
+    const int slot = n % C::QSLOTS;
+    // the slot is free once every reading warp has moved past item n - QSLOTS
+    if (n >= C::QSLOTS &&
+        !wait_bounded(&c.item_empty[slot], ((n / C::QSLOTS) - 1) & 1, c.abort_flag, c.lim, 175))
+        return false;
+    int w = (n & 1) ? wb : wa;
+    if (w >= p.num_items) w = -1;
+    c.items[slot] = w;
+    mbar_arrive(&c.item_full[slot]);  // release: the readers see the index after their wait
+    if (w < 0) return false;
+    // indices below gridDim.x are the CTAs' first items; the counter hands out the rest
+    if (n & 1)
+        wb = static_cast<int>(gridDim.x) + atomicAdd(p.queue, 1);
+    else
+        wa = static_cast<int>(gridDim.x) + atomicAdd(p.queue, 1);
+    int pair, bh;
+    dense_item_of<CAUSAL, GROUPED>(p, w, pair, bh);
+    set_dense_item<D, CAUSAL>(c, p, pair, bh);
+    return true;
 }
 
 // S_t = Q_t K_j^T for key tile j (tile-local step jj = j - j0(t)); after the tile's last QK of
@@ -605,7 +688,9 @@ __device__ __forceinline__ void fetch_group(uint8_t *tile, int rows, int g, int6
 // the other's loops.
 //
 // Dense inputs run persistently: the grid has one CTA per SM (at most one per work item), and
-// each CTA takes its work items in rounds (dense_item_at). Every role loops over the same items;
+// each CTA takes its work items in rounds (dense_item_at) or, non-causal over more than one
+// round with contiguous K/V and D <= 128, from the item queue in the same order. Every role
+// loops over the same items;
 // the producer loads an item's Q tiles as soon as the previous item's QKs on them are done, so
 // the next item's loads and first QKs overlap the current item's last steps and epilogue.
 // Packed inputs launch one CTA per 256 consecutive tokens (one item per CTA).
@@ -623,6 +708,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // Dense D = 256 runs in 2-CTA clusters (the host launches them so): the pair's two query tiles
     // share every K/V tile, each CTA loading half of it, and CTA 0 issues M = 256 MMAs for both.
     constexpr bool PAIR = (D == 256) && !PAGED && !PACKED;
+    // The item queue (dense non-causal inputs over contiguous K/V, more than one round; the host
+    // sets p.queue). Causal items keep the rounds: their lengths differ, and the snake deals them
+    // more evenly than taking them longest first from a queue (which also mixes up the head
+    // groups' order).
+    constexpr bool QUEUE = persistent && !PAIR && !PAGED && !CAUSAL;
+    const bool queued = QUEUE && p.queue != nullptr;
     Cta<D> c;
     c.dec = C::DECOUPLED;
     c.single = C::MAXQ == 1;
@@ -681,8 +772,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // been read, never held up behind the other tile's PV (which waits for that tile's P).
     const bool split_issue = c.dec && !c.fused;
     // Every role runs `for (int rd = 0; next_item(...); ++rd) { ...; c.advance(); }` over this
-    // CTA's work items (dense: the rounds of dense_item_at; packed: the one item set above),
-    // leaving the loop early when a wait gives up.
+    // CTA's work items (dense: the rounds of dense_item_at, or the queue: fetch_item in the TMA
+    // lane, take_item in the MMA and softmax warps; packed: the one item set above), leaving the
+    // loop early when a wait gives up.
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -702,8 +794,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     c.q_free = c.tail + 1;
     c.q_peer = c.q_free + 2;
     c.kv_peer = c.q_peer + 1;
+    c.item_full = c.kv_peer + NS;
+    c.item_empty = c.item_full + C::QSLOTS;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     c.abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    c.items = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
+    volatile int *item_sink = c.items + C::QSLOTS;  // the fetching lane's last indices, read before exit
     c.lim = p.timeout_ns;
 
     const int warp = threadIdx.x >> 5;
@@ -736,6 +832,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_init(c.q_peer, 1);
         for (int s = 0; s < NS; ++s) mbar_init(&c.kv_peer[s], 1);
         mbar_init(c.tail, 1);
+        for (int s = 0; s < C::QSLOTS; ++s) {
+            mbar_init(&c.item_full[s], 1);
+            // one arrival per reading warp: the softmax warps and the MMA-issuing warp(s)
+            mbar_init(&c.item_empty[s], C::NUM_SOFTMAX_WARPS + (split_issue ? 2 : 1));
+        }
         *c.abort_flag = 0;
         fence_mbar_init();
     }
@@ -1037,7 +1138,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             } else if (lane == 0) {
                 bool ok = true;
-                for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
+                // item queue: the indices of this CTA's first two items (this lane takes them all;
+                // the first is the CTA's own index, as in the first round)
+                int wa = 0, wb = 0;
+                if (queued) {
+                    wa = static_cast<int>(blockIdx.x);
+                    wb = static_cast<int>(gridDim.x) + atomicAdd(p.queue, 1);
+                }
+                for (int rd = 0; ok && (queued ? fetch_item<D, CAUSAL, GROUPED>(c, p, rd, wa, wb)
+                                               : next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent));
+                     ++rd) {
                     ok = load_q(0);
                     const int loads = c.loads();
                     for (int L = 0; ok && L < loads; ++L) {
@@ -1122,6 +1232,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                     c.advance();
                 }
+                // the last indices taken are read (so their atomics have completed) before the
+                // CTA reports itself done with the counter at exit
+                if (queued) *item_sink = wa ^ wb;
                 if (PAGED && bad_page) record_error(FA_ERR_INDEX, 150);
             }
             if (warp == C::WARP_TMA && lane == 0 && *c.abort_flag) {
@@ -1189,7 +1302,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             bool ok = true;
             const bool qk = !split_issue || warp == C::WARP_MMA;
             const bool pv = !split_issue || warp != C::WARP_MMA;
-            for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
+            for (int rd = 0; ok && (queued ? take_item<D, CAUSAL, GROUPED>(c, p, rd)
+                                           : next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent));
+                 ++rd) {
                 const int nl = max(c.nA, c.nB);  // key tiles of the item
                 if (c.single) {
                     const int n = c.nA;
@@ -1254,7 +1369,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // steps (the softmax warps are at their register limit there); the item is looked up
         // again for the epilogue.
         int gbase = 0;
-        for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
+        for (int rd = 0; ok && (queued ? take_item<D, CAUSAL, GROUPED>(c, p, rd)
+                                       : next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent));
+             ++rd) {
             const int n = c.steps(t);  // key tiles this warpgroup visits in the item
             if (n <= 0) continue;      // tile absent
             const int j0 = c.j0(t);
@@ -1453,7 +1570,17 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tc_fence_after_sync();
             // the item's coordinates again, computed afresh rather than carried through the key steps
             int eh, eb, eq0, eqbase;
-            item_coords<D, CAUSAL, GROUPED, PAIR>(p, rd, persistent, eh, eb, eq0, eqbase);
+            if (queued) {
+                // the item's slot is still this warp's: it is freed when the warp takes its next item
+                int qpair, qbh;
+                dense_item_of<CAUSAL, GROUPED>(p, c.items[rd % C::QSLOTS], qpair, qbh);
+                eb = qbh / p.H;
+                eh = qbh % p.H;
+                eq0 = qpair * C::MAXQ * BM;
+                eqbase = eb * p.seqlen + eq0;
+            } else {
+                item_coords<D, CAUSAL, GROUPED, PAIR>(p, rd, persistent, eh, eb, eq0, eqbase);
+            }
             const int64_t otok = static_cast<int64_t>(eqbase) + t * BM + r;
             const bool orow_ok = packed ? otok < p.total_tokens : (eq0 + t * BM + r < p.seqlen);
             const float inv_l = 1.f / l;
@@ -1547,6 +1674,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (p.gather && warp < C::NUM_SOFTMAX_WARPS) cp_async_wait_all();  // the query copies (abort paths)
     tc_fence_before_sync();
     __syncthreads();
+    if (queued && threadIdx.x == 0) {
+        // Every index this CTA takes has been taken (the fetching lane read the last ones before
+        // the barrier above); the last CTA to get here zeroes the counter for the next launch.
+        __threadfence();
+        if (atomicAdd(p.queue + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+            atomicExch(p.queue, 0);
+            atomicExch(p.queue + 1, 0);
+        }
+    }
     // pairs: neither CTA leaves (and frees shared memory or TMEM) while the other's MMAs, which
     // read both CTAs' tiles, or its arrivals may still be running
     if (PAIR) cluster_sync();
