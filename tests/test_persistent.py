@@ -102,3 +102,40 @@ def test_head_groups_match_single_heads(B, H):
     O, L = oracle.attention_dense(qh, kh, vh, causal=True, rows=rows)
     assert_o_close(out[b, idx, h].cpu(), O, dtype, "sampled rows")
     assert_lse_close(lse[b, h, idx].cpu(), L, "sampled rows")
+
+
+def test_item_queue_repeated_calls_on_two_streams():
+    """Non-causal B2 H40 S1024 D64 (320 items over the SMs) takes its items from the device item
+    queue. 70 calls in a row (more than the 64 counter slots, so every slot is reused after the
+    last CTA of its launch zeroed it), alternating between two streams without waiting, each
+    into a NaN-filled output: every output and LSE must equal, bit for bit, those of the first
+    call, and each (batch entry, head) those of a call on that pair alone (4 items, the static
+    rounds); one pair is checked against the oracle."""
+    B, S, H, D, dtype = 2, 1024, 40, 64, torch.bfloat16
+    dev = torch.device("cuda:0")
+    q, k, v = (t.to(dev) for t in fa_inputs.dense_qkv(B, S, H, D, dtype, seed=21))
+    ref, ref_lse = fa.fa_fwd(q, k, v)
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
+    outs = []
+    for i in range(70):
+        s = streams[i % 2]
+        with torch.cuda.stream(s):
+            o = torch.full_like(q, float("nan"))
+            l = torch.full((B, H, S), float("nan"), device=dev)
+            fa.fa_fwd(q, k, v, out=o, lse=l, stream=s)
+        outs.append((o, l))
+    torch.cuda.synchronize()
+    for i, (o, l) in enumerate(outs):
+        assert torch.equal(o, ref), f"output of call {i}"
+        assert torch.equal(l, ref_lse), f"LSE of call {i}"
+    for b, h in [(0, 0), (0, 39), (1, 17)]:
+        qs, ks, vs = (t[b:b + 1, :, h:h + 1].contiguous() for t in (q, k, v))
+        o1, l1 = fa.fa_fwd(qs, ks, vs)
+        torch.cuda.synchronize()
+        assert torch.equal(ref[b:b + 1, :, h:h + 1], o1), f"output of pair ({b}, {h})"
+        assert torch.equal(ref_lse[b:b + 1, h:h + 1], l1), f"LSE of pair ({b}, {h})"
+    qh, kh, vh = (t[1:2, :, 17:18].cpu() for t in (q, k, v))
+    O, L = oracle.attention_dense(qh, kh, vh, causal=False)
+    assert_o_close(ref[1:2, :, 17:18].cpu(), O, dtype, "pair (1, 17)")
+    assert_lse_close(ref_lse[1:2, 17:18].cpu(), L, "pair (1, 17)")
