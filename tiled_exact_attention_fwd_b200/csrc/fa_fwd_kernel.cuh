@@ -123,9 +123,9 @@ struct Cfg {
     // item_empty[QSLOTS] (the item queue's ring)
     static constexpr int QSLOTS = 4;
     static constexpr int NUM_BARS = 2 + 2 * NS + 2 + 2 + 2 + 1 + 2 + 1 + 2 + 1 + NS + 2 * QSLOTS;
-    // TMEM address, abort flag, the item queue's ring (QSLOTS item indices) and one more word
+    // TMEM address, abort flag, the item queue's ring (QSLOTS item indices)
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-    static constexpr int MISC_BYTES = 8 + 4 * QSLOTS + 8;
+    static constexpr int MISC_BYTES = 8 + 4 * QSLOTS;
     static constexpr int USED = OFF_MISC + MISC_BYTES;
     // More than half of the SM's shared memory, so exactly one CTA (and one 512-column
     // TMEM allocation) lives on an SM.
@@ -376,15 +376,14 @@ __device__ __forceinline__ bool next_item(Cta<D> &c, const FwdParams &p, int &r,
 }
 
 // ------------------------------------------------------------------ item queue
-// Dense non-causal inputs over more than one round (contiguous K/V, D <= 128) take their items
-// from a counter in global memory instead of round by round: item index w runs over the order
-// the rounds use, and a CTA that finishes early takes the next index, so CTAs that run faster
-// than others (their place on the chip, the L2 slices they read) end together. (All items
-// have the same length there; causal items keep the rounds, which deal their mixed lengths
-// more evenly.) The producer's TMA lane takes the indices (atomicAdd, one item
-// ahead, so the round trip overlaps an item) and puts each into a ring of QSLOTS slots in
-// shared memory (item_full); the MMA and softmax warps read it from there and free the slot
-// (item_empty, one arrival per warp) when they move on to their next item.
+// Dense inputs over more than one round (contiguous K/V, D <= 128) take their items from a
+// counter in global memory instead of round by round: item index w runs over the order the
+// rounds use (groups in turn; causal items longest first), and a CTA that finishes early takes
+// the next index, so CTAs that run faster than others (their place on the chip, the L2 slices
+// they read) end together. The producer's TMA lane takes each index when it needs it
+// (atomicAdd) and puts it into a ring of QSLOTS slots in shared memory (item_full); the MMA and
+// softmax warps read it from there and free the slot (item_empty, one arrival per warp) when
+// they move on to their next item.
 
 // (query-tile group, batch-entry-and-head) of item index w, in the rounds' order.
 template <bool CAUSAL, bool GROUPED>
@@ -426,26 +425,25 @@ __device__ __forceinline__ bool take_item(Cta<D> &c, const FwdParams &p, int n) 
     return true;
 }
 
-// The producer's TMA lane: publishes this CTA's n-th item (index wa for even n, wb for odd n,
-// taken one item earlier) and takes the index after next in its place.
+// The producer's TMA lane: takes this CTA's n-th item (its own index for the first, else the
+// next index of the counter) and publishes it. The index is taken only now, when the lane has
+// issued every load of the previous item (a few key steps before the CTA finishes it), not
+// earlier: a CTA holding a reserved item while another one runs out of work is what unbalances
+// the end of a launch. The lane is far enough ahead of the MMAs for the atomic's round trip.
 template <int D, bool CAUSAL, bool GROUPED>
-__device__ __forceinline__ bool fetch_item(Cta<D> &c, const FwdParams &p, int n, int &wa, int &wb) {
+__device__ __forceinline__ bool fetch_item(Cta<D> &c, const FwdParams &p, int n) {
     using C = Cfg<D>;
     const int slot = n % C::QSLOTS;
     // the slot is free once every reading warp has moved past item n - QSLOTS
     if (n >= C::QSLOTS &&
         !wait_bounded(&c.item_empty[slot], ((n / C::QSLOTS) - 1) & 1, c.abort_flag, c.lim, 175))
         return false;
-    int w = (n & 1) ? wb : wa;
+    // indices below gridDim.x are the CTAs' first items; the counter hands out the rest
+    int w = (n == 0) ? static_cast<int>(blockIdx.x) : static_cast<int>(gridDim.x) + atomicAdd(p.queue, 1);
     if (w >= p.num_items) w = -1;
     c.items[slot] = w;
     mbar_arrive(&c.item_full[slot]);  // release: the readers see the index after their wait
     if (w < 0) return false;
-    // indices below gridDim.x are the CTAs' first items; the counter hands out the rest
-    if (n & 1)
-        wb = static_cast<int>(gridDim.x) + atomicAdd(p.queue, 1);
-    else
-        wa = static_cast<int>(gridDim.x) + atomicAdd(p.queue, 1);
     int pair, bh;
     dense_item_of<CAUSAL, GROUPED>(p, w, pair, bh);
     set_dense_item<D, CAUSAL>(c, p, pair, bh);
@@ -688,9 +686,9 @@ __device__ __forceinline__ void fetch_group(uint8_t *tile, int rows, int g, int6
 // the other's loops.
 //
 // Dense inputs run persistently: the grid has one CTA per SM (at most one per work item), and
-// each CTA takes its work items in rounds (dense_item_at) or, non-causal over more than one
-// round with contiguous K/V and D <= 128, from the item queue in the same order. Every role
-// loops over the same items;
+// each CTA takes its work items in rounds (dense_item_at) or, over more than one round with
+// contiguous K/V and D <= 128, from the item queue in the same order. Every role loops over the
+// same items;
 // the producer loads an item's Q tiles as soon as the previous item's QKs on them are done, so
 // the next item's loads and first QKs overlap the current item's last steps and epilogue.
 // Packed inputs launch one CTA per 256 consecutive tokens (one item per CTA).
@@ -708,11 +706,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // Dense D = 256 runs in 2-CTA clusters (the host launches them so): the pair's two query tiles
     // share every K/V tile, each CTA loading half of it, and CTA 0 issues M = 256 MMAs for both.
     constexpr bool PAIR = (D == 256) && !PAGED && !PACKED;
-    // The item queue (dense non-causal inputs over contiguous K/V, more than one round; the host
-    // sets p.queue). Causal items keep the rounds: their lengths differ, and the snake deals them
-    // more evenly than taking them longest first from a queue (which also mixes up the head
-    // groups' order).
-    constexpr bool QUEUE = persistent && !PAIR && !PAGED && !CAUSAL;
+    // The item queue (dense inputs over contiguous K/V, more than one round; the host sets p.queue).
+    constexpr bool QUEUE = persistent && !PAIR && !PAGED;
     const bool queued = QUEUE && p.queue != nullptr;
     Cta<D> c;
     c.dec = C::DECOUPLED;
@@ -799,7 +794,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     c.abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     c.items = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
-    volatile int *item_sink = c.items + C::QSLOTS;  // the fetching lane's last indices, read before exit
     c.lim = p.timeout_ns;
 
     const int warp = threadIdx.x >> 5;
@@ -1138,14 +1132,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             } else if (lane == 0) {
                 bool ok = true;
-                // item queue: the indices of this CTA's first two items (this lane takes them all;
-                // the first is the CTA's own index, as in the first round)
-                int wa = 0, wb = 0;
-                if (queued) {
-                    wa = static_cast<int>(blockIdx.x);
-                    wb = static_cast<int>(gridDim.x) + atomicAdd(p.queue, 1);
-                }
-                for (int rd = 0; ok && (queued ? fetch_item<D, CAUSAL, GROUPED>(c, p, rd, wa, wb)
+                for (int rd = 0; ok && (queued ? fetch_item<D, CAUSAL, GROUPED>(c, p, rd)
                                                : next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent));
                      ++rd) {
                     ok = load_q(0);
@@ -1232,9 +1219,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                     c.advance();
                 }
-                // the last indices taken are read (so their atomics have completed) before the
-                // CTA reports itself done with the counter at exit
-                if (queued) *item_sink = wa ^ wb;
                 if (PAGED && bad_page) record_error(FA_ERR_INDEX, 150);
             }
             if (warp == C::WARP_TMA && lane == 0 && *c.abort_flag) {
@@ -1675,8 +1659,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_before_sync();
     __syncthreads();
     if (queued && threadIdx.x == 0) {
-        // Every index this CTA takes has been taken (the fetching lane read the last ones before
-        // the barrier above); the last CTA to get here zeroes the counter for the next launch.
+        // Every index this CTA takes has been taken (the fetching lane used each one before the
+        // barrier above); the last CTA to get here zeroes the counter for the next launch.
         __threadfence();
         if (atomicAdd(p.queue + 1, 1) == static_cast<int>(gridDim.x) - 1) {
             atomicExch(p.queue, 0);

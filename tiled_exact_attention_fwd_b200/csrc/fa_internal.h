@@ -38,10 +38,9 @@ struct FwdParams {
     // K/V of a few heads; head_group = batch * H (one group) unless K/V would not fit in L2.
     int head_group, num_groups, group_rounds;
     int out_align32;  // out is 32-byte aligned (the persistent epilogue then stores 32 bytes per lane)
-    // Dense non-causal inputs over more than one round (contiguous K/V, D <= 128): {next item
-    // index, CTAs done} in device memory, zero at launch; the CTAs take their items from it in
-    // the rounds' order instead of round by round, and the last CTA to finish zeroes it again.
-    // Else null.
+    // Dense inputs over more than one round (contiguous K/V, D <= 128): {next item index, CTAs
+    // done} in device memory, zero at launch; the CTAs take their items from it in the rounds'
+    // order instead of round by round, and the last CTA to finish zeroes it again. Else null.
     int *queue;
 };
 
