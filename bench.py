@@ -508,7 +508,7 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
         call()
     torch.cuda.synchronize(device)
     n_ev = 6
-    tot = [0.0] * 5
+    comp = [[], [], []]
     whole = []
     for it in range(iters):
         # keep the GPU busy while the host queues the whole call, so the events time the
@@ -525,9 +525,8 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
         ev[3].record(stream)
         torch.cuda.synchronize(device)
         whole.append(ev[0].elapsed_time(ev[3]) * 1e3)
-        tot[0] += ev[0].elapsed_time(ev[1]) * 1e3
-        tot[1] += ev[1].elapsed_time(ev[2]) * 1e3
-        tot[2] += ev[2].elapsed_time(ev[3]) * 1e3
+        for c in range(3):
+            comp[c].append(ev[c].elapsed_time(ev[c + 1]) * 1e3)
     # the same path as one launch (unpad and pad folded into the attention kernel)
     fused = []
     for it in range(iters):
@@ -550,10 +549,14 @@ def run_varlen_leg(fa, device, stream, iters, warmup, ws):
             "gpu_launches_per_call": 1,
             "three_launch_path": {"value": round(us3, 2), "unit": "us/call",
                                   "calls": "fa_unpad_qkv + fa_varlen_fwd + fa_pad",
-                                  "components_us_mean": {"unpad_qkv": round(tot[0] / iters, 2),
-                                                         "varlen_fwd": round(tot[1] / iters, 2),
-                                                         "pad_out": round(tot[2] / iters, 2)},
-                                  "varlen_fwd_tflops": round(flops / (tot[1] / iters * 1e-6) / 1e12, 2)}}
+                                  "components_us_median": {"unpad_qkv": round(statistics.median(comp[0]), 2),
+                                                           "varlen_fwd": round(statistics.median(comp[1]), 2),
+                                                           "pad_out": round(statistics.median(comp[2]), 2)},
+                                  "components_note": "each from the event before its launch to the event after "
+                                                     "it, so each includes the GPU's gap between the previous "
+                                                     "kernel's end and its own start (about 2 us), which a "
+                                                     "profiler's per-kernel duration leaves out",
+                                  "varlen_fwd_tflops": round(flops / (statistics.median(comp[1]) * 1e-6) / 1e12, 2)}}
 
 
 def run_padding_hbm_leg(fa, device, stream, iters):
