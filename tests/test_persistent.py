@@ -141,22 +141,25 @@ def test_item_queue_repeated_calls_on_two_streams():
     assert_lse_close(ref_lse[1:2, 17:18].cpu(), L, "pair (1, 17)")
 
 
+@pytest.mark.parametrize("D", [64, 256])
 @pytest.mark.parametrize("extra", [1, 0])
 @pytest.mark.parametrize("causal", [False, True])
-def test_item_queue_round_boundaries(extra, causal):
-    """Items = SMs + 1 (one CTA takes a second item from the queue) and exactly twice the SMs
-    (every CTA takes one more): S256 D64 has one item per (batch entry, head), so H sets the
-    item count. Each head must equal, bit for bit, a call on that head alone (one item, no
-    queue); two heads are checked against the oracle."""
+def test_item_queue_round_boundaries(D, extra, causal):
+    """Items = units + 1 (one unit takes a second item from the queue) and exactly twice the
+    units (every unit takes one more), a unit being a CTA (D = 64) or a 2-CTA cluster (D = 256,
+    whose CTA 0 takes the items for both): S256 has one item per (batch entry, head), so H
+    sets the item count. Each head must equal, bit for bit, a call on that head alone (one
+    item, no queue); two heads are checked against the oracle."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    H = sms + 1 if extra else 2 * sms
-    B, S, D, dtype = 1, 256, 64, torch.float16
+    units = sms // 2 if D == 256 else sms
+    H = units + 1 if extra else 2 * units
+    B, S, dtype = 1, 256, torch.float16
     dev = torch.device("cuda:0")
     q, k, v = (t.to(dev) for t in fa_inputs.dense_qkv(B, S, H, D, dtype, seed=31 + extra))
     out, lse = fa.fa_fwd(q, k, v, causal=causal)
     torch.cuda.synchronize()
     assert not torch.isnan(out).any()
-    for h in [0, 1, sms - 1, sms, H - 1]:
+    for h in [0, 1, units - 1, units, H - 1]:
         qs, ks, vs = (t[:, :, h:h + 1].contiguous() for t in (q, k, v))
         o1, l1 = fa.fa_fwd(qs, ks, vs, causal=causal)
         torch.cuda.synchronize()

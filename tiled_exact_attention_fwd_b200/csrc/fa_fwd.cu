@@ -50,9 +50,10 @@ cudaError_t launch_fwd(int D, bool bf16, bool causal, const CUtensorMap &tq, con
                        const CUtensorMap &tv, const FwdParams &p_in, dim3 grid, cudaStream_t st) {
     FwdParams p = p_in;
     p.queue = nullptr;
-    // Dense inputs over more than one round of the persistent grid take their items from a
-    // queue (the CTA pairs of D = 256 keep the static rounds).
-    if (!p.cu_seqlens && D != 256 && p.num_items > static_cast<int>(grid.x)) {
+    // Dense inputs over more than one round of the persistent grid (D = 256: of its CTA pairs)
+    // take their items from a queue.
+    const int units = (D == 256) ? static_cast<int>(grid.x / 2) : static_cast<int>(grid.x);
+    if (!p.cu_seqlens && p.num_items > units) {
         void *base = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&base, g_item_queue);  // on the current device
         if (e != cudaSuccess) return e;

@@ -450,6 +450,57 @@ __device__ __forceinline__ bool fetch_item(Cta<D> &c, const FwdParams &p, int n)
     return true;
 }
 
+// CTA pairs (D = 256): both CTAs of a cluster run the same items. CTA 0's producer lane takes
+// them and publishes each to both rings (CTA 1's slot written through its shared::cluster
+// address, then a release arrival on CTA 1's item_full); the reading warps of both CTAs free
+// a slot on CTA 0's item_empty (remote arrivals from CTA 1). Every wait is cluster-scope.
+template <int D, bool CAUSAL, bool GROUPED>
+__device__ __forceinline__ bool fetch_item_pair(Cta<D> &c, const FwdParams &p, int n) {
+    using C = Cfg<D>;
+    const int slot = n % C::QSLOTS;
+    if (n >= C::QSLOTS &&
+        !wait_bounded_cluster(&c.item_empty[slot], ((n / C::QSLOTS) - 1) & 1, c.abort_flag, c.lim, 176))
+        return false;
+    // a cluster's first item is its own index; the counter hands out the rest
+    const int clusters = static_cast<int>(gridDim.x >> 1);
+    int w = (n == 0) ? static_cast<int>(blockIdx.x >> 1) : clusters + atomicAdd(p.queue, 1);
+    if (w >= p.num_items) w = -1;
+    c.items[slot] = w;
+    mbar_arrive(&c.item_full[slot]);
+    st_cluster_u32(mapa_shared(const_cast<int *>(c.items + slot), 1), static_cast<uint32_t>(w));
+    mbar_arrive_cluster(mapa_shared(&c.item_full[slot], 1));  // release: orders the store above
+    if (w < 0) return false;
+    int pair, bh;
+    dense_item_of<CAUSAL, GROUPED>(p, w, pair, bh);
+    set_dense_item<D, CAUSAL, true>(c, p, pair, bh);
+    return true;
+}
+
+// A reading role's n-th item in a CTA pair: a whole warp, or one lane (one_lane: the lane-0
+// roles, CTA 1's producer and reporter).
+template <int D, bool CAUSAL, bool GROUPED>
+__device__ __forceinline__ bool take_item_pair(Cta<D> &c, const FwdParams &p, int n, bool one_lane) {
+    using C = Cfg<D>;
+    if (n > 0) {
+        if (!one_lane) __syncwarp();
+        if (one_lane || (threadIdx.x & 31) == 0) {
+            uint64_t *bar = &c.item_empty[(n - 1) % C::QSLOTS];
+            if (c.rank == 0)
+                mbar_arrive(bar);
+            else
+                mbar_arrive_cluster(mapa_shared(bar, 0));
+        }
+    }
+    if (!wait_bounded_cluster(&c.item_full[n % C::QSLOTS], (n / C::QSLOTS) & 1, c.abort_flag, c.lim, 171))
+        return false;
+    const int w = c.items[n % C::QSLOTS];
+    if (w < 0) return false;
+    int pair, bh;
+    dense_item_of<CAUSAL, GROUPED>(p, w, pair, bh);
+    set_dense_item<D, CAUSAL, true>(c, p, pair, bh);
+    return true;
+}
+
 // S_t = Q_t K_j^T for key tile j (tile-local step jj = j - j0(t)); after the tile's last QK of
 // the item, q_free[t] fires once the MMAs reading Q_t are done. Returns false when a wait gave up.
 template <int D, bool BF16>
@@ -707,7 +758,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // share every K/V tile, each CTA loading half of it, and CTA 0 issues M = 256 MMAs for both.
     constexpr bool PAIR = (D == 256) && !PAGED && !PACKED;
     // The item queue (dense inputs over contiguous K/V, more than one round; the host sets p.queue).
-    constexpr bool QUEUE = persistent && !PAIR && !PAGED;
+    constexpr bool QUEUE = persistent && !PAGED;
     const bool queued = QUEUE && p.queue != nullptr;
     Cta<D> c;
     c.dec = C::DECOUPLED;
@@ -828,8 +879,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_init(c.tail, 1);
         for (int s = 0; s < C::QSLOTS; ++s) {
             mbar_init(&c.item_full[s], 1);
-            // one arrival per reading warp: the softmax warps and the MMA-issuing warp(s)
-            mbar_init(&c.item_empty[s], C::NUM_SOFTMAX_WARPS + (split_issue ? 2 : 1));
+            // one arrival per reading warp: the softmax warps and the MMA-issuing warp(s); pairs
+            // (CTA 0's barrier): CTA 0's MMA and softmax warps, CTA 1's producer and reporter
+            // lanes and softmax warps
+            mbar_init(&c.item_empty[s], PAIR ? 2 * C::NUM_SOFTMAX_WARPS + 3
+                                             : C::NUM_SOFTMAX_WARPS + (split_issue ? 2 : 1));
         }
         *c.abort_flag = 0;
         fence_mbar_init();
@@ -1094,7 +1148,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // each on this CTA's own barriers (CTA 1's reporter warp passes them on to CTA 0). The
                 // ring slots and Q buffer are released by CTA 0's MMA commits.
                 bool ok = true;
-                for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
+                for (int rd = 0;
+                     ok && (queued ? (c.rank == 0 ? fetch_item_pair<D, CAUSAL, GROUPED>(c, p, rd)
+                                                  : take_item_pair<D, CAUSAL, GROUPED>(c, p, rd, true))
+                                   : next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent));
+                     ++rd) {
                     if (c.nq(0) > 0 && !wait_bounded_cluster(&c.q_free[0], (c.nq(0) - 1) & 1, c.abort_flag, c.lim, 110)) {
                         ok = false;
                         break;
@@ -1250,7 +1308,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (lane == 0) {
                 bool ok = true;
                 const uint32_t q_peer0 = mapa_shared(c.q_peer, 0);
-                for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
+                for (int rd = 0; ok && (queued ? take_item_pair<D, CAUSAL, GROUPED>(c, p, rd, true)
+                                               : next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent));
+                     ++rd) {
                     if (!(ok = wait_bounded(&c.q_full[0], c.nq(0) & 1, c.abort_flag, c.lim, 120))) break;
                     mbar_arrive_cluster(q_peer0);
                     const int loads = c.loads();
@@ -1266,7 +1326,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // ------------------------------------------------------------ pair MMA issuer (CTA 0)
             bool ok = true;
             if (c.rank == 0) {
-                for (int rd = 0; ok && next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent); ++rd) {
+                for (int rd = 0; ok && (queued ? take_item_pair<D, CAUSAL, GROUPED>(c, p, rd, false)
+                                               : next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent));
+                     ++rd) {
                     const int n = c.nA;
                     for (int idx = 0; ok && idx < 2 * n; ++idx) {
                         bool is_v;
@@ -1353,7 +1415,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // steps (the softmax warps are at their register limit there); the item is looked up
         // again for the epilogue.
         int gbase = 0;
-        for (int rd = 0; ok && (queued ? take_item<D, CAUSAL, GROUPED>(c, p, rd)
+        for (int rd = 0; ok && (queued ? (PAIR ? take_item_pair<D, CAUSAL, GROUPED>(c, p, rd, false)
+                                               : take_item<D, CAUSAL, GROUPED>(c, p, rd))
                                        : next_item<D, CAUSAL, GROUPED, PAIR>(c, p, rd, persistent));
              ++rd) {
             const int n = c.steps(t);  // key tiles this warpgroup visits in the item
@@ -1560,7 +1623,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 dense_item_of<CAUSAL, GROUPED>(p, c.items[rd % C::QSLOTS], qpair, qbh);
                 eb = qbh / p.H;
                 eh = qbh % p.H;
-                eq0 = qpair * C::MAXQ * BM;
+                eq0 = PAIR ? (2 * qpair + static_cast<int>(c.rank)) * BM : qpair * C::MAXQ * BM;
                 eqbase = eb * p.seqlen + eq0;
             } else {
                 item_coords<D, CAUSAL, GROUPED, PAIR>(p, rd, persistent, eh, eb, eq0, eqbase);
