@@ -89,6 +89,18 @@ def test_bwd_d256_long_causal_sampled_heads(cuda_device):
 
 
 @pytest.mark.gpu
+def test_bwd_d256_long_noncausal_sampled_heads(cuda_device):
+    """B1 H8 S1536 D256 non-causal fp16 (every key tile streams past every query tile), two
+    heads checked against the oracle over every row."""
+    B, S, H, D = 1, 1536, 8, 256
+    (q, k, v, do), (dq, dk, dv) = _run(B, S, H, D, torch.float16, False, seed=13, dev=cuda_device)
+    ref = oracle.attention_backward(q, k, v, do, causal=False, heads=[(0, 2), (0, 7)])
+    for (b, h), (rq, rk, rv) in ref.items():
+        for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+            _close(f"{name}[h={h}]", g[b, :, h], r, torch.float16)
+
+
+@pytest.mark.gpu
 def test_bwd_long_causal_sampled_heads(cuda_device):
     """B1 H32 S4096 D128 causal bf16 (the head-dim sweep's D=128 shape), two heads checked
     against the oracle over every row."""

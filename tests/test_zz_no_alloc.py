@@ -20,11 +20,12 @@ def test_oversize_problem_is_refused_before_any_launch():
 
 
 @pytest.mark.gpu
-def test_two_calls_match_the_workspace_entry_point(cuda_device):
+@pytest.mark.parametrize("D", [128, 256])
+def test_two_calls_match_the_workspace_entry_point(cuda_device, D):
     import tiled_exact_attention_fwd_b200 as fa
     dev = cuda_device
     for causal in (True, False):
-        B, S, H, D = 2, 300, 4, 128
+        B, S, H = 2, 300, 4
         q, k, v = (t.to(dev) for t in fa_inputs.dense_qkv(B, S, H, D, torch.bfloat16, seed=9))
         do = fa_inputs.normal((B, S, H, D), torch.bfloat16, seed=10).to(dev)
         out, lse = fa.fa_fwd(q, k, v, causal=causal)
