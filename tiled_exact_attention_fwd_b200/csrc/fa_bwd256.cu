@@ -16,8 +16,10 @@
 //   dQ:  X = Q_i K_u^T (S),  Y = dO_i V_u^T (dP);    dZ over X;    dQ += dZ K_u
 // X and Y are N = 64 SS MMAs over the 256 head columns (16 k-steps); the update is one TS MMA
 // (A = the 16-bit step from TMEM, B = the streamed half tile read MN-major, N = 256, K = 64).
-// TMEM: two 128-column buffers (X at +0, Y at +64) used by alternate steps, so X/Y of step
-// k+1 run while the elementwise warps work on step k, and the accumulator at column 256.
+// TMEM: two 128-column buffers (X at +0, Y at +64) used by alternate steps, so the next step's
+// products run while the elementwise warps work on this one, and the accumulator at column
+// 256. In dK and dQ the MMA warp issues X(k+1), the update of k, then Y(k+1), so that Y covers
+// the refill of the slot the update frees (see the issue loop).
 // Shared memory: the fixed tile(s) (64 KB each), the half tiles read by X in a two-slot ring,
 // the other stream in a one-slot ring (dK, dQ: Y is its only reader, so the slot is free once
 // Y completes, long before the next step needs it) or a two-slot ring (dV: read by the
@@ -304,35 +306,42 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (n > 0) {
             ok = wait_all(fix_full, 0, 510);
             if (ok) tc_fence_after_sync();
-            // X (and Y) of step k into TMEM buffer k % 2. Issue order: X/Y(k+1), then (once the
-            // elementwise warps are done with k) the update of k; the tensor core runs them in
-            // that order, so X/Y(k+2) overwrite buffer k % 2 only after the update of k has read it.
-            auto issue_xy = [&](int k) -> bool {
+            // X and Y of step k go into TMEM buffer k % 2; the update of step k reads it once the
+            // elementwise warps are done with k. Issue order, dV: X(k+1), then the update of k.
+            // dK and dQ: X(k+1), the update of k, then Y(k+1) — the update frees the slot of the
+            // stream X and the update read (step k's), whose refill for X(k+2) is a 32 KB load, and
+            // Y(k+1) runs while it lands (issued before the update, X(k+2) would wait for it in
+            // the tensor pipe on every step). The tensor core runs MMAs in issue order, so X/Y
+            // of step k+2 overwrite buffer k % 2 only after the update of k has read it.
+            auto issue_x = [&](int k) -> bool {
                 const int s0 = k & 1;
                 if (!wait_all(&r0_full[s0], (k >> 1) & 1, 520 + s0)) return false;
                 tc_fence_after_sync();
-                const uint32_t buf = tmem + (k & 1) * 128;
-                mma_scores<BF16>(buf, fix0, r0_tile(s0));
-                if constexpr (Kd::HAS_Y) {
-                    if (!wait_all(&r1_full[0], k & 1, 524)) return false;
-                    tc_fence_after_sync();
-                    mma_scores<BF16>(buf + STEP, fix1, r1_tile(0));
-                    umma_commit_elect(&r1_empty[0]);  // Y was the slot's only reader
-                } else {
+                mma_scores<BF16>(tmem + (k & 1) * 128, fix0, r0_tile(s0));
+                if constexpr (!Kd::HAS_Y) {
                     umma_commit_elect(&r0_empty[s0]);  // X was the slot's only reader
+                    umma_commit_elect(&s_full[k & 1]);
                 }
+                return true;
+            };
+            auto issue_y = [&](int k) -> bool {
+                if (!wait_all(&r1_full[0], k & 1, 524)) return false;
+                tc_fence_after_sync();
+                mma_scores<BF16>(tmem + (k & 1) * 128 + STEP, fix1, r1_tile(0));
+                umma_commit_elect(&r1_empty[0]);  // Y was the slot's only reader
                 umma_commit_elect(&s_full[k & 1]);
                 return true;
             };
-            if (ok) ok = issue_xy(0);
+            if (ok) ok = issue_x(0) && (!Kd::HAS_Y || issue_y(0));
             for (int k = 0; ok && k < n; ++k) {
-                if (k + 1 < n && !(ok = issue_xy(k + 1))) break;
+                if (k + 1 < n && !(ok = issue_x(k + 1))) break;
                 if (!(ok = wait_all(&p_ready[k & 1], (k >> 1) & 1, 530 + (k & 1)))) break;
                 tc_fence_after_sync();
                 const uint32_t zbuf = tmem + (k & 1) * 128;
                 if constexpr (Kd::HAS_Y) {
                     mma_update<BF16>(tmem + C::COL_ACC, zbuf, r0_tile(k & 1), k > 0);  // dK += dZ^T Q / dQ += dZ K
                     umma_commit_elect(&r0_empty[k & 1]);
+                    if (k + 1 < n && !(ok = issue_y(k + 1))) break;
                 } else {
                     const int s1 = k & 1;
                     if (!(ok = wait_all(&r1_full[s1], (k >> 1) & 1, 526 + s1))) break;
