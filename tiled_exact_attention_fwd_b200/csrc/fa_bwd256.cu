@@ -22,8 +22,9 @@
 // the refill of the slot the update frees (see the issue loop).
 // Shared memory: the fixed tile(s) (64 KB each), the half tiles read by X in a two-slot ring,
 // the other stream in a one-slot ring (dK, dQ: Y is its only reader, so the slot is free once
-// Y completes, long before the next step needs it) or a two-slot ring (dV: read by the
-// update), and the streamed queries' statistics (dV, dK) in three slots. The three kernels do
+// Y completes, long before the next step needs it) or a three-slot ring (dV: read by the
+// update, whose slot is refilled two steps ahead), and the streamed queries' statistics (dV,
+// dK) in three slots. The three kernels do
 // 8 score-sized products per tile pair where the D <= 128 kernels do 7 (S^T is recomputed by
 // dV and dK).
 // Warps 0-7 are elementwise (two threads per TMEM lane = row, 32 columns each), warp 8 lane 0
@@ -71,15 +72,15 @@ struct B256Kind {
     static constexpr bool COL_STATS = KIND != KIND_DQ;  // statistics belong to the streamed rows
     static constexpr int NFIX = HAS_Y ? 2 : 1;
     static constexpr int R0_SLOTS = 2;                  // read by X (and, dK / dQ, the update)
-    static constexpr int R1_SLOTS = HAS_Y ? 1 : 2;      // read by Y (dK, dQ) or the update (dV)
+    static constexpr int R1_SLOTS = HAS_Y ? 1 : 3;      // read by Y (dK, dQ) or the update (dV)
     static constexpr int STAT_SLOTS = 3;
     static constexpr int OFF_R0 = NFIX * C::FIX_BYTES;
     static constexpr int OFF_R1 = OFF_R0 + R0_SLOTS * C::HALF_BYTES;
     static constexpr int OFF_STAT = OFF_R1 + R1_SLOTS * C::HALF_BYTES;  // [slot][-lse*log2e | -delta][64]
     static constexpr int OFF_BAR = OFF_STAT + (COL_STATS ? STAT_SLOTS * 2 * C::STEP * 4 : 0);
-    // fix_full, r0_full[2], r0_empty[2], r1_full[2], r1_empty[2], s_full[2], p_ready[2],
+    // fix_full, r0_full[2], r0_empty[2], r1_full[3], r1_empty[3], s_full[2], p_ready[2],
     // stats_ready[3], done, drain
-    static constexpr int NUM_BARS = 18;
+    static constexpr int NUM_BARS = 20;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int USED = OFF_MISC + 16;
     static constexpr int SMEM_BYTES = USED + 1024;  // + alignment of the base to 1024 bytes
@@ -215,8 +216,8 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint8_t *fix0 = smem, *fix1 = smem + C::FIX_BYTES;
     float *stats = reinterpret_cast<float *>(smem + Kd::OFF_STAT);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Kd::OFF_BAR);
-    uint64_t *fix_full = bars, *r0_full = bars + 1, *r0_empty = bars + 3, *r1_full = bars + 5, *r1_empty = bars + 7;
-    uint64_t *s_full = bars + 9, *p_ready = bars + 11, *stats_ready = bars + 13, *done = bars + 16, *drain = bars + 17;
+    uint64_t *fix_full = bars, *r0_full = bars + 1, *r0_empty = bars + 3, *r1_full = bars + 5, *r1_empty = bars + 8;
+    uint64_t *s_full = bars + 11, *p_ready = bars + 13, *stats_ready = bars + 15, *done = bars + 18, *drain = bars + 19;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Kd::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Kd::OFF_MISC + 4);
     const uint64_t lim = p.timeout_ns;
@@ -229,10 +230,12 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int s = 0; s < 2; ++s) {
             mbar_init(&r0_full[s], 1);
             mbar_init(&r0_empty[s], 1);
-            mbar_init(&r1_full[s], 1);
-            mbar_init(&r1_empty[s], 1);
             mbar_init(&s_full[s], 1);
             mbar_init(&p_ready[s], C::NUM_EW);
+        }
+        for (int s = 0; s < 3; ++s) {
+            mbar_init(&r1_full[s], 1);
+            mbar_init(&r1_empty[s], 1);
         }
         for (int s = 0; s < Kd::STAT_SLOTS; ++s) mbar_init(&stats_ready[s], STEP);  // 64 publishing threads
         mbar_init(done, 1);
@@ -343,8 +346,8 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     umma_commit_elect(&r0_empty[k & 1]);
                     if (k + 1 < n && !(ok = issue_y(k + 1))) break;
                 } else {
-                    const int s1 = k & 1;
-                    if (!(ok = wait_all(&r1_full[s1], (k >> 1) & 1, 526 + s1))) break;
+                    const int s1 = k % Kd::R1_SLOTS;
+                    if (!(ok = wait_all(&r1_full[s1], (k / Kd::R1_SLOTS) & 1, 526 + s1))) break;
                     tc_fence_after_sync();
                     mma_update<BF16>(tmem + C::COL_ACC, zbuf, r1_tile(s1), k > 0);  // dV += P^T dO
                     umma_commit_elect(&r1_empty[s1]);
